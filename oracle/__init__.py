@@ -1,0 +1,187 @@
+"""CPU oracle of the fixed-codebook entropy coder (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may import this
+package. It wraps ``oracle.cpp`` (plain C++17, bit-serial) through ctypes and shares nothing with
+the CUDA library. ``build()`` compiles it with g++ into ``oracle/liboracle.so``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "oracle.cpp")
+LIB = os.path.join(HERE, "liboracle.so")
+
+ERR_ARG, ERR_UNCODABLE, ERR_CORRUPT, ERR_CODEBOOK, ERR_CAPACITY = 1, 4, 8, 16, 64
+KIND_HUFFMAN, KIND_QLC = 0, 1
+QLC_LMAX = 11
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.cpp with g++ (-O2, no GPU code) unless the library is newer than it."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.run(["g++", "-std=c++17", "-O2", "-fPIC", "-shared", "-Wall", "-o", tmp, SRC],
+                       check=True)
+        os.replace(tmp, LIB)
+    return LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(LIB)
+        P, u64, i32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int
+        sig = {
+            "orc_histogram": (None, [P, u64, P]),
+            "orc_huffman_lengths": (i32, [P, i32, i32, P]),
+            "orc_canonical_codes": (None, [P, P]),
+            "orc_qlc_build": (i32, [P, i32, P, P, P, P, P]),
+            "orc_hash_huffman": (u64, [i32, P]),
+            "orc_hash_qlc": (u64, [P, P]),
+            "orc_payload_offset": (u64, [u64]),
+            "orc_sync_offset": (u64, [u64]),
+            "orc_encode_bound": (u64, [u64]),
+            "orc_encode_huffman": (i32, [i32, P, P, u64, P, u64, P]),
+            "orc_decode_huffman": (i32, [i32, P, P, u64, P, u64]),
+            "orc_encode_qlc": (i32, [P, P, P, P, u64, P, u64, P]),
+            "orc_decode_qlc": (i32, [P, P, P, P, u64, P, u64]),
+            "orc_entropy": (ctypes.c_double, [P]),
+            "orc_fnv1a": (u64, [P, u64]),
+            "orc_mean_length": (ctypes.c_double, [P, P]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u8(x) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(x, dtype=np.uint8).reshape(-1))
+
+
+def histogram(x) -> np.ndarray:
+    x = _u8(x)
+    c = np.zeros(256, dtype=np.uint64)
+    lib().orc_histogram(_p(x), x.size, _p(c))
+    return c
+
+
+def huffman_lengths(counts, lmax: int = 12, cover_all: bool = True) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.uint64))
+    ln = np.zeros(256, dtype=np.uint8)
+    rc = lib().orc_huffman_lengths(_p(c), int(lmax), int(bool(cover_all)), _p(ln))
+    if rc:
+        raise ValueError("lmax too small for the alphabet")
+    return ln
+
+
+def canonical_codes(lengths) -> np.ndarray:
+    ln = _u8(lengths)
+    code = np.zeros(256, dtype=np.uint32)
+    lib().orc_canonical_codes(_p(ln), _p(code))
+    return code
+
+
+@dataclass
+class Codebook:
+    kind: int
+    lmax: int
+    len: np.ndarray        # u8[256]
+    code: np.ndarray       # u32[256]
+    bits: np.ndarray | None = None      # QLC u8[8]
+    start: np.ndarray | None = None     # QLC u16[9]
+    rank2sym: np.ndarray | None = None  # QLC u8[256]
+
+    @property
+    def hash(self) -> int:
+        L = lib()
+        if self.kind == KIND_HUFFMAN:
+            return int(L.orc_hash_huffman(self.lmax, _p(self.len)))
+        return int(L.orc_hash_qlc(_p(self.bits), _p(self.rank2sym)))
+
+
+def huffman_codebook(counts, lmax: int = 12, cover_all: bool = True) -> Codebook:
+    ln = huffman_lengths(counts, lmax, cover_all)
+    return Codebook(KIND_HUFFMAN, lmax, ln, canonical_codes(ln))
+
+
+def qlc_codebook(counts, max_distinct: int = 4) -> Codebook:
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.uint64))
+    bits = np.zeros(8, np.uint8)
+    start = np.zeros(9, np.uint16)
+    r2s = np.zeros(256, np.uint8)
+    ln = np.zeros(256, np.uint8)
+    code = np.zeros(256, np.uint32)
+    rc = lib().orc_qlc_build(_p(c), int(max_distinct), _p(bits), _p(start), _p(r2s), _p(ln), _p(code))
+    if rc:
+        raise ValueError("bad max_distinct")
+    return Codebook(KIND_QLC, QLC_LMAX, ln, code, bits, start, r2s)
+
+
+def payload_offset(n: int) -> int:
+    return int(lib().orc_payload_offset(n))
+
+
+def sync_offset(n: int) -> int:
+    return int(lib().orc_sync_offset(n))
+
+
+def encode_bound(n: int) -> int:
+    return int(lib().orc_encode_bound(n))
+
+
+def encode(cb: Codebook, x, cap: int | None = None) -> tuple[int, np.ndarray]:
+    """Bit-serial encode into the chunked stream; returns (status, stream bytes)."""
+    x = _u8(x)
+    cap = encode_bound(x.size) if cap is None else int(cap)
+    out = np.zeros(max(cap, 1), dtype=np.uint8)
+    written = ctypes.c_uint64(0)
+    if cb.kind == KIND_HUFFMAN:
+        st = lib().orc_encode_huffman(cb.lmax, _p(cb.len), _p(x), x.size, _p(out), cap,
+                                      ctypes.byref(written))
+    else:
+        st = lib().orc_encode_qlc(_p(cb.bits), _p(cb.start), _p(cb.rank2sym), _p(x), x.size,
+                                  _p(out), cap, ctypes.byref(written))
+    return int(st), out[: written.value] if written.value else out[: min(cap, 64)]
+
+
+def decode(cb: Codebook, stream, n: int) -> tuple[int, np.ndarray]:
+    """Bit-serial decode; returns (status, n bytes)."""
+    s = _u8(stream)
+    out = np.zeros(max(n, 1), dtype=np.uint8)
+    if cb.kind == KIND_HUFFMAN:
+        st = lib().orc_decode_huffman(cb.lmax, _p(cb.len), _p(s), s.size, _p(out), n)
+    else:
+        st = lib().orc_decode_qlc(_p(cb.bits), _p(cb.start), _p(cb.rank2sym), _p(s), s.size,
+                                  _p(out), n)
+    return int(st), out[:n]
+
+
+def fnv1a(data: bytes) -> int:
+    b = np.frombuffer(bytes(data), dtype=np.uint8).copy() if data else np.zeros(1, np.uint8)
+    return int(lib().orc_fnv1a(_p(b), len(data)))
+
+
+def entropy(counts) -> float:
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.uint64))
+    return float(lib().orc_entropy(_p(c)))
+
+
+def mean_length(counts, lengths) -> float:
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.uint64))
+    return float(lib().orc_mean_length(_p(c), _p(_u8(lengths))))
