@@ -353,7 +353,9 @@ int decode(const Header& h, const Dec& dec, const uint8_t* st, uint64_t bytes, u
   if (n != n_expected || rd64(st + 24) != n_chunks_of(n)) return kErrCorrupt;
   const uint64_t nc = n_chunks_of(n), S = sync_offset(n), P = payload_offset(n);
   const uint64_t total = rd64(st + 32);
-  if (P > bytes || total > (bytes - P) / 4) return kErrCorrupt;
+  // the stream holds the payload and its 2 guard words; word offsets are u32
+  if (P > bytes || (bytes - P) / 4 < 2 || total > (bytes - P) / 4 - 2 || total >= (1ull << 32))
+    return kErrCorrupt;
   int status = 0;
   for (uint64_t c = 0; c < nc; ++c) {
     const uint64_t lo = c * kChunk, hi = std::min(n, lo + kChunk);
