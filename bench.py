@@ -1,0 +1,399 @@
+#!/usr/bin/env python3
+"""Benchmark of the fixed-codebook entropy coder on B200: one JSON line on rank 0.
+
+Workload (one step): a 1 GiB batch of e4m3 bytes (fp32 N(0,1)*0.5, RNE-saturating cast), the
+fixed Huffman codebook (package-merge, Lmax 12) and the Quad Length Code built from the summed
+histogram of 4 earlier 1 MiB batches of the same law. A step runs the whole hot path on the batch:
+Huffman encode with the histogram fused in, Huffman decode, QLC encode, QLC decode. The metric is
+uncompressed bytes through the codec per second (4 x 1 GiB per step) and bits per symbol.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hx|reference]
+
+Timing: W untimed steps, then exactly K steps between a barrier + synchronize on both sides,
+CUDA events on the stream the kernels run on, max over ranks. The inputs (1 GiB) are larger than
+the 126 MB L2, so no flush is needed between steps. `--impl reference` times the CPU oracle (the
+reference implementation of this build) on a bounded sample of the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_BYTES = 1 << 30
+WORKLOAD = ("cfg4: 1 GiB e4m3 bytes of N(0,1)*0.5; fixed Huffman (Lmax 12) and QLC (8 areas) "
+            "from 4 prior 1 MiB batches; step = Huffman encode(+fused histogram) + decode + "
+            "QLC encode + decode")
+METRIC = "encode & decode GB/s (uncompressed) at 1 B200, % of HBM roofline; bits/symbol"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["lossless_entropy_coding_fixed_b200/csrc/hx_kernels.cu",
+                  "lossless_entropy_coding_fixed_b200/csrc/hx_tables.h"]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="hx", choices=["hx", "reference"])
+    p.add_argument("--n", type=int, default=N_BYTES, help="bytes per batch (default 1 GiB)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    k = rec.get("kernels", {}).get(kernel)
+    if not k or rec.get("n") is None:
+        return None
+    return k["dram_bytes_per_launch"] * (N_BYTES / rec["n"])
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc, self.out = index, None, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = None
+
+    def summary(self):
+        if not self.out:
+            return None
+        rows = [r.split(", ") for r in self.out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        if not sm:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+def cpu_reference(args, rank, ws):
+    """The oracle on a bounded sample of the workload (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import oracle
+    import datagen
+    sample = 1 << 20
+    counts = sum(oracle.histogram(b) for b in datagen.prior_batches(4))
+    hb, qb = oracle.huffman_codebook(counts), oracle.qlc_codebook(counts)
+    x = datagen.data(4, n=sample)
+
+    def step():
+        _, sh = oracle.encode(hb, x)
+        oracle.decode(hb, sh, x.size)
+        _, sq = oracle.encode(qb, x)
+        oracle.decode(qb, sq, x.size)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = 4 * sample * args.steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_bytes_per_step": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {sample} bytes of the 1 GiB batch per step, "
+                                   "single-thread bit-serial C++"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline_leg(counts):
+    """Time the oracle as it stands on a 64 MiB slice of the workload (~10-30 s, one core)."""
+    import oracle
+    import datagen
+    sample = 64 << 20
+    x = datagen.data(4, n=sample)
+    hb, qb = oracle.huffman_codebook(counts), oracle.qlc_codebook(counts)
+    t0 = time.perf_counter()
+    _, sh = oracle.encode(hb, x)
+    oracle.decode(hb, sh, x.size)
+    _, sq = oracle.encode(qb, x)
+    oracle.decode(qb, sq, x.size)
+    dt = time.perf_counter() - t0
+    return {"value": 4 * sample / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {sample >> 20} MiB of the batch through the same 4 codec calls "
+                      f"({dt:.1f} s, single-thread bit-serial C++)"}
+
+
+# ---------------------------------------------------------------------------------------------
+def main():
+    args = parse()
+    rank, local_rank, ws = dist_env()
+    if args.impl == "reference":
+        return cpu_reference(args, rank, ws)
+
+    import torch
+    import datagen
+    from lossless_entropy_coding_fixed_b200 import hx
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    n = args.n
+    # codebooks from the prior batches (host, off the data path)
+    pc = torch.zeros(256, dtype=torch.int32, device=dev)
+    for b in datagen.prior_batches(4):
+        hx.histogram(torch.from_numpy(b).to(dev), pc)
+    prior = pc.cpu().numpy().astype(np.uint64)
+    t0 = time.perf_counter()
+    hcb = hx.build_codebook(prior)
+    t1 = time.perf_counter()
+    qcb = hx.qlc_build(prior)
+    t2 = time.perf_counter()
+    x_host = datagen.data(4, n=n)
+    x = torch.from_numpy(x_host).to(dev)
+    ht, qt = hcb.upload(dev), qcb.upload(dev)
+    bound = hx.encode_bound(n)
+    sh = torch.empty(bound, dtype=torch.uint8, device=dev)
+    sq = torch.empty(bound, dtype=torch.uint8, device=dev)
+    scratch = torch.empty(hx.scratch_bytes(n), dtype=torch.uint8, device=dev)
+    y = torch.empty(n, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    # one fused-histogram row per timed step, so no counter is reset inside the timed region
+    hist = torch.zeros(args.steps + 1, 256, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ops = ["huffman_encode", "huffman_decode", "qlc_encode", "qlc_decode"]
+    ev = {o: [] for o in ops}
+
+    def step(record: bool, row: int = 0):
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
+        if record:
+            marks[0].record(stream)
+        hx.encode(ht, x, out=sh, scratch=scratch, hist=hist[row], status=status,
+                  kind=hx.KIND_HUFFMAN)
+        if record:
+            marks[1].record(stream)
+        hx.decode(ht, sh, n, out=y, status=status, kind=hx.KIND_HUFFMAN)
+        if record:
+            marks[2].record(stream)
+        hx.encode(qt, x, out=sq, scratch=scratch, status=status, kind=hx.KIND_QLC)
+        if record:
+            marks[3].record(stream)
+        hx.decode(qt, sq, n, out=y, status=status, kind=hx.KIND_QLC)
+        if record:
+            marks[4].record(stream)
+            for i, o in enumerate(ops):
+                ev[o].append((marks[i], marks[i + 1]))
+
+    for _ in range(max(3, args.warmup)):
+        step(False, args.steps)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, f"status {int(status.item())}"
+    # correctness of the timed configuration: both codecs round-trip the batch
+    hx.decode(ht, sh, n, out=y, status=status)
+    assert torch.equal(y, x)
+    hx.decode(qt, sq, n, out=y, status=status, kind=hx.KIND_QLC)
+    assert torch.equal(y, x)
+    torch.cuda.synchronize(dev)
+
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(True, i)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    if pg:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    assert int(status.item()) == 0, f"status {int(status.item())}"
+    per_op_ms = {o: sum(a.elapsed_time(b) for a, b in ev[o]) / args.steps for o in ops}
+
+    # sizes and bits per symbol
+    rows = hist[: args.steps].cpu().numpy().astype(np.uint64)
+    h = rows[0]
+    assert int(h.sum()) == n and (rows == h).all()
+    size_h, size_q = hx.stream_size(sh, n), hx.stream_size(sq, n)
+    payload_bits_h = hx.mean_length(h, hcb)
+    payload_bits_q = hx.mean_length(h, qcb)
+    per_shard = hx.mean_length(h, hx.build_codebook(h, seen_only=True))
+    H = hx.entropy(h)
+    alg_bytes = {"huffman_encode": n + size_h, "huffman_decode": size_h + n,
+                 "qlc_encode": n + size_q, "qlc_decode": size_q + n}
+    ms_per_step = elapsed_ms / args.steps
+    value = ws * 4 * n / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    dominant = max(ops, key=lambda o: per_op_ms[o])
+    achieved = alg_bytes[dominant] / (per_op_ms[dominant] * 1e-3) / 1e9
+    kernel_name = {"huffman_encode": "k_encode", "qlc_encode": "k_encode",
+                   "huffman_decode": "k_decode<0>", "qlc_decode": "k_decode<1>"}[dominant]
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_pin = torch.from_numpy(x_host).pin_memory()
+        out_h = torch.empty(bound, dtype=torch.uint8).pin_memory()
+        out_q = torch.empty(bound, dtype=torch.uint8).pin_memory()
+        st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+        hdr = torch.empty(64, dtype=torch.uint8).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_pin, non_blocking=True)
+            hx.encode(ht, x, out=sh, scratch=scratch, status=status, kind=hx.KIND_HUFFMAN)
+            hx.decode(ht, sh, n, out=y, status=status)
+            hx.encode(qt, x, out=sq, scratch=scratch, status=status, kind=hx.KIND_QLC)
+            hx.decode(qt, sq, n, out=y, status=status, kind=hx.KIND_QLC)
+            d2h = 0
+            for s_dev, s_host in ((sh, out_h), (sq, out_q)):
+                hdr.copy_(s_dev[:64], non_blocking=True)
+                torch.cuda.synchronize(dev)
+                size = hx.stream_bytes(n, int(hdr[32:40].numpy().view(np.uint64)[0]))
+                s_host[:size].copy_(s_dev[:size], non_blocking=True)
+                d2h += size + 64
+            st_host.copy_(status, non_blocking=True)
+            torch.cuda.synchronize(dev)
+            assert int(st_host.item()) == 0
+            return d2h + 4
+
+        e2e_step()
+        k_e2e = max(3, min(args.steps, 10))
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        d2h = 0
+        for _ in range(k_e2e):
+            d2h = e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = s0.elapsed_time(s1) / k_e2e
+        if pg:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": ws * 4 * n / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": n, "d2h_bytes_per_step": d2h, "steps": k_e2e,
+               "path": "pinned host batch -> H2D -> 4 codec calls -> D2H of both streams"}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_leg(prior)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "n_bytes_per_gpu": n, "chunk": 4096,
+                       "substreams": 8, "lmax": 12,
+                       "l2": "inputs larger than L2 (1 GiB per tensor vs 126 MB), no flush",
+                       "parallelism": f"replicas x{ws} (independent batches, no collective)"},
+            "ops": {o: {"ms": per_op_ms[o], "GB_per_s_uncompressed": n / (per_op_ms[o] * 1e-3) / 1e9,
+                        "hbm_GB_per_s_algorithmic": alg_bytes[o] / (per_op_ms[o] * 1e-3) / 1e9}
+                    for o in ops},
+            "bits_per_symbol": {"huffman_payload": payload_bits_h,
+                                "huffman_framed": size_h * 8 / n,
+                                "qlc_payload": payload_bits_q, "qlc_framed": size_q * 8 / n,
+                                "per_shard_huffman": per_shard, "entropy": H,
+                                "fixed_vs_per_shard": payload_bits_h / per_shard - 1,
+                                "fixed_vs_entropy": payload_bits_h / H - 1},
+            "host_codebook_build_us": {"huffman": (t1 - t0) * 1e6, "qlc": (t2 - t1) * 1e6},
+            "roofline": {"bound": "hbm", "kernel": kernel_name, "op": dominant,
+                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": recorded_traffic(kernel_name),
+                         "algorithmic_bytes_per_launch": alg_bytes[dominant]},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 6 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,167 @@
+/*
+ * hx.h -- C ABI of the fixed-codebook entropy coder for 8-bit tensor symbols (e4m3 / INT8 bytes)
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Method. "Single-Stage Huffman Encoder for ML Compression" (abstract): a Huffman codebook is
+ * fixed in advance from the average symbol distribution of previous batches, so the data path
+ * runs no frequency pass, builds no codebook and ships no codebook with the data. "Quad Length
+ * Codes for Lossless Compression of e4m3" (abstract, Tables 1-2): a variant whose code is a 3-bit
+ * area prefix followed by a fixed-width index inside the area, driven by a 256-entry table.
+ * "Lossless" is exact reconstruction of every input byte.
+ *
+ * Conventions for every call below.
+ *  - Pointers named d_* are device memory; all others are host memory. Every buffer belongs to
+ *    the caller: the library never allocates, frees or synchronises. Device work is enqueued on
+ *    `stream` (a cudaStream_t passed as void*; NULL = the legacy default stream) in call order.
+ *  - The return value (int) carries host-detected errors only: bad arguments, unsupported
+ *    alignment, launch failures. 0 = enqueued. Errors found in the data on the device (an
+ *    uncodable symbol, a corrupt stream, a codebook mismatch, a full output buffer) are OR-ed
+ *    into the caller's device word *d_status, which the caller zeroes before and reads after the
+ *    stream is synchronised. Data errors never trap the device: reads are clamped to the
+ *    buffers' valid ranges and every wait is bounded.
+ *  - d_in / d_out / d_stream must be 16-byte aligned (as every torch allocation is); n < 2^32.
+ *
+ * Stream format (version 1). All integers little-endian; offsets from the stream start.
+ *    0 u32 magic 0x31305848 ("HX01")   4 u8 version = 1   5 u8 kind (0 Huffman, 1 QLC)
+ *    6 u8 lmax (Huffman: the build's limit; QLC: 11)       7 u8 0
+ *    8 u32 chunk = 4096 symbols        12 u32 sub-streams per chunk = 8
+ *   16 u64 n                           24 u64 n_chunks = ceil(n / 4096)
+ *   32 u64 total_words                 40 u64 codebook hash (FNV-1a-64, see hx_codebook.hash)
+ *   48 16 zero bytes
+ *   64 u32 word_off[n_chunks + 1]: payload word where each chunk starts; [n_chunks] = total
+ *    S = round_up(64 + 4 * (n_chunks + 1), 16): u16 sync[n_chunks][8]. sync[c][0] = the number
+ *        of valid bits of chunk c; sync[c][k], k = 1..7, = bit offset of the chunk's symbol 512k
+ *        (the bit count when the chunk has no symbol 512k).
+ *    P = S + 16 * n_chunks = hx_payload_offset(n): u32 payload[total_words]. Codes are written
+ *        most-significant bit first (bit 31 of a word comes first) and each chunk is zero-padded
+ *        to a whole word; two zero guard words follow. Stream size = P + 4 * (total_words + 2).
+ */
+#ifndef HX_H
+#define HX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status bits: host return values and the device status word use the same codes. */
+typedef enum {
+  HX_OK = 0,
+  HX_ERR_ARG = 1,        /* invalid argument (null pointer, size, alignment, kind)          */
+  HX_ERR_CUDA = 2,       /* a CUDA runtime call or kernel launch failed                      */
+  HX_ERR_UNCODABLE = 4,  /* encode: an input byte has no code word (seen-only codebook)      */
+  HX_ERR_CORRUPT = 8,    /* decode: the stream is malformed or does not decode exactly      */
+  HX_ERR_CODEBOOK = 16,  /* decode: the stream was written with another codebook or kind    */
+  HX_ERR_TIMEOUT = 32,   /* encode: the chunk-offset scan waited past its bound              */
+  HX_ERR_CAPACITY = 64   /* encode: out_cap is too small; header.total_words holds the need */
+} hx_status;
+
+enum { HX_KIND_HUFFMAN = 0, HX_KIND_QLC = 1 };
+enum { HX_CHUNK = 4096, HX_SUBSTREAMS = 8, HX_LMAX_MAX = 12, HX_QLC_LMAX = 11 };
+enum { HX_CB_SEEN_ONLY = 1 }; /* hx_build_codebook flag: no code for bytes with count 0 */
+
+/* Bytes of the device table block that hx_codebook_upload writes and the codecs read. */
+#define HX_TABLES_BYTES 10240
+
+/* A codebook, built on the host. Huffman: len/code per byte value (canonical, RFC 1951 order).
+ * QLC: qlc_bits[a] index bits of area a, areas hold ranks [qlc_start[a], qlc_start[a+1]),
+ * rank2sym[r] the byte value of rank r; len/code are filled in as well (len = 3 + bits). */
+typedef struct {
+  uint8_t kind;          /* HX_KIND_HUFFMAN or HX_KIND_QLC                                */
+  uint8_t lmax;          /* Huffman: length limit of the build; QLC: 11                   */
+  uint8_t len[256];      /* code length in bits of each byte value, 0 = no code           */
+  uint16_t code[256];    /* code word, right-aligned in len bits                          */
+  uint8_t qlc_bits[8];   /* QLC only                                                      */
+  uint16_t qlc_start[9]; /* QLC only                                                      */
+  uint8_t rank2sym[256]; /* QLC only                                                      */
+  uint64_t hash;         /* FNV-1a-64 of [kind, lmax, len[256]] (Huffman) or of
+                            [kind, 11, qlc_bits[8], rank2sym[256]] (QLC); the stream header
+                            carries it in place of the codebook                            */
+} hx_codebook;
+
+/* Length-limited canonical Huffman codebook from summed counts.
+ * "Single-Stage Huffman Encoder for ML Compression", abstract: the counts are the sum over
+ * previous equal-size batches (the average distribution, up to scale). Every byte value gets a
+ * code (weight max(count, 1)) unless flags has HX_CB_SEEN_ONLY. Lengths come from package-merge
+ * (Larmore & Hirschberg 1990) with limit lmax in [1, 12]; ties: leaves by (count, byte value),
+ * a leaf before a package of equal weight. Codes are canonical (RFC 1951 section 3.2.2).
+ * counts: host u64[256]. Returns HX_ERR_ARG for a null pointer or an lmax the alphabet cannot
+ * fit in (2^lmax < number of coded symbols). */
+int hx_build_codebook(const uint64_t* counts, int lmax, uint32_t flags, hx_codebook* out);
+
+/* Quad Length Code from counts. "Quad Length Codes for Lossless Compression of e4m3", abstract
+ * and Tables 1-2: byte values ranked by count (descending, ties to the smaller value) fill 8
+ * areas in order; area a codes its symbols as a (3 bits) followed by the rank inside the area
+ * (qlc_bits[a] bits). Widths are non-decreasing, hold all 256 ranks, use at most max_distinct
+ * distinct values (4 = "quad"; 1..8), and minimise the mean code length; ties go to the
+ * lexicographically smallest width vector. flags must be 0. */
+int hx_qlc_build(const uint64_t* counts, int max_distinct, uint32_t flags, hx_codebook* out);
+
+/* Pack a codebook into the HX_TABLES_BYTES table block in host memory (host_tables). */
+int hx_codebook_tables(const hx_codebook* cb, void* host_tables);
+
+/* Pack and copy the table block to d_tables (HX_TABLES_BYTES of device memory) on `stream`.
+ * cb may be released when the call returns. */
+int hx_codebook_upload(const hx_codebook* cb, void* d_tables, void* stream);
+
+/* Histogram of byte values: d_counts[v] += occurrences of v in d_in[0..n). d_counts is a
+ * device u32[256] that accumulates (zero it first for a fresh count); n < 2^32.
+ * "Single-Stage Huffman Encoder for ML Compression", abstract (the frequency analysis whose
+ * running average defines the next fixed codebook). */
+int hx_histogram(const uint8_t* d_in, uint64_t n, uint32_t* d_counts, void* stream);
+
+/* Layout helpers (pure functions of n). */
+uint64_t hx_payload_offset(uint64_t n);   /* P above                                         */
+uint64_t hx_sync_offset(uint64_t n);      /* S above                                         */
+uint64_t hx_encode_bound(uint64_t n);     /* largest stream for n bytes: P + 4*(1536*chunks+2) */
+uint64_t hx_scratch_bytes(uint64_t n);    /* device scratch that hx_encode needs             */
+
+/* Encode d_in[0..n) with the fixed Huffman codebook in d_tables into the stream d_out.
+ * "Single-Stage Huffman Encoder for ML Compression", abstract (fixed codebook, nothing sent
+ * but the coded data and a hash of the codebook).
+ * d_out: out_cap bytes, at least hx_payload_offset(n) + 8. If the coded stream does not fit,
+ * HX_ERR_CAPACITY is raised in *d_status, the header (with total_words) and the index are
+ * still written, and the payload is not. d_scratch: hx_scratch_bytes(n) bytes of device memory,
+ * contents ignored on entry and clobbered. d_hist: NULL, or a device u32[256] that accumulates
+ * the histogram of d_in (as hx_histogram) in the same pass. d_status: device u32.
+ * Bytes with no code word raise HX_ERR_UNCODABLE and emit no bits. Tables of the wrong kind
+ * raise HX_ERR_ARG in *d_status. */
+int hx_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out, uint64_t out_cap,
+              void* d_scratch, uint32_t* d_hist, uint32_t* d_status, void* stream);
+
+/* Decode the stream d_stream (stream_bytes bytes) into d_out[0..n_expected).
+ * The header must match: magic, version, chunk, sub-streams, n == n_expected (else
+ * HX_ERR_CORRUPT), kind, lmax and hash == the tables' (else HX_ERR_CODEBOOK). Every chunk's
+ * index entries are checked, and each of its 8 sub-streams must decode to exactly the bit
+ * offset where the next one starts (else HX_ERR_CORRUPT; d_out is then unspecified).
+ * Returns HX_ERR_CORRUPT at once when stream_bytes cannot hold the index for n_expected. */
+int hx_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
+              uint64_t n_expected, uint32_t* d_status, void* stream);
+
+/* The same two calls for a QLC codebook (kind 1 tables): identical stream layout and rules.
+ * "Quad Length Codes for Lossless Compression of e4m3", abstract: decoding reads the 3-bit
+ * area, then the area's fixed number of index bits, then one 256-entry table. */
+int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                  uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
+                  void* stream);
+int hx_qlc_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
+                  uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream);
+
+/* Measurement helpers (host, fp64). Shannon entropy -sum p log2 p of counts[256] in bits per
+ * symbol ("Single-Stage Huffman Encoder for ML Compression", abstract: the ideal the fixed code
+ * is compared with), and the mean code length sum count*len / sum count of a codebook. Both
+ * return 0 for an all-zero histogram and -1 for a null pointer. */
+double hx_entropy(const uint64_t* counts);
+double hx_mean_length(const uint64_t* counts, const hx_codebook* cb);
+
+/* Library format version (1) and a static description of a status code. */
+int hx_version(void);
+const char* hx_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HX_H */

@@ -1,0 +1,284 @@
+// Host side of the hx library: codebook construction (package-merge, canonical codes, the QLC
+// area search), the codebook hash and the device table block. Runs on the CPU, off the data
+// path: "Single-Stage Huffman Encoder for ML Compression" (abstract) builds the codebook once
+// from earlier batches, so nothing here sits between a batch and its coded stream.
+#include <algorithm>
+#include <cmath>
+#include <cstddef>
+#include <cstring>
+#include <vector>
+
+#include "hx.h"
+#include "hx_tables.h"
+
+namespace {
+
+constexpr uint64_t kFnvBasis = 14695981039346656037ull;
+constexpr uint64_t kFnvPrime = 1099511628211ull;
+
+uint64_t fnv1a_update(uint64_t h, const uint8_t* p, size_t n) {
+  for (size_t i = 0; i < n; ++i) h = (h ^ p[i]) * kFnvPrime;
+  return h;
+}
+
+// ---- package-merge (Larmore & Hirschberg 1990) ------------------------------------------
+// Items live in a node pool: a leaf names its symbol, a package names its two parts. The
+// selected items are expanded once at the end to count how often each leaf appears.
+struct PmNode {
+  uint64_t weight;
+  int symbol;  // >= 0 for a leaf
+  int part0, part1;
+};
+
+bool lengths_by_package_merge(const uint64_t w[256], int lmax, uint8_t len[256]) {
+  std::memset(len, 0, 256);
+  std::vector<PmNode> pool;
+  std::vector<int> leaves;
+  for (int s = 0; s < 256; ++s)
+    if (w[s]) {
+      leaves.push_back((int)pool.size());
+      pool.push_back({w[s], s, -1, -1});
+    }
+  const size_t m = leaves.size();
+  if (m == 0) return true;
+  if (m == 1) {
+    len[pool[leaves[0]].symbol] = 1;
+    return true;
+  }
+  if (lmax < 1 || lmax > HX_LMAX_MAX || (size_t(1) << lmax) < m) return false;
+  std::stable_sort(leaves.begin(), leaves.end(),
+                   [&](int a, int b) { return pool[a].weight < pool[b].weight; });
+  std::vector<int> row(leaves), next;
+  for (int depth = 1; depth < lmax; ++depth) {
+    next.clear();
+    size_t li = 0, pi = 0;
+    const size_t npk = row.size() / 2;
+    // packages of this row are created lazily, in order, as the merge needs them
+    std::vector<int> pk(npk);
+    for (size_t i = 0; i < npk; ++i) {
+      const PmNode& a = pool[row[2 * i]];
+      const PmNode& b = pool[row[2 * i + 1]];
+      pk[i] = (int)pool.size();
+      pool.push_back({a.weight + b.weight, -1, row[2 * i], row[2 * i + 1]});
+    }
+    while (li < m || pi < npk) {
+      const bool take_leaf =
+          pi == npk || (li < m && pool[leaves[li]].weight <= pool[pk[pi]].weight);
+      next.push_back(take_leaf ? leaves[li++] : pk[pi++]);
+    }
+    row.swap(next);
+  }
+  std::vector<int> stack;
+  int depth_count[256] = {0};
+  for (size_t i = 0; i < 2 * m - 2; ++i) {
+    stack.push_back(row[i]);
+    while (!stack.empty()) {
+      const PmNode& nd = pool[stack.back()];
+      stack.pop_back();
+      if (nd.symbol >= 0) {
+        depth_count[nd.symbol]++;
+      } else {
+        stack.push_back(nd.part0);
+        stack.push_back(nd.part1);
+      }
+    }
+  }
+  for (int s = 0; s < 256; ++s) len[s] = (uint8_t)depth_count[s];
+  return true;
+}
+
+// Canonical code words from lengths, RFC 1951 section 3.2.2: shorter codes first, and within
+// one length in increasing symbol order.
+void canonical(const uint8_t len[256], uint16_t code[256]) {
+  uint32_t per_len[HX_LMAX_MAX + 1] = {0};
+  for (int s = 0; s < 256; ++s)
+    if (len[s]) per_len[len[s]]++;
+  uint32_t first[HX_LMAX_MAX + 1] = {0};
+  uint32_t v = 0;
+  for (int l = 1; l <= HX_LMAX_MAX; ++l) {
+    v = (v + per_len[l - 1]) << 1;
+    first[l] = v;
+  }
+  for (int s = 0; s < 256; ++s) code[s] = len[s] ? (uint16_t)first[len[s]]++ : 0;
+}
+
+// ---- QLC area search -------------------------------------------------------------------
+struct QlcSearch {
+  unsigned __int128 prefix[257];  // prefix[r] = total weight of ranks < r
+  int max_distinct;
+  int cur[8];
+  int best[8];
+  bool found = false;
+  unsigned __int128 best_cost = 0;
+
+  // Width vectors are visited depth-first with non-decreasing widths: lexicographic order, so
+  // the first vector reaching the minimum is the smallest one.
+  void visit(int area, int min_width, int distinct, int covered, unsigned __int128 cost) {
+    if (area == 8) {
+      if (covered == 256 && (!found || cost < best_cost)) {
+        found = true;
+        best_cost = cost;
+        std::memcpy(best, cur, sizeof cur);
+      }
+      return;
+    }
+    for (int b = min_width; b <= 8; ++b) {
+      const int d = distinct + ((area == 0 || b != cur[area - 1]) ? 1 : 0);
+      if (d > max_distinct) continue;
+      const int take = std::min(1 << b, 256 - covered);
+      cur[area] = b;
+      visit(area + 1, b, d, covered + take,
+            cost + (prefix[covered + take] - prefix[covered]) * (unsigned)(3 + b));
+    }
+  }
+};
+
+int fill_qlc(const uint64_t counts[256], int max_distinct, hx_codebook* out) {
+  int rank[256];
+  for (int s = 0; s < 256; ++s) rank[s] = s;
+  std::stable_sort(rank, rank + 256, [&](int a, int b) { return counts[a] > counts[b]; });
+  QlcSearch q;
+  q.max_distinct = max_distinct;
+  q.prefix[0] = 0;
+  for (int r = 0; r < 256; ++r) q.prefix[r + 1] = q.prefix[r] + counts[rank[r]];
+  q.visit(0, 0, 0, 0, 0);
+  if (!q.found) return HX_ERR_ARG;
+  std::memset(out, 0, sizeof *out);
+  out->kind = HX_KIND_QLC;
+  out->lmax = HX_QLC_LMAX;
+  int r = 0;
+  for (int a = 0; a < 8; ++a) {
+    out->qlc_bits[a] = (uint8_t)q.best[a];
+    out->qlc_start[a] = (uint16_t)r;
+    const int take = std::min(1 << q.best[a], 256 - r);
+    for (int i = 0; i < take; ++i, ++r) {
+      const int s = rank[r];
+      out->len[s] = (uint8_t)(3 + q.best[a]);
+      out->code[s] = (uint16_t)((a << q.best[a]) | i);
+    }
+  }
+  out->qlc_start[8] = (uint16_t)r;
+  for (int i = 0; i < 256; ++i) out->rank2sym[i] = (uint8_t)rank[i];
+  const uint8_t head[2] = {HX_KIND_QLC, HX_QLC_LMAX};
+  uint64_t h = fnv1a_update(kFnvBasis, head, 2);
+  h = fnv1a_update(h, out->qlc_bits, 8);
+  out->hash = fnv1a_update(h, out->rank2sym, 256);
+  return HX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hx_build_codebook(const uint64_t* counts, int lmax, uint32_t flags, hx_codebook* out) {
+  if (!counts || !out || (flags & ~(uint32_t)HX_CB_SEEN_ONLY)) return HX_ERR_ARG;
+  uint64_t w[256];
+  for (int s = 0; s < 256; ++s)
+    w[s] = (flags & HX_CB_SEEN_ONLY) ? counts[s] : std::max<uint64_t>(counts[s], 1);
+  hx_codebook cb;
+  std::memset(&cb, 0, sizeof cb);
+  if (!lengths_by_package_merge(w, lmax, cb.len)) return HX_ERR_ARG;
+  cb.kind = HX_KIND_HUFFMAN;
+  cb.lmax = (uint8_t)lmax;
+  canonical(cb.len, cb.code);
+  const uint8_t head[2] = {HX_KIND_HUFFMAN, (uint8_t)lmax};
+  cb.hash = fnv1a_update(fnv1a_update(kFnvBasis, head, 2), cb.len, 256);
+  *out = cb;
+  return HX_OK;
+}
+
+int hx_qlc_build(const uint64_t* counts, int max_distinct, uint32_t flags, hx_codebook* out) {
+  if (!counts || !out || flags || max_distinct < 1 || max_distinct > 8) return HX_ERR_ARG;
+  return fill_qlc(counts, max_distinct, out);
+}
+
+int hx_codebook_tables(const hx_codebook* cb, void* host_tables) {
+  if (!cb || !host_tables) return HX_ERR_ARG;
+  if (cb->kind != HX_KIND_HUFFMAN && cb->kind != HX_KIND_QLC) return HX_ERR_ARG;
+  std::memset(host_tables, 0, HX_TABLES_BYTES);
+  hx::Tables* t = static_cast<hx::Tables*>(host_tables);
+  for (int s = 0; s < 256; ++s) {
+    const int l = cb->len[s];
+    if (l > HX_LMAX_MAX || (l && (cb->code[s] >> l))) return HX_ERR_ARG;
+    t->enc[s] = ((uint32_t)cb->code[s] << 4) | (uint32_t)l;
+    if (!l) continue;
+    const uint32_t lo = (uint32_t)cb->code[s] << (HX_LMAX_MAX - l);
+    const uint32_t hi = lo + (1u << (HX_LMAX_MAX - l));
+    for (uint32_t wv = lo; wv < hi; ++wv) {
+      if (t->dec[wv]) return HX_ERR_ARG;  // not a prefix code
+      t->dec[wv] = (uint16_t)((l << 8) | s);
+    }
+  }
+  if (cb->kind == HX_KIND_QLC) {
+    std::memcpy(t->rank2sym, cb->rank2sym, 256);
+    for (int a = 0; a < 8; ++a) {
+      const uint32_t first = cb->qlc_start[a], fill = cb->qlc_start[a + 1] - cb->qlc_start[a];
+      if (cb->qlc_bits[a] > 8 || cb->qlc_start[a + 1] < cb->qlc_start[a] ||
+          fill > (1u << cb->qlc_bits[a]))
+        return HX_ERR_ARG;
+      t->qlc_area[a] = first | (fill << 9) | ((uint32_t)cb->qlc_bits[a] << 18);
+      t->qlc_bits_packed |= (uint32_t)cb->qlc_bits[a] << (4 * a);
+    }
+  }
+  t->kind = cb->kind;
+  t->lmax = cb->lmax;
+  t->magic = hx::kTablesMagic;
+  t->hash = cb->hash;
+  return HX_OK;
+}
+
+uint64_t hx_sync_offset(uint64_t n) {
+  const uint64_t chunks = (n + HX_CHUNK - 1) / HX_CHUNK;
+  return (64 + 4 * (chunks + 1) + 15) / 16 * 16;
+}
+
+uint64_t hx_payload_offset(uint64_t n) {
+  return hx_sync_offset(n) + 16 * ((n + HX_CHUNK - 1) / HX_CHUNK);
+}
+
+uint64_t hx_encode_bound(uint64_t n) {
+  const uint64_t chunks = (n + HX_CHUNK - 1) / HX_CHUNK;
+  return hx_payload_offset(n) + 4 * (chunks * (HX_CHUNK * HX_LMAX_MAX / 32) + 2);
+}
+
+double hx_entropy(const uint64_t* counts) {
+  if (!counts) return -1;
+  long double total = 0;
+  for (int s = 0; s < 256; ++s) total += counts[s];
+  if (total == 0) return 0;
+  double h = 0;
+  for (int s = 0; s < 256; ++s)
+    if (counts[s]) {
+      const double p = (double)(counts[s] / total);
+      h -= p * std::log2(p);
+    }
+  return h;
+}
+
+double hx_mean_length(const uint64_t* counts, const hx_codebook* cb) {
+  if (!counts || !cb) return -1;
+  long double total = 0, bits = 0;
+  for (int s = 0; s < 256; ++s) {
+    total += counts[s];
+    bits += (long double)counts[s] * cb->len[s];
+  }
+  return total == 0 ? 0 : (double)(bits / total);
+}
+
+int hx_version(void) { return 1; }
+
+const char* hx_status_string(int code) {
+  switch (code) {
+    case HX_OK: return "ok";
+    case HX_ERR_ARG: return "invalid argument";
+    case HX_ERR_CUDA: return "CUDA error";
+    case HX_ERR_UNCODABLE: return "input byte without a code word";
+    case HX_ERR_CORRUPT: return "corrupt stream";
+    case HX_ERR_CODEBOOK: return "stream written with another codebook";
+    case HX_ERR_TIMEOUT: return "chunk-offset scan timed out";
+    case HX_ERR_CAPACITY: return "output buffer too small";
+    default: return "several errors (bit set)";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,33 @@
+// Device table block of the hx library (private to the library; HX_TABLES_BYTES bytes).
+// Written on the host by hx_codebook_tables / hx_codebook_upload, read by the kernels.
+#pragma once
+#include <stdint.h>
+
+#include "hx.h"
+
+namespace hx {
+
+constexpr uint32_t kTablesMagic = 0x42545848u;  // "HXTB"
+
+struct Tables {
+  // Encoder: per byte value (code << 4) | len; len 0 = no code word.
+  uint32_t enc[256];
+  // Huffman decoder: for every 12-bit window w, (len << 8) | sym of the code word that w starts
+  // with; 0 when no code word is a prefix of w. (Filled for QLC codebooks as well.)
+  uint16_t dec[4096];
+  // QLC: byte value of each rank.
+  uint8_t rank2sym[256];
+  // QLC area a: first rank (bits 0-8) | number of ranks it holds (bits 9-17) | index bits (18-21).
+  uint32_t qlc_area[8];
+  // QLC: index bits of area a in nibble a.
+  uint32_t qlc_bits_packed;
+  uint32_t kind;
+  uint32_t lmax;
+  uint32_t magic;
+  uint64_t hash;
+};
+
+static_assert(sizeof(Tables) <= HX_TABLES_BYTES, "table block too large");
+static_assert(offsetof(Tables, dec) % 16 == 0, "decode table must be 16-byte aligned");
+
+}  // namespace hx

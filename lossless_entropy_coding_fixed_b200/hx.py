@@ -1,0 +1,275 @@
+"""Python binding of the hx C ABI (include/hx.h): argument marshalling only.
+
+Every step of the coder runs in libhx.so: the codebook builder on the host, the histogram,
+encode and decode kernels on the GPU. PyTorch supplies device memory and the current CUDA
+stream; tensors are passed as raw pointers. There is no fallback: if the library is missing or
+cannot load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import build as _build
+
+HX_OK, HX_ERR_ARG, HX_ERR_CUDA = 0, 1, 2
+HX_ERR_UNCODABLE, HX_ERR_CORRUPT, HX_ERR_CODEBOOK, HX_ERR_TIMEOUT, HX_ERR_CAPACITY = 4, 8, 16, 32, 64
+KIND_HUFFMAN, KIND_QLC = 0, 1
+CHUNK, SUBSTREAMS, LMAX_MAX, QLC_LMAX = 4096, 8, 12, 11
+CB_SEEN_ONLY = 1
+TABLES_BYTES = 10240
+
+HEADER = os.path.join(_build.INCLUDE, "hx.h")
+
+
+class HxError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: status {code} ({status_string(code)})")
+        self.code = code
+
+
+class _Codebook(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_uint8), ("lmax", ctypes.c_uint8),
+                ("len", ctypes.c_uint8 * 256), ("code", ctypes.c_uint16 * 256),
+                ("qlc_bits", ctypes.c_uint8 * 8), ("qlc_start", ctypes.c_uint16 * 9),
+                ("rank2sym", ctypes.c_uint8 * 256), ("hash", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions include/hx.h declares."""
+    with open(HEADER) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return re.findall(r"^\s*(?:int|uint64_t|double|const char\*)\s+(hx_\w+)\s*\(", text,
+                      flags=re.M)
+
+
+def lib():
+    """Load libhx.so (building it first when the sources are newer). Raises if it cannot."""
+    global _lib
+    if _lib is None:
+        if not _build.up_to_date():
+            _build.build()
+        L = ctypes.CDLL(_build.LIB)
+        P, u64, i32, u32 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int, ctypes.c_uint32
+        CB = ctypes.POINTER(_Codebook)
+        sig = {
+            "hx_build_codebook": (i32, [P, i32, u32, CB]),
+            "hx_qlc_build": (i32, [P, i32, u32, CB]),
+            "hx_codebook_tables": (i32, [CB, P]),
+            "hx_codebook_upload": (i32, [CB, P, P]),
+            "hx_histogram": (i32, [P, u64, P, P]),
+            "hx_payload_offset": (u64, [u64]),
+            "hx_sync_offset": (u64, [u64]),
+            "hx_encode_bound": (u64, [u64]),
+            "hx_scratch_bytes": (u64, [u64]),
+            "hx_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
+            "hx_decode": (i32, [P, P, u64, P, u64, P, P]),
+            "hx_qlc_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
+            "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
+            "hx_entropy": (ctypes.c_double, [P]),
+            "hx_mean_length": (ctypes.c_double, [P, CB]),
+            "hx_version": (i32, []),
+            "hx_status_string": (ctypes.c_char_p, [i32]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().hx_status_string(int(code)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc:
+        raise HxError(rc, what)
+
+
+# ------------------------------------------------------------------------------ codebooks (host)
+@dataclass
+class Codebook:
+    """A host codebook (hx_codebook)."""
+    raw: _Codebook
+
+    @property
+    def kind(self) -> int:
+        return self.raw.kind
+
+    @property
+    def lmax(self) -> int:
+        return self.raw.lmax
+
+    @property
+    def len(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.raw.len), np.uint8).copy()
+
+    @property
+    def code(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.raw.code), np.uint16).copy()
+
+    @property
+    def qlc_bits(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.raw.qlc_bits), np.uint8).copy()
+
+    @property
+    def qlc_start(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.raw.qlc_start), np.uint16).copy()
+
+    @property
+    def rank2sym(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.raw.rank2sym), np.uint8).copy()
+
+    @property
+    def hash(self) -> int:
+        return int(self.raw.hash)
+
+    def tables(self) -> bytes:
+        buf = (ctypes.c_uint8 * TABLES_BYTES)()
+        _check(lib().hx_codebook_tables(ctypes.byref(self.raw), buf), "hx_codebook_tables")
+        return bytes(buf)
+
+    def upload(self, device=None):
+        """The table block as a device uint8 tensor (HX_TABLES_BYTES), copied on the current stream."""
+        import torch
+        t = torch.empty(TABLES_BYTES, dtype=torch.uint8, device=device or "cuda")
+        _check(lib().hx_codebook_upload(ctypes.byref(self.raw), t.data_ptr(), _stream(t)),
+               "hx_codebook_upload")
+        return t
+
+
+def _counts(counts) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.uint64).reshape(-1))
+    if c.size != 256:
+        raise ValueError("counts must have 256 entries")
+    return c
+
+
+def build_codebook(counts, lmax: int = 12, seen_only: bool = False) -> Codebook:
+    c = _counts(counts)
+    raw = _Codebook()
+    _check(lib().hx_build_codebook(c.ctypes.data, int(lmax), CB_SEEN_ONLY if seen_only else 0,
+                                   ctypes.byref(raw)), "hx_build_codebook")
+    return Codebook(raw)
+
+
+def qlc_build(counts, max_distinct: int = 4) -> Codebook:
+    c = _counts(counts)
+    raw = _Codebook()
+    _check(lib().hx_qlc_build(c.ctypes.data, int(max_distinct), 0, ctypes.byref(raw)),
+           "hx_qlc_build")
+    return Codebook(raw)
+
+
+def entropy(counts) -> float:
+    """Shannon entropy of a 256-bin histogram, bits per symbol."""
+    c = _counts(counts)
+    return float(lib().hx_entropy(c.ctypes.data))
+
+
+def mean_length(counts, cb: Codebook) -> float:
+    """Mean code length (bits per symbol) of `cb` on data with this histogram."""
+    c = _counts(counts)
+    return float(lib().hx_mean_length(c.ctypes.data, ctypes.byref(cb.raw)))
+
+
+# ------------------------------------------------------------------------------ layout helpers
+def payload_offset(n: int) -> int:
+    return int(lib().hx_payload_offset(n))
+
+
+def sync_offset(n: int) -> int:
+    return int(lib().hx_sync_offset(n))
+
+
+def encode_bound(n: int) -> int:
+    return int(lib().hx_encode_bound(n))
+
+
+def scratch_bytes(n: int) -> int:
+    return int(lib().hx_scratch_bytes(n))
+
+
+def stream_bytes(n: int, total_words: int) -> int:
+    return payload_offset(n) + 4 * (int(total_words) + 2)
+
+
+# ------------------------------------------------------------------------------ device calls
+def _stream(t) -> int:
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dev_u8(x, what):
+    import torch
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.uint8 and x.is_contiguous()):
+        raise TypeError(f"{what} must be a contiguous CUDA uint8 tensor")
+    return x
+
+
+def new_status(device=None):
+    import torch
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def histogram(x, counts=None):
+    """counts (int32[256] on the device) += histogram of x; returns counts."""
+    import torch
+    x = _dev_u8(x, "x")
+    if counts is None:
+        counts = torch.zeros(256, dtype=torch.int32, device=x.device)
+    _check(lib().hx_histogram(x.data_ptr(), x.numel(), counts.data_ptr(), _stream(x)), "hx_histogram")
+    return counts
+
+
+def encode(tables, x, out=None, scratch=None, hist=None, status=None, kind: int = KIND_HUFFMAN):
+    """Encode device bytes x with the device table block `tables`.
+
+    Returns (out, status): out holds the stream (its first stream_size(out, n) bytes are
+    meaningful), status is the device status word (0 when every check passed)."""
+    import torch
+    x = _dev_u8(x, "x")
+    n = x.numel()
+    if out is None:
+        out = torch.empty(encode_bound(n), dtype=torch.uint8, device=x.device)
+    if scratch is None:
+        scratch = torch.empty(scratch_bytes(n), dtype=torch.uint8, device=x.device)
+    if status is None:
+        status = new_status(x.device)
+    fn = lib().hx_encode if kind == KIND_HUFFMAN else lib().hx_qlc_encode
+    _check(fn(tables.data_ptr(), x.data_ptr(), n, out.data_ptr(), out.numel(), scratch.data_ptr(),
+              hist.data_ptr() if hist is not None else None, status.data_ptr(), _stream(x)),
+           "hx_encode")
+    return out, status
+
+
+def decode(tables, stream, n: int, out=None, status=None, kind: int = KIND_HUFFMAN, nbytes=None):
+    """Decode n bytes from the device stream. Returns (out, status)."""
+    import torch
+    stream = _dev_u8(stream, "stream")
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=torch.uint8, device=stream.device)[:n]
+    if status is None:
+        status = new_status(stream.device)
+    fn = lib().hx_decode if kind == KIND_HUFFMAN else lib().hx_qlc_decode
+    _check(fn(tables.data_ptr(), stream.data_ptr(), int(nbytes or stream.numel()),
+              out.data_ptr() if n else stream.data_ptr(), n, status.data_ptr(), _stream(stream)),
+           "hx_decode")
+    return out, status
+
+
+def total_words(stream) -> int:
+    """total_words from a stream header (reads 8 bytes back: synchronises with the stream)."""
+    return int(np.frombuffer(stream[32:40].cpu().numpy().tobytes(), np.uint64)[0])
+
+
+def stream_size(stream, n: int) -> int:
+    return stream_bytes(n, total_words(stream))
