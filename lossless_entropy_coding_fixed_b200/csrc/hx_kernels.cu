@@ -122,6 +122,9 @@ __device__ inline void write_header(const EncodeArgs& a) {
   h64[5] = a.tables->hash;
   h64[6] = 0;
   h64[7] = 0;
+  // zero the alignment gap between word_off[n_chunks] and the 16-byte aligned sync table
+  const uint64_t gap = 64 + 4 * (n_chunks_of(a.n) + 1);
+  for (uint64_t i = gap; i < sync_offset(a.n); i += 4) h32[i / 4] = 0;
 }
 
 // Decoupled look-back: publish this chunk's word count, then add up predecessors until one
