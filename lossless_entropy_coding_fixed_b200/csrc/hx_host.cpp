@@ -206,7 +206,7 @@ int hx_codebook_tables(const hx_codebook* cb, void* host_tables) {
     const uint32_t hi = lo + (1u << (HX_LMAX_MAX - l));
     for (uint32_t wv = lo; wv < hi; ++wv) {
       if (t->dec[wv]) return HX_ERR_ARG;  // not a prefix code
-      t->dec[wv] = (uint16_t)((l << 8) | s);
+      t->dec[wv] = (uint16_t)((s << 8) | l);
     }
   }
   if (cb->kind == HX_KIND_QLC) {
@@ -220,6 +220,9 @@ int hx_codebook_tables(const hx_codebook* cb, void* host_tables) {
       t->qlc_bits_packed |= (uint32_t)cb->qlc_bits[a] << (4 * a);
     }
   }
+  t->complete = 1;
+  for (int wv = 0; wv < 4096; ++wv)
+    if (!t->dec[wv]) t->complete = 0;
   t->kind = cb->kind;
   t->lmax = cb->lmax;
   t->magic = hx::kTablesMagic;

@@ -1,22 +1,34 @@
 // CUDA kernels of the hx library (sm_100a) and the C entry points that launch them.
 //
-//   k_histogram   byte histogram: 16-byte loads, one private 256-bin table per warp in shared
-//                 memory, one global atomic per non-empty bin and block.
-//   k_encode      one 4096-symbol chunk per block iteration (persistent grid, chunks taken in
-//                 order from an atomic ticket): code/length lookup from a shared-memory table,
-//                 warp + block prefix sums of the code lengths (warp k = sub-stream k, so the
-//                 warp prefixes are the sync offsets), packing through a 64-bit accumulator into
-//                 shared memory, the chunk's word offset from a single-pass decoupled look-back
-//                 scan (Merrill & Garland 2016) with a bounded wait, then coalesced word stores.
-//   k_decode      one thread per sub-stream (8 per chunk, 32 chunks per 256-thread block): a
-//                 64-bit bit window refilled from the payload, one lookup per symbol in the
-//                 4096-entry shared-memory table (Huffman) or a 3-bit area + index read (QLC),
-//                 16 output bytes per 16-byte store. Every sub-stream must end exactly where the
-//                 next one starts.
-//
 // The method: "Single-Stage Huffman Encoder for ML Compression" (abstract) -- a codebook fixed
 // from earlier batches, so the coder runs with no frequency pass and ships no codebook; "Quad
 // Length Codes for Lossless Compression of e4m3" (abstract, Tables 1-2) -- the area code.
+//
+//   k_histogram  byte histogram: 16-byte loads, one private 256-bin table per warp in shared
+//                memory, one global atomic per non-empty bin and block.
+//
+//   k_encode     persistent; one 4096-symbol chunk per block iteration, chunks taken in order
+//                from an atomic ticket. Input chunks arrive in a 4-stage shared-memory ring by
+//                bulk asynchronous copies (cp.async.bulk + mbarrier), issued as soon as a stage
+//                is free. The code/length table is replicated once per lane ([symbol][lane]), so
+//                a warp's 32 lookups never share a bank; its high half counts the symbols, so a
+//                single shared atomic both reads the code and adds to the fused histogram.
+//                Warp prefix sums of the code lengths (warp k = sub-stream k: the warp prefixes
+//                are the sync offsets) and packing through a 64-bit accumulator into a shared
+//                output buffer; the chunk's size goes out at once as a flag word. Block 0 of the
+//                (cooperatively launched, so co-resident) grid is the scanner: it turns the run
+//                of published sizes into word offsets 2048 chunks per step with a block-wide
+//                prefix sum -- a single-pass chained scan whose serial part moves a whole
+//                window at a time. One iteration later, so the wait overlaps the next chunk's
+//                work, the encoder reads its offset and stores the chunk with coalesced words.
+//
+//   k_decode     one thread per sub-stream (8 per chunk, 32 chunks per 256-thread block). The
+//                payload is read 16 bytes at a time with the next 16 bytes already in flight; a
+//                64-bit bit window feeds one lookup per symbol in the 4096-entry shared table.
+//                Huffman takes symbol and length from the table; QLC takes the length from the
+//                3-bit area through a register-held width table (3 + width) and only the symbol
+//                from the table. 32 decoded bytes leave as two 16-byte stores (a whole 32-byte
+//                sector). Every sub-stream must end exactly where the next one starts.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -35,12 +47,20 @@ constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
 constexpr int kEncThreads = 256;  // 16 symbols per thread; warp k codes sub-stream k
 constexpr int kDecThreads = 256;  // 8 threads per chunk, 32 chunks per block
 constexpr int kHistThreads = 256;
-constexpr unsigned long long kLookbackLimitNs = 1000000000ull;  // 1 s bound on any wait
+constexpr int kStages = 4;        // encode input ring
+constexpr int kLag = 3;           // encode: a chunk is stored kLag iterations after it is packed
+constexpr int kLutCopies = 32;    // encode: table copies; lane l reads copy l % kLutCopies
+constexpr int kOutBufs = kLag + 2;  // encode output buffers
+// 12-bit counters; a copy gains at most 16 per chunk from each lane that reads it
+constexpr uint32_t kHistFlushChunks = 255 / (32 / kLutCopies);
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s bound on any wait
 
-// look-back flag word: [63:62] state, [61:0] value (words)
-constexpr unsigned long long kFlagAggregate = 1ull << 62;
-constexpr unsigned long long kFlagInclusive = 2ull << 62;
+// per-chunk flag word: [63:62] state, [61:0] value. An encoder block publishes the chunk's
+// size in words (kFlagSize); the scanner block replaces it by the chunk's word offset (kFlagDone).
+constexpr unsigned long long kFlagSize = 1ull << 62;
+constexpr unsigned long long kFlagDone = 2ull << 62;
 constexpr unsigned long long kFlagValue = (1ull << 62) - 1;
+constexpr int kScanPerThread = 8;  // scanner window: 256 threads x 8 flags
 
 __host__ __device__ inline uint64_t n_chunks_of(uint64_t n) { return (n + kChunk - 1) / kChunk; }
 __host__ __device__ inline uint64_t sync_offset(uint64_t n) {
@@ -50,6 +70,7 @@ __host__ __device__ inline uint64_t payload_offset(uint64_t n) {
   return sync_offset(n) + 16 * n_chunks_of(n);
 }
 
+// ---------------------------------------------------------------------------------- PTX helpers
 __device__ inline unsigned long long ld_relaxed(const unsigned long long* p) {
   unsigned long long v;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -62,6 +83,55 @@ __device__ inline unsigned long long global_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
+}
+__device__ inline uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+__device__ inline void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bulk copy global -> shared (no multicast), completion counted on `bar`.
+__device__ inline void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ inline void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ inline void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Wait for phase `parity` of `bar`; false after kWaitLimitNs.
+__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  return true;
 }
 
 // ---------------------------------------------------------------------------------- histogram
@@ -109,7 +179,21 @@ struct EncodeArgs {
   uint32_t kind;
 };
 
-// Every header field but total_words (written by the block that codes the last chunk).
+struct EncSmem {
+  // [symbol][copy]: (count << 20) | (code << 8) | len. One copy per lane: no bank conflicts;
+  // len in the low byte lets 16 entries be summed into a bit count (16 * 12 < 256).
+  uint32_t lut[256 * kLutCopies];
+  alignas(128) uint8_t in[kStages][kChunk];
+  uint32_t out[kOutBufs][kMaxChunkWords];
+  alignas(16) uint32_t warp_bits[kOutBufs][kEncThreads / 32];
+  uint32_t chunk_of[kOutBufs];
+  uint32_t ticket[kStages];
+  uint32_t next[2];    // chunk of the next iteration's stage (0xffffffff: stop), double-buffered
+  uint64_t bar[kStages];
+  uint32_t offset[2];  // word offset of the chunk stored this iteration, double-buffered
+};
+
+// Every header field but total_words (written by the block that finishes the last chunk).
 __device__ inline void write_header(const EncodeArgs& a) {
   uint32_t* h32 = reinterpret_cast<uint32_t*>(a.out);
   uint64_t* h64 = reinterpret_cast<uint64_t*>(a.out);
@@ -127,202 +211,368 @@ __device__ inline void write_header(const EncodeArgs& a) {
   for (uint64_t i = gap; i < sync_offset(a.n); i += 4) h32[i / 4] = 0;
 }
 
-// Decoupled look-back: publish this chunk's word count, then add up predecessors until one
-// with an inclusive prefix is found. Chunks are taken in ticket order, so every predecessor is
-// already running and will publish; the wait is still bounded (HX_ERR_TIMEOUT).
-__device__ uint32_t chunk_word_offset(const EncodeArgs& a, uint32_t c, uint32_t words) {
-  if (c == 0) {
-    st_relaxed(a.flags, kFlagInclusive | words);
-    return 0;
-  }
-  st_relaxed(a.flags + c, kFlagAggregate | words);
-  unsigned long long excl = 0;
-  int64_t j = (int64_t)c - 1;
+// The scanner block: walks the flag words in order, 2048 at a time. The longest run of
+// published sizes at the front of the window gets a block-wide exclusive prefix sum; each of
+// those chunks gets its word offset (flag kFlagDone, and word_off[] in the stream). Encoder
+// blocks publish a size without waiting, so the run always grows; waits are bounded in time.
+__device__ void scan_chunk_offsets(const EncodeArgs& a, uint32_t nchunks, uint32_t* s_red,
+                                   uint32_t* s_stop) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
+  const uint64_t P = payload_offset(a.n);
+  uint64_t F = 0, running = 0;
   unsigned long long t0 = 0;
-  while (j >= 0) {
-    const unsigned long long f = ld_relaxed(a.flags + j);
-    const unsigned long long state = f & ~kFlagValue;
-    if (state == 0) {
-      const unsigned long long now = global_ns();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > kLookbackLimitNs) {
-        atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
-        break;
+  while (F < nchunks) {
+    uint32_t val[kScanPerThread];
+    uint32_t first = kScanPerThread * kEncThreads;  // first index in the window without a size
+#pragma unroll
+    for (int j = kScanPerThread - 1; j >= 0; --j) {
+      const uint64_t idx = F + (uint64_t)tid * kScanPerThread + j;
+      unsigned long long f = 0;
+      if (idx < nchunks) f = ld_relaxed(a.flags + idx);
+      val[j] = (uint32_t)(f & kFlagValue);
+      if ((f & ~kFlagValue) != kFlagSize) first = (uint32_t)tid * kScanPerThread + j;
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, d));
+    if (lane == 0) s_red[warp] = first;
+    __syncthreads();
+    uint32_t cnt = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kEncThreads / 32; ++w) cnt = min(cnt, s_red[w]);
+    __syncthreads();
+    if (cnt == 0) {  // nothing new yet: thread 0 keeps the clock, so all threads agree
+      if (tid == 0) {
+        const unsigned long long now = global_ns();
+        if (t0 == 0) t0 = now;
+        *s_stop = now - t0 > kWaitLimitNs;
+        if (*s_stop) atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
       }
-      __nanosleep(64);
+      __syncthreads();
+      if (*s_stop) return;
+      __nanosleep(100);
       continue;
     }
-    excl += f & kFlagValue;
-    if (state == kFlagInclusive) break;
-    --j;
-  }
-  st_relaxed(a.flags + c, kFlagInclusive | (excl + words));
-  return (uint32_t)excl;
-}
-
-__global__ void __launch_bounds__(kEncThreads) k_encode(EncodeArgs a) {
-  __shared__ uint32_t s_lut[256];
-  __shared__ uint32_t s_hist[256];
-  __shared__ uint32_t s_buf[kMaxChunkWords];
-  __shared__ uint32_t s_warp_bits[kEncThreads / 32];
-  __shared__ uint32_t s_chunk, s_offset;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint64_t n = a.n;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
-    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
-    return;
-  }
-  {
-    uint32_t e = a.tables->enc[tid];
-    if ((e & 15u) > HX_LMAX_MAX) {  // keeps a damaged table block inside the staging buffer
-      e = 0;
-      atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+    t0 = 0;
+    // exclusive prefix over window indices < cnt (thread-contiguous: index = 8 tid + j)
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < kScanPerThread; ++j)
+      if ((uint32_t)tid * kScanPerThread + j < cnt) mine += val[j];
+    uint32_t incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += t;
     }
-    s_lut[tid] = e;
+    if (lane == 31) s_red[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, window_total = 0;
+#pragma unroll
+    for (int w = 0; w < kEncThreads / 32; ++w) {
+      before += w < warp ? s_red[w] : 0u;
+      window_total += s_red[w];
+    }
+    __syncthreads();
+    uint64_t off = running + before + incl - mine;
+#pragma unroll
+    for (int j = 0; j < kScanPerThread; ++j) {
+      const uint32_t e = (uint32_t)tid * kScanPerThread + j;
+      if (e < cnt) {
+        word_off[F + e] = (uint32_t)off;
+        st_relaxed(a.flags + F + e, kFlagDone | off);
+        off += val[j];
+      }
+    }
+    running += window_total;
+    F += cnt;
   }
-  s_hist[tid] = 0;
-  if (blockIdx.x == 0 && tid == 0 && nchunks == 0) {
-    write_header(a);
-    reinterpret_cast<uint64_t*>(a.out)[4] = 0;
-    reinterpret_cast<uint32_t*>(a.out + 64)[0] = 0;
-    const uint64_t P = payload_offset(0);
-    if (P + 8 <= a.cap) {
-      reinterpret_cast<uint32_t*>(a.out + P)[0] = 0;
-      reinterpret_cast<uint32_t*>(a.out + P)[1] = 0;
+  if (tid == 0) {
+    word_off[nchunks] = (uint32_t)running;
+    reinterpret_cast<uint64_t*>(a.out)[4] = running;
+    uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
+    if (P + 4 * (running + 2) <= a.cap) {
+      payload[running] = 0;
+      payload[running + 1] = 0;
     } else {
       atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
     }
   }
+}
+
+// Word offset of chunk c from the scanner (one thread polls); bounded in time.
+__device__ uint32_t wait_chunk_offset(const EncodeArgs& a, uint32_t c) {
+  unsigned long long f = ld_relaxed(a.flags + c);
+  if ((f & ~kFlagValue) == kFlagDone) return (uint32_t)(f & kFlagValue);
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    __nanosleep(64);
+    f = ld_relaxed(a.flags + c);
+    if ((f & ~kFlagValue) == kFlagDone) return (uint32_t)(f & kFlagValue);
+    if (global_ns() - t0 > kWaitLimitNs) {
+      atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
+      return 0;
+    }
+  }
+}
+
+// The 16 symbols of one thread -> table entries (and the fused histogram); returns the summed
+// entries, whose low byte is the thread's bit count. FULL: all 16 symbols exist.
+template <bool HIST, bool FULL>
+__device__ __forceinline__ uint32_t lookup16(uint32_t* lut_lane, const uint32_t w[4],
+                                             uint32_t valid, uint32_t e[16]) {
+  uint32_t sum = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t sym = (w[j >> 2] >> (8 * (j & 3))) & 0xffu;
+    uint32_t ent = 0;
+    if (FULL || (uint32_t)j < valid) {
+      uint32_t* slot = lut_lane + sym * kLutCopies;
+      ent = HIST ? atomicAdd(slot, 1u << 20) : *slot;
+    }
+    e[j] = ent;
+    sum += ent;
+  }
+  return sum;
+}
+
+// Pack 16 (code, len) entries MSB-first starting at bit `off` of buf: two codes are joined in a
+// 32-bit register (<= 24 bits), then appended to a 64-bit accumulator (hi:lo) with funnel
+// shifts. Words this thread owns are stored; the first and last, shared with neighbours, OR-ed.
+__device__ __forceinline__ void pack16(const uint32_t e[16], uint32_t off, uint32_t* buf) {
+  uint32_t widx = off >> 5;
+  uint32_t nacc = off & 31;  // the first bits belong to the previous thread (zeros here)
+  bool shared_first = nacc != 0;
+  uint32_t hi = 0, lo = 0;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t e0 = e[2 * p], e1 = e[2 * p + 1];
+    const uint32_t l1 = e1 & 0xffu;
+    const uint32_t pl = (e0 & 0xffu) + l1;
+    const uint32_t pc = (((e0 >> 8) & 0xfffu) << l1) | ((e1 >> 8) & 0xfffu);
+    hi = __funnelshift_l(lo, hi, pl);
+    lo = (lo << pl) | pc;
+    nacc += pl;
+    if (nacc >= 32) {
+      nacc -= 32;
+      const uint32_t word = __funnelshift_r(lo, hi, nacc);
+      if (shared_first) atomicOr(&buf[widx], word);
+      else buf[widx] = word;
+      shared_first = false;
+      ++widx;
+    }
+  }
+  if (nacc) atomicOr(&buf[widx], lo << (32 - nacc));
+}
+
+template <bool HIST, bool COMPLETE>
+__device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
+  const uint32_t full_chunks = (uint32_t)(n / kChunk);
   const uint64_t P = payload_offset(n);
-  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
   uint4* sync = reinterpret_cast<uint4*>(a.out + sync_offset(n));
   uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
-  const bool want_hist = a.hist != nullptr;
-  bool uncodable = false;
+  uint32_t* lut_lane = sm.lut + lane % kLutCopies;
 
-  for (;;) {
-    if (tid == 0) s_chunk = atomicAdd(a.ticket, 1u);
-    for (int i = tid; i < (int)kMaxChunkWords; i += kEncThreads) s_buf[i] = 0;
-    __syncthreads();
-    const uint32_t c = s_chunk;
-    if (c >= nchunks) break;
-    const uint64_t base = (uint64_t)c * kChunk;
-    const uint32_t count = n - base < kChunk ? (uint32_t)(n - base) : kChunk;
-    const uint32_t first = (uint32_t)tid * 16;
-
-    // 16 symbols of this thread
-    uint32_t w[4];
-    if (count == kChunk) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(a.in + base) + tid);
-      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  // stage s takes ticket t; full chunks arrive by bulk copy, others by plain loads
+  auto refill = [&](int s, uint32_t t) {
+    sm.ticket[s] = t;
+    if (t < full_chunks) {
+      mbar_arrive_expect_tx(&sm.bar[s], kChunk);
+      bulk_load(sm.in[s], a.in + (uint64_t)t * kChunk, kChunk, &sm.bar[s]);
     } else {
+      mbar_arrive(&sm.bar[s]);
+    }
+  };
+  // Only thread 0 waits on a stage's mbarrier; the block barrier that follows hands the
+  // stage (and the uniform go/stop decision) to every thread.
+  auto await_stage = [&](uint32_t it_next) {
+    const int s = (int)(it_next % kStages);
+    uint32_t c = 0xffffffffu;
+    if (mbar_wait(&sm.bar[s], (it_next / kStages) & 1u)) c = sm.ticket[s];
+    else atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
+    sm.next[it_next & 1] = c;
+  };
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) refill(s, atomicAdd(a.ticket, 1u));
+    await_stage(0);
+  }
+  __syncthreads();
+
+  bool uncodable = false;
+  uint32_t since_flush = 0;
+
+  // Stores of the chunk packed kLag iterations earlier (buffer b), once its offset is known.
+  auto store_chunk = [&](int b, uint32_t woff) {
+    const uint32_t c = sm.chunk_of[b];
+    const uint4 t0 = *reinterpret_cast<const uint4*>(&sm.warp_bits[b][0]);
+    const uint4 t1 = *reinterpret_cast<const uint4*>(&sm.warp_bits[b][4]);
+    const uint32_t total = t0.x + t0.y + t0.z + t0.w + t1.x + t1.y + t1.z + t1.w;
+    const uint32_t words = (total + 31) >> 5;
+    const bool fits = P + 4ull * ((uint64_t)woff + words + 2) <= a.cap;
+    uint32_t* buf = sm.out[b];
+    for (uint32_t i = tid; i < words; i += kEncThreads) {
+      if (fits) payload[woff + i] = buf[i];
+      buf[i] = 0;
+    }
+    if (tid == 0) {
+      const uint32_t p1 = t0.x, p2 = p1 + t0.y, p3 = p2 + t0.z, p4 = p3 + t0.w;
+      const uint32_t p5 = p4 + t1.x, p6 = p5 + t1.y, p7 = p6 + t1.z;
+      sync[c] = make_uint4(total | (p1 << 16), p2 | (p3 << 16), p4 | (p5 << 16), p6 | (p7 << 16));
+      if (!fits) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
+      if (c == 0) write_header(a);
+    }
+  };
+
+  auto flush_hist = [&]() {  // counts in the lane tables -> global, then clear them
+    __syncthreads();
+    uint32_t sum = 0;
+    for (int l = 0; l < kLutCopies; ++l) {
+      const uint32_t e = sm.lut[tid * kLutCopies + l];
+      sum += e >> 20;
+      sm.lut[tid * kLutCopies + l] = e & 0xfffffu;
+    }
+    if (sum) atomicAdd(&a.hist[tid], sum);
+    __syncthreads();
+  };
+
+  uint32_t it = 0;
+  for (;; ++it) {
+    const int s = (int)(it % kStages);
+    const int ob = (int)(it % kOutBufs);
+    const uint32_t c = sm.next[it & 1];
+    if (c >= nchunks) break;  // uniform: written before the last block barrier
+
+    // thread 0 starts its two global round trips now and needs the answers only after the
+    // symbol work: the ticket for this stage's refill and the flag of the lagged chunk
+    uint32_t next_ticket = 0;
+    unsigned long long lag_flag = 0;
+    if (tid == 0) {
+      next_ticket = atomicAdd(a.ticket, 1u);
+      if (it >= kLag) lag_flag = ld_relaxed(a.flags + sm.chunk_of[(it - kLag) % kOutBufs]);
+    }
+    uint32_t w[4];
+    uint32_t e[16];
+    uint32_t sum;
+    if (c < full_chunks) {
+      const uint4 v = reinterpret_cast<const uint4*>(sm.in[s])[tid];
+      w[0] = v.x;
+      w[1] = v.y;
+      w[2] = v.z;
+      w[3] = v.w;
+      sum = lookup16<HIST, true>(lut_lane, w, 16, e);
+    } else {  // the ragged last chunk, from global memory
+      const uint64_t base = (uint64_t)c * kChunk;
+      const uint32_t first = (uint32_t)tid * 16;
+      const uint32_t count = (uint32_t)(n - base);
+      const uint32_t valid = count > first ? min(16u, count - first) : 0u;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t x = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const uint32_t i = first + 4 * q + b;
-          if (i < count) x |= (uint32_t)a.in[base + i] << (8 * b);
-        }
+        for (int b = 0; b < 4; ++b)
+          if ((uint32_t)(4 * q + b) < valid)
+            x |= (uint32_t)a.in[base + first + 4 * q + b] << (8 * b);
         w[q] = x;
       }
-    }
-    const uint32_t valid = count > first ? min(16u, count - first) : 0u;
-    uint32_t e[16];
-    uint32_t bits = 0;
+      sum = lookup16<HIST, false>(lut_lane, w, valid, e);
+      if (!COMPLETE)
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const uint32_t sym = (w[j >> 2] >> (8 * (j & 3))) & 0xff;
-      const bool here = (uint32_t)j < valid;
-      const uint32_t ent = here ? s_lut[sym] : 0u;
-      uncodable |= here && (ent & 15u) == 0;
-      if (want_hist && here) atomicAdd(&s_hist[sym], 1u);
-      e[j] = ent;
-      bits += ent & 15u;
+        for (int j = 0; j < 16; ++j) uncodable |= (uint32_t)j < valid && (e[j] & 0xffu) == 0;
     }
-
-    // bit offset of this thread inside the chunk: warp scan, then the warps before it
+    if (!COMPLETE && c < full_chunks)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) uncodable |= (e[j] & 0xffu) == 0;
+    const uint32_t bits = sum & 0xffu;
     uint32_t incl = bits;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
       if (lane >= d) incl += t;
     }
-    if (lane == 31) s_warp_bits[warp] = incl;
-    __syncthreads();
-    uint32_t warp_base = 0, total = 0;
-#pragma unroll
-    for (int k = 0; k < kEncThreads / 32; ++k) {
-      const uint32_t t = s_warp_bits[k];
-      warp_base += k < warp ? t : 0u;
-      total += t;
-    }
-    const uint32_t off = warp_base + incl - bits;
-
-    // pack: whole words this thread owns are stored, shared boundary words are OR-ed
-    if (bits) {
-      uint32_t widx = off >> 5;
-      const uint32_t lead = off & 31;
-      uint64_t acc = 0;
-      uint32_t nacc = lead;
-      bool first_word = true;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const uint32_t len = e[j] & 15u;
-        acc = (acc << len) | (e[j] >> 4);
-        nacc += len;
-        if (nacc >= 32) {
-          nacc -= 32;
-          const uint32_t word = (uint32_t)(acc >> nacc);
-          if (first_word && lead) atomicOr(&s_buf[widx], word);
-          else s_buf[widx] = word;
-          first_word = false;
-          ++widx;
-        }
-      }
-      if (nacc) atomicOr(&s_buf[widx], (uint32_t)(acc << (32 - nacc)));
-    }
-    const uint32_t words = (total + 31) >> 5;
-    __syncthreads();
-
-    if (tid == 0) s_offset = chunk_word_offset(a, c, words);
-    __syncthreads();
-    const uint32_t woff = s_offset;
-    const bool fits = P + 4ull * ((uint64_t)woff + words + 2) <= a.cap;
-    if (fits) {
-      for (uint32_t i = tid; i < words; i += kEncThreads) payload[woff + i] = s_buf[i];
-    }
+    if (lane == 31) sm.warp_bits[ob][warp] = incl;
     if (tid == 0) {
-      word_off[c] = woff;
-      uint32_t pre[HX_SUBSTREAMS];
-      uint32_t acc = 0;
-#pragma unroll
-      for (int k = 0; k < HX_SUBSTREAMS; ++k) {
-        pre[k] = acc;
-        acc += s_warp_bits[k];
-      }
-      sync[c] = make_uint4(total | (pre[1] << 16), pre[2] | (pre[3] << 16), pre[4] | (pre[5] << 16),
-                           pre[6] | (pre[7] << 16));
-      if (!fits) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
-      if (c == 0) write_header(a);
-      if (c == nchunks - 1) {
-        const uint32_t end = woff + words;
-        word_off[nchunks] = end;
-        reinterpret_cast<uint64_t*>(a.out)[4] = end;
-        if (fits) {
-          payload[end] = 0;
-          payload[end + 1] = 0;
-        }
-      }
+      if (it >= kLag)  // offset of the chunk packed kLag iterations ago
+        sm.offset[it & 1] = (lag_flag & ~kFlagValue) == kFlagDone
+                                ? (uint32_t)(lag_flag & kFlagValue)
+                                : wait_chunk_offset(a, sm.chunk_of[(it - kLag) % kOutBufs]);
+      await_stage(it + 1);
     }
-    __syncthreads();
+    __syncthreads();  // warp totals ready; stage s read by all; next stage handed over
+
+    const uint4 t0 = *reinterpret_cast<const uint4*>(&sm.warp_bits[ob][0]);
+    const uint4 t1 = *reinterpret_cast<const uint4*>(&sm.warp_bits[ob][4]);
+    const uint32_t tw[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+    uint32_t warp_base = 0;
+#pragma unroll
+    for (int k = 0; k < kEncThreads / 32; ++k) warp_base += k < warp ? tw[k] : 0u;
+    if (tid == 0) {
+      const uint32_t total = t0.x + t0.y + t0.z + t0.w + t1.x + t1.y + t1.z + t1.w;
+      st_relaxed(a.flags + c, kFlagSize | ((total + 31) >> 5));
+      sm.chunk_of[ob] = c;
+      fence_proxy_async();  // this stage's generic reads before the async refill
+      refill(s, next_ticket);
+    }
+    if (bits) pack16(e, warp_base + incl - bits, sm.out[ob]);
+    if (it >= kLag) store_chunk((int)((it - kLag) % kOutBufs), sm.offset[it & 1]);
+    if (HIST && ++since_flush == kHistFlushChunks) {
+      flush_hist();
+      since_flush = 0;
+    }
   }
-  if (uncodable) atomicOr(a.status, (uint32_t)HX_ERR_UNCODABLE);
-  if (want_hist) {
+  if (tid == 0 && sm.next[it & 1] == 0xffffffffu)  // timed out: let copies still in flight land
+    for (uint32_t j = 1; j < (uint32_t)kStages; ++j)
+      mbar_wait(&sm.bar[(it + j) % kStages], ((it + j) / kStages) & 1u);
+  // drain: the last kLag packed chunks
+  for (uint32_t k = it > kLag ? it - kLag : 0; k < it; ++k) {
     __syncthreads();
-    if (s_hist[tid]) atomicAdd(&a.hist[tid], s_hist[tid]);
+    if (tid == 0) sm.offset[0] = wait_chunk_offset(a, sm.chunk_of[k % kOutBufs]);
+    __syncthreads();
+    store_chunk((int)(k % kOutBufs), sm.offset[0]);
+  }
+  if (!COMPLETE && uncodable) atomicOr(a.status, (uint32_t)HX_ERR_UNCODABLE);
+  if (HIST) flush_hist();
+}
+
+__global__ void __launch_bounds__(kEncThreads) k_encode(EncodeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  EncSmem& sm = *reinterpret_cast<EncSmem*>(smem_raw);
+  const int tid = threadIdx.x;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(a.n);
+  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
+    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+    return;
+  }
+  if (blockIdx.x == 0) {  // block 0 scans the chunk sizes into word offsets
+    if (nchunks == 0 && tid == 0) write_header(a);
+    scan_chunk_offsets(a, nchunks, sm.warp_bits[0], &sm.offset[0]);
+    return;
+  }
+  bool complete = true;
+  for (int i = tid; i < 256 * kLutCopies; i += kEncThreads) {
+    const uint32_t t = a.tables->enc[i / kLutCopies];  // (code << 4) | len
+    uint32_t e = ((t >> 4) << 8) | (t & 15u);
+    if ((t & 15u) > HX_LMAX_MAX || t > 0xffffu) {  // a damaged table block stays harmless
+      e = 0;
+      atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+    }
+    complete &= (e & 0xffu) != 0;
+    sm.lut[i] = e;
+  }
+  for (int i = tid; i < kOutBufs * (int)kMaxChunkWords; i += kEncThreads) (&sm.out[0][0])[i] = 0;
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+    fence_barrier_init();
+  }
+  complete = __syncthreads_and(complete);
+  if (a.hist) {
+    if (complete) encode_chunks<true, true>(a, sm);
+    else encode_chunks<true, false>(a, sm);
+  } else {
+    if (complete) encode_chunks<false, true>(a, sm);
+    else encode_chunks<false, false>(a, sm);
   }
 }
 
@@ -343,7 +593,7 @@ struct DecodeArgs {
   uint32_t kind;
 };
 
-// Header checks shared by every block; returns total_words, or -1 after raising the status.
+// Header checks shared by every block; returns total_words, or -status.
 __device__ int64_t check_header(const DecodeArgs& a) {
   const uint32_t* h32 = reinterpret_cast<const uint32_t*>(a.st);
   const uint64_t* h64 = reinterpret_cast<const uint64_t*>(a.st);
@@ -362,35 +612,146 @@ __device__ int64_t check_header(const DecodeArgs& a) {
   return (int64_t)total;
 }
 
-template <int KIND>
-__global__ void __launch_bounds__(kDecThreads) k_decode(DecodeArgs a) {
-  __shared__ __align__(16) uint16_t s_lut[KIND == HX_KIND_HUFFMAN ? 4096 : 2];
-  __shared__ uint8_t s_r2s[256];
-  __shared__ uint32_t s_area[8];
-  __shared__ int64_t s_total;
-  const int tid = threadIdx.x;
-  if (tid == 0) s_total = check_header(a);
+// A quad (16 bytes) of payload words that is not wholly inside the caller's buffer: words past
+// the buffer read as 0. Out of line: only the last quad of a stream can take this path.
+__device__ __noinline__ uint4 tail_quad(const uint32_t* words, uint64_t q, uint64_t wlimit) {
+  uint32_t v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t wi = 4 * q + i;
+    v[i] = wi < wlimit ? __ldg(words + wi) : 0u;
+  }
+  return make_uint4(v[0], v[1], v[2], v[3]);
+}
+
+// Payload words of one sub-stream, MSB-first, through a 64-bit bit window held as two 32-bit
+// halves (wh:wl) whose top `avail` bits are valid. Words come from a reservoir: `cur` holds the
+// next `left` words, `nxt` the quad after them, so the next 16 bytes are always in flight.
+// FAST: every quad the current group can touch lies wholly inside the buffer.
+struct SubstreamReader {
+  const uint4* quads;
+  const uint32_t* words;
+  uint64_t qsafe, wlimit;
+  uint64_t qn;  // next quad to request
+  uint4 cur, nxt;
+  uint32_t left, taken;
+  uint32_t wh, wl;
+  int avail;
+
+  template <bool FAST>
+  __device__ __forceinline__ uint4 quad(uint64_t q) const {
+    if (FAST) return __ldg(quads + q);
+    return q < qsafe ? __ldg(quads + q) : tail_quad(words, q, wlimit);
+  }
+  template <bool FAST>
+  __device__ __forceinline__ uint32_t take() {
+    const uint32_t w = cur.x;
+    cur.x = cur.y;
+    cur.y = cur.z;
+    cur.z = cur.w;
+    ++taken;
+    if (--left == 0) {
+      cur = nxt;
+      nxt = quad<FAST>(qn++);
+      left = 4;
+    }
+    return w;
+  }
+  // afterwards >= 32 valid bits: room for two codes of <= 12 bits
+  template <bool FAST>
+  __device__ __forceinline__ void refill() {
+    if (avail < 32) {
+      const uint32_t w = take<FAST>();
+      wh |= w >> avail;                             // the word lands at bits [32-avail, 64-avail)
+      wl |= __funnelshift_lc(0u, w, 32 - avail);   // its low part (nothing when avail == 0)
+      avail += 32;
+    }
+  }
+  __device__ __forceinline__ void consume(uint32_t len) {  // len <= 15
+    wh = __funnelshift_l(wl, wh, len);
+    wl <<= len;
+    avail -= (int)len;
+  }
+  __device__ void start(uint64_t first_bit) {
+    const uint64_t fw = first_bit >> 5;
+    qn = fw >> 2;
+    cur = quad<false>(qn);
+    nxt = quad<false>(qn + 1);
+    qn += 2;
+    left = 4;
+    for (uint32_t skip = (uint32_t)(fw & 3); skip > 0; --skip) take<false>();
+    taken = 0;
+    wh = take<false>();
+    wl = take<false>();
+    const uint32_t sh = (uint32_t)(first_bit & 31);
+    wh = __funnelshift_l(wl, wh, sh);
+    wl <<= sh;
+    avail = 64 - (int)sh;
+  }
+  // index (in payload bits) of the next bit not yet consumed
+  __device__ uint64_t position(uint64_t first_bit) const {
+    return 32 * ((first_bit >> 5) + taken) - (uint64_t)avail;
+  }
+};
+
+// One symbol from the top of the window, returned as a table entry whose byte 1 is the symbol.
+// Huffman: the 4096-entry table gives symbol and length. QLC: the length is 3 + the width of the
+// area named by the top 3 bits (a register lookup, so the window advance waits on no memory
+// access); the symbol comes from the same kind of table.
+template <int KIND, bool COMPLETE>
+__device__ __forceinline__ uint32_t next_symbol(SubstreamReader& rd, bool& invalid,
+                                                const uint16_t* lut, const uint32_t* area,
+                                                uint32_t qbits) {
+  const uint32_t e = lut[rd.wh >> 20];
+  uint32_t len;
   if (KIND == HX_KIND_HUFFMAN) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.tables->dec);
-    uint4* dst = reinterpret_cast<uint4*>(s_lut);
-    for (int i = tid; i < 4096 * 2 / 16; i += kDecThreads) dst[i] = src[i];
+    len = e & 15u;
+    if (!COMPLETE) invalid |= len == 0;
   } else {
-    s_r2s[tid] = a.tables->rank2sym[tid];
-    if (tid < 8) s_area[tid] = a.tables->qlc_area[tid];
+    const uint32_t ar = rd.wh >> 29;
+    const uint32_t b = (qbits >> (4 * ar)) & 15u;
+    len = 3 + b;
+    if (!COMPLETE) invalid |= ((rd.wh >> (29 - b)) & ((1u << b) - 1u)) >= ((area[ar] >> 9) & 511u);
   }
-  __syncthreads();
-  const int64_t total = s_total;
-  if (total < 0) {
-    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)(-total));
-    return;
+  rd.consume(len);
+  return e;
+}
+
+// 32 symbols -> 32 output bytes (two 16-byte stores, one whole sector). Each symbol's byte is
+// moved into place with one byte permute.
+template <int KIND, bool COMPLETE, bool FAST>
+__device__ __forceinline__ void decode_group32(SubstreamReader& rd, bool& invalid, uint4* d4,
+                                               const uint16_t* lut, const uint32_t* area,
+                                               uint32_t qbits) {
+  uint32_t o[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    rd.refill<FAST>();
+    uint32_t v = next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits) >> 8;
+    v = __byte_perm(v, next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits), 0x3250);
+    rd.refill<FAST>();
+    v = __byte_perm(v, next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits), 0x3510);
+    v = __byte_perm(v, next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits), 0x5210);
+    o[q] = v;
   }
-  const uint32_t qbits = a.tables->qlc_bits_packed;
+  d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int KIND, bool COMPLETE>
+__device__ void decode_chunks(const DecodeArgs& a, const uint16_t* lut, const uint32_t* area,
+                              uint32_t qbits, uint32_t total) {
+  const int tid = threadIdx.x;
   const uint64_t n = a.n;
   const uint64_t nchunks = n_chunks_of(n);
+  const uint64_t P = payload_offset(n);
   const uint32_t* word_off = reinterpret_cast<const uint32_t*>(a.st + 64);
   const uint4* sync = reinterpret_cast<const uint4*>(a.st + sync_offset(n));
-  const uint32_t* payload = reinterpret_cast<const uint32_t*>(a.st + payload_offset(n));
-  const uint32_t last_word = (uint32_t)total + 1;  // the second guard word
+  SubstreamReader rd;
+  rd.words = reinterpret_cast<const uint32_t*>(a.st + P);
+  rd.quads = reinterpret_cast<const uint4*>(a.st + P);
+  rd.wlimit = (a.bytes - P) / 4;  // payload words inside the buffer
+  rd.qsafe = (a.bytes - P) / 16;  // quads [0, qsafe) lie wholly inside it
   const int k = tid & 7;
 
   for (uint64_t c = (uint64_t)blockIdx.x * (kDecThreads / 8) + (tid >> 3); c < nchunks;
@@ -404,68 +765,59 @@ __global__ void __launch_bounds__(kDecThreads) k_decode(DecodeArgs a) {
     const uint32_t nbits = sy.x & 0xffffu;
     const uint32_t count = n - c * kChunk < kChunk ? (uint32_t)(n - c * kChunk) : kChunk;
     const uint32_t nsub = (count + kSubLen - 1) / kSubLen;
-    bool bad = w0 > w1 || w1 > (uint32_t)total || nbits > 32u * (w1 - w0) ||
-               (nbits + 31) / 32 != w1 - w0;
+    bool bad = w0 > w1 || w1 > total || nbits > 32u * (w1 - w0) || (nbits + 31) / 32 != w1 - w0;
     const uint32_t mine = (uint32_t)k < nsub ? min(kSubLen, count - k * kSubLen) : 0u;
     if (mine == 0) {
       bad |= k > 0 && sync_at(k) != nbits;
     } else if (!bad) {
       const uint32_t start = k == 0 ? 0u : sync_at(k);
       const uint32_t end = (uint32_t)k + 1 < nsub ? sync_at(k + 1) : nbits;
-      uint32_t widx = w0 + (start >> 5);
-      auto fetch = [&](uint32_t i) -> uint32_t { return __ldg(payload + min(i, last_word)); };
-      uint64_t win = ((uint64_t)fetch(widx) << 32) | fetch(widx + 1);
-      win <<= (start & 31);
-      int avail = 64 - (int)(start & 31);
-      widx += 2;
-      uint32_t used = 0;
+      const uint64_t first_bit = 32ull * w0 + start;
+      rd.start(first_bit);
       bool invalid = false;
       uint8_t* dst = a.out + c * kChunk + (uint64_t)k * kSubLen;
-
-      auto step = [&]() -> uint32_t {
-        if (avail < 32) {
-          win |= (uint64_t)fetch(widx++) << (32 - avail);
-          avail += 32;
-        }
-        uint32_t sym, len;
-        if (KIND == HX_KIND_HUFFMAN) {
-          const uint32_t e = s_lut[win >> 52];
-          len = e >> 8;
-          sym = e & 0xff;
-          invalid |= len == 0;
-        } else {
-          const uint32_t area = (uint32_t)(win >> 61);
-          const uint32_t b = (qbits >> (4 * area)) & 15u;
-          const uint32_t idx = (uint32_t)(win >> (61 - b)) & ((1u << b) - 1u);
-          const uint32_t info = s_area[area];
-          invalid |= idx >= ((info >> 9) & 511u);
-          sym = s_r2s[((info & 511u) + idx) & 255u];
-          len = 3 + b;
-        }
-        win <<= len;
-        avail -= (int)len;
-        used += len;
-        return sym;
-      };
-
-      const uint32_t groups = mine / 16;
+      const uint32_t groups = mine / 32;
       for (uint32_t g = 0; g < groups; ++g) {
-        uint32_t o[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t v = step();
-          v |= step() << 8;
-          v |= step() << 16;
-          v |= step() << 24;
-          o[q] = v;
-        }
-        reinterpret_cast<uint4*>(dst)[g] = make_uint4(o[0], o[1], o[2], o[3]);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * g);
+        // a group takes at most 12 words: 3 more quads past the one requested last
+        if (rd.qn + 3 < rd.qsafe)
+          decode_group32<KIND, COMPLETE, true>(rd, invalid, d4, lut, area, qbits);
+        else
+          decode_group32<KIND, COMPLETE, false>(rd, invalid, d4, lut, area, qbits);
       }
-      for (uint32_t i = groups * 16; i < mine; ++i) dst[i] = (uint8_t)step();
-      bad |= invalid || start + used != end;
+      for (uint32_t i = groups * 32; i < mine; ++i) {
+        rd.refill<false>();
+        dst[i] = (uint8_t)(next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits) >> 8);
+      }
+      // the sub-stream must end exactly where the next one starts
+      bad |= invalid || rd.position(first_bit) != 32ull * w0 + end;
     }
     if (bad) atomicOr(a.status, (uint32_t)HX_ERR_CORRUPT);
   }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kDecThreads, 5) k_decode(DecodeArgs a) {
+  __shared__ __align__(16) uint16_t s_lut[4096];
+  __shared__ uint32_t s_area[8];
+  __shared__ int64_t s_total;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_total = check_header(a);
+  const uint4* src = reinterpret_cast<const uint4*>(a.tables->dec);
+  uint4* dst = reinterpret_cast<uint4*>(s_lut);
+  for (int i = tid; i < 4096 * 2 / 16; i += kDecThreads) dst[i] = src[i];
+  if (tid < 8) s_area[tid] = a.tables->qlc_area[tid];
+  __syncthreads();
+  const int64_t total = s_total;
+  if (total < 0) {
+    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)(-total));
+    return;
+  }
+  const uint32_t qbits = a.tables->qlc_bits_packed;
+  if (a.tables->complete)
+    decode_chunks<KIND, true>(a, s_lut, s_area, qbits, (uint32_t)total);
+  else
+    decode_chunks<KIND, false>(a, s_lut, s_area, qbits, (uint32_t)total);
 }
 
 // ---------------------------------------------------------------------------------- launch
@@ -486,14 +838,19 @@ bool device_info(DeviceInfo* out) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return false;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.enc_per_sm, k_encode, kEncThreads, 0) !=
-            cudaSuccess ||
+    if (cudaFuncSetAttribute(k_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(EncSmem)) != cudaSuccess)
+      return false;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.enc_per_sm, k_encode, kEncThreads,
+                                                      sizeof(EncSmem)) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.huff_per_sm, k_decode<HX_KIND_HUFFMAN>,
                                                       kDecThreads, 0) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qlc_per_sm, k_decode<HX_KIND_QLC>,
                                                       kDecThreads, 0) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
                                                       0) != cudaSuccess)
+      return false;
+    if (d.enc_per_sm < 1 || d.huff_per_sm < 1 || d.qlc_per_sm < 1 || d.hist_per_sm < 1)
       return false;
     d.sms = sms;
   }
@@ -521,9 +878,13 @@ int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint
   k_zero_scratch<<<(nchunks + 255) / 256 + (nchunks == 0), 256, 0, s>>>(flags, nchunks, ticket);
   EncodeArgs a{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
                out_cap, flags, ticket, d_hist, d_status, kind};
-  const uint32_t grid =
-      (uint32_t)std::max<uint64_t>(1, std::min<uint64_t>(nchunks, (uint64_t)info.sms * info.enc_per_sm));
-  k_encode<<<grid, kEncThreads, 0, s>>>(a);
+  // block 0 scans, the others encode; all must be resident at once (cooperative launch)
+  const uint32_t grid = 1 + (uint32_t)std::max<uint64_t>(
+      1, std::min<uint64_t>(nchunks, (uint64_t)info.sms * info.enc_per_sm - 1));
+  void* params[] = {&a};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_encode), dim3(grid),
+                                  dim3(kEncThreads), params, sizeof(EncSmem), s) != cudaSuccess)
+    return launched() | HX_ERR_CUDA;
   return launched();
 }
 

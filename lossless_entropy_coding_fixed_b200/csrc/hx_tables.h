@@ -12,8 +12,8 @@ constexpr uint32_t kTablesMagic = 0x42545848u;  // "HXTB"
 struct Tables {
   // Encoder: per byte value (code << 4) | len; len 0 = no code word.
   uint32_t enc[256];
-  // Huffman decoder: for every 12-bit window w, (len << 8) | sym of the code word that w starts
-  // with; 0 when no code word is a prefix of w. (Filled for QLC codebooks as well.)
+  // Decoder: for every 12-bit window w, (sym << 8) | len of the code word that w starts with;
+  // 0 when no code word is a prefix of w. (Filled for QLC codebooks as well.)
   uint16_t dec[4096];
   // QLC: byte value of each rank.
   uint8_t rank2sym[256];
@@ -24,6 +24,9 @@ struct Tables {
   uint32_t kind;
   uint32_t lmax;
   uint32_t magic;
+  // 1 when every 12-bit window starts with a code word (Kraft sum 1): decode needs no check
+  // for unused code words.
+  uint32_t complete;
   uint64_t hash;
 };
 

@@ -104,7 +104,7 @@ def test_table_block_consistent(orc, kind):
     coded = np.nonzero(ln)[0]
     for w in range(4096):
         e = int(dec[w])
-        l, s = e >> 8, e & 0xff
+        s, l = e >> 8, e & 0xff
         if e == 0:  # no code word starts this window (only possible for an incomplete code)
             assert not any((w >> (12 - ln[t])) == code[t] for t in coded)
         else:
