@@ -149,6 +149,24 @@ int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d
 int hx_qlc_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
                   uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream);
 
+/* Allocation-free encode. The pages have no counterpart to this call: it exists for callers
+ * that cannot allocate device memory when they encode -- for example code that runs under a
+ * framework whose caching allocator has already reserved the device's memory (a stray
+ * cudaMalloc there can fail or fragment the pool), or a latency-critical path that cannot afford
+ * the implicit device synchronisation of cudaMalloc/cudaFree. It behaves exactly like hx_encode
+ * with Huffman tables (same stream, same status bits) but takes no scratch argument: its scratch
+ * lives in a fixed device array inside the library, sized for n <= HX_NOALLOC_MAX_BYTES, that
+ * every GPU which loads the library keeps until the process exits.
+ *  - n > HX_NOALLOC_MAX_BYTES is refused with HX_ERR_ARG; nothing is enqueued.
+ *  - The first call on a device looks up that array's device address (once per device, with
+ *    the device current); make that first call before any stream capture on the device.
+ *  - All calls share the one array, and each call clears what must start at zero. Calls whose
+ *    work overlaps on the GPU (other streams, other host threads) race on it: serialise them.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine. */
+#define HX_NOALLOC_MAX_BYTES (128ull << 20)
+int hx_encode_noalloc(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                      uint64_t out_cap, uint32_t* d_hist, uint32_t* d_status, void* stream);
+
 /* Measurement helpers (host, fp64). Shannon entropy -sum p log2 p of counts[256] in bits per
  * symbol ("Single-Stage Huffman Encoder for ML Compression", abstract: the ideal the fixed code
  * is compared with), and the mean code length sum count*len / sum count of a codebook. Both

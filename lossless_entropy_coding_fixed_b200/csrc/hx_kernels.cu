@@ -914,9 +914,46 @@ int decode_common(uint32_t kind, const void* d_tables, const void* d_stream, uin
 
 }  // namespace
 
+// Scratch of hx_encode_noalloc: one flag word per chunk plus the ticket, for up to
+// HX_NOALLOC_MAX_BYTES of input. Host code must not pass this name to a kernel (on the host it is
+// only a stand-in); its device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[8 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64];  // device address of g_noalloc_scratch, per device
+}  // namespace
+
 extern "C" {
 
 uint64_t hx_scratch_bytes(uint64_t n) { return 8 * n_chunks_of(n) + 16; }
+
+// For callers that cannot allocate device memory at encode time (a framework's caching
+// allocator owns the device memory, or a path that cannot take cudaMalloc's implicit
+// synchronisation): hx_encode with Huffman tables, its scratch in g_noalloc_scratch. The first
+// call on a device fetches that array's address with the device current; every call zeroes the
+// part it uses (k_zero_scratch) and calls that overlap on the GPU race on the shared array.
+int hx_encode_noalloc(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                      uint64_t out_cap, uint32_t* d_hist, uint32_t* d_status, void* stream) {
+  if (n > HX_NOALLOC_MAX_BYTES) return HX_ERR_ARG;
+  static_assert(sizeof(g_noalloc_scratch) >= 8 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16,
+                "scratch array smaller than hx_scratch_bytes(HX_NOALLOC_MAX_BYTES)");
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HX_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HX_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return encode_common(HX_KIND_HUFFMAN, d_tables, d_in, n, d_out, out_cap, scratch, d_hist,
+                       d_status, stream);
+}
 
 int hx_codebook_upload(const hx_codebook* cb, void* d_tables, void* stream) {
   if (!d_tables) return HX_ERR_ARG;

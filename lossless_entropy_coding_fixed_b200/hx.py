@@ -73,6 +73,7 @@ def lib():
             "hx_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_qlc_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
             "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
+            "hx_encode_noalloc": (i32, [P, P, u64, P, u64, P, P, P]),
             "hx_entropy": (ctypes.c_double, [P]),
             "hx_mean_length": (ctypes.c_double, [P, CB]),
             "hx_version": (i32, []),
@@ -248,6 +249,23 @@ def encode(tables, x, out=None, scratch=None, hist=None, status=None, kind: int 
     _check(fn(tables.data_ptr(), x.data_ptr(), n, out.data_ptr(), out.numel(), scratch.data_ptr(),
               hist.data_ptr() if hist is not None else None, status.data_ptr(), _stream(x)),
            "hx_encode")
+    return out, status
+
+
+NOALLOC_MAX_BYTES = 128 << 20
+
+
+def encode_noalloc(tables, x, out, hist=None, status=None):
+    """hx_encode_noalloc: Huffman encode whose scratch lives in the library (no allocation inside
+    the call; `out` and `status` are the caller's). For callers that cannot allocate device
+    memory at encode time. n <= NOALLOC_MAX_BYTES; calls overlapping on the GPU race."""
+    x = _dev_u8(x, "x")
+    out = _dev_u8(out, "out")
+    if status is None:
+        status = new_status(x.device)
+    _check(lib().hx_encode_noalloc(tables.data_ptr(), x.data_ptr(), x.numel(), out.data_ptr(),
+                                   out.numel(), hist.data_ptr() if hist is not None else None,
+                                   status.data_ptr(), _stream(x)), "hx_encode_noalloc")
     return out, status
 
 
