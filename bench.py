@@ -57,6 +57,21 @@ def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
 
 
+def max_over_ranks(ms: float, pg, device) -> float:
+    """The slowest rank's time: every rank calls this at the same point (a MAX all-reduce)."""
+    if pg is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world: int, bytes_per_rank_step: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank moves its own batch each step (weak scaling)."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
@@ -280,11 +295,7 @@ def main():
         torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
-    elapsed_ms = start.elapsed_time(end)
-    if pg:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), pg, dev)
     assert int(status.item()) == 0, f"status {int(status.item())}"
     per_op_ms = {o: sum(a.elapsed_time(b) for a, b in ev[o]) / args.steps for o in ops}
 
@@ -300,7 +311,7 @@ def main():
     alg_bytes = {"huffman_encode": n + size_h, "huffman_decode": size_h + n,
                  "qlc_encode": n + size_q, "qlc_decode": size_q + n}
     ms_per_step = elapsed_ms / args.steps
-    value = ws * 4 * n / (ms_per_step * 1e-3) / 1e9
+    value = job_gbs(ws, 4 * n, ms_per_step)
     peak, peak_kind = hbm_peak()
     dominant = max(ops, key=lambda o: per_op_ms[o])
     achieved = alg_bytes[dominant] / (per_op_ms[dominant] * 1e-3) / 1e9
@@ -346,12 +357,8 @@ def main():
             d2h = e2e_step()
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = s0.elapsed_time(s1) / k_e2e
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": ws * 4 * n / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / k_e2e, pg, dev)
+        e2e = {"value": job_gbs(ws, 4 * n, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": n, "d2h_bytes_per_step": d2h, "steps": k_e2e,
                "path": "pinned host batch -> H2D -> 4 codec calls -> D2H of both streams"}
 

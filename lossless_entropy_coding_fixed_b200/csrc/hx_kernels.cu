@@ -7,28 +7,27 @@
 //   k_histogram  byte histogram: 16-byte loads, one private 256-bin table per warp in shared
 //                memory, one global atomic per non-empty bin and block.
 //
-//   k_encode     persistent; one 4096-symbol chunk per block iteration, chunks taken in order
-//                from an atomic ticket. Input chunks arrive in a 4-stage shared-memory ring by
-//                bulk asynchronous copies (cp.async.bulk + mbarrier), issued as soon as a stage
-//                is free. The code/length table is replicated once per lane ([symbol][lane]), so
-//                a warp's 32 lookups never share a bank; its high half counts the symbols, so a
-//                single shared atomic both reads the code and adds to the fused histogram.
+//   k_encode     persistent; one 4096-symbol chunk per block iteration, encoder block e of E
+//                taking chunks e, e+E, e+2E, ... Input chunks arrive in a 3-stage shared-memory
+//                ring by bulk asynchronous copies (cp.async.bulk + mbarrier), issued as soon as a
+//                stage is free. The code/length table is replicated 16 times ([symbol][copy]),
+//                so a warp's 32 lookups meet at most two to a bank; its high bits count the
+//                symbols, so a single shared atomic both reads the code and adds to the fused
+//                histogram.
 //                Warp prefix sums of the code lengths (warp k = sub-stream k: the warp prefixes
 //                are the sync offsets) and packing through a 64-bit accumulator into a shared
-//                output buffer; the chunk's size goes out at once as a flag word. Block 0 of the
-//                (cooperatively launched, so co-resident) grid is the scanner: it turns the run
-//                of published sizes into word offsets 2048 chunks per step with a block-wide
-//                prefix sum -- a single-pass chained scan whose serial part moves a whole
-//                window at a time. One iteration later, so the wait overlaps the next chunk's
-//                work, the encoder reads its offset and stores the chunk with coalesced words.
+//                output buffer; the chunk's size goes out at once as a flag word. A chunk is
+//                stored a few iterations later, when every block has published the sizes of its
+//                wave: each block sums the wave's sizes itself (no serial scan, no dedicated
+//                block) and keeps a running total of earlier waves, which gives the offset.
 //
 //   k_decode     one thread per sub-stream (8 per chunk, 32 chunks per 256-thread block). The
-//                payload is read 16 bytes at a time with the next 16 bytes already in flight; a
-//                64-bit bit window feeds one lookup per symbol in the 4096-entry shared table.
-//                Huffman takes symbol and length from the table; QLC takes the length from the
-//                3-bit area through a register-held width table (3 + width) and only the symbol
-//                from the table. 32 decoded bytes leave as two 16-byte stores (a whole 32-byte
-//                sector). Every sub-stream must end exactly where the next one starts.
+//                payload is read word by word, a few words ahead of use (predicated loads, no
+//                lane-dependent branch); a 64-bit bit window feeds one lookup per symbol in the
+//                4096-entry shared table, which gives symbol and length for either kind (for a
+//                QLC code it is precomputed from the area widths and the rank table). 32
+//                decoded bytes leave as two 16-byte stores (a whole 32-byte sector). Every
+//                sub-stream must end exactly where the next one starts.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -47,20 +46,19 @@ constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
 constexpr int kEncThreads = 256;  // 16 symbols per thread; warp k codes sub-stream k
 constexpr int kDecThreads = 256;  // 8 threads per chunk, 32 chunks per block
 constexpr int kHistThreads = 256;
-constexpr int kStages = 4;        // encode input ring
-constexpr int kLag = 3;           // encode: a chunk is stored kLag iterations after it is packed
-constexpr int kLutCopies = 32;    // encode: table copies; lane l reads copy l % kLutCopies
+constexpr int kStages = 3;        // encode input ring
+constexpr int kLag = 2;           // encode: a chunk is stored kLag iterations after it is coded
+constexpr int kLutCopies = 16;    // encode: table copies; lane l reads copy l % kLutCopies
 constexpr int kOutBufs = kLag + 2;  // encode output buffers
 // 12-bit counters; a copy gains at most 16 per chunk from each lane that reads it
-constexpr uint32_t kHistFlushChunks = 255 / (32 / kLutCopies);
+constexpr uint32_t kHistFlushChunks = 4095 / (16 * (32 / kLutCopies));
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s bound on any wait
 
-// per-chunk flag word: [63:62] state, [61:0] value. An encoder block publishes the chunk's
-// size in words (kFlagSize); the scanner block replaces it by the chunk's word offset (kFlagDone).
+// per-chunk flag word: [63:62] state, [61:0] value. The block that codes a chunk publishes its
+// size in words (kFlagSize).
 constexpr unsigned long long kFlagSize = 1ull << 62;
-constexpr unsigned long long kFlagDone = 2ull << 62;
 constexpr unsigned long long kFlagValue = (1ull << 62) - 1;
-constexpr int kScanPerThread = 8;  // scanner window: 256 threads x 8 flags
+constexpr uint32_t kMaxEncodeBlocks = 2 * kEncThreads;  // a wave's sizes: two per thread
 
 __host__ __device__ inline uint64_t n_chunks_of(uint64_t n) { return (n + kChunk - 1) / kChunk; }
 __host__ __device__ inline uint64_t sync_offset(uint64_t n) {
@@ -180,17 +178,16 @@ struct EncodeArgs {
 };
 
 struct EncSmem {
-  // [symbol][copy]: (count << 20) | (code << 8) | len. One copy per lane: no bank conflicts;
-  // len in the low byte lets 16 entries be summed into a bit count (16 * 12 < 256).
+  // [symbol][copy]: (code << 20) | (count << 8) | len. Lane l reads copy l % kLutCopies, so a
+  // warp's lookups meet at most 32 / kLutCopies to a bank; len in the low byte lets 16 entries
+  // be summed into a bit count (16 * 12 < 256); the code comes out with one shift.
   uint32_t lut[256 * kLutCopies];
   alignas(128) uint8_t in[kStages][kChunk];
   uint32_t out[kOutBufs][kMaxChunkWords];
   alignas(16) uint32_t warp_bits[kOutBufs][kEncThreads / 32];
-  uint32_t chunk_of[kOutBufs];
-  uint32_t ticket[kStages];
-  uint32_t next[2];    // chunk of the next iteration's stage (0xffffffff: stop), double-buffered
+  alignas(8) uint32_t wave_red[2][2 * (kEncThreads / 32)];  // per warp (total, prefix), by parity
   uint64_t bar[kStages];
-  uint32_t offset[2];  // word offset of the chunk stored this iteration, double-buffered
+  uint32_t stop;  // a bulk copy did not complete in time
 };
 
 // Every header field but total_words (written by the block that finishes the last chunk).
@@ -211,104 +208,14 @@ __device__ inline void write_header(const EncodeArgs& a) {
   for (uint64_t i = gap; i < sync_offset(a.n); i += 4) h32[i / 4] = 0;
 }
 
-// The scanner block: walks the flag words in order, 2048 at a time. The longest run of
-// published sizes at the front of the window gets a block-wide exclusive prefix sum; each of
-// those chunks gets its word offset (flag kFlagDone, and word_off[] in the stream). Encoder
-// blocks publish a size without waiting, so the run always grows; waits are bounded in time.
-__device__ void scan_chunk_offsets(const EncodeArgs& a, uint32_t nchunks, uint32_t* s_red,
-                                   uint32_t* s_stop) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
-  const uint64_t P = payload_offset(a.n);
-  uint64_t F = 0, running = 0;
-  unsigned long long t0 = 0;
-  while (F < nchunks) {
-    uint32_t val[kScanPerThread];
-    uint32_t first = kScanPerThread * kEncThreads;  // first index in the window without a size
-#pragma unroll
-    for (int j = kScanPerThread - 1; j >= 0; --j) {
-      const uint64_t idx = F + (uint64_t)tid * kScanPerThread + j;
-      unsigned long long f = 0;
-      if (idx < nchunks) f = ld_relaxed(a.flags + idx);
-      val[j] = (uint32_t)(f & kFlagValue);
-      if ((f & ~kFlagValue) != kFlagSize) first = (uint32_t)tid * kScanPerThread + j;
-    }
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, d));
-    if (lane == 0) s_red[warp] = first;
-    __syncthreads();
-    uint32_t cnt = s_red[0];
-#pragma unroll
-    for (int w = 1; w < kEncThreads / 32; ++w) cnt = min(cnt, s_red[w]);
-    __syncthreads();
-    if (cnt == 0) {  // nothing new yet: thread 0 keeps the clock, so all threads agree
-      if (tid == 0) {
-        const unsigned long long now = global_ns();
-        if (t0 == 0) t0 = now;
-        *s_stop = now - t0 > kWaitLimitNs;
-        if (*s_stop) atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
-      }
-      __syncthreads();
-      if (*s_stop) return;
-      __nanosleep(100);
-      continue;
-    }
-    t0 = 0;
-    // exclusive prefix over window indices < cnt (thread-contiguous: index = 8 tid + j)
-    uint32_t mine = 0;
-#pragma unroll
-    for (int j = 0; j < kScanPerThread; ++j)
-      if ((uint32_t)tid * kScanPerThread + j < cnt) mine += val[j];
-    uint32_t incl = mine;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += t;
-    }
-    if (lane == 31) s_red[warp] = incl;
-    __syncthreads();
-    uint32_t before = 0, window_total = 0;
-#pragma unroll
-    for (int w = 0; w < kEncThreads / 32; ++w) {
-      before += w < warp ? s_red[w] : 0u;
-      window_total += s_red[w];
-    }
-    __syncthreads();
-    uint64_t off = running + before + incl - mine;
-#pragma unroll
-    for (int j = 0; j < kScanPerThread; ++j) {
-      const uint32_t e = (uint32_t)tid * kScanPerThread + j;
-      if (e < cnt) {
-        word_off[F + e] = (uint32_t)off;
-        st_relaxed(a.flags + F + e, kFlagDone | off);
-        off += val[j];
-      }
-    }
-    running += window_total;
-    F += cnt;
-  }
-  if (tid == 0) {
-    word_off[nchunks] = (uint32_t)running;
-    reinterpret_cast<uint64_t*>(a.out)[4] = running;
-    uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
-    if (P + 4 * (running + 2) <= a.cap) {
-      payload[running] = 0;
-      payload[running + 1] = 0;
-    } else {
-      atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
-    }
-  }
-}
-
-// Word offset of chunk c from the scanner (one thread polls); bounded in time.
-__device__ uint32_t wait_chunk_offset(const EncodeArgs& a, uint32_t c) {
-  unsigned long long f = ld_relaxed(a.flags + c);
-  if ((f & ~kFlagValue) == kFlagDone) return (uint32_t)(f & kFlagValue);
+// Size flag of chunk c, waiting (bounded in time) until its block has published it.
+__device__ uint32_t wait_chunk_size(const EncodeArgs& a, uint32_t c, unsigned long long f) {
+  if ((f & ~kFlagValue) == kFlagSize) return (uint32_t)(f & kFlagValue);
   const unsigned long long t0 = global_ns();
   while (true) {
-    __nanosleep(64);
+    __nanosleep(32);
     f = ld_relaxed(a.flags + c);
-    if ((f & ~kFlagValue) == kFlagDone) return (uint32_t)(f & kFlagValue);
+    if ((f & ~kFlagValue) == kFlagSize) return (uint32_t)(f & kFlagValue);
     if (global_ns() - t0 > kWaitLimitNs) {
       atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
       return 0;
@@ -328,7 +235,7 @@ __device__ __forceinline__ uint32_t lookup16(uint32_t* lut_lane, const uint32_t 
     uint32_t ent = 0;
     if (FULL || (uint32_t)j < valid) {
       uint32_t* slot = lut_lane + sym * kLutCopies;
-      ent = HIST ? atomicAdd(slot, 1u << 20) : *slot;
+      ent = HIST ? atomicAdd(slot, 1u << 8) : *slot;
     }
     e[j] = ent;
     sum += ent;
@@ -338,80 +245,141 @@ __device__ __forceinline__ uint32_t lookup16(uint32_t* lut_lane, const uint32_t 
 
 // Pack 16 (code, len) entries MSB-first starting at bit `off` of buf: two codes are joined in a
 // 32-bit register (<= 24 bits), then appended to a 64-bit accumulator (hi:lo) with funnel
-// shifts. Words this thread owns are stored; the first and last, shared with neighbours, OR-ed.
+// shifts. Every finished word is OR-ed into the zeroed buffer (the first and last may be shared
+// with neighbours), so the emit is one predicated step with no lane-dependent branch.
 __device__ __forceinline__ void pack16(const uint32_t e[16], uint32_t off, uint32_t* buf) {
   uint32_t widx = off >> 5;
   uint32_t nacc = off & 31;  // the first bits belong to the previous thread (zeros here)
-  bool shared_first = nacc != 0;
   uint32_t hi = 0, lo = 0;
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
     const uint32_t e0 = e[2 * p], e1 = e[2 * p + 1];
     const uint32_t l1 = e1 & 0xffu;
     const uint32_t pl = (e0 & 0xffu) + l1;
-    const uint32_t pc = (((e0 >> 8) & 0xfffu) << l1) | ((e1 >> 8) & 0xfffu);
+    const uint32_t pc = ((e0 >> 20) << l1) | (e1 >> 20);
     hi = __funnelshift_l(lo, hi, pl);
     lo = (lo << pl) | pc;
     nacc += pl;
-    if (nacc >= 32) {
-      nacc -= 32;
-      const uint32_t word = __funnelshift_r(lo, hi, nacc);
-      if (shared_first) atomicOr(&buf[widx], word);
-      else buf[widx] = word;
-      shared_first = false;
-      ++widx;
-    }
+    const bool full = nacc >= 32;
+    nacc -= full ? 32u : 0u;
+    if (full) atomicOr(&buf[widx], __funnelshift_r(lo, hi, nacc));
+    widx += full ? 1u : 0u;
   }
   if (nacc) atomicOr(&buf[widx], lo << (32 - nacc));
 }
 
+// Encoder block e of E takes chunks e, e + E, e + 2E, ... in order: iteration k codes chunk
+// kE + e, and the chunks kE .. kE + E - 1 form wave k. Stage k % kStages of the input ring
+// holds the chunk of iteration k, loaded by a bulk copy kStages iterations ahead.
+//
+// Word offsets without a serial scan: a chunk is stored kLag iterations after it is coded.
+// Then every block reads the sizes that all blocks published for that wave (two per thread,
+// requested before the symbol work), and one block-wide sum gives both the wave's total and
+// the words of the chunks before its own in the wave. Each block adds the wave totals up as it
+// goes, so the offset of its chunk is that running total plus its in-wave prefix. All blocks
+// are resident (cooperative launch), so every size a block waits for is being computed.
 template <bool HIST, bool COMPLETE>
 __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint64_t n = a.n;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
   const uint32_t full_chunks = (uint32_t)(n / kChunk);
+  const uint32_t E = gridDim.x, eb = blockIdx.x;
   const uint64_t P = payload_offset(n);
+  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
   uint4* sync = reinterpret_cast<uint4*>(a.out + sync_offset(n));
   uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
   uint32_t* lut_lane = sm.lut + lane % kLutCopies;
+  auto chunk_of = [&](uint32_t k) -> uint32_t { return k * E + eb; };
 
-  // stage s takes ticket t; full chunks arrive by bulk copy, others by plain loads
-  auto refill = [&](int s, uint32_t t) {
-    sm.ticket[s] = t;
-    if (t < full_chunks) {
-      mbar_arrive_expect_tx(&sm.bar[s], kChunk);
-      bulk_load(sm.in[s], a.in + (uint64_t)t * kChunk, kChunk, &sm.bar[s]);
+  // stage k % kStages <- chunk of iteration k (bulk copy for a full chunk; else a plain arrive)
+  auto issue = [&](uint32_t k) {
+    const uint32_t c = chunk_of(k);
+    uint64_t* bar = &sm.bar[k % kStages];
+    if (c < full_chunks) {
+      mbar_arrive_expect_tx(bar, kChunk);
+      bulk_load(sm.in[k % kStages], a.in + (uint64_t)c * kChunk, kChunk, bar);
     } else {
-      mbar_arrive(&sm.bar[s]);
+      mbar_arrive(bar);
     }
   };
-  // Only thread 0 waits on a stage's mbarrier; the block barrier that follows hands the
-  // stage (and the uniform go/stop decision) to every thread.
-  auto await_stage = [&](uint32_t it_next) {
-    const int s = (int)(it_next % kStages);
-    uint32_t c = 0xffffffffu;
-    if (mbar_wait(&sm.bar[s], (it_next / kStages) & 1u)) c = sm.ticket[s];
-    else atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
-    sm.next[it_next & 1] = c;
+  // only thread 0 waits on a stage; the block barrier after it hands the stage to every thread
+  auto await_stage = [&](uint32_t k) {
+    if (chunk_of(k) < nchunks && !mbar_wait(&sm.bar[k % kStages], (k / kStages) & 1u)) {
+      sm.stop = 1;
+      atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
+    }
+  };
+  // size flags of wave w that this thread sums: its chunks tid and tid + kEncThreads
+  auto load_wave = [&](uint32_t w, unsigned long long f[2]) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t j = (uint32_t)tid + i * kEncThreads;
+      const uint64_t c = (uint64_t)w * E + j;
+      f[i] = (j < E && c < nchunks) ? ld_relaxed(a.flags + c) : kFlagSize;
+    }
+  };
+  // this thread's part of the wave total and of the block's in-wave prefix, reduced per warp
+  auto reduce_wave = [&](uint32_t w, unsigned long long f[2], uint32_t parity) {
+    uint32_t tot = 0, pre = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t j = (uint32_t)tid + i * kEncThreads;
+      const uint32_t v = wait_chunk_size(a, w * E + j, f[i]);
+      tot += v;
+      pre += j < eb ? v : 0u;
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, d);
+      pre += __shfl_xor_sync(0xffffffffu, pre, d);
+    }
+    if (lane == 0) {
+      sm.wave_red[parity][2 * warp] = tot;
+      sm.wave_red[parity][2 * warp + 1] = pre;
+    }
   };
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) refill(s, atomicAdd(a.ticket, 1u));
+    sm.stop = 0;
+    for (uint32_t k = 0; k < (uint32_t)kStages; ++k) issue(k);
     await_stage(0);
+    if (nchunks == 0 && eb == 0) {  // an empty stream: header, index and guards only
+      write_header(a);
+      reinterpret_cast<uint64_t*>(a.out)[4] = 0;
+      word_off[0] = 0;
+      payload[0] = 0;  // the host checked cap >= P + 8
+      payload[1] = 0;
+    }
   }
   __syncthreads();
 
   bool uncodable = false;
   uint32_t since_flush = 0;
+  uint64_t running = 0;  // words of all waves before the one being stored
 
-  // Stores of the chunk packed kLag iterations earlier (buffer b), once its offset is known.
-  auto store_chunk = [&](int b, uint32_t woff) {
-    const uint32_t c = sm.chunk_of[b];
+  // Stores of the chunk of iteration k (output buffer k % kOutBufs); its wave's sums are in
+  // wave_red[parity]. Every thread computes the same offset.
+  auto store_chunk = [&](uint32_t k, uint32_t parity) {
+    // lanes 0..7 fetch one warp's (total, prefix) pair each; a shuffle sum spreads the result
+    uint2 wr = lane < kEncThreads / 32
+                   ? *reinterpret_cast<const uint2*>(&sm.wave_red[parity][2 * lane])
+                   : make_uint2(0u, 0u);
+#pragma unroll
+    for (int d = 4; d > 0; d >>= 1) {
+      wr.x += __shfl_xor_sync(0xffffffffu, wr.x, d);
+      wr.y += __shfl_xor_sync(0xffffffffu, wr.y, d);
+    }
+    const uint32_t wave_total = __shfl_sync(0xffffffffu, wr.x, 0);
+    const uint32_t before = __shfl_sync(0xffffffffu, wr.y, 0);
+    const uint64_t woff = running + before;
+    running += wave_total;
+    const int b = (int)(k % kOutBufs);
+    const uint32_t c = chunk_of(k);
     const uint4 t0 = *reinterpret_cast<const uint4*>(&sm.warp_bits[b][0]);
     const uint4 t1 = *reinterpret_cast<const uint4*>(&sm.warp_bits[b][4]);
     const uint32_t total = t0.x + t0.y + t0.z + t0.w + t1.x + t1.y + t1.z + t1.w;
     const uint32_t words = (total + 31) >> 5;
-    const bool fits = P + 4ull * ((uint64_t)woff + words + 2) <= a.cap;
+    const bool fits = P + 4ull * (woff + words + 2) <= a.cap;
     uint32_t* buf = sm.out[b];
     for (uint32_t i = tid; i < words; i += kEncThreads) {
       if (fits) payload[woff + i] = buf[i];
@@ -421,8 +389,18 @@ __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
       const uint32_t p1 = t0.x, p2 = p1 + t0.y, p3 = p2 + t0.z, p4 = p3 + t0.w;
       const uint32_t p5 = p4 + t1.x, p6 = p5 + t1.y, p7 = p6 + t1.z;
       sync[c] = make_uint4(total | (p1 << 16), p2 | (p3 << 16), p4 | (p5 << 16), p6 | (p7 << 16));
+      word_off[c] = (uint32_t)woff;
       if (!fits) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
       if (c == 0) write_header(a);
+      if (c == nchunks - 1) {  // the last chunk closes the index
+        const uint64_t end = woff + words;
+        word_off[nchunks] = (uint32_t)end;
+        reinterpret_cast<uint64_t*>(a.out)[4] = end;
+        if (fits) {
+          payload[end] = 0;
+          payload[end + 1] = 0;
+        }
+      }
     }
   };
 
@@ -431,28 +409,23 @@ __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
     uint32_t sum = 0;
     for (int l = 0; l < kLutCopies; ++l) {
       const uint32_t e = sm.lut[tid * kLutCopies + l];
-      sum += e >> 20;
-      sm.lut[tid * kLutCopies + l] = e & 0xfffffu;
+      sum += (e >> 8) & 0xfffu;
+      sm.lut[tid * kLutCopies + l] = e & ~(0xfffu << 8);
     }
     if (sum) atomicAdd(&a.hist[tid], sum);
     __syncthreads();
   };
 
-  uint32_t it = 0;
-  for (;; ++it) {
-    const int s = (int)(it % kStages);
-    const int ob = (int)(it % kOutBufs);
-    const uint32_t c = sm.next[it & 1];
-    if (c >= nchunks) break;  // uniform: written before the last block barrier
+  uint32_t k = 0;
+  for (;; ++k) {
+    const uint32_t c = chunk_of(k);
+    if (c >= nchunks || sm.stop) break;  // uniform: sm.stop is set before a block barrier
+    const int s = (int)(k % kStages);
+    const int ob = (int)(k % kOutBufs);
+    const bool lagged = k >= kLag;
+    unsigned long long wf[2];
+    if (lagged) load_wave(k - kLag, wf);  // answers are needed only after the symbol work
 
-    // thread 0 starts its two global round trips now and needs the answers only after the
-    // symbol work: the ticket for this stage's refill and the flag of the lagged chunk
-    uint32_t next_ticket = 0;
-    unsigned long long lag_flag = 0;
-    if (tid == 0) {
-      next_ticket = atomicAdd(a.ticket, 1u);
-      if (it >= kLag) lag_flag = ld_relaxed(a.flags + sm.chunk_of[(it - kLag) % kOutBufs]);
-    }
     uint32_t w[4];
     uint32_t e[16];
     uint32_t sum;
@@ -463,6 +436,9 @@ __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
       w[2] = v.z;
       w[3] = v.w;
       sum = lookup16<HIST, true>(lut_lane, w, 16, e);
+      if (!COMPLETE)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) uncodable |= (e[j] & 0xffu) == 0;
     } else {  // the ragged last chunk, from global memory
       const uint64_t base = (uint64_t)c * kChunk;
       const uint32_t first = (uint32_t)tid * 16;
@@ -482,9 +458,6 @@ __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) uncodable |= (uint32_t)j < valid && (e[j] & 0xffu) == 0;
     }
-    if (!COMPLETE && c < full_chunks)
-#pragma unroll
-      for (int j = 0; j < 16; ++j) uncodable |= (e[j] & 0xffu) == 0;
     const uint32_t bits = sum & 0xffu;
     uint32_t incl = bits;
 #pragma unroll
@@ -493,50 +466,49 @@ __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
       if (lane >= d) incl += t;
     }
     if (lane == 31) sm.warp_bits[ob][warp] = incl;
-    if (tid == 0) {
-      if (it >= kLag)  // offset of the chunk packed kLag iterations ago
-        sm.offset[it & 1] = (lag_flag & ~kFlagValue) == kFlagDone
-                                ? (uint32_t)(lag_flag & kFlagValue)
-                                : wait_chunk_offset(a, sm.chunk_of[(it - kLag) % kOutBufs]);
-      await_stage(it + 1);
-    }
-    __syncthreads();  // warp totals ready; stage s read by all; next stage handed over
+    if (lagged) reduce_wave(k - kLag, wf, k & 1);
+    if (tid == 0) await_stage(k + 1);
+    __syncthreads();  // warp totals and wave sums ready; stage s read; next stage handed over
 
-    const uint4 t0 = *reinterpret_cast<const uint4*>(&sm.warp_bits[ob][0]);
-    const uint4 t1 = *reinterpret_cast<const uint4*>(&sm.warp_bits[ob][4]);
-    const uint32_t tw[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-    uint32_t warp_base = 0;
+    // lanes 0..7 hold the warp totals; a shuffle scan gives this warp's base and the total
+    uint32_t wt = lane < kEncThreads / 32 ? sm.warp_bits[ob][lane] : 0u;
 #pragma unroll
-    for (int k = 0; k < kEncThreads / 32; ++k) warp_base += k < warp ? tw[k] : 0u;
+    for (int d = 1; d < kEncThreads / 32; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, wt, d);
+      if (lane >= d) wt += t;
+    }
+    const uint32_t warp_base = __shfl_sync(0xffffffffu, wt, (warp + 31) & 31) & (warp ? ~0u : 0u);
+    const uint32_t total = __shfl_sync(0xffffffffu, wt, kEncThreads / 32 - 1);
     if (tid == 0) {
-      const uint32_t total = t0.x + t0.y + t0.z + t0.w + t1.x + t1.y + t1.z + t1.w;
       st_relaxed(a.flags + c, kFlagSize | ((total + 31) >> 5));
-      sm.chunk_of[ob] = c;
       fence_proxy_async();  // this stage's generic reads before the async refill
-      refill(s, next_ticket);
+      issue(k + kStages);
     }
     if (bits) pack16(e, warp_base + incl - bits, sm.out[ob]);
-    if (it >= kLag) store_chunk((int)((it - kLag) % kOutBufs), sm.offset[it & 1]);
+    if (lagged) store_chunk(k - kLag, k & 1);
     if (HIST && ++since_flush == kHistFlushChunks) {
       flush_hist();
       since_flush = 0;
     }
   }
-  if (tid == 0 && sm.next[it & 1] == 0xffffffffu)  // timed out: let copies still in flight land
-    for (uint32_t j = 1; j < (uint32_t)kStages; ++j)
-      mbar_wait(&sm.bar[(it + j) % kStages], ((it + j) / kStages) & 1u);
-  // drain: the last kLag packed chunks
-  for (uint32_t k = it > kLag ? it - kLag : 0; k < it; ++k) {
+  if (tid == 0 && sm.stop)  // timed out: let copies still in flight land
+    for (uint32_t j = 0; j < (uint32_t)kStages; ++j)
+      if (chunk_of(k + j) < full_chunks)
+        mbar_wait(&sm.bar[(k + j) % kStages], ((k + j) / kStages) & 1u);
+  // drain: the last kLag coded chunks
+  for (uint32_t j = k > kLag ? k - kLag : 0; j < k; ++j) {
+    unsigned long long wf[2];
+    load_wave(j, wf);
     __syncthreads();
-    if (tid == 0) sm.offset[0] = wait_chunk_offset(a, sm.chunk_of[k % kOutBufs]);
+    reduce_wave(j, wf, 0);
     __syncthreads();
-    store_chunk((int)(k % kOutBufs), sm.offset[0]);
+    store_chunk(j, 0);
   }
   if (!COMPLETE && uncodable) atomicOr(a.status, (uint32_t)HX_ERR_UNCODABLE);
   if (HIST) flush_hist();
 }
 
-__global__ void __launch_bounds__(kEncThreads) k_encode(EncodeArgs a) {
+__global__ void __launch_bounds__(kEncThreads, 3) k_encode(EncodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   EncSmem& sm = *reinterpret_cast<EncSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -545,15 +517,10 @@ __global__ void __launch_bounds__(kEncThreads) k_encode(EncodeArgs a) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
     return;
   }
-  if (blockIdx.x == 0) {  // block 0 scans the chunk sizes into word offsets
-    if (nchunks == 0 && tid == 0) write_header(a);
-    scan_chunk_offsets(a, nchunks, sm.warp_bits[0], &sm.offset[0]);
-    return;
-  }
   bool complete = true;
   for (int i = tid; i < 256 * kLutCopies; i += kEncThreads) {
     const uint32_t t = a.tables->enc[i / kLutCopies];  // (code << 4) | len
-    uint32_t e = ((t >> 4) << 8) | (t & 15u);
+    uint32_t e = ((t >> 4) << 20) | (t & 15u);
     if ((t & 15u) > HX_LMAX_MAX || t > 0xffffu) {  // a damaged table block stays harmless
       e = 0;
       atomicOr(a.status, (uint32_t)HX_ERR_ARG);
@@ -612,58 +579,33 @@ __device__ int64_t check_header(const DecodeArgs& a) {
   return (int64_t)total;
 }
 
-// A quad (16 bytes) of payload words that is not wholly inside the caller's buffer: words past
-// the buffer read as 0. Out of line: only the last quad of a stream can take this path.
-__device__ __noinline__ uint4 tail_quad(const uint32_t* words, uint64_t q, uint64_t wlimit) {
-  uint32_t v[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint64_t wi = 4 * q + i;
-    v[i] = wi < wlimit ? __ldg(words + wi) : 0u;
-  }
-  return make_uint4(v[0], v[1], v[2], v[3]);
-}
-
 // Payload words of one sub-stream, MSB-first, through a 64-bit bit window held as two 32-bit
-// halves (wh:wl) whose top `avail` bits are valid. Words come from a reservoir: `cur` holds the
-// next `left` words, `nxt` the quad after them, so the next 16 bytes are always in flight.
-// FAST: every quad the current group can touch lies wholly inside the buffer.
+// halves (wh:wl) whose top `avail` bits are valid. The next kPrefetch words are already
+// requested (pf[]): a refill takes pf[0] and requests one more word -- one predicated load and
+// register moves, no branch that depends on the other lanes. Words past the caller's buffer
+// read as 0.
+constexpr int kPrefetch = 2;
 struct SubstreamReader {
-  const uint4* quads;
   const uint32_t* words;
-  uint64_t qsafe, wlimit;
-  uint64_t qn;  // next quad to request
-  uint4 cur, nxt;
-  uint32_t left, taken;
+  uint64_t wlimit;  // payload words inside the buffer
+  uint64_t wi;      // index of the word in pf[0]
+  uint32_t pf[kPrefetch];
   uint32_t wh, wl;
   int avail;
 
-  template <bool FAST>
-  __device__ __forceinline__ uint4 quad(uint64_t q) const {
-    if (FAST) return __ldg(quads + q);
-    return q < qsafe ? __ldg(quads + q) : tail_quad(words, q, wlimit);
-  }
-  template <bool FAST>
-  __device__ __forceinline__ uint32_t take() {
-    const uint32_t w = cur.x;
-    cur.x = cur.y;
-    cur.y = cur.z;
-    cur.z = cur.w;
-    ++taken;
-    if (--left == 0) {
-      cur = nxt;
-      nxt = quad<FAST>(qn++);
-      left = 4;
-    }
-    return w;
+  __device__ __forceinline__ uint32_t word(uint64_t i) const {
+    return i < wlimit ? __ldg(words + i) : 0u;
   }
   // afterwards >= 32 valid bits: room for two codes of <= 12 bits
-  template <bool FAST>
   __device__ __forceinline__ void refill() {
     if (avail < 32) {
-      const uint32_t w = take<FAST>();
-      wh |= w >> avail;                             // the word lands at bits [32-avail, 64-avail)
-      wl |= __funnelshift_lc(0u, w, 32 - avail);   // its low part (nothing when avail == 0)
+      const uint32_t w = pf[0];
+#pragma unroll
+      for (int i = 0; i + 1 < kPrefetch; ++i) pf[i] = pf[i + 1];
+      pf[kPrefetch - 1] = word(wi + kPrefetch);
+      ++wi;
+      wh |= w >> avail;                            // the word lands at bits [32-avail, 64-avail)
+      wl |= __funnelshift_lc(0u, w, 32 - avail);  // its low part (nothing when avail == 0)
       avail += 32;
     }
   }
@@ -674,73 +616,56 @@ struct SubstreamReader {
   }
   __device__ void start(uint64_t first_bit) {
     const uint64_t fw = first_bit >> 5;
-    qn = fw >> 2;
-    cur = quad<false>(qn);
-    nxt = quad<false>(qn + 1);
-    qn += 2;
-    left = 4;
-    for (uint32_t skip = (uint32_t)(fw & 3); skip > 0; --skip) take<false>();
-    taken = 0;
-    wh = take<false>();
-    wl = take<false>();
     const uint32_t sh = (uint32_t)(first_bit & 31);
+    wh = word(fw);
+    wl = word(fw + 1);
+    wi = fw + 2;
+#pragma unroll
+    for (int i = 0; i < kPrefetch; ++i) pf[i] = word(wi + i);
     wh = __funnelshift_l(wl, wh, sh);
     wl <<= sh;
     avail = 64 - (int)sh;
   }
   // index (in payload bits) of the next bit not yet consumed
-  __device__ uint64_t position(uint64_t first_bit) const {
-    return 32 * ((first_bit >> 5) + taken) - (uint64_t)avail;
-  }
+  __device__ uint64_t position() const { return 32 * wi - (uint64_t)avail; }
 };
 
-// One symbol from the top of the window, returned as a table entry whose byte 1 is the symbol.
-// Huffman: the 4096-entry table gives symbol and length. QLC: the length is 3 + the width of the
-// area named by the top 3 bits (a register lookup, so the window advance waits on no memory
-// access); the symbol comes from the same kind of table.
-template <int KIND, bool COMPLETE>
+// One symbol from the top of the window: the 4096-entry table gives (symbol << 8) | length for
+// both kinds. For a QLC table the length is 3 + the width of the area in the top 3 bits; the
+// table holds it already, so reading it there costs less than recomputing it. An entry of 0
+// (no code word starts the window) only occurs for an incomplete code.
+template <bool COMPLETE>
 __device__ __forceinline__ uint32_t next_symbol(SubstreamReader& rd, bool& invalid,
-                                                const uint16_t* lut, const uint32_t* area,
-                                                uint32_t qbits) {
+                                                const uint16_t* lut) {
   const uint32_t e = lut[rd.wh >> 20];
-  uint32_t len;
-  if (KIND == HX_KIND_HUFFMAN) {
-    len = e & 15u;
-    if (!COMPLETE) invalid |= len == 0;
-  } else {
-    const uint32_t ar = rd.wh >> 29;
-    const uint32_t b = (qbits >> (4 * ar)) & 15u;
-    len = 3 + b;
-    if (!COMPLETE) invalid |= ((rd.wh >> (29 - b)) & ((1u << b) - 1u)) >= ((area[ar] >> 9) & 511u);
-  }
+  const uint32_t len = e & 15u;
+  if (!COMPLETE) invalid |= len == 0;
   rd.consume(len);
   return e;
 }
 
-// 32 symbols -> 32 output bytes (two 16-byte stores, one whole sector). Each symbol's byte is
-// moved into place with one byte permute.
-template <int KIND, bool COMPLETE, bool FAST>
+// 32 symbols -> 32 output bytes (two 16-byte streaming stores, one whole sector). Each symbol's
+// byte is moved into place with one byte permute.
+template <bool COMPLETE>
 __device__ __forceinline__ void decode_group32(SubstreamReader& rd, bool& invalid, uint4* d4,
-                                               const uint16_t* lut, const uint32_t* area,
-                                               uint32_t qbits) {
+                                               const uint16_t* lut) {
   uint32_t o[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    rd.refill<FAST>();
-    uint32_t v = next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits) >> 8;
-    v = __byte_perm(v, next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits), 0x3250);
-    rd.refill<FAST>();
-    v = __byte_perm(v, next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits), 0x3510);
-    v = __byte_perm(v, next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits), 0x5210);
+    rd.refill();
+    uint32_t v = next_symbol<COMPLETE>(rd, invalid, lut) >> 8;
+    v = __byte_perm(v, next_symbol<COMPLETE>(rd, invalid, lut), 0x3250);
+    rd.refill();
+    v = __byte_perm(v, next_symbol<COMPLETE>(rd, invalid, lut), 0x3510);
+    v = __byte_perm(v, next_symbol<COMPLETE>(rd, invalid, lut), 0x5210);
     o[q] = v;
   }
-  d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
-  d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  __stcs(d4, make_uint4(o[0], o[1], o[2], o[3]));
+  __stcs(d4 + 1, make_uint4(o[4], o[5], o[6], o[7]));
 }
 
-template <int KIND, bool COMPLETE>
-__device__ void decode_chunks(const DecodeArgs& a, const uint16_t* lut, const uint32_t* area,
-                              uint32_t qbits, uint32_t total) {
+template <bool COMPLETE>
+__device__ void decode_chunks(const DecodeArgs& a, const uint16_t* lut, uint32_t total) {
   const int tid = threadIdx.x;
   const uint64_t n = a.n;
   const uint64_t nchunks = n_chunks_of(n);
@@ -749,9 +674,7 @@ __device__ void decode_chunks(const DecodeArgs& a, const uint16_t* lut, const ui
   const uint4* sync = reinterpret_cast<const uint4*>(a.st + sync_offset(n));
   SubstreamReader rd;
   rd.words = reinterpret_cast<const uint32_t*>(a.st + P);
-  rd.quads = reinterpret_cast<const uint4*>(a.st + P);
   rd.wlimit = (a.bytes - P) / 4;  // payload words inside the buffer
-  rd.qsafe = (a.bytes - P) / 16;  // quads [0, qsafe) lie wholly inside it
   const int k = tid & 7;
 
   for (uint64_t c = (uint64_t)blockIdx.x * (kDecThreads / 8) + (tid >> 3); c < nchunks;
@@ -777,47 +700,39 @@ __device__ void decode_chunks(const DecodeArgs& a, const uint16_t* lut, const ui
       bool invalid = false;
       uint8_t* dst = a.out + c * kChunk + (uint64_t)k * kSubLen;
       const uint32_t groups = mine / 32;
-      for (uint32_t g = 0; g < groups; ++g) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * g);
-        // a group takes at most 12 words: 3 more quads past the one requested last
-        if (rd.qn + 3 < rd.qsafe)
-          decode_group32<KIND, COMPLETE, true>(rd, invalid, d4, lut, area, qbits);
-        else
-          decode_group32<KIND, COMPLETE, false>(rd, invalid, d4, lut, area, qbits);
-      }
+      for (uint32_t g = 0; g < groups; ++g)
+        decode_group32<COMPLETE>(rd, invalid, reinterpret_cast<uint4*>(dst + 32 * g), lut);
       for (uint32_t i = groups * 32; i < mine; ++i) {
-        rd.refill<false>();
-        dst[i] = (uint8_t)(next_symbol<KIND, COMPLETE>(rd, invalid, lut, area, qbits) >> 8);
+        rd.refill();
+        dst[i] = (uint8_t)(next_symbol<COMPLETE>(rd, invalid, lut) >> 8);
       }
       // the sub-stream must end exactly where the next one starts
-      bad |= invalid || rd.position(first_bit) != 32ull * w0 + end;
+      bad |= invalid || rd.position() != 32ull * w0 + end;
     }
     if (bad) atomicOr(a.status, (uint32_t)HX_ERR_CORRUPT);
   }
 }
 
+// KIND is checked against the stream header and the tables; the symbol loop is the same.
 template <int KIND>
 __global__ void __launch_bounds__(kDecThreads, 5) k_decode(DecodeArgs a) {
   __shared__ __align__(16) uint16_t s_lut[4096];
-  __shared__ uint32_t s_area[8];
   __shared__ int64_t s_total;
   const int tid = threadIdx.x;
   if (tid == 0) s_total = check_header(a);
   const uint4* src = reinterpret_cast<const uint4*>(a.tables->dec);
   uint4* dst = reinterpret_cast<uint4*>(s_lut);
   for (int i = tid; i < 4096 * 2 / 16; i += kDecThreads) dst[i] = src[i];
-  if (tid < 8) s_area[tid] = a.tables->qlc_area[tid];
   __syncthreads();
   const int64_t total = s_total;
   if (total < 0) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)(-total));
     return;
   }
-  const uint32_t qbits = a.tables->qlc_bits_packed;
   if (a.tables->complete)
-    decode_chunks<KIND, true>(a, s_lut, s_area, qbits, (uint32_t)total);
+    decode_chunks<true>(a, s_lut, (uint32_t)total);
   else
-    decode_chunks<KIND, false>(a, s_lut, s_area, qbits, (uint32_t)total);
+    decode_chunks<false>(a, s_lut, (uint32_t)total);
 }
 
 // ---------------------------------------------------------------------------------- launch
@@ -878,9 +793,11 @@ int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint
   k_zero_scratch<<<(nchunks + 255) / 256 + (nchunks == 0), 256, 0, s>>>(flags, nchunks, ticket);
   EncodeArgs a{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
                out_cap, flags, ticket, d_hist, d_status, kind};
-  // block 0 scans, the others encode; all must be resident at once (cooperative launch)
-  const uint32_t grid = 1 + (uint32_t)std::max<uint64_t>(
-      1, std::min<uint64_t>(nchunks, (uint64_t)info.sms * info.enc_per_sm - 1));
+  // blocks take chunks round-robin and wait for each other's sizes: all must be resident at
+  // once (cooperative launch), and a wave's sizes are summed two per thread
+  const uint32_t grid = (uint32_t)std::max<uint64_t>(
+      1, std::min<uint64_t>({(uint64_t)nchunks, (uint64_t)info.sms * info.enc_per_sm,
+                             (uint64_t)kMaxEncodeBlocks}));
   void* params[] = {&a};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_encode), dim3(grid),
                                   dim3(kEncThreads), params, sizeof(EncSmem), s) != cudaSuccess)

@@ -1,0 +1,64 @@
+"""bench.py's host logic on CPU: the max-over-ranks timing across 2 gloo ranks (the N > 1 path
+has no data-path collective, only this reduction), the whole-job throughput, and the reference
+(oracle) arm on a bounded sample, including its silent exit on ranks other than 0."""
+import io
+import json
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+from types import SimpleNamespace
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, out):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        ms = bench.max_over_ranks(10.0 + 5.0 * rank, dist, torch.device("cpu"))
+        out[rank] = ms
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank, args=(2, port, out), nprocs=2, join=True)
+        assert dict(out) == {0: 15.0, 1: 15.0}
+
+
+def test_job_throughput_is_whole_job():
+    assert bench.job_gbs(1, 4 << 30, 1.0) == pytest.approx(4 * 1.073741824e9 / 1e-3 / 1e9)
+    assert bench.job_gbs(8, 1 << 30, 2.0) == pytest.approx(8 * bench.job_gbs(1, 1 << 30, 2.0))
+    assert bench.max_over_ranks(3.5, None, None) == 3.5
+
+
+def test_reference_arm_runs_oracle_on_rank0_only():
+    args = SimpleNamespace(steps=2, warmup=1)
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        assert bench.cpu_reference(args, rank=1, ws=2) == 0
+    assert buf.getvalue() == ""
+    with redirect_stdout(buf):
+        assert bench.cpu_reference(args, rank=0, ws=1) == 0
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["higher_is_better"] is True
