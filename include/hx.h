@@ -141,8 +141,10 @@ int hx_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
               uint64_t n_expected, uint32_t* d_status, void* stream);
 
 /* The same two calls for a QLC codebook (kind 1 tables): identical stream layout and rules.
- * "Quad Length Codes for Lossless Compression of e4m3", abstract: decoding reads the 3-bit
- * area, then the area's fixed number of index bits, then one 256-entry table. */
+ * "Quad Length Codes for Lossless Compression of e4m3", abstract: a code word is the 3-bit
+ * area, then the area's fixed number of index bits; the index picks the symbol through a
+ * 256-entry rank table. The GPU decoder folds these three steps into one lookup in a 4096-entry
+ * window table that hx_codebook_tables precomputes from the area widths and the rank table. */
 int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
                   uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
                   void* stream);
