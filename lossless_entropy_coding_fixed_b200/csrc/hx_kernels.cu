@@ -7,27 +7,28 @@
 //   k_histogram  byte histogram: 16-byte loads, one private 256-bin table per warp in shared
 //                memory, one global atomic per non-empty bin and block.
 //
-//   k_encode     persistent; one 4096-symbol chunk per block iteration, encoder block e of E
-//                taking chunks e, e+E, e+2E, ... Input chunks arrive in a 3-stage shared-memory
-//                ring by bulk asynchronous copies (cp.async.bulk + mbarrier), issued as soon as a
-//                stage is free. The code/length table is replicated 16 times ([symbol][copy]),
-//                so a warp's 32 lookups meet at most two to a bank; its high bits count the
-//                symbols, so a single shared atomic both reads the code and adds to the fused
-//                histogram.
-//                Warp prefix sums of the code lengths (warp k = sub-stream k: the warp prefixes
-//                are the sync offsets) and packing through a 64-bit accumulator into a shared
-//                output buffer; the chunk's size goes out at once as a flag word. A chunk is
-//                stored a few iterations later, when every block has published the sizes of its
-//                wave: each block sums the wave's sizes itself (no serial scan, no dedicated
-//                block) and keeps a running total of earlier waves, which gives the offset.
+//   k_measure    code lengths only (the first of two passes over the input): a warp measures one
+//                4096-symbol chunk -- lane l looks up 16 bytes of each sub-stream in its own copy
+//                of the length table (no bank conflicts) -- and writes the chunk's sync row; a
+//                block owns a contiguous run of chunks and scans their word counts into
+//                block-local offsets. The fused histogram rides on the same lookups (a shared
+//                atomic that returns the length adds to a per-copy count).
+//
+//   k_pack       every block scans the measure blocks' totals into offsets, so no block waits
+//                for another. A warp codes a whole chunk, one sub-stream (512 symbols, 16 per
+//                lane) at a time: table lookup, warp prefix sum of the lane bit counts, two codes
+//                joined per 32-bit register and appended to a 64-bit accumulator, finished words
+//                OR-ed into the warp's shared buffer; then the chunk goes out with coalesced
+//                stores at its final offset.
 //
 //   k_decode     one thread per sub-stream (8 per chunk, 32 chunks per 256-thread block). The
-//                payload is read word by word, a few words ahead of use (predicated loads, no
-//                lane-dependent branch); a 64-bit bit window feeds one lookup per symbol in the
-//                4096-entry shared table, which gives symbol and length for either kind (for a
-//                QLC code it is precomputed from the area widths and the rank table). 32
-//                decoded bytes leave as two 16-byte stores (a whole 32-byte sector). Every
-//                sub-stream must end exactly where the next one starts.
+//                two payload words in use and a bit offset into them give the next 32 bits with
+//                one funnel shift, enough for two codes; two more words are already requested
+//                (predicated 4-byte loads, no lane-dependent branch). One lookup per symbol in
+//                the 4096-entry shared table gives symbol and length for either kind (for a QLC
+//                code it is precomputed from the area widths and the rank table). 32 decoded
+//                bytes leave as one 32-byte store (a whole sector). Every sub-stream must end
+//                exactly where the next one starts.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -43,22 +44,8 @@ constexpr uint32_t kMagic = 0x31305848u;  // "HX01"
 constexpr uint32_t kChunk = HX_CHUNK;
 constexpr uint32_t kSubLen = HX_CHUNK / HX_SUBSTREAMS;
 constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
-constexpr int kEncThreads = 256;  // 16 symbols per thread; warp k codes sub-stream k
 constexpr int kDecThreads = 256;  // 8 threads per chunk, 32 chunks per block
 constexpr int kHistThreads = 256;
-constexpr int kStages = 3;        // encode input ring
-constexpr int kLag = 2;           // encode: a chunk is stored kLag iterations after it is coded
-constexpr int kLutCopies = 16;    // encode: table copies; lane l reads copy l % kLutCopies
-constexpr int kOutBufs = kLag + 2;  // encode output buffers
-// 12-bit counters; a copy gains at most 16 per chunk from each lane that reads it
-constexpr uint32_t kHistFlushChunks = 4095 / (16 * (32 / kLutCopies));
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s bound on any wait
-
-// per-chunk flag word: [63:62] state, [61:0] value. The block that codes a chunk publishes its
-// size in words (kFlagSize).
-constexpr unsigned long long kFlagSize = 1ull << 62;
-constexpr unsigned long long kFlagValue = (1ull << 62) - 1;
-constexpr uint32_t kMaxEncodeBlocks = 2 * kEncThreads;  // a wave's sizes: two per thread
 
 __host__ __device__ inline uint64_t n_chunks_of(uint64_t n) { return (n + kChunk - 1) / kChunk; }
 __host__ __device__ inline uint64_t sync_offset(uint64_t n) {
@@ -66,70 +53,6 @@ __host__ __device__ inline uint64_t sync_offset(uint64_t n) {
 }
 __host__ __device__ inline uint64_t payload_offset(uint64_t n) {
   return sync_offset(n) + 16 * n_chunks_of(n);
-}
-
-// ---------------------------------------------------------------------------------- PTX helpers
-__device__ inline unsigned long long ld_relaxed(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ inline void st_relaxed(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ inline unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ inline uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-               : "memory");
-}
-__device__ inline void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bulk copy global -> shared (no multicast), completion counted on `bar`.
-__device__ inline void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ inline void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ inline void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-// Wait for phase `parity` of `bar`; false after kWaitLimitNs.
-__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (global_ns() - t0 > kWaitLimitNs) return false;
-  return true;
 }
 
 // ---------------------------------------------------------------------------------- histogram
@@ -164,33 +87,30 @@ __global__ void __launch_bounds__(kHistThreads) k_histogram(const uint8_t* __res
 }
 
 // ---------------------------------------------------------------------------------- encode
+// Two passes over the input, with no block waiting for another:
+//   k_measure  code lengths only. Every chunk's sub-stream bit counts become its sync row (the
+//              stream's index) and its word count; a measure block owns a contiguous run of
+//              chunks, scans their word counts into block-local offsets (scratch) and records
+//              its total. The fused histogram is counted here.
+//   k_pack     every block scans the measure blocks' totals (a few thousand at most) into their
+//              offsets; then one warp codes one whole chunk, sub-stream by sub-stream, into a
+//              shared-memory buffer and stores it at its final place in the payload.
 struct EncodeArgs {
   const hx::Tables* tables;
   const uint8_t* in;
   uint64_t n;
   uint8_t* out;
   uint64_t cap;
-  unsigned long long* flags;  // scratch: one look-back word per chunk
-  uint32_t* ticket;           // scratch: next chunk to take
-  uint32_t* hist;             // optional fused histogram
+  uint32_t* local;   // scratch: block-local word offset of every chunk
+  uint32_t* btotal;  // scratch: words of each measure block
+  uint32_t mblocks;  // measure blocks
+  uint32_t cpb;      // chunks per measure block
+  uint32_t* hist;    // optional fused histogram
   uint32_t* status;
   uint32_t kind;
 };
 
-struct EncSmem {
-  // [symbol][copy]: (code << 20) | (count << 8) | len. Lane l reads copy l % kLutCopies, so a
-  // warp's lookups meet at most 32 / kLutCopies to a bank; len in the low byte lets 16 entries
-  // be summed into a bit count (16 * 12 < 256); the code comes out with one shift.
-  uint32_t lut[256 * kLutCopies];
-  alignas(128) uint8_t in[kStages][kChunk];
-  uint32_t out[kOutBufs][kMaxChunkWords];
-  alignas(16) uint32_t warp_bits[kOutBufs][kEncThreads / 32];
-  alignas(8) uint32_t wave_red[2][2 * (kEncThreads / 32)];  // per warp (total, prefix), by parity
-  uint64_t bar[kStages];
-  uint32_t stop;  // a bulk copy did not complete in time
-};
-
-// Every header field but total_words (written by the block that finishes the last chunk).
+// Every header field but total_words.
 __device__ inline void write_header(const EncodeArgs& a) {
   uint32_t* h32 = reinterpret_cast<uint32_t*>(a.out);
   uint64_t* h64 = reinterpret_cast<uint64_t*>(a.out);
@@ -208,39 +128,194 @@ __device__ inline void write_header(const EncodeArgs& a) {
   for (uint64_t i = gap; i < sync_offset(a.n); i += 4) h32[i / 4] = 0;
 }
 
-// Size flag of chunk c, waiting (bounded in time) until its block has published it.
-__device__ uint32_t wait_chunk_size(const EncodeArgs& a, uint32_t c, unsigned long long f) {
-  if ((f & ~kFlagValue) == kFlagSize) return (uint32_t)(f & kFlagValue);
-  const unsigned long long t0 = global_ns();
-  while (true) {
-    __nanosleep(32);
-    f = ld_relaxed(a.flags + c);
-    if ((f & ~kFlagValue) == kFlagSize) return (uint32_t)(f & kFlagValue);
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
-      return 0;
-    }
+// The tables' code word of byte value `sym` as (code, len); a damaged entry (a length above the
+// limit or a code longer than its length) reads as no code word and raises HX_ERR_ARG.
+__device__ inline uint32_t checked_code(const EncodeArgs& a, uint32_t sym, uint32_t* code) {
+  const uint32_t t = a.tables->enc[sym];  // (code << 4) | len
+  const uint32_t len = t & 15u, c = t >> 4;
+  if (len > HX_LMAX_MAX || (c >> len) != 0) {
+    atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+    *code = 0;
+    return 0;
   }
+  *code = c;
+  return len;
 }
 
-// The 16 symbols of one thread -> table entries (and the fused histogram); returns the summed
-// entries, whose low byte is the thread's bit count. FULL: all 16 symbols exist.
-template <bool HIST, bool FULL>
-__device__ __forceinline__ uint32_t lookup16(uint32_t* lut_lane, const uint32_t w[4],
-                                             uint32_t valid, uint32_t e[16]) {
-  uint32_t sum = 0;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t sym = (w[j >> 2] >> (8 * (j & 3))) & 0xffu;
-    uint32_t ent = 0;
-    if (FULL || (uint32_t)j < valid) {
-      uint32_t* slot = lut_lane + sym * kLutCopies;
-      ent = HIST ? atomicAdd(slot, 1u << 8) : *slot;
-    }
-    e[j] = ent;
-    sum += ent;
+// The 16 bytes of sub-stream k that lane `lane` codes: a 16-byte load for a whole chunk, byte
+// loads (0 past the end) for the ragged last one. Returns how many of the 16 exist.
+__device__ __forceinline__ uint32_t load16(const EncodeArgs& a, uint32_t c, uint32_t k,
+                                           uint32_t lane, bool whole, uint4& v) {
+  const uint64_t first = (uint64_t)c * kChunk + k * kSubLen + lane * 16;
+  if (whole) {
+    v = __ldg(reinterpret_cast<const uint4*>(a.in + first));
+    return 16;
   }
-  return sum;
+  uint32_t w[4] = {0, 0, 0, 0};
+  const uint32_t valid = first < a.n ? (uint32_t)min((uint64_t)16, a.n - first) : 0u;
+  for (uint32_t j = 0; j < valid; ++j) w[j >> 2] |= (uint32_t)a.in[first + j] << (8 * (j & 3));
+  v = make_uint4(w[0], w[1], w[2], w[3]);
+  return valid;
+}
+
+__device__ __forceinline__ uint32_t byte_of(const uint4& v, int j) {
+  const uint32_t w = j < 4 ? v.x : j < 8 ? v.y : j < 12 ? v.z : v.w;
+  return (w >> (8 * (j & 3))) & 0xffu;
+}
+
+__device__ __forceinline__ uint32_t warp_sum(uint32_t x) {
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) x += __shfl_xor_sync(0xffffffffu, x, d);
+  return x;
+}
+
+// Exclusive scan of cnt[0..m) in place with the whole block (m <= 16 * blockDim.x); returns the
+// sum. `red` holds one word per warp.
+template <int THREADS>
+__device__ uint32_t block_exclusive_scan(uint32_t* cnt, uint32_t m, uint32_t* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t seg = (m + THREADS - 1) / THREADS;
+  const uint32_t lo = min(m, tid * seg), hi = min(m, lo + seg);
+  uint32_t s = 0;
+  for (uint32_t i = lo; i < hi; ++i) s += cnt[i];
+  uint32_t incl = s;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += t;
+  }
+  if (lane == 31) red[warp] = incl;
+  __syncthreads();
+  uint32_t before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < THREADS / 32; ++w) {
+    const uint32_t r = red[w];
+    before += w < warp ? r : 0u;
+    total += r;
+  }
+  uint32_t run = before + incl - s;
+  for (uint32_t i = lo; i < hi; ++i) {
+    const uint32_t v = cnt[i];
+    cnt[i] = run;
+    run += v;
+  }
+  __syncthreads();
+  return total;
+}
+
+constexpr int kMeasureThreads = 256;
+constexpr int kMeasureCopies = 32;            // lane l reads copy l: no bank conflicts
+constexpr uint32_t kMaxChunksPerBlock = 4096;  // chunks of one measure block
+constexpr uint32_t kMaxMeasureBlocks = 2048;
+// 16-bit counters; a round (one chunk per warp) adds at most 8 * 128 to a copy
+constexpr uint32_t kMeasureFlushRounds = 65535 / ((kMeasureThreads / 32) * 128);
+
+struct MeasureSmem {
+  uint32_t lut[256 * kMeasureCopies];  // [symbol][copy]: (count << 16) | len
+  uint32_t cnt[kMaxChunksPerBlock];    // words per chunk, then block-local word offsets
+  uint32_t red[kMeasureThreads / 32];
+};
+
+// One chunk's sync row and word count (lane 0 writes them); WHOLE: all 4096 bytes exist.
+template <bool HIST, bool COMPLETE, bool WHOLE>
+__device__ __forceinline__ uint32_t measure_chunk(const EncodeArgs& a, uint32_t c, uint32_t* lut_lane,
+                                                  uint4* sync, bool& uncodable) {
+  const uint32_t lane = threadIdx.x & 31;
+  uint4 v[HX_SUBSTREAMS];
+  uint32_t valid[HX_SUBSTREAMS];
+#pragma unroll
+  for (int k = 0; k < HX_SUBSTREAMS; ++k) valid[k] = load16(a, c, k, lane, WHOLE, v[k]);
+  uint32_t row[HX_SUBSTREAMS];  // bit offset of each sub-stream in the chunk
+  uint32_t run = 0;
+#pragma unroll
+  for (int k = 0; k < HX_SUBSTREAMS; ++k) {
+    row[k] = run;
+    uint32_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (WHOLE || (uint32_t)j < valid[k]) {
+        uint32_t* slot = lut_lane + byte_of(v[k], j) * kMeasureCopies;
+        const uint32_t e = HIST ? atomicAdd(slot, 1u << 16) : *slot;
+        sum += e & 0xffffu;
+        if (!COMPLETE) uncodable |= (e & 0xffu) == 0;
+      }
+    }
+    run += warp_sum(sum);
+  }
+  if (lane == 0)
+    sync[c] = make_uint4(run | (row[1] << 16), row[2] | (row[3] << 16), row[4] | (row[5] << 16),
+                         row[6] | (row[7] << 16));
+  return run;
+}
+
+template <bool HIST, bool COMPLETE>
+__device__ void measure_chunks(const EncodeArgs& a, MeasureSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
+  const uint32_t full_chunks = (uint32_t)(n / kChunk);
+  const uint32_t c0 = blockIdx.x * a.cpb;
+  const uint32_t m = c0 < nchunks ? min(a.cpb, nchunks - c0) : 0u;
+  uint4* sync = reinterpret_cast<uint4*>(a.out + sync_offset(n));
+  uint32_t* lut_lane = sm.lut + lane;
+  bool uncodable = false;
+
+  auto flush_hist = [&]() {  // counts of the table copies -> global, then clear them
+    __syncthreads();
+    uint32_t sum = 0;
+    for (int l = 0; l < kMeasureCopies; ++l) {
+      const uint32_t e = sm.lut[tid * kMeasureCopies + l];
+      sum += e >> 16;
+      sm.lut[tid * kMeasureCopies + l] = e & 0xffffu;
+    }
+    if (sum) atomicAdd(&a.hist[tid], sum);
+    __syncthreads();
+  };
+
+  // round r: warp w measures the block's chunk 8r + w
+  const uint32_t rounds = (m + 7) / 8;
+  for (uint32_t r = 0; r < rounds; ++r) {
+    const uint32_t i = r * 8 + warp;
+    if (i < m) {
+      const uint32_t c = c0 + i;
+      const uint32_t bits =
+          c < full_chunks ? measure_chunk<HIST, COMPLETE, true>(a, c, lut_lane, sync, uncodable)
+                          : measure_chunk<HIST, COMPLETE, false>(a, c, lut_lane, sync, uncodable);
+      if (lane == 0) sm.cnt[i] = (bits + 31) >> 5;
+    }
+    if (HIST && (r + 1) % kMeasureFlushRounds == 0) flush_hist();
+  }
+  __syncthreads();
+  const uint32_t total = block_exclusive_scan<kMeasureThreads>(sm.cnt, m, sm.red);
+  for (uint32_t i = tid; i < m; i += kMeasureThreads) a.local[c0 + i] = sm.cnt[i];
+  if (tid == 0) a.btotal[blockIdx.x] = total;
+  if (!COMPLETE && uncodable) atomicOr(a.status, (uint32_t)HX_ERR_UNCODABLE);
+  if (HIST) flush_hist();
+}
+
+__global__ void __launch_bounds__(kMeasureThreads, 4) k_measure(EncodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  MeasureSmem& sm = *reinterpret_cast<MeasureSmem*>(smem_raw);
+  const int tid = threadIdx.x;
+  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
+    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+    return;
+  }
+  bool complete = true;
+  for (int i = tid; i < 256 * kMeasureCopies; i += kMeasureThreads) {
+    uint32_t code;
+    const uint32_t len = checked_code(a, i / kMeasureCopies, &code);
+    complete &= len != 0;
+    sm.lut[i] = len;
+  }
+  complete = __syncthreads_and(complete);
+  if (a.hist) {
+    if (complete) measure_chunks<true, true>(a, sm);
+    else measure_chunks<true, false>(a, sm);
+  } else {
+    if (complete) measure_chunks<false, true>(a, sm);
+    else measure_chunks<false, false>(a, sm);
+  }
 }
 
 // Pack 16 (code, len) entries MSB-first starting at bit `off` of buf: two codes are joined in a
@@ -249,7 +324,7 @@ __device__ __forceinline__ uint32_t lookup16(uint32_t* lut_lane, const uint32_t 
 // with neighbours), so the emit is one predicated step with no lane-dependent branch.
 __device__ __forceinline__ void pack16(const uint32_t e[16], uint32_t off, uint32_t* buf) {
   uint32_t widx = off >> 5;
-  uint32_t nacc = off & 31;  // the first bits belong to the previous thread (zeros here)
+  uint32_t nacc = off & 31;  // the first bits belong to the previous lane (zeros here)
   uint32_t hi = 0, lo = 0;
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
@@ -268,195 +343,37 @@ __device__ __forceinline__ void pack16(const uint32_t e[16], uint32_t off, uint3
   if (nacc) atomicOr(&buf[widx], lo << (32 - nacc));
 }
 
-// Encoder block e of E takes chunks e, e + E, e + 2E, ... in order: iteration k codes chunk
-// kE + e, and the chunks kE .. kE + E - 1 form wave k. Stage k % kStages of the input ring
-// holds the chunk of iteration k, loaded by a bulk copy kStages iterations ahead.
-//
-// Word offsets without a serial scan: a chunk is stored kLag iterations after it is coded.
-// Then every block reads the sizes that all blocks published for that wave (two per thread,
-// requested before the symbol work), and one block-wide sum gives both the wave's total and
-// the words of the chunks before its own in the wave. Each block adds the wave totals up as it
-// goes, so the offset of its chunk is that running total plus its in-wave prefix. All blocks
-// are resident (cooperative launch), so every size a block waits for is being computed.
-template <bool HIST, bool COMPLETE>
-__device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint64_t n = a.n;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  const uint32_t full_chunks = (uint32_t)(n / kChunk);
-  const uint32_t E = gridDim.x, eb = blockIdx.x;
-  const uint64_t P = payload_offset(n);
-  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
-  uint4* sync = reinterpret_cast<uint4*>(a.out + sync_offset(n));
-  uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
-  uint32_t* lut_lane = sm.lut + lane % kLutCopies;
-  auto chunk_of = [&](uint32_t k) -> uint32_t { return k * E + eb; };
+constexpr int kPackThreads = 256;
+constexpr int kPackCopies = 16;  // lane l reads copy l % 16: at most two lookups to a bank
 
-  // stage k % kStages <- chunk of iteration k (bulk copy for a full chunk; else a plain arrive)
-  auto issue = [&](uint32_t k) {
-    const uint32_t c = chunk_of(k);
-    uint64_t* bar = &sm.bar[k % kStages];
-    if (c < full_chunks) {
-      mbar_arrive_expect_tx(bar, kChunk);
-      bulk_load(sm.in[k % kStages], a.in + (uint64_t)c * kChunk, kChunk, bar);
-    } else {
-      mbar_arrive(bar);
-    }
-  };
-  // only thread 0 waits on a stage; the block barrier after it hands the stage to every thread
-  auto await_stage = [&](uint32_t k) {
-    if (chunk_of(k) < nchunks && !mbar_wait(&sm.bar[k % kStages], (k / kStages) & 1u)) {
-      sm.stop = 1;
-      atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
-    }
-  };
-  // size flags of wave w that this thread sums: its chunks tid and tid + kEncThreads
-  auto load_wave = [&](uint32_t w, unsigned long long f[2]) {
+struct PackSmem {
+  // [symbol][copy]: (code << 20) | len; the low byte of 16 summed entries is their bit count
+  uint32_t lut[256 * kPackCopies];
+  uint32_t out[kPackThreads / 32][kMaxChunkWords];  // one chunk per warp
+  uint32_t bpre[kMaxMeasureBlocks];                  // word offset of each measure block
+  uint32_t red[kPackThreads / 32];
+  uint32_t total;
+};
+
+// Codes chunk c into buf (zeroed, the warp's own); returns its bit count. WHOLE: all 4096
+// bytes exist.
+template <bool WHOLE>
+__device__ __forceinline__ uint32_t pack_chunk(const EncodeArgs& a, uint32_t c,
+                                               const uint32_t* lut_lane, uint32_t* buf) {
+  const uint32_t lane = threadIdx.x & 31;
+  uint4 v[HX_SUBSTREAMS];
+  uint32_t valid[HX_SUBSTREAMS];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t j = (uint32_t)tid + i * kEncThreads;
-      const uint64_t c = (uint64_t)w * E + j;
-      f[i] = (j < E && c < nchunks) ? ld_relaxed(a.flags + c) : kFlagSize;
-    }
-  };
-  // this thread's part of the wave total and of the block's in-wave prefix, reduced per warp
-  auto reduce_wave = [&](uint32_t w, unsigned long long f[2], uint32_t parity) {
-    uint32_t tot = 0, pre = 0;
+  for (int k = 0; k < HX_SUBSTREAMS; ++k) valid[k] = load16(a, c, k, lane, WHOLE, v[k]);
+  uint32_t base = 0;  // bits of the chunk before sub-stream k
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t j = (uint32_t)tid + i * kEncThreads;
-      const uint32_t v = wait_chunk_size(a, w * E + j, f[i]);
-      tot += v;
-      pre += j < eb ? v : 0u;
-    }
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) {
-      tot += __shfl_xor_sync(0xffffffffu, tot, d);
-      pre += __shfl_xor_sync(0xffffffffu, pre, d);
-    }
-    if (lane == 0) {
-      sm.wave_red[parity][2 * warp] = tot;
-      sm.wave_red[parity][2 * warp + 1] = pre;
-    }
-  };
-  if (tid == 0) {
-    sm.stop = 0;
-    for (uint32_t k = 0; k < (uint32_t)kStages; ++k) issue(k);
-    await_stage(0);
-    if (nchunks == 0 && eb == 0) {  // an empty stream: header, index and guards only
-      write_header(a);
-      reinterpret_cast<uint64_t*>(a.out)[4] = 0;
-      word_off[0] = 0;
-      payload[0] = 0;  // the host checked cap >= P + 8
-      payload[1] = 0;
-    }
-  }
-  __syncthreads();
-
-  bool uncodable = false;
-  uint32_t since_flush = 0;
-  uint64_t running = 0;  // words of all waves before the one being stored
-
-  // Stores of the chunk of iteration k (output buffer k % kOutBufs); its wave's sums are in
-  // wave_red[parity]. Every thread computes the same offset.
-  auto store_chunk = [&](uint32_t k, uint32_t parity) {
-    // lanes 0..7 fetch one warp's (total, prefix) pair each; a shuffle sum spreads the result
-    uint2 wr = lane < kEncThreads / 32
-                   ? *reinterpret_cast<const uint2*>(&sm.wave_red[parity][2 * lane])
-                   : make_uint2(0u, 0u);
-#pragma unroll
-    for (int d = 4; d > 0; d >>= 1) {
-      wr.x += __shfl_xor_sync(0xffffffffu, wr.x, d);
-      wr.y += __shfl_xor_sync(0xffffffffu, wr.y, d);
-    }
-    const uint32_t wave_total = __shfl_sync(0xffffffffu, wr.x, 0);
-    const uint32_t before = __shfl_sync(0xffffffffu, wr.y, 0);
-    const uint64_t woff = running + before;
-    running += wave_total;
-    const int b = (int)(k % kOutBufs);
-    const uint32_t c = chunk_of(k);
-    const uint4 t0 = *reinterpret_cast<const uint4*>(&sm.warp_bits[b][0]);
-    const uint4 t1 = *reinterpret_cast<const uint4*>(&sm.warp_bits[b][4]);
-    const uint32_t total = t0.x + t0.y + t0.z + t0.w + t1.x + t1.y + t1.z + t1.w;
-    const uint32_t words = (total + 31) >> 5;
-    const bool fits = P + 4ull * (woff + words + 2) <= a.cap;
-    uint32_t* buf = sm.out[b];
-    for (uint32_t i = tid; i < words; i += kEncThreads) {
-      if (fits) payload[woff + i] = buf[i];
-      buf[i] = 0;
-    }
-    if (tid == 0) {
-      const uint32_t p1 = t0.x, p2 = p1 + t0.y, p3 = p2 + t0.z, p4 = p3 + t0.w;
-      const uint32_t p5 = p4 + t1.x, p6 = p5 + t1.y, p7 = p6 + t1.z;
-      sync[c] = make_uint4(total | (p1 << 16), p2 | (p3 << 16), p4 | (p5 << 16), p6 | (p7 << 16));
-      word_off[c] = (uint32_t)woff;
-      if (!fits) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
-      if (c == 0) write_header(a);
-      if (c == nchunks - 1) {  // the last chunk closes the index
-        const uint64_t end = woff + words;
-        word_off[nchunks] = (uint32_t)end;
-        reinterpret_cast<uint64_t*>(a.out)[4] = end;
-        if (fits) {
-          payload[end] = 0;
-          payload[end + 1] = 0;
-        }
-      }
-    }
-  };
-
-  auto flush_hist = [&]() {  // counts in the lane tables -> global, then clear them
-    __syncthreads();
-    uint32_t sum = 0;
-    for (int l = 0; l < kLutCopies; ++l) {
-      const uint32_t e = sm.lut[tid * kLutCopies + l];
-      sum += (e >> 8) & 0xfffu;
-      sm.lut[tid * kLutCopies + l] = e & ~(0xfffu << 8);
-    }
-    if (sum) atomicAdd(&a.hist[tid], sum);
-    __syncthreads();
-  };
-
-  uint32_t k = 0;
-  for (;; ++k) {
-    const uint32_t c = chunk_of(k);
-    if (c >= nchunks || sm.stop) break;  // uniform: sm.stop is set before a block barrier
-    const int s = (int)(k % kStages);
-    const int ob = (int)(k % kOutBufs);
-    const bool lagged = k >= kLag;
-    unsigned long long wf[2];
-    if (lagged) load_wave(k - kLag, wf);  // answers are needed only after the symbol work
-
-    uint32_t w[4];
+  for (int k = 0; k < HX_SUBSTREAMS; ++k) {
     uint32_t e[16];
-    uint32_t sum;
-    if (c < full_chunks) {
-      const uint4 v = reinterpret_cast<const uint4*>(sm.in[s])[tid];
-      w[0] = v.x;
-      w[1] = v.y;
-      w[2] = v.z;
-      w[3] = v.w;
-      sum = lookup16<HIST, true>(lut_lane, w, 16, e);
-      if (!COMPLETE)
+    uint32_t sum = 0;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) uncodable |= (e[j] & 0xffu) == 0;
-    } else {  // the ragged last chunk, from global memory
-      const uint64_t base = (uint64_t)c * kChunk;
-      const uint32_t first = (uint32_t)tid * 16;
-      const uint32_t count = (uint32_t)(n - base);
-      const uint32_t valid = count > first ? min(16u, count - first) : 0u;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t x = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          if ((uint32_t)(4 * q + b) < valid)
-            x |= (uint32_t)a.in[base + first + 4 * q + b] << (8 * b);
-        w[q] = x;
-      }
-      sum = lookup16<HIST, false>(lut_lane, w, valid, e);
-      if (!COMPLETE)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) uncodable |= (uint32_t)j < valid && (e[j] & 0xffu) == 0;
+    for (int j = 0; j < 16; ++j) {
+      e[j] = (WHOLE || (uint32_t)j < valid[k]) ? lut_lane[byte_of(v[k], j) * kPackCopies] : 0u;
+      sum += e[j];
     }
     const uint32_t bits = sum & 0xffu;
     uint32_t incl = bits;
@@ -465,88 +382,64 @@ __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
       const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
       if (lane >= d) incl += t;
     }
-    if (lane == 31) sm.warp_bits[ob][warp] = incl;
-    if (lagged) reduce_wave(k - kLag, wf, k & 1);
-    if (tid == 0) await_stage(k + 1);
-    __syncthreads();  // warp totals and wave sums ready; stage s read; next stage handed over
-
-    // lanes 0..7 hold the warp totals; a shuffle scan gives this warp's base and the total
-    uint32_t wt = lane < kEncThreads / 32 ? sm.warp_bits[ob][lane] : 0u;
-#pragma unroll
-    for (int d = 1; d < kEncThreads / 32; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, wt, d);
-      if (lane >= d) wt += t;
-    }
-    const uint32_t warp_base = __shfl_sync(0xffffffffu, wt, (warp + 31) & 31) & (warp ? ~0u : 0u);
-    const uint32_t total = __shfl_sync(0xffffffffu, wt, kEncThreads / 32 - 1);
-    if (tid == 0) {
-      st_relaxed(a.flags + c, kFlagSize | ((total + 31) >> 5));
-      fence_proxy_async();  // this stage's generic reads before the async refill
-      issue(k + kStages);
-    }
-    if (bits) pack16(e, warp_base + incl - bits, sm.out[ob]);
-    if (lagged) store_chunk(k - kLag, k & 1);
-    if (HIST && ++since_flush == kHistFlushChunks) {
-      flush_hist();
-      since_flush = 0;
-    }
+    if (bits) pack16(e, base + incl - bits, buf);
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  if (tid == 0 && sm.stop)  // timed out: let copies still in flight land
-    for (uint32_t j = 0; j < (uint32_t)kStages; ++j)
-      if (chunk_of(k + j) < full_chunks)
-        mbar_wait(&sm.bar[(k + j) % kStages], ((k + j) / kStages) & 1u);
-  // drain: the last kLag coded chunks
-  for (uint32_t j = k > kLag ? k - kLag : 0; j < k; ++j) {
-    unsigned long long wf[2];
-    load_wave(j, wf);
-    __syncthreads();
-    reduce_wave(j, wf, 0);
-    __syncthreads();
-    store_chunk(j, 0);
-  }
-  if (!COMPLETE && uncodable) atomicOr(a.status, (uint32_t)HX_ERR_UNCODABLE);
-  if (HIST) flush_hist();
+  return base;
 }
 
-__global__ void __launch_bounds__(kEncThreads, 3) k_encode(EncodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  EncSmem& sm = *reinterpret_cast<EncSmem*>(smem_raw);
-  const int tid = threadIdx.x;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(a.n);
-  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
-    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
-    return;
-  }
-  bool complete = true;
-  for (int i = tid; i < 256 * kLutCopies; i += kEncThreads) {
-    const uint32_t t = a.tables->enc[i / kLutCopies];  // (code << 4) | len
-    uint32_t e = ((t >> 4) << 20) | (t & 15u);
-    if ((t & 15u) > HX_LMAX_MAX || t > 0xffffu) {  // a damaged table block stays harmless
-      e = 0;
-      atomicOr(a.status, (uint32_t)HX_ERR_ARG);
-    }
-    complete &= (e & 0xffu) != 0;
-    sm.lut[i] = e;
-  }
-  for (int i = tid; i < kOutBufs * (int)kMaxChunkWords; i += kEncThreads) (&sm.out[0][0])[i] = 0;
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
-    fence_barrier_init();
-  }
-  complete = __syncthreads_and(complete);
-  if (a.hist) {
-    if (complete) encode_chunks<true, true>(a, sm);
-    else encode_chunks<true, false>(a, sm);
-  } else {
-    if (complete) encode_chunks<false, true>(a, sm);
-    else encode_chunks<false, false>(a, sm);
-  }
-}
+__global__ void __launch_bounds__(kPackThreads, 3) k_pack(EncodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  PackSmem& sm = *reinterpret_cast<PackSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) return;  // k_measure said so
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
+  const uint32_t full_chunks = (uint32_t)(n / kChunk);
+  const uint64_t P = payload_offset(n);
+  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
+  uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
 
-__global__ void k_zero_scratch(unsigned long long* flags, uint32_t nchunks, uint32_t* ticket) {
-  const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < nchunks) flags[i] = 0;
-  if (i == 0) *ticket = 0;
+  for (int i = tid; i < 256 * kPackCopies; i += kPackThreads) {
+    uint32_t code;
+    const uint32_t len = checked_code(a, i / kPackCopies, &code);
+    sm.lut[i] = (code << 20) | len;
+  }
+  for (int i = tid; i < (kPackThreads / 32) * (int)kMaxChunkWords; i += kPackThreads)
+    (&sm.out[0][0])[i] = 0;
+  for (uint32_t i = tid; i < a.mblocks; i += kPackThreads) sm.bpre[i] = a.btotal[i];
+  __syncthreads();
+  const uint32_t total = block_exclusive_scan<kPackThreads>(sm.bpre, a.mblocks, sm.red);
+  const bool fits = P + 4ull * ((uint64_t)total + 2) <= a.cap;
+  if (blockIdx.x == 0 && tid == 0) {
+    write_header(a);
+    reinterpret_cast<uint64_t*>(a.out)[4] = total;
+    word_off[nchunks] = total;
+    if (fits) {
+      payload[total] = 0;
+      payload[total + 1] = 0;
+    } else {
+      atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
+    }
+  }
+
+  const uint32_t* lut_lane = sm.lut + lane % kPackCopies;
+  uint32_t* buf = sm.out[warp];
+  const uint32_t stride = gridDim.x * (kPackThreads / 32);
+  for (uint32_t c = blockIdx.x * (kPackThreads / 32) + warp; c < nchunks; c += stride) {
+    const uint32_t woff = sm.bpre[c / a.cpb] + a.local[c];
+    if (lane == 0) word_off[c] = woff;
+    const uint32_t base = c < full_chunks ? pack_chunk<true>(a, c, lut_lane, buf)
+                                          : pack_chunk<false>(a, c, lut_lane, buf);
+    __syncwarp();
+    const uint32_t words = (base + 31) >> 5;
+    for (uint32_t i = lane; i < words; i += 32) {
+      // woff + words <= total unless the input changed since k_measure read it
+      if (fits && woff + i < total) payload[woff + i] = buf[i];
+      buf[i] = 0;
+    }
+    __syncwarp();
+  }
 }
 
 // ---------------------------------------------------------------------------------- decode
@@ -579,102 +472,139 @@ __device__ int64_t check_header(const DecodeArgs& a) {
   return (int64_t)total;
 }
 
-// Payload words of one sub-stream, MSB-first, through a 64-bit bit window held as two 32-bit
-// halves (wh:wl) whose top `avail` bits are valid. The next kPrefetch words are already
-// requested (pf[]): a refill takes pf[0] and requests one more word -- one predicated load and
-// register moves, no branch that depends on the other lanes. Words past the caller's buffer
-// read as 0.
-constexpr int kPrefetch = 2;
-struct SubstreamReader {
+// A sub-stream's payload words, MSB-first. The two words in use (w0:w1) and an offset bo < 32
+// into w0 give the next 32 bits with one funnel shift -- enough for two codes of <= 12 bits, so
+// every second symbol costs no extraction. Two further words are already requested (pf0, pf1);
+// once bo passes 32 the words move up and one more is requested: one predicated 4-byte load
+// per payload word. The word index is 32-bit, so an address is one multiply-add off the payload
+// base. CHECKED readers treat words past the caller's buffer as 0; the others never reach them
+// (checked once per sub-stream).
+template <bool CHECKED>
+struct SubstreamBits {
   const uint32_t* words;
-  uint64_t wlimit;  // payload words inside the buffer
-  uint64_t wi;      // index of the word in pf[0]
-  uint32_t pf[kPrefetch];
-  uint32_t wh, wl;
-  int avail;
+  uint32_t wlimit;  // payload words inside the buffer (used when CHECKED)
+  uint32_t wi;      // index of the next word to request
+  uint32_t w0, w1, pf0, pf1;
+  uint32_t bo;
 
-  __device__ __forceinline__ uint32_t word(uint64_t i) const {
-    return i < wlimit ? __ldg(words + i) : 0u;
+  // a miss brings 256 bytes into L2: the rest of this sub-stream's line and the next one
+  __device__ __forceinline__ static uint32_t load(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L2::256B.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
   }
-  // afterwards >= 32 valid bits: room for two codes of <= 12 bits
-  __device__ __forceinline__ void refill() {
-    if (avail < 32) {
-      const uint32_t w = pf[0];
-#pragma unroll
-      for (int i = 0; i + 1 < kPrefetch; ++i) pf[i] = pf[i + 1];
-      pf[kPrefetch - 1] = word(wi + kPrefetch);
-      ++wi;
-      wh |= w >> avail;                            // the word lands at bits [32-avail, 64-avail)
-      wl |= __funnelshift_lc(0u, w, 32 - avail);  // its low part (nothing when avail == 0)
-      avail += 32;
+  __device__ __forceinline__ uint32_t word(uint32_t i) const {
+    if (CHECKED) return i < wlimit ? load(words + i) : 0u;
+    return load(words + i);
+  }
+  __device__ __forceinline__ void start(uint32_t fw, uint32_t first_bo) {
+    w0 = word(fw);
+    w1 = word(fw + 1);
+    pf0 = word(fw + 2);
+    pf1 = word(fw + 3);
+    wi = fw + 4;
+    bo = first_bo;
+  }
+  __device__ __forceinline__ uint32_t peek() const { return __funnelshift_l(w1, w0, bo); }
+  // after at most 24 more bits: bo < 56, so one word restores bo < 32
+  __device__ __forceinline__ void advance(uint32_t nbits) {
+    bo += nbits;
+    if (bo >= 32) {
+      bo -= 32;
+      w0 = w1;
+      w1 = pf0;
+      pf0 = pf1;
+      pf1 = word(wi++);
     }
   }
-  __device__ __forceinline__ void consume(uint32_t len) {  // len <= 15
-    wh = __funnelshift_l(wl, wh, len);
-    wl <<= len;
-    avail -= (int)len;
-  }
-  __device__ void start(uint64_t first_bit) {
-    const uint64_t fw = first_bit >> 5;
-    const uint32_t sh = (uint32_t)(first_bit & 31);
-    wh = word(fw);
-    wl = word(fw + 1);
-    wi = fw + 2;
-#pragma unroll
-    for (int i = 0; i < kPrefetch; ++i) pf[i] = word(wi + i);
-    wh = __funnelshift_l(wl, wh, sh);
-    wl <<= sh;
-    avail = 64 - (int)sh;
-  }
   // index (in payload bits) of the next bit not yet consumed
-  __device__ uint64_t position() const { return 32 * wi - (uint64_t)avail; }
+  __device__ __forceinline__ uint64_t position() const { return 32ull * (wi - 4) + bo; }
+};
+// Words a reader may request for one sub-stream: 4 at the start, then one per 32 bits of at
+// most kSubLen codes of at most 15 bits (the table's length field).
+constexpr uint32_t kReaderReach = 4 + (kSubLen * 15 + 31) / 32;
+
+// The decode table in shared memory: for every 12-bit window, (symbol << 8) | length of the code
+// word it starts with; 0 when none does (an incomplete code).
+struct DecLut {
+  const uint16_t* full;
+  __device__ __forceinline__ uint32_t operator()(uint32_t x) const { return full[x >> 20]; }
 };
 
-// One symbol from the top of the window: the 4096-entry table gives (symbol << 8) | length for
-// both kinds. For a QLC table the length is 3 + the width of the area in the top 3 bits; the
-// table holds it already, so reading it there costs less than recomputing it. An entry of 0
-// (no code word starts the window) only occurs for an incomplete code.
-template <bool COMPLETE>
-__device__ __forceinline__ uint32_t next_symbol(SubstreamReader& rd, bool& invalid,
-                                                const uint16_t* lut) {
-  const uint32_t e = lut[rd.wh >> 20];
-  const uint32_t len = e & 15u;
-  if (!COMPLETE) invalid |= len == 0;
-  rd.consume(len);
-  return e;
+// Two symbols from the reader: table entries (symbol << 8) | length for either kind (for a QLC
+// table the length is 3 + the width of the area in the top 3 bits; the table holds it already).
+// An entry of 0 (no code word starts the window) only occurs for an incomplete code.
+template <bool COMPLETE, bool CHECKED>
+__device__ __forceinline__ void decode_pair(SubstreamBits<CHECKED>& rd, bool& invalid,
+                                            const DecLut& lut, uint32_t& e1, uint32_t& e2) {
+  const uint32_t x = rd.peek();
+  e1 = lut(x);
+  const uint32_t l1 = e1 & 15u;
+  e2 = lut(x << l1);
+  const uint32_t l2 = e2 & 15u;
+  if (!COMPLETE) invalid |= l1 == 0 || l2 == 0;
+  rd.advance(l1 + l2);
 }
 
-// 32 symbols -> 32 output bytes (two 16-byte streaming stores, one whole sector). Each symbol's
-// byte is moved into place with one byte permute.
-template <bool COMPLETE>
-__device__ __forceinline__ void decode_group32(SubstreamReader& rd, bool& invalid, uint4* d4,
-                                               const uint16_t* lut) {
+// 32 symbols -> 32 output bytes, one 32-byte streaming store (a whole sector) when the output is
+// 32-byte aligned, else two 16-byte stores. The symbol bytes are gathered with byte permutes.
+template <bool COMPLETE, bool CHECKED>
+__device__ __forceinline__ void decode_group32(SubstreamBits<CHECKED>& rd, bool& invalid,
+                                               uint8_t* dst, bool out32, const DecLut& lut) {
   uint32_t o[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    rd.refill();
-    uint32_t v = next_symbol<COMPLETE>(rd, invalid, lut) >> 8;
-    v = __byte_perm(v, next_symbol<COMPLETE>(rd, invalid, lut), 0x3250);
-    rd.refill();
-    v = __byte_perm(v, next_symbol<COMPLETE>(rd, invalid, lut), 0x3510);
-    v = __byte_perm(v, next_symbol<COMPLETE>(rd, invalid, lut), 0x5210);
-    o[q] = v;
+    uint32_t e1, e2, e3, e4;
+    decode_pair<COMPLETE>(rd, invalid, lut, e1, e2);
+    decode_pair<COMPLETE>(rd, invalid, lut, e3, e4);
+    o[q] = __byte_perm(__byte_perm(e1, e2, 0x0051), __byte_perm(e3, e4, 0x0051), 0x5410);
   }
-  __stcs(d4, make_uint4(o[0], o[1], o[2], o[3]));
-  __stcs(d4 + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  if (out32) {
+    asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(o[0]),
+                 "r"(o[1]), "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                 : "memory");
+  } else {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    __stcs(d4, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcs(d4 + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
+// Decodes `mine` symbols of one sub-stream to dst; returns the reader's final bit position.
+template <bool COMPLETE, bool CHECKED>
+__device__ __forceinline__ uint64_t decode_substream(const uint32_t* words, uint32_t wlimit,
+                                                     uint64_t first_bit, uint32_t mine,
+                                                     uint8_t* dst, bool out32, bool& invalid,
+                                                     const DecLut& lut) {
+  SubstreamBits<CHECKED> rd;
+  rd.words = words;
+  rd.wlimit = wlimit;
+  rd.start((uint32_t)(first_bit >> 5), (uint32_t)(first_bit & 31));
+  const uint32_t groups = mine / 32;
+  for (uint32_t g = 0; g < groups; ++g)
+    decode_group32<COMPLETE>(rd, invalid, dst + 32 * g, out32, lut);
+  for (uint32_t i = groups * 32; i < mine; ++i) {
+    const uint32_t e = lut(rd.peek());
+    if (!COMPLETE) invalid |= (e & 15u) == 0;
+    rd.advance(e & 15u);
+    dst[i] = (uint8_t)(e >> 8);
+  }
+  return rd.position();
 }
 
 template <bool COMPLETE>
-__device__ void decode_chunks(const DecodeArgs& a, const uint16_t* lut, uint32_t total) {
+__device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut& lut,
+                                              uint32_t total) {
   const int tid = threadIdx.x;
   const uint64_t n = a.n;
   const uint64_t nchunks = n_chunks_of(n);
   const uint64_t P = payload_offset(n);
   const uint32_t* word_off = reinterpret_cast<const uint32_t*>(a.st + 64);
   const uint4* sync = reinterpret_cast<const uint4*>(a.st + sync_offset(n));
-  SubstreamReader rd;
-  rd.words = reinterpret_cast<const uint32_t*>(a.st + P);
-  rd.wlimit = (a.bytes - P) / 4;  // payload words inside the buffer
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(a.st + P);
+  // payload words inside the buffer, capped at 2^32 - 1 (no payload word lies beyond 2^32 - 2)
+  const uint32_t wlimit = (uint32_t)min((a.bytes - P) / 4, (uint64_t)0xffffffffull);
+  const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;
   const int k = tid & 7;
 
   for (uint64_t c = (uint64_t)blockIdx.x * (kDecThreads / 8) + (tid >> 3); c < nchunks;
@@ -695,19 +625,18 @@ __device__ void decode_chunks(const DecodeArgs& a, const uint16_t* lut, uint32_t
     } else if (!bad) {
       const uint32_t start = k == 0 ? 0u : sync_at(k);
       const uint32_t end = (uint32_t)k + 1 < nsub ? sync_at(k + 1) : nbits;
-      const uint64_t first_bit = 32ull * w0 + start;
-      rd.start(first_bit);
+      const uint64_t first_bit = 32ull * w0 + start;  // w0 <= total < 2^32
       bool invalid = false;
       uint8_t* dst = a.out + c * kChunk + (uint64_t)k * kSubLen;
-      const uint32_t groups = mine / 32;
-      for (uint32_t g = 0; g < groups; ++g)
-        decode_group32<COMPLETE>(rd, invalid, reinterpret_cast<uint4*>(dst + 32 * g), lut);
-      for (uint32_t i = groups * 32; i < mine; ++i) {
-        rd.refill();
-        dst[i] = (uint8_t)(next_symbol<COMPLETE>(rd, invalid, lut) >> 8);
-      }
+      uint64_t pos;
+      if ((first_bit >> 5) + kReaderReach <= wlimit)
+        pos = decode_substream<COMPLETE, false>(words, wlimit, first_bit, mine, dst, out32,
+                                                invalid, lut);
+      else
+        pos = decode_substream<COMPLETE, true>(words, wlimit, first_bit, mine, dst, out32,
+                                               invalid, lut);
       // the sub-stream must end exactly where the next one starts
-      bad |= invalid || rd.position() != 32ull * w0 + end;
+      bad |= invalid || pos != 32ull * w0 + end;
     }
     if (bad) atomicOr(a.status, (uint32_t)HX_ERR_CORRUPT);
   }
@@ -729,17 +658,41 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_decode(DecodeArgs a) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)(-total));
     return;
   }
+  const DecLut lut{s_lut};
   if (a.tables->complete)
-    decode_chunks<true>(a, s_lut, (uint32_t)total);
+    decode_chunks<true>(a, lut, (uint32_t)total);
   else
-    decode_chunks<false>(a, s_lut, (uint32_t)total);
+    decode_chunks<false>(a, lut, (uint32_t)total);
 }
 
 // ---------------------------------------------------------------------------------- launch
 struct DeviceInfo {
   int sms = 0;
-  int enc_per_sm = 0, huff_per_sm = 0, qlc_per_sm = 0, hist_per_sm = 0;
+  int measure_per_sm = 0, pack_per_sm = 0, huff_per_sm = 0, qlc_per_sm = 0, hist_per_sm = 0;
 };
+
+// Sets the shared-memory carveout of `fn` to the smallest share that still holds `per_sm` blocks,
+// the rest going to L1; keeps the default if that would lower the occupancy.
+bool prefer_l1(int dev, const void* fn, int per_sm, int threads) {
+  cudaFuncAttributes fa;
+  int max_smem = 0;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
+      cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      max_smem <= 0)
+    return false;
+  const long need = (long)per_sm * (long)(fa.sharedSizeBytes + 1024);  // + the per-block reserve
+  const int pct = (int)std::min<long>(100, (need * 100 + max_smem - 1) / max_smem + 1);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, pct) != cudaSuccess)
+    return false;
+  int now = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&now, fn, threads, 0) != cudaSuccess)
+    return false;
+  if (now < per_sm)
+    return cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutDefault) == cudaSuccess;
+  return true;
+}
 
 std::mutex g_info_mutex;
 DeviceInfo g_info[64];
@@ -753,11 +706,16 @@ bool device_info(DeviceInfo* out) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return false;
-    if (cudaFuncSetAttribute(k_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(EncSmem)) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_measure, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(MeasureSmem)) != cudaSuccess ||
+        cudaFuncSetAttribute(k_pack, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(PackSmem)) != cudaSuccess)
       return false;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.enc_per_sm, k_encode, kEncThreads,
-                                                      sizeof(EncSmem)) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.measure_per_sm, k_measure,
+                                                      kMeasureThreads,
+                                                      sizeof(MeasureSmem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.pack_per_sm, k_pack, kPackThreads,
+                                                      sizeof(PackSmem)) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.huff_per_sm, k_decode<HX_KIND_HUFFMAN>,
                                                       kDecThreads, 0) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qlc_per_sm, k_decode<HX_KIND_QLC>,
@@ -765,7 +723,15 @@ bool device_info(DeviceInfo* out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
                                                       0) != cudaSuccess)
       return false;
-    if (d.enc_per_sm < 1 || d.huff_per_sm < 1 || d.qlc_per_sm < 1 || d.hist_per_sm < 1)
+    if (d.measure_per_sm < 1 || d.pack_per_sm < 1 || d.huff_per_sm < 1 || d.qlc_per_sm < 1 ||
+        d.hist_per_sm < 1)
+      return false;
+    // The decoder's payload reads hit L1 about half the time: give L1 all the on-chip memory
+    // that the resident decode blocks do not need for their tables.
+    if (!prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_HUFFMAN>), d.huff_per_sm,
+                   kDecThreads) ||
+        !prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_QLC>), d.qlc_per_sm,
+                   kDecThreads))
       return false;
     d.sms = sms;
   }
@@ -788,20 +754,26 @@ int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint
   if (!device_info(&info)) return HX_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  auto* flags = static_cast<unsigned long long*>(d_scratch);
-  auto* ticket = reinterpret_cast<uint32_t*>(flags + nchunks);
-  k_zero_scratch<<<(nchunks + 255) / 256 + (nchunks == 0), 256, 0, s>>>(flags, nchunks, ticket);
+  // measure blocks: at least one wave of resident blocks, at most kMaxChunksPerBlock chunks each
+  // (n < 2^32 gives at most 2^20 chunks, so 256 blocks always suffice)
+  uint32_t mblocks = (uint32_t)std::min<uint64_t>(
+      {(uint64_t)nchunks, (uint64_t)kMaxMeasureBlocks,
+       std::max<uint64_t>((uint64_t)info.sms * info.measure_per_sm,
+                          (nchunks + kMaxChunksPerBlock - 1) / kMaxChunksPerBlock)});
+  const uint32_t cpb = mblocks ? (nchunks + mblocks - 1) / mblocks : 1;
+  if (mblocks) mblocks = (nchunks + cpb - 1) / cpb;  // no block without chunks
+  // scratch: u32 local[nchunks], then u32 btotal[mblocks] (mblocks <= nchunks)
+  auto* local = static_cast<uint32_t*>(d_scratch);
   EncodeArgs a{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
-               out_cap, flags, ticket, d_hist, d_status, kind};
-  // blocks take chunks round-robin and wait for each other's sizes: all must be resident at
-  // once (cooperative launch), and a wave's sizes are summed two per thread
+               out_cap, local, local + nchunks, mblocks, cpb, d_hist, d_status, kind};
+  if (mblocks) {
+    k_measure<<<mblocks, kMeasureThreads, sizeof(MeasureSmem), s>>>(a);
+    if (cudaPeekAtLastError() != cudaSuccess) return launched();
+  }
   const uint32_t grid = (uint32_t)std::max<uint64_t>(
-      1, std::min<uint64_t>({(uint64_t)nchunks, (uint64_t)info.sms * info.enc_per_sm,
-                             (uint64_t)kMaxEncodeBlocks}));
-  void* params[] = {&a};
-  if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(k_encode), dim3(grid),
-                                  dim3(kEncThreads), params, sizeof(EncSmem), s) != cudaSuccess)
-    return launched() | HX_ERR_CUDA;
+      1, std::min<uint64_t>((nchunks + kPackThreads / 32 - 1) / (kPackThreads / 32),
+                            (uint64_t)info.sms * info.pack_per_sm));
+  k_pack<<<grid, kPackThreads, sizeof(PackSmem), s>>>(a);
   return launched();
 }
 
@@ -831,9 +803,10 @@ int decode_common(uint32_t kind, const void* d_tables, const void* d_stream, uin
 
 }  // namespace
 
-// Scratch of hx_encode_noalloc: one flag word per chunk plus the ticket, for up to
-// HX_NOALLOC_MAX_BYTES of input. Host code must not pass this name to a kernel (on the host it is
-// only a stand-in); its device address comes from cudaGetSymbolAddress, once per device.
+// Scratch of hx_encode_noalloc: hx_scratch_bytes(HX_NOALLOC_MAX_BYTES) bytes (a block-local word
+// offset per chunk and the measure blocks' totals). Host code must not pass this name to a kernel
+// (on the host it is only a stand-in); its device address comes from cudaGetSymbolAddress, once
+// per device.
 static __device__ __align__(256) unsigned char
     g_noalloc_scratch[8 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16];
 
@@ -849,8 +822,8 @@ uint64_t hx_scratch_bytes(uint64_t n) { return 8 * n_chunks_of(n) + 16; }
 // For callers that cannot allocate device memory at encode time (a framework's caching
 // allocator owns the device memory, or a path that cannot take cudaMalloc's implicit
 // synchronisation): hx_encode with Huffman tables, its scratch in g_noalloc_scratch. The first
-// call on a device fetches that array's address with the device current; every call zeroes the
-// part it uses (k_zero_scratch) and calls that overlap on the GPU race on the shared array.
+// call on a device fetches that array's address with the device current; every call writes each
+// scratch word before reading it, and calls that overlap on the GPU race on the shared array.
 int hx_encode_noalloc(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
                       uint64_t out_cap, uint32_t* d_hist, uint32_t* d_status, void* stream) {
   if (n > HX_NOALLOC_MAX_BYTES) return HX_ERR_ARG;
