@@ -15,11 +15,13 @@
 //                atomic that returns the length adds to a per-copy count).
 //
 //   k_pack       every block scans the measure blocks' totals into offsets, so no block waits
-//                for another. A warp codes a whole chunk, one sub-stream (512 symbols, 16 per
-//                lane) at a time: table lookup, warp prefix sum of the lane bit counts, two codes
-//                joined per 32-bit register and appended to a 64-bit accumulator, finished words
-//                OR-ed into the warp's shared buffer; then the chunk goes out with coalesced
-//                stores at its final offset.
+//                for another. A warp codes a whole chunk, lane p its piece p (128 bytes, a
+//                quarter sub-stream) starting at the bit that a warp prefix sum of the measured
+//                piece bit counts gives: one table lookup per symbol, two codes joined per 32-bit
+//                register and appended to a 64-bit accumulator, each finished word stored in the
+//                warp's shared buffer (a word two pieces share is stored by the piece that
+//                finishes it and the other ORs its bits in after a warp barrier). The chunk then
+//                leaves with coalesced stores at its final offset.
 //
 //   k_decode     one thread per sub-stream (8 per chunk, 32 chunks per 256-thread block). The
 //                two payload words in use and a bit offset into them give the next 32 bits with
@@ -43,7 +45,6 @@ namespace {
 constexpr uint32_t kMagic = 0x31305848u;  // "HX01"
 constexpr uint32_t kChunk = HX_CHUNK;
 constexpr uint32_t kSubLen = HX_CHUNK / HX_SUBSTREAMS;
-constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
 constexpr int kDecThreads = 256;  // 8 threads per chunk, 32 chunks per block
 constexpr int kHistThreads = 256;
 
@@ -103,6 +104,7 @@ struct EncodeArgs {
   uint64_t cap;
   uint32_t* local;   // scratch: block-local word offset of every chunk
   uint32_t* btotal;  // scratch: words of each measure block
+  uint16_t* pieces;  // scratch: bit count of each 128-byte piece, 32 per chunk
   uint32_t mblocks;  // measure blocks
   uint32_t cpb;      // chunks per measure block
   uint32_t* hist;    // optional fused histogram
@@ -158,17 +160,6 @@ __device__ __forceinline__ uint32_t load16(const EncodeArgs& a, uint32_t c, uint
   return valid;
 }
 
-__device__ __forceinline__ uint32_t byte_of(const uint4& v, int j) {
-  const uint32_t w = j < 4 ? v.x : j < 8 ? v.y : j < 12 ? v.z : v.w;
-  return (w >> (8 * (j & 3))) & 0xffu;
-}
-
-__device__ __forceinline__ uint32_t warp_sum(uint32_t x) {
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) x += __shfl_xor_sync(0xffffffffu, x, d);
-  return x;
-}
-
 // Exclusive scan of cnt[0..m) in place with the whole block (m <= 16 * blockDim.x); returns the
 // sum. `red` holds one word per warp.
 template <int THREADS>
@@ -216,32 +207,67 @@ struct MeasureSmem {
   uint32_t red[kMeasureThreads / 32];
 };
 
-// One chunk's sync row and word count (lane 0 writes them); WHOLE: all 4096 bytes exist.
+// Byte offset of table entry sym * 32 + lane in a [symbol][32] u32 table, for byte J (0..3) of w:
+// one shift and one AND-OR (lane4 = lane * 4 < 128).
+template <int J>
+__device__ __forceinline__ uint32_t lut_off(uint32_t w, uint32_t lane4) {
+  return ((J == 0 ? (w << 7) : (w >> (8 * J - 7))) & 0x7f80u) | lane4;
+}
+
+// Sum of the table entries of the 16 bytes in v (count of them: `valid`); the low 16 bits of the
+// sum are the bit count (<= 16 * 12). With HIST each lookup is a shared atomic that also adds 1
+// to the entry's count (bits 16..31).
 template <bool HIST, bool COMPLETE, bool WHOLE>
-__device__ __forceinline__ uint32_t measure_chunk(const EncodeArgs& a, uint32_t c, uint32_t* lut_lane,
+__device__ __forceinline__ uint32_t measure16(char* lut, uint32_t lane4, const uint4& v,
+                                              uint32_t valid, bool& uncodable) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t sum = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (WHOLE || (uint32_t)(4 * q + j) < valid) {
+        const uint32_t off = j == 0   ? lut_off<0>(w[q], lane4)
+                             : j == 1 ? lut_off<1>(w[q], lane4)
+                             : j == 2 ? lut_off<2>(w[q], lane4)
+                                      : lut_off<3>(w[q], lane4);
+        uint32_t* slot = reinterpret_cast<uint32_t*>(lut + off);
+        const uint32_t e = HIST ? atomicAdd(slot, 1u << 16) : *slot;
+        sum += e;
+        if (!COMPLETE) uncodable |= (e & 0xffu) == 0;
+      }
+    }
+  }
+  return sum & 0xffffu;
+}
+
+// One chunk's sync row (lane 0 writes it) and the bit counts of its 32 pieces of 128 bytes
+// (piece p = bytes 128p .. 128p + 127: a quarter of sub-stream p / 4); returns its bit count.
+// WHOLE: all 4096 bytes exist.
+template <bool HIST, bool COMPLETE, bool WHOLE>
+__device__ __forceinline__ uint32_t measure_chunk(const EncodeArgs& a, uint32_t c, char* lut,
                                                   uint4* sync, bool& uncodable) {
-  const uint32_t lane = threadIdx.x & 31;
+  const uint32_t lane = threadIdx.x & 31, lane4 = lane * 4;
   uint4 v[HX_SUBSTREAMS];
   uint32_t valid[HX_SUBSTREAMS];
 #pragma unroll
   for (int k = 0; k < HX_SUBSTREAMS; ++k) valid[k] = load16(a, c, k, lane, WHOLE, v[k]);
   uint32_t row[HX_SUBSTREAMS];  // bit offset of each sub-stream in the chunk
-  uint32_t run = 0;
+  uint32_t run = 0, piece = 0;
 #pragma unroll
   for (int k = 0; k < HX_SUBSTREAMS; ++k) {
     row[k] = run;
-    uint32_t sum = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (WHOLE || (uint32_t)j < valid[k]) {
-        uint32_t* slot = lut_lane + byte_of(v[k], j) * kMeasureCopies;
-        const uint32_t e = HIST ? atomicAdd(slot, 1u << 16) : *slot;
-        sum += e & 0xffffu;
-        if (!COMPLETE) uncodable |= (e & 0xffu) == 0;
-      }
-    }
-    run += warp_sum(sum);
+    // lanes 8q .. 8q + 7 hold quarter q of sub-stream k: three steps sum each quarter
+    uint32_t x = measure16<HIST, COMPLETE, WHOLE>(lut, lane4, v[k], valid[k], uncodable);
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    if ((lane & 7) == (uint32_t)k) piece = x;  // lane 8q + k keeps piece 4k + q
+    x += __shfl_xor_sync(0xffffffffu, x, 8);
+    x += __shfl_xor_sync(0xffffffffu, x, 16);
+    run += x;
   }
+  a.pieces[(uint64_t)c * 32 + (lane & 7) * 4 + (lane >> 3)] = (uint16_t)piece;
   if (lane == 0)
     sync[c] = make_uint4(run | (row[1] << 16), row[2] | (row[3] << 16), row[4] | (row[5] << 16),
                          row[6] | (row[7] << 16));
@@ -257,7 +283,7 @@ __device__ void measure_chunks(const EncodeArgs& a, MeasureSmem& sm) {
   const uint32_t c0 = blockIdx.x * a.cpb;
   const uint32_t m = c0 < nchunks ? min(a.cpb, nchunks - c0) : 0u;
   uint4* sync = reinterpret_cast<uint4*>(a.out + sync_offset(n));
-  uint32_t* lut_lane = sm.lut + lane;
+  char* lut = reinterpret_cast<char*>(sm.lut);
   bool uncodable = false;
 
   auto flush_hist = [&]() {  // counts of the table copies -> global, then clear them
@@ -279,8 +305,8 @@ __device__ void measure_chunks(const EncodeArgs& a, MeasureSmem& sm) {
     if (i < m) {
       const uint32_t c = c0 + i;
       const uint32_t bits =
-          c < full_chunks ? measure_chunk<HIST, COMPLETE, true>(a, c, lut_lane, sync, uncodable)
-                          : measure_chunk<HIST, COMPLETE, false>(a, c, lut_lane, sync, uncodable);
+          c < full_chunks ? measure_chunk<HIST, COMPLETE, true>(a, c, lut, sync, uncodable)
+                          : measure_chunk<HIST, COMPLETE, false>(a, c, lut, sync, uncodable);
       if (lane == 0) sm.cnt[i] = (bits + 31) >> 5;
     }
     if (HIST && (r + 1) % kMeasureFlushRounds == 0) flush_hist();
@@ -293,7 +319,7 @@ __device__ void measure_chunks(const EncodeArgs& a, MeasureSmem& sm) {
   if (HIST) flush_hist();
 }
 
-__global__ void __launch_bounds__(kMeasureThreads, 4) k_measure(EncodeArgs a) {
+__global__ void __launch_bounds__(kMeasureThreads, 3) k_measure(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   MeasureSmem& sm = *reinterpret_cast<MeasureSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -318,17 +344,37 @@ __global__ void __launch_bounds__(kMeasureThreads, 4) k_measure(EncodeArgs a) {
   }
 }
 
-// Pack 16 (code, len) entries MSB-first starting at bit `off` of buf: two codes are joined in a
-// 32-bit register (<= 24 bits), then appended to a 64-bit accumulator (hi:lo) with funnel
-// shifts. Every finished word is OR-ed into the zeroed buffer (the first and last may be shared
-// with neighbours), so the emit is one predicated step with no lane-dependent branch.
-__device__ __forceinline__ void pack16(const uint32_t e[16], uint32_t off, uint32_t* buf) {
-  uint32_t widx = off >> 5;
-  uint32_t nacc = off & 31;  // the first bits belong to the previous lane (zeros here)
-  uint32_t hi = 0, lo = 0;
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const uint32_t e0 = e[2 * p], e1 = e[2 * p + 1];
+constexpr int kPackThreads = 256;  // a warp per chunk; lane p codes piece p (128 bytes)
+constexpr int kPackCopies = 16;    // lane l reads copy l % 16: at most two lookups to a bank
+constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
+constexpr uint32_t kMaxPieceBits = 128 * HX_LMAX_MAX;
+
+struct PackSmem {
+  uint32_t lut[256 * kPackCopies];                  // [symbol][copy]: (code << 20) | len
+  uint32_t out[kPackThreads / 32][kMaxChunkWords];  // one chunk per warp
+  uint32_t bpre[kMaxMeasureBlocks];                  // word offset of each measure block
+  uint32_t red[kPackThreads / 32];
+};
+
+// Table entry of byte J (0..3) of w for this lane: byte offset sym * 64 + (lane % 16) * 4 into
+// the [symbol][16] table, by one shift and one AND-OR.
+template <int J>
+__device__ __forceinline__ uint32_t lut_entry(const char* lut, uint32_t w, uint32_t lane4) {
+  const uint32_t off = ((J == 0 ? (w << 6) : (w >> (8 * J - 6))) & 0x3fc0u) | lane4;
+  return *reinterpret_cast<const uint32_t*>(lut + off);
+}
+
+// Codes m (<= 128) bytes at src as the bits [s, s + its length) of the chunk's word buffer:
+// two codes are joined in a 32-bit register (<= 24 bits), appended to a 64-bit accumulator
+// (hi:lo) with funnel shifts, and every word this piece finishes is stored whole (bits of earlier
+// pieces in it as zeros). Returns the unfinished last word's bits in the low *nacc bits; *widx
+// is its index.
+template <bool WHOLE>
+__device__ __forceinline__ uint32_t pack_piece(const uint8_t* src, uint32_t m, const char* lut,
+                                               uint32_t lane4, uint32_t* buf, uint32_t s,
+                                               uint32_t* widx_out, uint32_t* nacc_out) {
+  uint32_t widx = s >> 5, nacc = s & 31, hi = 0, lo = 0;
+  auto put2 = [&](uint32_t e0, uint32_t e1) {
     const uint32_t l1 = e1 & 0xffu;
     const uint32_t pl = (e0 & 0xffu) + l1;
     const uint32_t pc = ((e0 >> 20) << l1) | (e1 >> 20);
@@ -337,76 +383,63 @@ __device__ __forceinline__ void pack16(const uint32_t e[16], uint32_t off, uint3
     nacc += pl;
     const bool full = nacc >= 32;
     nacc -= full ? 32u : 0u;
-    if (full) atomicOr(&buf[widx], __funnelshift_r(lo, hi, nacc));
+    if (full) buf[widx] = __funnelshift_r(lo, hi, nacc);
     widx += full ? 1u : 0u;
-  }
-  if (nacc) atomicOr(&buf[widx], lo << (32 - nacc));
-}
-
-constexpr int kPackThreads = 256;
-constexpr int kPackCopies = 16;  // lane l reads copy l % 16: at most two lookups to a bank
-
-struct PackSmem {
-  // [symbol][copy]: (code << 20) | len; the low byte of 16 summed entries is their bit count
-  uint32_t lut[256 * kPackCopies];
-  uint32_t out[kPackThreads / 32][kMaxChunkWords];  // one chunk per warp
-  uint32_t bpre[kMaxMeasureBlocks];                  // word offset of each measure block
-  uint32_t red[kPackThreads / 32];
-  uint32_t total;
-};
-
-// Codes chunk c into buf (zeroed, the warp's own); returns its bit count. WHOLE: all 4096
-// bytes exist.
-template <bool WHOLE>
-__device__ __forceinline__ uint32_t pack_chunk(const EncodeArgs& a, uint32_t c,
-                                               const uint32_t* lut_lane, uint32_t* buf) {
-  const uint32_t lane = threadIdx.x & 31;
-  uint4 v[HX_SUBSTREAMS];
-  uint32_t valid[HX_SUBSTREAMS];
-#pragma unroll
-  for (int k = 0; k < HX_SUBSTREAMS; ++k) valid[k] = load16(a, c, k, lane, WHOLE, v[k]);
-  uint32_t base = 0;  // bits of the chunk before sub-stream k
-#pragma unroll
-  for (int k = 0; k < HX_SUBSTREAMS; ++k) {
-    uint32_t e[16];
-    uint32_t sum = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      e[j] = (WHOLE || (uint32_t)j < valid[k]) ? lut_lane[byte_of(v[k], j) * kPackCopies] : 0u;
-      sum += e[j];
+  };
+  auto put_word = [&](uint32_t w, uint32_t count) {  // bytes 0..count-1 of w
+    uint32_t e[4];
+    e[0] = (WHOLE || count > 0) ? lut_entry<0>(lut, w, lane4) : 0u;
+    e[1] = (WHOLE || count > 1) ? lut_entry<1>(lut, w, lane4) : 0u;
+    e[2] = (WHOLE || count > 2) ? lut_entry<2>(lut, w, lane4) : 0u;
+    e[3] = (WHOLE || count > 3) ? lut_entry<3>(lut, w, lane4) : 0u;
+    put2(e[0], e[1]);
+    put2(e[2], e[3]);
+  };
+  if (WHOLE) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4 v = __ldg(s4);
+#pragma unroll 1
+    for (uint32_t g = 0; g < 8; ++g) {
+      const uint4 cur = v;
+      if (g + 1 < 8) v = __ldg(s4 + g + 1);
+      put_word(cur.x, 4);
+      put_word(cur.y, 4);
+      put_word(cur.z, 4);
+      put_word(cur.w, 4);
     }
-    const uint32_t bits = sum & 0xffu;
-    uint32_t incl = bits;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += t;
+  } else {
+    for (uint32_t i = 0; i < m; i += 4) {
+      const uint32_t cnt = min(4u, m - i);
+      uint32_t w = 0;
+      for (uint32_t j = 0; j < cnt; ++j) w |= (uint32_t)src[i + j] << (8 * j);
+      put_word(w, cnt);
     }
-    if (bits) pack16(e, base + incl - bits, buf);
-    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  return base;
+  *widx_out = widx;
+  *nacc_out = nacc;
+  return lo;
 }
 
 __global__ void __launch_bounds__(kPackThreads, 3) k_pack(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PackSmem& sm = *reinterpret_cast<PackSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lane4 = (lane % kPackCopies) * 4;
   if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) return;  // k_measure said so
   const uint64_t n = a.n;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
   const uint32_t full_chunks = (uint32_t)(n / kChunk);
   const uint64_t P = payload_offset(n);
   uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
+  const uint4* sync = reinterpret_cast<const uint4*>(a.out + sync_offset(n));
   uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
+  const char* lut = reinterpret_cast<const char*>(sm.lut);
 
   for (int i = tid; i < 256 * kPackCopies; i += kPackThreads) {
     uint32_t code;
     const uint32_t len = checked_code(a, i / kPackCopies, &code);
     sm.lut[i] = (code << 20) | len;
   }
-  for (int i = tid; i < (kPackThreads / 32) * (int)kMaxChunkWords; i += kPackThreads)
-    (&sm.out[0][0])[i] = 0;
   for (uint32_t i = tid; i < a.mblocks; i += kPackThreads) sm.bpre[i] = a.btotal[i];
   __syncthreads();
   const uint32_t total = block_exclusive_scan<kPackThreads>(sm.bpre, a.mblocks, sm.red);
@@ -422,22 +455,49 @@ __global__ void __launch_bounds__(kPackThreads, 3) k_pack(EncodeArgs a) {
       atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
     }
   }
+  const uint32_t limit = fits ? total : 0u;  // no payload store at all when it does not fit
 
-  const uint32_t* lut_lane = sm.lut + lane % kPackCopies;
   uint32_t* buf = sm.out[warp];
   const uint32_t stride = gridDim.x * (kPackThreads / 32);
   for (uint32_t c = blockIdx.x * (kPackThreads / 32) + warp; c < nchunks; c += stride) {
     const uint32_t woff = sm.bpre[c / a.cpb] + a.local[c];
     if (lane == 0) word_off[c] = woff;
-    const uint32_t base = c < full_chunks ? pack_chunk<true>(a, c, lut_lane, buf)
-                                          : pack_chunk<false>(a, c, lut_lane, buf);
-    __syncwarp();
-    const uint32_t words = (base + 31) >> 5;
-    for (uint32_t i = lane; i < words; i += 32) {
-      // woff + words <= total unless the input changed since k_measure read it
-      if (fits && woff + i < total) payload[woff + i] = buf[i];
-      buf[i] = 0;
+    // this piece's first bit: a warp prefix sum of the piece bit counts
+    const uint32_t mine = min((uint32_t)a.pieces[(uint64_t)c * 32 + lane], kMaxPieceBits);
+    uint32_t incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += t;
     }
+    const uint32_t chunk_bits = __shfl_sync(0xffffffffu, incl, 31);
+    const uint32_t s = incl - mine;
+    const uint32_t words = (chunk_bits + 31) >> 5;
+    if (chunk_bits != (__ldg(reinterpret_cast<const uint32_t*>(sync + c)) & 0xffffu)) {
+      // the scratch disagrees with the index k_measure wrote: leave the chunk's words unwritten
+      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+      continue;
+    }
+    uint32_t widx = 0, nacc = 0, tail = 0;
+    const uint8_t* src = a.in + (uint64_t)c * kChunk + lane * 128;
+    if (c < full_chunks) {
+      tail = pack_piece<true>(src, 128, lut, lane4, buf, s, &widx, &nacc);
+    } else {
+      const uint64_t first = (uint64_t)c * kChunk + lane * 128;
+      const uint32_t m = first < n ? (uint32_t)min((uint64_t)128, n - first) : 0u;
+      tail = pack_piece<false>(src, m, lut, lane4, buf, s, &widx, &nacc);
+    }
+    // The piece's unfinished word: the chunk's last word is stored whole (zero padding); any
+    // other is OR-ed, after a warp barrier, into the word that a later piece stored whole.
+    const bool has_tail = mine != 0 && nacc != 0;
+    const bool last = mine != 0 && incl == chunk_bits;
+    tail = has_tail ? tail << (32 - nacc) : 0u;
+    if (has_tail && last) buf[widx] = tail;
+    __syncwarp();
+    if (has_tail && !last) atomicOr(buf + widx, tail);
+    __syncwarp();
+    for (uint32_t i = lane; i < words; i += 32)
+      if (woff + i < limit) payload[woff + i] = buf[i];
     __syncwarp();
   }
 }
@@ -762,10 +822,11 @@ int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint
                           (nchunks + kMaxChunksPerBlock - 1) / kMaxChunksPerBlock)});
   const uint32_t cpb = mblocks ? (nchunks + mblocks - 1) / mblocks : 1;
   if (mblocks) mblocks = (nchunks + cpb - 1) / cpb;  // no block without chunks
-  // scratch: u32 local[nchunks], then u32 btotal[mblocks] (mblocks <= nchunks)
+  // scratch: u32 local[nchunks], u32 btotal[mblocks] (mblocks <= nchunks), u16 pieces[32 nchunks]
   auto* local = static_cast<uint32_t*>(d_scratch);
+  auto* pieces = reinterpret_cast<uint16_t*>(local + 2 * (uint64_t)nchunks);
   EncodeArgs a{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
-               out_cap, local, local + nchunks, mblocks, cpb, d_hist, d_status, kind};
+               out_cap, local, local + nchunks, pieces, mblocks, cpb, d_hist, d_status, kind};
   if (mblocks) {
     k_measure<<<mblocks, kMeasureThreads, sizeof(MeasureSmem), s>>>(a);
     if (cudaPeekAtLastError() != cudaSuccess) return launched();
@@ -803,12 +864,12 @@ int decode_common(uint32_t kind, const void* d_tables, const void* d_stream, uin
 
 }  // namespace
 
-// Scratch of hx_encode_noalloc: hx_scratch_bytes(HX_NOALLOC_MAX_BYTES) bytes (a block-local word
-// offset per chunk and the measure blocks' totals). Host code must not pass this name to a kernel
+// Scratch of hx_encode_noalloc: hx_scratch_bytes(HX_NOALLOC_MAX_BYTES) bytes (per chunk a
+// block-local word offset and 32 piece bit counts; the measure blocks' totals). Host code must not pass this name to a kernel
 // (on the host it is only a stand-in); its device address comes from cudaGetSymbolAddress, once
 // per device.
 static __device__ __align__(256) unsigned char
-    g_noalloc_scratch[8 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16];
+    g_noalloc_scratch[72 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16];
 
 namespace {
 std::mutex g_noalloc_mutex;
@@ -817,7 +878,7 @@ void* g_noalloc_ptr[64];  // device address of g_noalloc_scratch, per device
 
 extern "C" {
 
-uint64_t hx_scratch_bytes(uint64_t n) { return 8 * n_chunks_of(n) + 16; }
+uint64_t hx_scratch_bytes(uint64_t n) { return 72 * n_chunks_of(n) + 16; }
 
 // For callers that cannot allocate device memory at encode time (a framework's caching
 // allocator owns the device memory, or a path that cannot take cudaMalloc's implicit
@@ -827,7 +888,7 @@ uint64_t hx_scratch_bytes(uint64_t n) { return 8 * n_chunks_of(n) + 16; }
 int hx_encode_noalloc(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
                       uint64_t out_cap, uint32_t* d_hist, uint32_t* d_status, void* stream) {
   if (n > HX_NOALLOC_MAX_BYTES) return HX_ERR_ARG;
-  static_assert(sizeof(g_noalloc_scratch) >= 8 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16,
+  static_assert(sizeof(g_noalloc_scratch) >= 72 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16,
                 "scratch array smaller than hx_scratch_bytes(HX_NOALLOC_MAX_BYTES)");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HX_ERR_CUDA;
