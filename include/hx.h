@@ -18,7 +18,7 @@
  *    uncodable symbol, a corrupt stream, a codebook mismatch, a full output buffer) are OR-ed
  *    into the caller's device word *d_status, which the caller zeroes before and reads after the
  *    stream is synchronised. Data errors never trap the device: reads are clamped to the
- *    buffers' valid ranges and every wait is bounded.
+ *    buffers' valid ranges, and no kernel waits for another block.
  *  - d_in / d_out / d_stream must be 16-byte aligned (as every torch allocation is); n < 2^32.
  *
  * Stream format (version 1). All integers little-endian; offsets from the stream start.
@@ -54,7 +54,7 @@ typedef enum {
   HX_ERR_UNCODABLE = 4,  /* encode: an input byte has no code word (seen-only codebook)      */
   HX_ERR_CORRUPT = 8,    /* decode: the stream is malformed or does not decode exactly      */
   HX_ERR_CODEBOOK = 16,  /* decode: the stream was written with another codebook or kind    */
-  HX_ERR_TIMEOUT = 32,   /* encode: the chunk-offset scan waited past its bound              */
+  HX_ERR_TIMEOUT = 32,   /* reserved: a bounded device wait ran out (no current kernel waits) */
   HX_ERR_CAPACITY = 64   /* encode: out_cap is too small; header.total_words holds the need */
 } hx_status;
 
@@ -150,6 +150,23 @@ int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d
                   void* stream);
 int hx_qlc_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
                   uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream);
+
+/* The two passes of an encode, for callers that schedule or time them apart; hx_encode (kind 0)
+ * and hx_qlc_encode (kind 1) are exactly hx_encode_measure followed by hx_encode_pack. The pages
+ * do not split the encoder: the split is this library's way to give every chunk its offset with
+ * no block waiting for another. kind: 0 Huffman, 1 QLC (must match the tables).
+ *  - hx_encode_measure: code lengths only. Writes the index's sync rows into d_out, per-chunk
+ *    word counts and per-piece bit counts into d_scratch, and (d_hist non-NULL) accumulates the
+ *    histogram of d_in.
+ *  - hx_encode_pack: from those, the header, the word offsets and the payload.
+ * Give both the same arguments, in this order, on one stream; d_in, d_scratch and d_out must not
+ * change in between. Errors as for hx_encode. */
+int hx_encode_measure(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
+                      void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
+                      uint32_t* d_status, void* stream);
+int hx_encode_pack(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
+                   void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_status,
+                   void* stream);
 
 /* Allocation-free encode. The pages have no counterpart to this call: it exists for callers
  * that cannot allocate device memory when they encode -- for example code that runs under a

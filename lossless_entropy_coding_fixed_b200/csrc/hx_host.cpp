@@ -278,7 +278,7 @@ const char* hx_status_string(int code) {
     case HX_ERR_UNCODABLE: return "input byte without a code word";
     case HX_ERR_CORRUPT: return "corrupt stream";
     case HX_ERR_CODEBOOK: return "stream written with another codebook";
-    case HX_ERR_TIMEOUT: return "chunk-offset scan timed out";
+    case HX_ERR_TIMEOUT: return "a bounded device wait ran out";
     case HX_ERR_CAPACITY: return "output buffer too small";
     default: return "several errors (bit set)";
   }

@@ -803,39 +803,60 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 int launched() { return cudaGetLastError() == cudaSuccess ? HX_OK : HX_ERR_CUDA; }
 
-int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
-                  void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
-                  uint32_t* d_status, void* stream) {
+// Checks the arguments and fills the kernel arguments of one encode (both passes compute the same
+// from the same call arguments). Returns HX_OK or a host error.
+int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
+                EncodeArgs* a, DeviceInfo* info) {
   if (!d_tables || !d_out || !d_scratch || !d_status || (n && !d_in)) return HX_ERR_ARG;
+  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC) return HX_ERR_ARG;
   if (n >= (1ull << 32) || out_cap < payload_offset(n) + 8) return HX_ERR_ARG;
   if (!aligned16(d_in) || !aligned16(d_out) || !aligned16(d_scratch) || !aligned16(d_tables))
     return HX_ERR_ARG;
-  DeviceInfo info;
-  if (!device_info(&info)) return HX_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!device_info(info)) return HX_ERR_CUDA;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
   // measure blocks: at least one wave of resident blocks, at most kMaxChunksPerBlock chunks each
   // (n < 2^32 gives at most 2^20 chunks, so 256 blocks always suffice)
   uint32_t mblocks = (uint32_t)std::min<uint64_t>(
       {(uint64_t)nchunks, (uint64_t)kMaxMeasureBlocks,
-       std::max<uint64_t>((uint64_t)info.sms * info.measure_per_sm,
+       std::max<uint64_t>((uint64_t)info->sms * info->measure_per_sm,
                           (nchunks + kMaxChunksPerBlock - 1) / kMaxChunksPerBlock)});
   const uint32_t cpb = mblocks ? (nchunks + mblocks - 1) / mblocks : 1;
   if (mblocks) mblocks = (nchunks + cpb - 1) / cpb;  // no block without chunks
   // scratch: u32 local[nchunks], u32 btotal[mblocks] (mblocks <= nchunks), u16 pieces[32 nchunks]
   auto* local = static_cast<uint32_t*>(d_scratch);
   auto* pieces = reinterpret_cast<uint16_t*>(local + 2 * (uint64_t)nchunks);
-  EncodeArgs a{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
-               out_cap, local, local + nchunks, pieces, mblocks, cpb, d_hist, d_status, kind};
-  if (mblocks) {
-    k_measure<<<mblocks, kMeasureThreads, sizeof(MeasureSmem), s>>>(a);
-    if (cudaPeekAtLastError() != cudaSuccess) return launched();
-  }
+  *a = EncodeArgs{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
+                  out_cap, local, local + nchunks, pieces, mblocks, cpb, d_hist, d_status, kind};
+  return HX_OK;
+}
+
+int launch_measure(const EncodeArgs& a, cudaStream_t s) {
+  if (a.mblocks) k_measure<<<a.mblocks, kMeasureThreads, sizeof(MeasureSmem), s>>>(a);
+  return launched();
+}
+
+int launch_pack(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
+  const uint32_t nchunks = (uint32_t)n_chunks_of(a.n);
   const uint32_t grid = (uint32_t)std::max<uint64_t>(
       1, std::min<uint64_t>((nchunks + kPackThreads / 32 - 1) / (kPackThreads / 32),
                             (uint64_t)info.sms * info.pack_per_sm));
   k_pack<<<grid, kPackThreads, sizeof(PackSmem), s>>>(a);
   return launched();
+}
+
+int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
+                  void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
+                  uint32_t* d_status, void* stream) {
+  EncodeArgs a;
+  DeviceInfo info;
+  const int rc = encode_args(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
+                             &a, &info);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int m = launch_measure(a, s);
+  if (m) return m;
+  return launch_pack(a, info, s);
 }
 
 int decode_common(uint32_t kind, const void* d_tables, const void* d_stream, uint64_t bytes,
@@ -941,6 +962,26 @@ int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d
                   void* stream) {
   return encode_common(HX_KIND_QLC, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist,
                        d_status, stream);
+}
+
+int hx_encode_measure(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
+                      void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
+                      uint32_t* d_status, void* stream) {
+  EncodeArgs a;
+  DeviceInfo info;
+  const int rc = encode_args(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
+                             &a, &info);
+  return rc ? rc : launch_measure(a, static_cast<cudaStream_t>(stream));
+}
+
+int hx_encode_pack(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
+                   void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_status,
+                   void* stream) {
+  EncodeArgs a;
+  DeviceInfo info;
+  const int rc = encode_args(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, nullptr,
+                             d_status, &a, &info);
+  return rc ? rc : launch_pack(a, info, static_cast<cudaStream_t>(stream));
 }
 
 int hx_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,

@@ -74,6 +74,8 @@ def lib():
             "hx_qlc_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
             "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_encode_noalloc": (i32, [P, P, u64, P, u64, P, P, P]),
+            "hx_encode_measure": (i32, [u32, P, P, u64, P, u64, P, P, P, P]),
+            "hx_encode_pack": (i32, [u32, P, P, u64, P, u64, P, P, P]),
             "hx_entropy": (ctypes.c_double, [P]),
             "hx_mean_length": (ctypes.c_double, [P, CB]),
             "hx_version": (i32, []),
@@ -249,6 +251,28 @@ def encode(tables, x, out=None, scratch=None, hist=None, status=None, kind: int 
     _check(fn(tables.data_ptr(), x.data_ptr(), n, out.data_ptr(), out.numel(), scratch.data_ptr(),
               hist.data_ptr() if hist is not None else None, status.data_ptr(), _stream(x)),
            "hx_encode")
+    return out, status
+
+
+def encode_passes(tables, x, out, scratch, hist=None, status=None, kind: int = KIND_HUFFMAN,
+                  between=None):
+    """The same encode as encode(), as its two calls: hx_encode_measure, then hx_encode_pack.
+    `between`, if given, is called (host side) after the first is enqueued -- e.g. to record an
+    event. Returns (out, status)."""
+    x = _dev_u8(x, "x")
+    out = _dev_u8(out, "out")
+    if status is None:
+        status = new_status(x.device)
+    n, s = x.numel(), _stream(x)
+    _check(lib().hx_encode_measure(kind, tables.data_ptr(), x.data_ptr(), n, out.data_ptr(),
+                                   out.numel(), scratch.data_ptr(),
+                                   hist.data_ptr() if hist is not None else None,
+                                   status.data_ptr(), s), "hx_encode_measure")
+    if between is not None:
+        between()
+    _check(lib().hx_encode_pack(kind, tables.data_ptr(), x.data_ptr(), n, out.data_ptr(),
+                                out.numel(), scratch.data_ptr(), status.data_ptr(), s),
+           "hx_encode_pack")
     return out, status
 
 

@@ -185,6 +185,24 @@ def test_wrong_kind_tables(books):
     assert st == hx.HX_ERR_ARG
 
 
+@pytest.mark.parametrize("kind", ["huffman", "qlc"])
+@pytest.mark.parametrize("n", [4096 * 5 + 777, (1 << 20) - 5])
+def test_encode_passes_equal_oracle(orc, books, kind, n):
+    """hx_encode_measure then hx_encode_pack (timed apart by bench.py) write the oracle's stream."""
+    cb, tables, ocb, k = books[kind]
+    x = datagen.data(1, n=n)
+    ost, ref = orc.encode(ocb, x)
+    xd = dev(x)
+    out = torch.empty(hx.encode_bound(n), dtype=torch.uint8, device="cuda")
+    scratch = torch.empty(hx.scratch_bytes(n), dtype=torch.uint8, device="cuda")
+    hist = torch.zeros(256, dtype=torch.int32, device="cuda")
+    out, st = hx.encode_passes(tables, xd, out, scratch, hist=hist, kind=k)
+    torch.cuda.synchronize()
+    assert int(st.item()) == ost == 0
+    assert (out[:ref.size].cpu().numpy() == ref).all()
+    assert (hist.cpu().numpy().astype(np.uint64) == orc.histogram(x)).all()
+
+
 def test_deterministic_repeat(books):
     cb, tables, ocb, k = books["huffman"]
     x = datagen.data(4, n=(1 << 23) + 12345)
@@ -194,13 +212,13 @@ def test_deterministic_repeat(books):
 
 
 # --------------------------------------------------------------------------- damaged streams
-@pytest.fixture(scope="module")
-def damaged_setup(orc, books):
-    cb, tables, ocb, k = books["huffman"]
+@pytest.fixture(scope="module", params=["huffman", "qlc"])
+def damaged_setup(orc, books, request):
+    cb, tables, ocb, k = books[request.param]
     x = datagen.data(1, n=7 * 4096 + 777)
     st, s = orc.encode(ocb, x)
     assert st == 0
-    return tables, ocb, x, s
+    return tables, ocb, x, s, k
 
 
 def _damage_cases(s, n, orc):
@@ -224,30 +242,32 @@ def _damage_cases(s, n, orc):
 
 
 def test_damaged_index_and_header_statuses_match_oracle(orc, damaged_setup):
-    tables, ocb, x, s = damaged_setup
+    tables, ocb, x, s, k = damaged_setup
     for i, t in enumerate(_damage_cases(s, x.size, orc)):
         ost, _ = orc.decode(ocb, t, x.size)
-        st, _ = gpu_decode(tables, t, x.size, 0)
+        st, _ = gpu_decode(tables, t, x.size, k)
         assert ost != 0, i
         assert st == ost, (i, st, ost)
 
 
 def test_payload_bit_flips_match_oracle(orc, damaged_setup):
-    tables, ocb, x, s = damaged_setup
+    tables, ocb, x, s, k = damaged_setup
     P = orc.payload_offset(x.size)
     rng = np.random.default_rng(1)
     for _ in range(40):
         t = s.copy()
         t[int(rng.integers(P, s.size - 8))] ^= np.uint8(1 << int(rng.integers(0, 8)))
         ost, oy = orc.decode(ocb, t, x.size)
-        st, y = gpu_decode(tables, t, x.size, 0)
+        st, y = gpu_decode(tables, t, x.size, k)
         assert st == ost
         if st == 0:
             assert (y == oy).all()
 
 
 def test_other_codebook_rejected(orc, damaged_setup, cuda):
-    tables, ocb, x, s = damaged_setup
+    tables, ocb, x, s, k = damaged_setup
+    if k != hx.KIND_HUFFMAN:
+        pytest.skip("a Huffman table block against a Huffman stream")
     other = hx.build_codebook(datagen.random_counts(99)).upload(cuda)
     st, _ = gpu_decode(other, s, x.size, 0)
     assert st == hx.HX_ERR_CODEBOOK == orc.decode(orc.huffman_codebook(datagen.random_counts(99)), s, x.size)[0]
