@@ -345,23 +345,23 @@ __global__ void __launch_bounds__(kMeasureThreads, 3) k_measure(EncodeArgs a) {
 }
 
 constexpr int kPackThreads = 256;  // a warp per chunk; lane p codes piece p (128 bytes)
-constexpr int kPackCopies = 16;    // lane l reads copy l % 16: at most two lookups to a bank
+constexpr int kPackCopies = 32;    // lane l reads copy l: no bank conflicts
 constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
 constexpr uint32_t kMaxPieceBits = 128 * HX_LMAX_MAX;
 
 struct PackSmem {
   uint32_t lut[256 * kPackCopies];                  // [symbol][copy]: (code << 20) | len
-  uint32_t out[kPackThreads / 32][kMaxChunkWords];  // one chunk per warp
+  // one chunk per warp; word w of the chunk sits at w + (its offset & 3), so that 16-byte
+  // aligned runs of the payload are 16-byte aligned here too
+  alignas(16) uint32_t out[kPackThreads / 32][kMaxChunkWords + 4];
   uint32_t bpre[kMaxMeasureBlocks];                  // word offset of each measure block
   uint32_t red[kPackThreads / 32];
 };
 
-// Table entry of byte J (0..3) of w for this lane: byte offset sym * 64 + (lane % 16) * 4 into
-// the [symbol][16] table, by one shift and one AND-OR.
+// Table entry of byte J (0..3) of w for this lane (copy `lane` of the [symbol][32] table).
 template <int J>
 __device__ __forceinline__ uint32_t lut_entry(const char* lut, uint32_t w, uint32_t lane4) {
-  const uint32_t off = ((J == 0 ? (w << 6) : (w >> (8 * J - 6))) & 0x3fc0u) | lane4;
-  return *reinterpret_cast<const uint32_t*>(lut + off);
+  return *reinterpret_cast<const uint32_t*>(lut + lut_off<J>(w, lane4));
 }
 
 // Codes m (<= 128) bytes at src as the bits [s, s + its length) of the chunk's word buffer:
@@ -420,11 +420,11 @@ __device__ __forceinline__ uint32_t pack_piece(const uint8_t* src, uint32_t m, c
   return lo;
 }
 
-__global__ void __launch_bounds__(kPackThreads, 3) k_pack(EncodeArgs a) {
+__global__ void __launch_bounds__(kPackThreads, 2) k_pack(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PackSmem& sm = *reinterpret_cast<PackSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lane4 = (lane % kPackCopies) * 4;
+  const uint32_t lane4 = lane * 4;
   if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) return;  // k_measure said so
   const uint64_t n = a.n;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
@@ -457,11 +457,12 @@ __global__ void __launch_bounds__(kPackThreads, 3) k_pack(EncodeArgs a) {
   }
   const uint32_t limit = fits ? total : 0u;  // no payload store at all when it does not fit
 
-  uint32_t* buf = sm.out[warp];
+  uint32_t* const wbuf = sm.out[warp];
   const uint32_t stride = gridDim.x * (kPackThreads / 32);
   for (uint32_t c = blockIdx.x * (kPackThreads / 32) + warp; c < nchunks; c += stride) {
     const uint32_t woff = sm.bpre[c / a.cpb] + a.local[c];
     if (lane == 0) word_off[c] = woff;
+    uint32_t* buf = wbuf + (woff & 3);
     // this piece's first bit: a warp prefix sum of the piece bit counts
     const uint32_t mine = min((uint32_t)a.pieces[(uint64_t)c * 32 + lane], kMaxPieceBits);
     uint32_t incl = mine;
@@ -496,8 +497,14 @@ __global__ void __launch_bounds__(kPackThreads, 3) k_pack(EncodeArgs a) {
     __syncwarp();
     if (has_tail && !last) atomicOr(buf + widx, tail);
     __syncwarp();
-    for (uint32_t i = lane; i < words; i += 32)
-      if (woff + i < limit) payload[woff + i] = buf[i];
+    // out: a ragged head and tail word by word, the 16-byte aligned middle as uint4
+    const uint32_t end = min(woff + words, limit);
+    const uint32_t g0 = min((woff + 3) & ~3u, end), g1 = max(end & ~3u, g0);
+    if (woff + lane < g0) payload[woff + lane] = buf[lane];
+    if (g1 + lane < end) payload[g1 + lane] = buf[g1 - woff + lane];
+    const uint4* b4 = reinterpret_cast<const uint4*>(buf + (g0 - woff));
+    uint4* p4 = reinterpret_cast<uint4*>(payload + g0);
+    for (uint32_t q = lane; q < (g1 - g0) / 4; q += 32) p4[q] = b4[q];
     __syncwarp();
   }
 }

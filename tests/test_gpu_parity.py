@@ -113,13 +113,21 @@ def test_adversarial_inputs(orc, kind, cuda):
     k = cb.kind
     longest = int(np.argmax(ocb.len))
     shortest = int(np.argmin(np.where(ocb.len > 0, ocb.len, 99)))
+    # chunks coded longer than 8 bits per symbol take the encoder's direct path; mixed runs
+    # interleave direct and buffered chunks
+    mixed = np.concatenate([np.full(4096, longest if i % 3 else shortest, np.uint8)
+                            for i in range(7)] + [np.full(1000, longest, np.uint8)])
     for x in (np.full(5 * 4096 + 7, longest, np.uint8), np.full(5 * 4096 + 7, shortest, np.uint8),
-              datagen.uniform_bytes(9 * 4096 + 77, 5)):
+              datagen.uniform_bytes(9 * 4096 + 77, 5), mixed):
         ref = orc.encode(ocb, x)[1]
         got, st, _ = gpu_encode(tables, x, k)
         assert st == 0 and (got == ref).all()
         st, y = gpu_decode(tables, ref, x.size, k)
         assert st == 0 and (y == x).all()
+    # a full output buffer on the direct path: the header and index are written, no payload
+    need = orc.encode(ocb, mixed)[1].size
+    got, st, total = gpu_encode(tables, mixed, k, cap=need - 8)
+    assert st == hx.HX_ERR_CAPACITY and hx.stream_bytes(mixed.size, total) == need
 
 
 @pytest.mark.parametrize("lmax", [8, 9, 11])
