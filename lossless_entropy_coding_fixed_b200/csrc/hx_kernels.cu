@@ -709,9 +709,11 @@ __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut&
   }
 }
 
-// KIND is checked against the stream header and the tables; the symbol loop is the same.
+// KIND is checked against the stream header and the tables; the symbol loop is the same. (The
+// register budgets are the measured best per kind: 48 for Huffman, 64 for QLC.)
 template <int KIND>
-__global__ void __launch_bounds__(kDecThreads, 5) k_decode(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, KIND == HX_KIND_QLC ? 4 : 5)
+    k_decode(DecodeArgs a) {
   __shared__ __align__(16) uint16_t s_lut[4096];
   __shared__ int64_t s_total;
   const int tid = threadIdx.x;
