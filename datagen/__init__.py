@@ -195,6 +195,15 @@ def prior_batches(cfg: int, layer: int = 0):
         yield tensor_bytes(family, dtype, SIZES[cfg], 2000 + 100 * cfg + j, scale)
 
 
+def online_batch(t: int, n: int, switch: int = 10) -> np.ndarray:
+    """Batch t of the online-loop workload: e4m3 activations whose scale drifts 3 % per batch
+    (N(0, 0.5 * 1.03^t)) up to batch `switch`, then the cfg-2 FFN mixture law (an abrupt change).
+    Seed 7000 + t."""
+    if t < switch:
+        return tensor_bytes("normal", "e4m3", n, 7000 + t, 0.5 * 1.03 ** t)
+    return tensor_bytes("ffn_mix", "e4m3", n, 7000 + t, 1.0)
+
+
 def uniform_bytes(n: int, seed: int) -> np.ndarray:
     """n independent uniform bytes (edge-case and adversarial tests)."""
     return np.random.default_rng(seed).integers(0, 256, n, dtype=np.uint8)

@@ -151,6 +151,19 @@ int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d
 int hx_qlc_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
                   uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream);
 
+/* Decode with a set of table blocks: the device picks, by the codebook hash in the stream's
+ * header, the block to decode with (the first of the right kind whose lmax and hash match), so
+ * a receiver that keeps several codebook versions needs no host round trip to choose. d_tables:
+ * a HOST array of n_tables device pointers (1 <= n_tables <= HX_MAX_TABLE_SET), each a
+ * HX_TABLES_BYTES block; blocks that are not valid tables of this kind are skipped. No match
+ * raises HX_ERR_CODEBOOK. Otherwise as hx_decode / hx_qlc_decode (kind 0 / 1), which are this
+ * call with a set of one. "Single-Stage Huffman Encoder for ML Compression", abstract (sender and
+ * receiver share the codebook; only its identity travels with the data). */
+#define HX_MAX_TABLE_SET 8
+int hx_decode_set(uint32_t kind, const void* const* d_tables, uint32_t n_tables,
+                  const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
+                  uint64_t n_expected, uint32_t* d_status, void* stream);
+
 /* The two passes of an encode, for callers that schedule or time them apart; hx_encode (kind 0)
  * and hx_qlc_encode (kind 1) are exactly hx_encode_measure followed by hx_encode_pack. The pages
  * do not split the encoder: the split is this library's way to give every chunk its offset with
@@ -185,6 +198,73 @@ int hx_encode_pack(uint32_t kind, const void* d_tables, const uint8_t* d_in, uin
 #define HX_NOALLOC_MAX_BYTES (128ull << 20)
 int hx_encode_noalloc(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
                       uint64_t out_cap, uint32_t* d_hist, uint32_t* d_status, void* stream);
+
+/* ---- Online single-stage loop -----------------------------------------------------------
+ * "Single-Stage Huffman Encoder for ML Compression", abstract: the codebook for a batch comes
+ * from the average symbol distribution of previous batches, so the data path has no frequency
+ * pass and no codebook build, and no codebook travels with the data. A session runs that loop:
+ * batch t (the t-th hx_session_encode call, from 0) is coded with the codebook built from the
+ * summed histograms of batches t-lag-m+1 .. t-lag (m = history), which the encoder itself
+ * counted (the fused histogram); before any batch is observed, from initial_counts (NULL: all
+ * ones). Drift refresh (the "Shannonic" review of range-partitioned coding: rebuild when the
+ * code stops fitting the data): when batch j is observed, drift_j = mean code length of batch j
+ * under the codebook that coded it / its entropy - 1; if drift > cfg.drift > 0 the history
+ * restarts from batch j alone. The schedule depends only on the histograms, never on timing.
+ *
+ * hx_planner is that bookkeeping alone, on the host (no device): hx_planner_codebook(t) returns
+ * batch t's codebook once batches 0 .. t-lag (and no later one) have been observed, in order,
+ * with hx_planner_observe. */
+typedef struct {
+  uint32_t kind;          /* HX_KIND_HUFFMAN or HX_KIND_QLC                                   */
+  uint32_t lmax;          /* Huffman: length limit 1..12 (0 = 12)                             */
+  uint32_t max_distinct;  /* QLC: distinct widths 1..8 (0 = 4)                                */
+  uint32_t flags;         /* Huffman: 0 or HX_CB_SEEN_ONLY; QLC: 0                            */
+  uint32_t history;       /* m, batches summed: 1..64                                         */
+  uint32_t lag;           /* batch t uses histograms of batches <= t - lag: 1..8              */
+  double drift;           /* refresh threshold (fraction above entropy); <= 0: never refresh  */
+} hx_session_config;
+
+typedef struct {
+  uint64_t hash;          /* codebook hash the batch was coded with                           */
+  uint32_t slot;          /* device table slot that held it                                   */
+  int32_t observed;       /* 1 once its histogram has been folded into the plan               */
+  int32_t refreshed;      /* 1 if it triggered a drift refresh                                */
+  uint32_t pad;
+  uint64_t symbols;       /* bytes counted (once observed)                                    */
+  double drift;           /* its drift (NaN until observed, or for an all-empty batch)        */
+} hx_batch_info;
+
+typedef struct hx_planner hx_planner;
+int hx_planner_create(const hx_session_config* cfg, const uint64_t* initial_counts,
+                      hx_planner** out);
+int hx_planner_codebook(hx_planner* p, uint64_t batch, hx_codebook* out);
+int hx_planner_observe(hx_planner* p, uint64_t batch, const uint64_t* counts, int* refreshed,
+                       double* drift);
+void hx_planner_destroy(hx_planner* p);
+
+/* A session owns host state (the plan; pinned host buffers for lag + 1 histograms and one table
+ * block per slot; CUDA events); the device memory is the caller's: d_slots, n_slots table blocks
+ * of HX_TABLES_BYTES (lag + 1 <= n_slots <= HX_MAX_TABLE_SET, 16-byte aligned), which create
+ * zeroes (cudaMemset, synchronous). Use a session from one host thread and one stream.
+ *  - hx_session_encode: waits (host) for the histogram of batch t - lag if the device has not
+ *    finished it, builds batch t's codebook when the history changed and uploads it to the next
+ *    slot, zeroes d_hist (device u32[256]) and encodes into d_out with the fused histogram (as
+ *    hx_encode / hx_qlc_encode: same arguments, scratch, status), then copies d_hist to the host.
+ *  - hx_session_decode: hx_decode_set over the slots. A stream stays decodable until its slot is
+ *    reused, n_slots codebook changes later (after that: HX_ERR_CODEBOOK).
+ *  - hx_session_drain: folds every histogram still in flight (waits for the stream).
+ *  - hx_session_batch_info: what batch t was coded with, and its drift once observed. */
+typedef struct hx_session hx_session;
+int hx_session_create(const hx_session_config* cfg, const uint64_t* initial_counts,
+                      void* const* d_slots, uint32_t n_slots, hx_session** out);
+int hx_session_encode(hx_session* s, const uint8_t* d_in, uint64_t n, void* d_out,
+                      uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
+                      void* stream);
+int hx_session_decode(hx_session* s, const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
+                      uint64_t n_expected, uint32_t* d_status, void* stream);
+int hx_session_drain(hx_session* s);
+int hx_session_batch_info(const hx_session* s, uint64_t batch, hx_batch_info* out);
+void hx_session_destroy(hx_session* s);
 
 /* Measurement helpers (host, fp64). Shannon entropy -sum p log2 p of counts[256] in bits per
  * symbol ("Single-Stage Huffman Encoder for ML Compression", abstract: the ideal the fixed code

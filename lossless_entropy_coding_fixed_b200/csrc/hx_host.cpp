@@ -32,58 +32,61 @@ struct PmNode {
 
 bool lengths_by_package_merge(const uint64_t w[256], int lmax, uint8_t len[256]) {
   std::memset(len, 0, 256);
+  // leaves first (pool[0..m)), then each row's packages; a row holds at most 2m - 1 <= 511 items
+  constexpr int kPool = 256 + (HX_LMAX_MAX - 1) * 256;
   std::vector<PmNode> pool;
-  std::vector<int> leaves;
+  pool.reserve(kPool);
+  int leaves[256];
+  size_t m = 0;
   for (int s = 0; s < 256; ++s)
     if (w[s]) {
-      leaves.push_back((int)pool.size());
+      leaves[m++] = (int)pool.size();
       pool.push_back({w[s], s, -1, -1});
     }
-  const size_t m = leaves.size();
   if (m == 0) return true;
   if (m == 1) {
     len[pool[leaves[0]].symbol] = 1;
     return true;
   }
   if (lmax < 1 || lmax > HX_LMAX_MAX || (size_t(1) << lmax) < m) return false;
-  std::stable_sort(leaves.begin(), leaves.end(),
+  std::stable_sort(leaves, leaves + m,
                    [&](int a, int b) { return pool[a].weight < pool[b].weight; });
-  std::vector<int> row(leaves), next;
+  int rows[2][512];
+  int* row = rows[0];
+  int* next = rows[1];
+  size_t nrow = m;
+  std::copy(leaves, leaves + m, row);
   for (int depth = 1; depth < lmax; ++depth) {
-    next.clear();
-    size_t li = 0, pi = 0;
-    const size_t npk = row.size() / 2;
-    // packages of this row are created lazily, in order, as the merge needs them
-    std::vector<int> pk(npk);
+    // this row's packages, in order; then merge them with the leaves (a leaf first on a tie)
+    const size_t npk = nrow / 2, first = pool.size();
     for (size_t i = 0; i < npk; ++i) {
-      const PmNode& a = pool[row[2 * i]];
-      const PmNode& b = pool[row[2 * i + 1]];
-      pk[i] = (int)pool.size();
-      pool.push_back({a.weight + b.weight, -1, row[2 * i], row[2 * i + 1]});
+      const int a = row[2 * i], b = row[2 * i + 1];
+      pool.push_back({pool[a].weight + pool[b].weight, -1, a, b});
     }
+    size_t li = 0, pi = 0, k = 0;
     while (li < m || pi < npk) {
       const bool take_leaf =
-          pi == npk || (li < m && pool[leaves[li]].weight <= pool[pk[pi]].weight);
-      next.push_back(take_leaf ? leaves[li++] : pk[pi++]);
+          pi == npk || (li < m && pool[leaves[li]].weight <= pool[first + pi].weight);
+      next[k++] = take_leaf ? leaves[li++] : (int)(first + pi++);
     }
-    row.swap(next);
+    std::swap(row, next);
+    nrow = k;
   }
-  std::vector<int> stack;
-  int depth_count[256] = {0};
+  // the first 2m - 2 items of the top row; a leaf's length is how often it occurs in them
+  int stack[2 * HX_LMAX_MAX + 2];
   for (size_t i = 0; i < 2 * m - 2; ++i) {
-    stack.push_back(row[i]);
-    while (!stack.empty()) {
-      const PmNode& nd = pool[stack.back()];
-      stack.pop_back();
+    int sp = 0;
+    stack[sp++] = row[i];
+    while (sp) {
+      const PmNode& nd = pool[stack[--sp]];
       if (nd.symbol >= 0) {
-        depth_count[nd.symbol]++;
+        len[nd.symbol]++;
       } else {
-        stack.push_back(nd.part0);
-        stack.push_back(nd.part1);
+        stack[sp++] = nd.part0;
+        stack[sp++] = nd.part1;
       }
     }
   }
-  for (int s = 0; s < 256; ++s) len[s] = (uint8_t)depth_count[s];
   return true;
 }
 
@@ -114,6 +117,13 @@ struct QlcSearch {
   // Width vectors are visited depth-first with non-decreasing widths: lexicographic order, so
   // the first vector reaching the minimum is the smallest one.
   void visit(int area, int min_width, int distinct, int covered, unsigned __int128 cost) {
+    // costs only grow along a path, and a later vector of equal cost never replaces the best
+    if (found && cost >= best_cost) return;
+    if (covered == 256 && area < 8) {
+      // every completion costs the same; the smallest repeats the last width (no new value)
+      for (int a = area; a < 8; ++a) cur[a] = min_width;
+      area = 8;
+    }
     if (area == 8) {
       if (covered == 256 && (!found || cost < best_cost)) {
         found = true;

@@ -510,8 +510,12 @@ __global__ void __launch_bounds__(kPackThreads, 2) k_pack(EncodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------------- decode
+// The decoder takes a set of table blocks and codes with the one whose hash the header names
+// (hx_decode: a set of one).
+constexpr int kMaxTableSet = HX_MAX_TABLE_SET;
 struct DecodeArgs {
-  const hx::Tables* tables;
+  const hx::Tables* set[kMaxTableSet];
+  uint32_t nset;
   const uint8_t* st;
   uint64_t bytes;
   uint8_t* out;
@@ -520,17 +524,28 @@ struct DecodeArgs {
   uint32_t kind;
 };
 
-// Header checks shared by every block; returns total_words, or -status.
-__device__ int64_t check_header(const DecodeArgs& a) {
+// Header checks shared by every block; returns total_words, or -status, and the table block the
+// header's codebook hash picks. A set of one keeps the single-table order of checks: a block of
+// the wrong kind is an argument error before the stream is looked at.
+__device__ int64_t check_header(const DecodeArgs& a, const hx::Tables** picked) {
   const uint32_t* h32 = reinterpret_cast<const uint32_t*>(a.st);
   const uint64_t* h64 = reinterpret_cast<const uint64_t*>(a.st);
   const uint32_t vk = h32[1];
-  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) return -(int64_t)HX_ERR_ARG;
+  if (a.nset == 1 && (a.set[0]->magic != hx::kTablesMagic || a.set[0]->kind != a.kind))
+    return -(int64_t)HX_ERR_ARG;
   if (h32[0] != kMagic || (vk & 0xff) != 1 || h32[2] != kChunk || h32[3] != HX_SUBSTREAMS)
     return -(int64_t)HX_ERR_CORRUPT;
-  if (((vk >> 8) & 0xff) != a.kind || ((vk >> 16) & 0xff) != a.tables->lmax ||
-      h64[5] != a.tables->hash)
-    return -(int64_t)HX_ERR_CODEBOOK;
+  if (((vk >> 8) & 0xff) != a.kind) return -(int64_t)HX_ERR_CODEBOOK;
+  *picked = nullptr;
+  for (uint32_t i = 0; i < a.nset && i < (uint32_t)kMaxTableSet; ++i) {
+    const hx::Tables* t = a.set[i];
+    if (t->magic == hx::kTablesMagic && t->kind == a.kind && ((vk >> 16) & 0xff) == t->lmax &&
+        h64[5] == t->hash) {
+      *picked = t;
+      break;
+    }
+  }
+  if (!*picked) return -(int64_t)HX_ERR_CODEBOOK;
   if (h64[2] != a.n || h64[3] != n_chunks_of(a.n)) return -(int64_t)HX_ERR_CORRUPT;
   const uint64_t P = payload_offset(a.n);
   const uint64_t total = h64[4];
@@ -716,19 +731,22 @@ __global__ void __launch_bounds__(kDecThreads, KIND == HX_KIND_QLC ? 4 : 5)
     k_decode(DecodeArgs a) {
   __shared__ __align__(16) uint16_t s_lut[4096];
   __shared__ int64_t s_total;
+  __shared__ const hx::Tables* s_tables;
   const int tid = threadIdx.x;
-  if (tid == 0) s_total = check_header(a);
-  const uint4* src = reinterpret_cast<const uint4*>(a.tables->dec);
-  uint4* dst = reinterpret_cast<uint4*>(s_lut);
-  for (int i = tid; i < 4096 * 2 / 16; i += kDecThreads) dst[i] = src[i];
+  if (tid == 0) s_total = check_header(a, &s_tables);
   __syncthreads();
   const int64_t total = s_total;
   if (total < 0) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)(-total));
     return;
   }
+  const hx::Tables* tables = s_tables;
+  const uint4* src = reinterpret_cast<const uint4*>(tables->dec);
+  uint4* dst = reinterpret_cast<uint4*>(s_lut);
+  for (int i = tid; i < 4096 * 2 / 16; i += kDecThreads) dst[i] = src[i];
+  __syncthreads();
   const DecLut lut{s_lut};
-  if (a.tables->complete)
+  if (tables->complete)
     decode_chunks<true>(a, lut, (uint32_t)total);
   else
     decode_chunks<false>(a, lut, (uint32_t)total);
@@ -868,11 +886,14 @@ int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint
   return launch_pack(a, info, s);
 }
 
-int decode_common(uint32_t kind, const void* d_tables, const void* d_stream, uint64_t bytes,
-                  uint8_t* d_out, uint64_t n, uint32_t* d_status, void* stream) {
-  if (!d_tables || !d_stream || !d_status || (n && !d_out)) return HX_ERR_ARG;
+int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const void* d_stream,
+                  uint64_t bytes, uint8_t* d_out, uint64_t n, uint32_t* d_status, void* stream) {
+  if (!d_set || nset < 1 || nset > (uint32_t)kMaxTableSet) return HX_ERR_ARG;
+  for (uint32_t i = 0; i < nset; ++i)
+    if (!d_set[i] || !aligned16(d_set[i])) return HX_ERR_ARG;
+  if (!d_stream || !d_status || (n && !d_out)) return HX_ERR_ARG;
   if (n >= (1ull << 32)) return HX_ERR_ARG;
-  if (!aligned16(d_stream) || !aligned16(d_out) || !aligned16(d_tables)) return HX_ERR_ARG;
+  if (!aligned16(d_stream) || !aligned16(d_out)) return HX_ERR_ARG;
   if (bytes < payload_offset(n) + 8) return HX_ERR_CORRUPT;
   DeviceInfo info;
   if (!device_info(&info)) return HX_ERR_CUDA;
@@ -883,8 +904,15 @@ int decode_common(uint32_t kind, const void* d_tables, const void* d_stream, uin
   const uint64_t want = (nchunks + per_block - 1) / per_block;
   const uint32_t grid =
       (uint32_t)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)info.sms * per_sm));
-  DecodeArgs a{static_cast<const hx::Tables*>(d_tables), static_cast<const uint8_t*>(d_stream),
-               bytes, d_out, n, d_status, kind};
+  DecodeArgs a{};
+  for (uint32_t i = 0; i < nset; ++i) a.set[i] = static_cast<const hx::Tables*>(d_set[i]);
+  a.nset = nset;
+  a.st = static_cast<const uint8_t*>(d_stream);
+  a.bytes = bytes;
+  a.out = d_out;
+  a.n = n;
+  a.status = d_status;
+  a.kind = kind;
   if (kind == HX_KIND_HUFFMAN)
     k_decode<HX_KIND_HUFFMAN><<<grid, kDecThreads, 0, s>>>(a);
   else
@@ -995,14 +1023,22 @@ int hx_encode_pack(uint32_t kind, const void* d_tables, const uint8_t* d_in, uin
 
 int hx_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
               uint64_t n_expected, uint32_t* d_status, void* stream) {
-  return decode_common(HX_KIND_HUFFMAN, d_tables, d_stream, stream_bytes, d_out, n_expected,
+  return decode_common(HX_KIND_HUFFMAN, &d_tables, 1, d_stream, stream_bytes, d_out, n_expected,
                        d_status, stream);
 }
 
 int hx_qlc_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
                   uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream) {
-  return decode_common(HX_KIND_QLC, d_tables, d_stream, stream_bytes, d_out, n_expected, d_status,
-                       stream);
+  return decode_common(HX_KIND_QLC, &d_tables, 1, d_stream, stream_bytes, d_out, n_expected,
+                       d_status, stream);
+}
+
+int hx_decode_set(uint32_t kind, const void* const* d_tables, uint32_t n_tables,
+                  const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
+                  uint64_t n_expected, uint32_t* d_status, void* stream) {
+  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC) return HX_ERR_ARG;
+  return decode_common(kind, d_tables, n_tables, d_stream, stream_bytes, d_out, n_expected,
+                       d_status, stream);
 }
 
 }  // extern "C"

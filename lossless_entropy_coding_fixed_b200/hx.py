@@ -75,6 +75,17 @@ def lib():
             "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_encode_noalloc": (i32, [P, P, u64, P, u64, P, P, P]),
             "hx_encode_measure": (i32, [u32, P, P, u64, P, u64, P, P, P, P]),
+            "hx_decode_set": (i32, [u32, P, u32, P, u64, P, u64, P, P]),
+            "hx_planner_create": (i32, [ctypes.POINTER(_SessionConfig), P, P]),
+            "hx_planner_codebook": (i32, [P, u64, CB]),
+            "hx_planner_observe": (i32, [P, u64, P, P, P]),
+            "hx_planner_destroy": (None, [P]),
+            "hx_session_create": (i32, [ctypes.POINTER(_SessionConfig), P, P, u32, P]),
+            "hx_session_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
+            "hx_session_decode": (i32, [P, P, u64, P, u64, P, P]),
+            "hx_session_drain": (i32, [P]),
+            "hx_session_batch_info": (i32, [P, u64, ctypes.POINTER(_BatchInfo)]),
+            "hx_session_destroy": (None, [P]),
             "hx_encode_pack": (i32, [u32, P, P, u64, P, u64, P, P, P]),
             "hx_entropy": (ctypes.c_double, [P]),
             "hx_mean_length": (ctypes.c_double, [P, CB]),
@@ -95,6 +106,18 @@ def status_string(code: int) -> str:
 def _check(rc: int, what: str) -> None:
     if rc:
         raise HxError(rc, what)
+
+
+class _SessionConfig(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_uint32), ("lmax", ctypes.c_uint32),
+                ("max_distinct", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("history", ctypes.c_uint32), ("lag", ctypes.c_uint32), ("drift", ctypes.c_double)]
+
+
+class _BatchInfo(ctypes.Structure):
+    _fields_ = [("hash", ctypes.c_uint64), ("slot", ctypes.c_uint32), ("observed", ctypes.c_int32),
+                ("refreshed", ctypes.c_int32), ("pad", ctypes.c_uint32),
+                ("symbols", ctypes.c_uint64), ("drift", ctypes.c_double)]
 
 
 # ------------------------------------------------------------------------------ codebooks (host)
@@ -315,3 +338,114 @@ def total_words(stream) -> int:
 
 def stream_size(stream, n: int) -> int:
     return stream_bytes(n, total_words(stream))
+
+
+MAX_TABLE_SET = 8
+
+
+def decode_set(kind: int, tables, stream, n: int, out=None, status=None, nbytes=None):
+    """hx_decode_set: decode with whichever of the device table blocks `tables` the stream's
+    header hash names (picked on the device). Returns (out, status)."""
+    import torch
+    stream = _dev_u8(stream, "stream")
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=torch.uint8, device=stream.device)[:n]
+    if status is None:
+        status = new_status(stream.device)
+    ptrs = (ctypes.c_void_p * len(tables))(*[t.data_ptr() for t in tables])
+    _check(lib().hx_decode_set(kind, ptrs, len(tables), stream.data_ptr(),
+                               int(nbytes or stream.numel()),
+                               out.data_ptr() if n else stream.data_ptr(), n, status.data_ptr(),
+                               _stream(stream)), "hx_decode_set")
+    return out, status
+
+
+def _config(kind, history, lag, drift, lmax=12, max_distinct=4, seen_only=False):
+    return _SessionConfig(kind=kind, lmax=lmax if kind == KIND_HUFFMAN else 0,
+                          max_distinct=max_distinct if kind == KIND_QLC else 0,
+                          flags=CB_SEEN_ONLY if seen_only else 0, history=history, lag=lag,
+                          drift=float(drift))
+
+
+class Planner:
+    """hx_planner: the online loop's bookkeeping on the host (which codebook codes batch t)."""
+
+    def __init__(self, kind=KIND_HUFFMAN, history=4, lag=2, drift=0.0, initial_counts=None,
+                 **kw):
+        self._cfg = _config(kind, history, lag, drift, **kw)
+        init = None if initial_counts is None else _counts(initial_counts)
+        h = ctypes.c_void_p()
+        _check(lib().hx_planner_create(ctypes.byref(self._cfg),
+                                       None if init is None else init.ctypes.data,
+                                       ctypes.byref(h)), "hx_planner_create")
+        self._h = h
+
+    def codebook(self, batch: int) -> Codebook:
+        raw = _Codebook()
+        _check(lib().hx_planner_codebook(self._h, batch, ctypes.byref(raw)), "hx_planner_codebook")
+        return Codebook(raw)
+
+    def observe(self, batch: int, counts) -> tuple[bool, float]:
+        c = _counts(counts)
+        r, d = ctypes.c_int(), ctypes.c_double()
+        _check(lib().hx_planner_observe(self._h, batch, c.ctypes.data, ctypes.byref(r),
+                                        ctypes.byref(d)), "hx_planner_observe")
+        return bool(r.value), float(d.value)
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h and _lib is not None:
+            _lib.hx_planner_destroy(h)
+
+
+class Session:
+    """hx_session: encode a sequence of batches, each with the codebook of earlier batches'
+    fused histograms; decode picks the table by the stream's codebook hash. The table slots,
+    the histogram buffer and the status word are device tensors this object holds."""
+
+    def __init__(self, device, kind=KIND_HUFFMAN, history=4, lag=2, drift=0.0,
+                 initial_counts=None, slots=None, **kw):
+        import torch
+        self._cfg = _config(kind, history, lag, drift, **kw)
+        self.kind = kind
+        nslots = slots or min(MAX_TABLE_SET, lag + 2)
+        self.slots = [torch.empty(TABLES_BYTES, dtype=torch.uint8, device=device)
+                      for _ in range(nslots)]
+        self.hist = torch.zeros(256, dtype=torch.int32, device=device)
+        init = None if initial_counts is None else _counts(initial_counts)
+        ptrs = (ctypes.c_void_p * nslots)(*[t.data_ptr() for t in self.slots])
+        h = ctypes.c_void_p()
+        _check(lib().hx_session_create(ctypes.byref(self._cfg),
+                                       None if init is None else init.ctypes.data, ptrs, nslots,
+                                       ctypes.byref(h)), "hx_session_create")
+        self._h = h
+
+    def encode(self, x, out, scratch, status):
+        x = _dev_u8(x, "x")
+        _check(lib().hx_session_encode(self._h, x.data_ptr(), x.numel(), out.data_ptr(),
+                                       out.numel(), scratch.data_ptr(), self.hist.data_ptr(),
+                                       status.data_ptr(), _stream(x)), "hx_session_encode")
+        return out
+
+    def decode(self, stream, n: int, out, status, nbytes=None):
+        stream = _dev_u8(stream, "stream")
+        _check(lib().hx_session_decode(self._h, stream.data_ptr(), int(nbytes or stream.numel()),
+                                       out.data_ptr() if n else stream.data_ptr(), n,
+                                       status.data_ptr(), _stream(stream)), "hx_session_decode")
+        return out
+
+    def drain(self):
+        _check(lib().hx_session_drain(self._h), "hx_session_drain")
+
+    def info(self, batch: int) -> dict:
+        b = _BatchInfo()
+        _check(lib().hx_session_batch_info(self._h, batch, ctypes.byref(b)),
+               "hx_session_batch_info")
+        return {"hash": int(b.hash), "slot": int(b.slot), "observed": bool(b.observed),
+                "refreshed": bool(b.refreshed), "symbols": int(b.symbols),
+                "drift": float(b.drift)}
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h and _lib is not None:
+            _lib.hx_session_destroy(h)

@@ -185,3 +185,47 @@ def entropy(counts) -> float:
 def mean_length(counts, lengths) -> float:
     c = np.ascontiguousarray(np.asarray(counts, dtype=np.uint64))
     return float(lib().orc_mean_length(_p(c), _p(_u8(lengths))))
+
+
+def session_schedule(hists, kind: int = KIND_HUFFMAN, history: int = 4, lag: int = 2,
+                     drift: float = 0.0, initial_counts=None, lmax: int = 12,
+                     max_distinct: int = 4, cover_all: bool = True):
+    """The online single-stage loop, written out batch by batch.
+
+    "Single-Stage Huffman Encoder for ML Compression", abstract: a batch is coded with the
+    codebook of the average distribution of earlier batches. Batch t's codebook is built from the
+    summed histograms of the batches observed once batch t - lag has been observed (at most the
+    last `history` of them; `initial_counts`, or all ones, before any). Observing batch j computes
+    its drift, mean code length under the codebook that coded it over its entropy, minus one;
+    above `drift` (> 0) the history restarts from batch j (the drift refresh of the "Shannonic"
+    review). Returns (codebook per batch, (refreshed, drift) per batch)."""
+    init = np.ones(256, np.uint64) if initial_counts is None else np.asarray(initial_counts, np.uint64)
+
+    def build(c):
+        if kind == KIND_HUFFMAN:
+            return huffman_codebook(c, lmax, cover_all)
+        return qlc_codebook(c, max_distinct)
+
+    window, books, seen = [], [], []
+
+    def observe(j):
+        h = np.asarray(hists[j], np.uint64)
+        H = entropy(h)
+        d, refresh = float("nan"), False
+        if H > 0:
+            d = mean_length(h, books[j].len) / H - 1.0
+            refresh = drift > 0 and d > drift
+        if refresh:
+            window.clear()
+        window.append(h)
+        del window[:-history]
+        seen.append((refresh, d))
+
+    for t in range(len(hists)):
+        if t >= lag:
+            observe(t - lag)
+        counts = np.sum(window, axis=0, dtype=np.uint64) if window else init
+        books.append(build(counts))
+    for j in range(max(0, len(hists) - lag), len(hists)):
+        observe(j)
+    return books, seen
