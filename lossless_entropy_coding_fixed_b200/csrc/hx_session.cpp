@@ -12,11 +12,14 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <condition_variable>
 #include <cstring>
 #include <deque>
 #include <limits>
 #include <map>
+#include <mutex>
 #include <new>
+#include <thread>
 #include <vector>
 
 #include "hx.h"
@@ -31,8 +34,12 @@ struct hx_planner {
   hx_codebook current;
 };
 
+// The session's host work (waiting for a batch's histogram, folding it into the plan, building
+// and packing the next codebook) runs on a worker thread, so the calling thread only enqueues
+// device work; hx_session_encode(t) waits only if batch t's codebook is not ready yet.
 struct hx_session {
-  hx_planner plan;
+  hx_planner plan;  // the worker's
+  int device = 0;
   void* slots[HX_MAX_TABLE_SET];        // device table blocks (caller's memory)
   uint64_t slot_hash[HX_MAX_TABLE_SET];  // 0 = empty
   uint32_t nslots = 0, cur = 0;
@@ -40,8 +47,21 @@ struct hx_session {
   uint32_t* hist_host = nullptr;        // pinned: lag + 1 histograms in flight
   cudaEvent_t* events = nullptr;        // one per in-flight histogram
   uint32_t ring = 0;                    // lag + 1
-  uint64_t batch = 0;                   // next batch to encode
+  uint64_t batch = 0;                   // next batch to encode (caller's thread)
+
+  struct Ready {
+    hx_codebook cb;
+    std::vector<unsigned char> tables;
+  };
+  std::mutex mu;
+  std::condition_variable cv;
+  uint64_t enqueued = 0;             // batches whose histogram copy is enqueued
+  uint64_t folded = 0;               // batches the worker has folded
+  std::map<uint64_t, Ready> ready;   // codebooks built for batches not yet encoded
   std::vector<hx_batch_info> info;
+  int error = HX_OK;                 // first error of the worker
+  bool stop = false;
+  std::thread worker;
 };
 
 namespace {
@@ -116,27 +136,71 @@ int planner_observe(hx_planner* p, uint64_t j, const uint64_t* counts, int* refr
   return HX_OK;
 }
 
-// Folds the histogram of batch j (its copy to pinned memory has been enqueued) into the plan.
+// Worker: builds and packs the codebook of batch t into the ready map.
+int session_prepare(hx_session* s, uint64_t t) {
+  hx_session::Ready r;
+  int rc = planner_codebook(&s->plan, t, &r.cb);
+  if (rc) return rc;
+  r.tables.resize(HX_TABLES_BYTES);
+  rc = hx_codebook_tables(&r.cb, r.tables.data());
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(s->mu);
+  s->ready.emplace(t, std::move(r));
+  return HX_OK;
+}
+
+// Worker: folds the histogram of batch j (its copy to pinned memory has been enqueued).
 int session_fold(hx_session* s, uint64_t j) {
   const uint32_t r = (uint32_t)(j % s->ring);
   if (cudaEventSynchronize(s->events[r]) != cudaSuccess) return HX_ERR_CUDA;
   uint64_t counts[256];
-  for (int v = 0; v < 256; ++v) counts[v] = s->hist_host[r * 256 + v];
+  uint64_t total = 0;
+  for (int v = 0; v < 256; ++v) total += counts[v] = s->hist_host[r * 256 + v];
   int refreshed = 0;
   double drift = 0;
   const int rc = planner_observe(&s->plan, j, counts, &refreshed, &drift);
   if (rc) return rc;
+  std::lock_guard<std::mutex> lock(s->mu);
   hx_batch_info& b = s->info[j];
   b.observed = 1;
   b.refreshed = refreshed;
   b.drift = drift;
-  uint64_t total = 0;
-  for (int v = 0; v < 256; ++v) total += counts[v];
   b.symbols = total;
   return HX_OK;
 }
 
+void session_worker(hx_session* s) {
+  cudaSetDevice(s->device);
+  int rc = HX_OK;
+  // batches 0 .. lag-1 are coded before any histogram is back
+  for (uint64_t t = 0; t < s->plan.cfg.lag && rc == HX_OK; ++t) rc = session_prepare(s, t);
+  for (uint64_t j = 0; rc == HX_OK; ++j) {
+    {
+      std::unique_lock<std::mutex> lock(s->mu);
+      s->cv.notify_all();
+      s->cv.wait(lock, [&] { return s->enqueued > j || s->stop; });
+      if (s->enqueued <= j) break;  // stopped with nothing left to fold
+    }
+    rc = session_fold(s, j);
+    if (rc == HX_OK) rc = session_prepare(s, j + s->plan.cfg.lag);
+    std::lock_guard<std::mutex> lock(s->mu);
+    s->folded = j + 1;
+  }
+  std::lock_guard<std::mutex> lock(s->mu);
+  if (rc != HX_OK && s->error == HX_OK) s->error = rc;
+  s->stop = true;
+  s->cv.notify_all();
+}
+
 void session_free(hx_session* s) {
+  if (s->worker.joinable()) {
+    {
+      std::lock_guard<std::mutex> lock(s->mu);
+      s->stop = true;
+    }
+    s->cv.notify_all();
+    s->worker.join();
+  }
   if (s->events)
     for (uint32_t i = 0; i < s->ring; ++i)
       if (s->events[i]) cudaEventDestroy(s->events[i]);
@@ -220,6 +284,16 @@ int hx_session_create(const hx_session_config* cfg, const uint64_t* initial_coun
       session_free(s);
       return HX_ERR_CUDA;
     }
+  if (cudaGetDevice(&s->device) != cudaSuccess) {
+    session_free(s);
+    return HX_ERR_CUDA;
+  }
+  try {
+    s->worker = std::thread(session_worker, s);
+  } catch (...) {
+    session_free(s);
+    return HX_ERR_ARG;
+  }
   *out = s;
   return HX_OK;
 }
@@ -234,26 +308,27 @@ int hx_session_encode(hx_session* s, const uint8_t* d_in, uint64_t n, void* d_ou
   if (!s || !d_hist) return HX_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const uint64_t t = s->batch;
-  const uint32_t lag = s->plan.cfg.lag;
-  // 1. the histograms this batch's codebook averages: batches up to t - lag
-  while (t >= lag && s->plan.next_obs <= t - lag) {
-    const int rc = session_fold(s, s->plan.next_obs);
-    if (rc) return rc;
+  // 1. batch t's codebook, built by the worker from the histograms up to batch t - lag
+  hx_session::Ready r;
+  {
+    std::unique_lock<std::mutex> lock(s->mu);
+    s->cv.wait(lock, [&] { return s->ready.count(t) || s->stop; });
+    auto it = s->ready.find(t);
+    if (it == s->ready.end()) return s->error ? s->error : HX_ERR_ARG;
+    r = std::move(it->second);
+    s->ready.erase(it);
   }
-  // 2. the codebook, uploaded to the next slot when it changed
-  hx_codebook cb;
-  int rc = planner_codebook(&s->plan, t, &cb);
-  if (rc) return rc;
-  if (s->slot_hash[s->cur] != cb.hash) {
+  // 2. uploaded to the next slot when it changed
+  int rc;
+  if (s->slot_hash[s->cur] != r.cb.hash) {
     const uint32_t next = s->slot_hash[s->cur] == 0 ? s->cur : (s->cur + 1) % s->nslots;
     unsigned char* host = s->staging + (size_t)next * HX_TABLES_BYTES;
-    rc = hx_codebook_tables(&cb, host);
-    if (rc) return rc;
+    std::memcpy(host, r.tables.data(), HX_TABLES_BYTES);
     if (cudaMemcpyAsync(s->slots[next], host, HX_TABLES_BYTES, cudaMemcpyHostToDevice, st) !=
         cudaSuccess)
       return HX_ERR_CUDA;
     s->cur = next;
-    s->slot_hash[next] = cb.hash;
+    s->slot_hash[next] = r.cb.hash;
   }
   // 3. encode with it, counting this batch's histogram
   if (cudaMemsetAsync(d_hist, 0, 256 * sizeof(uint32_t), st) != cudaSuccess) return HX_ERR_CUDA;
@@ -263,17 +338,22 @@ int hx_session_encode(hx_session* s, const uint8_t* d_in, uint64_t n, void* d_ou
            : hx_qlc_encode(s->slots[s->cur], d_in, n, d_out, out_cap, d_scratch, d_hist,
                            d_status, stream);
   if (rc) return rc;
-  // 4. the histogram goes to the host for the batch lag batches later
-  const uint32_t r = (uint32_t)(t % s->ring);
-  if (cudaMemcpyAsync(s->hist_host + (size_t)r * 256, d_hist, 256 * sizeof(uint32_t),
+  // 4. the histogram goes to the host, where the worker folds it
+  const uint32_t ri = (uint32_t)(t % s->ring);
+  if (cudaMemcpyAsync(s->hist_host + (size_t)ri * 256, d_hist, 256 * sizeof(uint32_t),
                       cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaEventRecord(s->events[r], st) != cudaSuccess)
+      cudaEventRecord(s->events[ri], st) != cudaSuccess)
     return HX_ERR_CUDA;
   hx_batch_info b{};
-  b.hash = cb.hash;
+  b.hash = r.cb.hash;
   b.slot = s->cur;
   b.drift = std::numeric_limits<double>::quiet_NaN();
-  s->info.push_back(b);
+  {
+    std::lock_guard<std::mutex> lock(s->mu);
+    s->info.push_back(b);
+    s->enqueued = t + 1;
+  }
+  s->cv.notify_all();
   s->batch = t + 1;
   return HX_OK;
 }
@@ -287,16 +367,17 @@ int hx_session_decode(hx_session* s, const void* d_stream, uint64_t stream_bytes
 
 int hx_session_drain(hx_session* s) {
   if (!s) return HX_ERR_ARG;
-  while (s->plan.next_obs < s->batch) {
-    const int rc = session_fold(s, s->plan.next_obs);
-    if (rc) return rc;
-  }
-  return HX_OK;
+  std::unique_lock<std::mutex> lock(s->mu);
+  s->cv.wait(lock, [&] { return s->folded >= s->enqueued || s->stop; });
+  return s->error;
 }
 
 int hx_session_batch_info(const hx_session* s, uint64_t batch, hx_batch_info* out) {
-  if (!s || !out || batch >= s->info.size()) return HX_ERR_ARG;
-  *out = s->info[batch];
+  if (!s || !out) return HX_ERR_ARG;
+  hx_session* m = const_cast<hx_session*>(s);
+  std::lock_guard<std::mutex> lock(m->mu);
+  if (batch >= m->info.size()) return HX_ERR_ARG;
+  *out = m->info[batch];
   return HX_OK;
 }
 
