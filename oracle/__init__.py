@@ -18,7 +18,8 @@ SRC = os.path.join(HERE, "oracle.cpp")
 LIB = os.path.join(HERE, "liboracle.so")
 
 ERR_ARG, ERR_UNCODABLE, ERR_CORRUPT, ERR_CODEBOOK, ERR_CAPACITY = 1, 4, 8, 16, 64
-KIND_HUFFMAN, KIND_QLC = 0, 1
+KIND_HUFFMAN, KIND_QLC, KIND_SHANNONIC = 0, 1, 2
+SHN_K, SHN_L, SHN_R = 16, 128, 7
 QLC_LMAX = 11
 
 _lib = None
@@ -57,6 +58,13 @@ def lib():
             "orc_entropy": (ctypes.c_double, [P]),
             "orc_fnv1a": (u64, [P, u64]),
             "orc_mean_length": (ctypes.c_double, [P, P]),
+            "orc_shannonic_build": (i32, [P, i32, i32, P, P, P]),
+            "orc_shannonic_partition": (i32, [P, i32, i32, P]),
+            "orc_shannonic_normalise": (i32, [P, i32, P]),
+            "orc_hash_shannonic": (u64, [i32, P, P]),
+            "orc_shannonic_encode_bound": (u64, [u64]),
+            "orc_encode_shannonic": (i32, [i32, P, P, P, u64, P, u64, P]),
+            "orc_decode_shannonic": (i32, [i32, P, P, P, u64, P, u64]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -145,9 +153,64 @@ def encode_bound(n: int) -> int:
     return int(lib().orc_encode_bound(n))
 
 
-def encode(cb: Codebook, x, cap: int | None = None) -> tuple[int, np.ndarray]:
+@dataclass
+class ShannonicBook:
+    """[SHN] ranges lo[0..nr] over the byte values and their tANS frequencies f (sum 128)."""
+    nr: int
+    lo: np.ndarray  # i32[nr + 1]
+    f: np.ndarray   # i32[nr]
+    kind: int = KIND_SHANNONIC
+
+    @property
+    def hash(self) -> int:
+        return int(lib().orc_hash_shannonic(self.nr, _p(self.lo), _p(self.f)))
+
+    @property
+    def offset_bits(self) -> np.ndarray:
+        return np.array([int(np.ceil(np.log2(b - a))) if b - a > 1 else 0
+                         for a, b in zip(self.lo[:-1], self.lo[1:])])
+
+
+def shannonic_codebook(counts, K: int = SHN_K, cover_all: bool = True) -> ShannonicBook:
+    c = np.ascontiguousarray(np.asarray(counts, dtype=np.uint64))
+    nr = ctypes.c_int()
+    lo = np.zeros(SHN_K + 1, np.int32)
+    f = np.zeros(SHN_K, np.int32)
+    if lib().orc_shannonic_build(_p(c), int(K), int(cover_all), ctypes.byref(nr), _p(lo), _p(f)):
+        raise ValueError("no Shannonic codebook for these counts")
+    k = nr.value
+    return ShannonicBook(k, lo[:k + 1].copy(), f[:k].copy())
+
+
+def shannonic_partition(weights, K: int) -> np.ndarray:
+    """The dynamic programme's partition of any alphabet (boundaries lo[0..nr])."""
+    w = np.ascontiguousarray(np.asarray(weights, dtype=np.uint64))
+    lo = np.zeros(K + 1, np.int32)
+    k = lib().orc_shannonic_partition(_p(w), w.size, int(K), _p(lo))
+    return lo[:k + 1].copy()
+
+
+def shannonic_normalise(range_weights) -> np.ndarray:
+    wr = np.ascontiguousarray(np.asarray(range_weights, dtype=np.uint64))
+    f = np.zeros(wr.size, np.int32)
+    lib().orc_shannonic_normalise(_p(wr), wr.size, _p(f))
+    return f
+
+
+def shannonic_encode_bound(n: int) -> int:
+    return int(lib().orc_shannonic_encode_bound(n))
+
+
+def encode(cb, x, cap: int | None = None) -> tuple[int, np.ndarray]:
     """Bit-serial encode into the chunked stream; returns (status, stream bytes)."""
     x = _u8(x)
+    if cb.kind == KIND_SHANNONIC:
+        cap = shannonic_encode_bound(x.size) if cap is None else int(cap)
+        out = np.zeros(max(cap, 1), dtype=np.uint8)
+        written = ctypes.c_uint64(0)
+        st = lib().orc_encode_shannonic(cb.nr, _p(cb.lo), _p(cb.f), _p(x), x.size, _p(out), cap,
+                                        ctypes.byref(written))
+        return int(st), out[: written.value] if written.value else out[: min(cap, 64)]
     cap = encode_bound(x.size) if cap is None else int(cap)
     out = np.zeros(max(cap, 1), dtype=np.uint8)
     written = ctypes.c_uint64(0)
@@ -160,11 +223,13 @@ def encode(cb: Codebook, x, cap: int | None = None) -> tuple[int, np.ndarray]:
     return int(st), out[: written.value] if written.value else out[: min(cap, 64)]
 
 
-def decode(cb: Codebook, stream, n: int) -> tuple[int, np.ndarray]:
+def decode(cb, stream, n: int) -> tuple[int, np.ndarray]:
     """Bit-serial decode; returns (status, n bytes)."""
     s = _u8(stream)
     out = np.zeros(max(n, 1), dtype=np.uint8)
-    if cb.kind == KIND_HUFFMAN:
+    if cb.kind == KIND_SHANNONIC:
+        st = lib().orc_decode_shannonic(cb.nr, _p(cb.lo), _p(cb.f), _p(s), s.size, _p(out), n)
+    elif cb.kind == KIND_HUFFMAN:
         st = lib().orc_decode_huffman(cb.lmax, _p(cb.len), _p(s), s.size, _p(out), n)
     else:
         st = lib().orc_decode_qlc(_p(cb.bits), _p(cb.start), _p(cb.rank2sym), _p(s), s.size,

@@ -14,6 +14,11 @@
 //         probability and codes them with a fixed number of index bits.
 //   [PM]  Larmore & Hirschberg (1990), package-merge for length-limited prefix codes.
 //   [RFC] RFC 1951 section 3.2.2, canonical Huffman codes from code lengths.
+//   [SHN] the "Shannonic" review page (method and runtime sections): the 256 byte values split
+//         by dynamic programming into at most K = 16 contiguous ranges that minimise the range
+//         entropy plus the fixed-width offset bits; the range index is coded by 128-state tANS
+//         (J. Duda, asymmetric numeral systems, table variant), the offset in ceil(log2 size)
+//         bits.
 //
 // Readings where the pages are silent (all stated once more in the design notes):
 //   - averaging over equal-size batches == summing their counts; every byte gets a code
@@ -384,6 +389,301 @@ int decode(const Header& h, const Dec& dec, const uint8_t* st, uint64_t bytes, u
   return status;
 }
 
+// ---- [SHN] range partition + 128-state tANS --------------------------------------------------
+// Readings (the page gives the objective, K = 16 and L = 128, not the details):
+//   - ranges are contiguous in byte value; weights max(count, 1) (every byte codable); at most K
+//     ranges; cost of range [a, b) with weight W_ab (of W in all) is
+//     W_ab * log2(W / W_ab) + W_ab * ceil(log2(b - a)), summed; the dynamic programme takes, for
+//     each prefix, the smallest split point reaching the strict minimum, and the smallest range
+//     count reaching it;
+//   - tANS frequencies: f_r = max(1, floor(W_r L / W)); a shortfall goes +1 at a time to the
+//     largest remainders W_r L mod W (ties to the lower range, cycling), an excess -1 at a time
+//     from the largest f_r > 1 (ties to the lower range);
+//   - spread: positions 0, 83, 166 mod 128, ... (step L/2 + L/8 + 3) take range 0 f_0 times,
+//     then range 1, ...; decoding state L + u holds range spread[u], and the k-th state of range
+//     r (in increasing u) is reached from x_s = f_r + k;
+//   - a sub-stream is encoded from its last symbol to its first, starting in state L: the offset
+//     (ceil(log2 size) bits), then the low nb bits of the state (nb making state >> nb fall in
+//     [f_r, 2 f_r)), then the state becomes the k-th state of the range, k = (state >> nb) - f_r;
+//     after the first symbol the state minus L goes out in 7 bits. Bits are appended MSB-first,
+//     so a decoder reads each sub-stream backwards from its end and must finish in state L
+//     exactly at the sub-stream's first bit.
+constexpr int kShR = 7, kShL = 1 << kShR, kShK = 16, kShStep = kShL / 2 + kShL / 8 + 3;
+constexpr uint8_t kKindShannonic = 2;
+
+int ceil_log2(int v) {
+  int b = 0;
+  while ((1 << b) < v) ++b;
+  return b;
+}
+
+// Optimal partition of weights[0..n) into at most K contiguous ranges; lo[0..nr] boundaries.
+int partition(const uint64_t* w, int n, int K, int* lo) {
+  std::vector<uint64_t> P(n + 1, 0);
+  for (int i = 0; i < n; ++i) P[i + 1] = P[i] + w[i];
+  const double W = (double)P[n];
+  auto cost = [&](int a, int b) {
+    const uint64_t wab = P[b] - P[a];
+    if (wab == 0) return 0.0;
+    return (double)wab * std::log2(W / (double)wab) + (double)wab * (double)ceil_log2(b - a);
+  };
+  const double inf = 1e300;
+  std::vector<std::vector<double>> best(K + 1, std::vector<double>(n + 1, inf));
+  std::vector<std::vector<int>> from(K + 1, std::vector<int>(n + 1, -1));
+  for (int b = 1; b <= n; ++b) best[1][b] = cost(0, b), from[1][b] = 0;
+  for (int k = 2; k <= K; ++k)
+    for (int b = k; b <= n; ++b)
+      for (int a = k - 1; a < b; ++a) {
+        const double c = best[k - 1][a] + cost(a, b);
+        if (c < best[k][b]) best[k][b] = c, from[k][b] = a;
+      }
+  int kbest = 1;
+  for (int k = 2; k <= K && k <= n; ++k)
+    if (best[k][n] < best[kbest][n]) kbest = k;
+  int b = n;
+  for (int k = kbest; k >= 1; --k) {
+    lo[k] = b;
+    b = from[k][b];
+  }
+  lo[0] = 0;
+  return kbest;
+}
+
+struct Shn {
+  int nr;
+  int lo[kShK + 1];
+  int f[kShK];
+  int spread[kShL];
+  int range_of[256];
+};
+
+void shn_tables(Shn& t) {
+  int pos = 0;
+  for (int r = 0; r < t.nr; ++r)
+    for (int j = 0; j < t.f[r]; ++j) {
+      t.spread[pos] = r;
+      pos = (pos + kShStep) % kShL;
+    }
+  for (int r = 0; r < t.nr; ++r)
+    for (int v = t.lo[r]; v < t.lo[r + 1]; ++v) t.range_of[v] = r;
+}
+
+void normalise(const uint64_t* wr, int nr, int* f) {
+  uint64_t W = 0;
+  for (int r = 0; r < nr; ++r) W += wr[r];
+  int sum = 0;
+  std::vector<uint64_t> rem(nr);
+  for (int r = 0; r < nr; ++r) {
+    const uint64_t q = wr[r] * kShL / W;
+    rem[r] = wr[r] * kShL - q * W;
+    f[r] = std::max<int>(1, (int)q);
+    sum += f[r];
+  }
+  while (sum < kShL) {  // largest remainder first, ties to the lower range; then cycle
+    std::vector<int> order(nr);
+    for (int r = 0; r < nr; ++r) order[r] = r;
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return rem[a] > rem[b]; });
+    for (int i = 0; i < nr && sum < kShL; ++i) ++f[order[i]], ++sum;
+  }
+  while (sum > kShL) {
+    int big = -1;
+    for (int r = 0; r < nr; ++r)
+      if (f[r] > 1 && (big < 0 || f[r] > f[big])) big = r;
+    --f[big];
+    --sum;
+  }
+}
+
+bool shn_build(const uint64_t* counts, int K, bool cover_all, Shn& t) {
+  uint64_t w[256];
+  for (int s = 0; s < 256; ++s) w[s] = cover_all ? std::max<uint64_t>(counts[s], 1) : counts[s];
+  uint64_t W = 0;
+  for (int s = 0; s < 256; ++s) W += w[s];
+  if (W == 0 || K < 1 || K > kShK) return false;
+  t.nr = partition(w, 256, K, t.lo);
+  uint64_t wr[kShK] = {0};
+  for (int r = 0; r < t.nr; ++r)
+    for (int v = t.lo[r]; v < t.lo[r + 1]; ++v) wr[r] += w[v];
+  for (int r = 0; r < t.nr; ++r)
+    if (wr[r] == 0) return false;  // seen-only weights left a range empty
+  normalise(wr, t.nr, t.f);
+  shn_tables(t);
+  return true;
+}
+
+uint64_t shn_hash(const Shn& t) {
+  std::vector<uint8_t> b = {kKindShannonic, (uint8_t)kShR, (uint8_t)t.nr};
+  for (int r = 1; r < t.nr; ++r) b.push_back((uint8_t)t.lo[r]);
+  for (int r = 0; r < t.nr; ++r) b.push_back((uint8_t)t.f[r]);
+  return fnv1a(b);
+}
+
+// The k-th decoding state of range r (k from 0, increasing u).
+int shn_state_of(const Shn& t, int r, int k) {
+  for (int u = 0; u < kShL; ++u)
+    if (t.spread[u] == r && k-- == 0) return kShL + u;
+  return -1;
+}
+
+int floor_log2(int v) {
+  int b = -1;
+  while (v) v >>= 1, ++b;
+  return b;
+}
+
+void shn_encode_substream(const Shn& t, const uint8_t* x, uint64_t m, BitWriter& bw) {
+  int state = kShL;
+  for (uint64_t i = m; i-- > 0;) {
+    const int s = x[i], r = t.range_of[s];
+    bw.put((uint32_t)(s - t.lo[r]), ceil_log2(t.lo[r + 1] - t.lo[r]));
+    int nb = 0;
+    while ((state >> nb) >= 2 * t.f[r]) ++nb;  // state >> nb lands in [f_r, 2 f_r)
+    bw.put((uint32_t)(state & ((1 << nb) - 1)), nb);
+    state = shn_state_of(t, r, (state >> nb) - t.f[r]);
+  }
+  bw.put((uint32_t)(state - kShL), kShR);
+}
+
+struct BackReader {  // reads a sub-stream from its end towards its first bit
+  const uint8_t* payload;
+  uint64_t start, pos;
+  bool past = false;
+  uint32_t get(int nb) {
+    if (pos - start < (uint64_t)nb) { past = true; return 0; }
+    uint32_t v = 0;
+    for (uint64_t q = pos - nb; q < pos; ++q)
+      v = (v << 1) | ((rd32(payload + 4 * (q / 32)) >> (31 - q % 32)) & 1u);
+    pos -= nb;
+    return v;
+  }
+};
+
+// Decodes m symbols of a sub-stream occupying chunk bits [start, end); false if it is not one.
+bool shn_decode_substream(const Shn& t, const uint8_t* payload, uint64_t start, uint64_t end,
+                          uint8_t* out, uint64_t m) {
+  int next[kShK];
+  for (int r = 0; r < t.nr; ++r) next[r] = t.f[r];
+  int dec_xs[kShL];  // x_s of each decoding state
+  for (int u = 0; u < kShL; ++u) dec_xs[u] = next[t.spread[u]]++;
+  BackReader br{payload, start, end};
+  int state = kShL + (int)br.get(kShR);
+  for (uint64_t i = 0; i < m; ++i) {
+    const int u = state - kShL, r = t.spread[u], xs = dec_xs[u];
+    const int nb = kShR - floor_log2(xs);
+    const int low = (int)br.get(nb);
+    const int off = (int)br.get(ceil_log2(t.lo[r + 1] - t.lo[r]));
+    if (br.past || t.lo[r] + off >= t.lo[r + 1]) return false;
+    out[i] = (uint8_t)(t.lo[r] + off);
+    state = (xs << nb) + low;
+  }
+  return state == kShL && br.pos == start;
+}
+
+int shn_encode(const Shn& t, const uint8_t* x, uint64_t n, uint8_t* out, uint64_t cap,
+               uint64_t* written) {
+  const uint64_t nc = n_chunks_of(n), S = sync_offset(n), P = payload_offset(n);
+  *written = 0;
+  if (cap < P) return kErrCapacity;
+  std::vector<uint32_t> word_off(nc + 1, 0);
+  std::vector<uint16_t> sync(nc * kSubstreams, 0);
+  std::vector<uint32_t> payload;
+  for (uint64_t c = 0; c < nc; ++c) {
+    BitWriter bw;
+    const uint64_t lo = c * kChunk, hi = std::min(n, lo + kChunk);
+    const uint64_t nsub = (hi - lo + kSubLen - 1) / kSubLen;
+    uint16_t starts[kSubstreams] = {0};
+    for (uint64_t k = 0; k < nsub; ++k) {
+      starts[k] = (uint16_t)bw.nbits;
+      const uint64_t a = lo + k * kSubLen, b = std::min(hi, a + kSubLen);
+      shn_encode_substream(t, x + a, b - a, bw);
+    }
+    sync[c * kSubstreams + 0] = (uint16_t)bw.nbits;
+    for (uint64_t k = 1; k < kSubstreams; ++k)
+      sync[c * kSubstreams + k] = k < nsub ? starts[k] : (uint16_t)bw.nbits;
+    word_off[c] = (uint32_t)payload.size();
+    payload.insert(payload.end(), bw.words.begin(), bw.words.end());
+  }
+  word_off[nc] = (uint32_t)payload.size();
+  const uint64_t total = payload.size();
+  const uint64_t need = P + 4 * (total + 2);
+  std::memset(out, 0, (size_t)std::min<uint64_t>(cap, P));
+  wr32(out + 0, kMagic);
+  out[4] = kVersion;
+  out[5] = kKindShannonic;
+  out[6] = (uint8_t)kShR;
+  out[7] = 0;
+  wr32(out + 8, (uint32_t)kChunk);
+  wr32(out + 12, (uint32_t)kSubstreams);
+  wr64(out + 16, n);
+  wr64(out + 24, nc);
+  wr64(out + 32, total);
+  wr64(out + 40, shn_hash(t));
+  if (need > cap) return kErrCapacity;
+  for (uint64_t c = 0; c <= nc; ++c) wr32(out + 64 + 4 * c, word_off[c]);
+  for (uint64_t i = 0; i < nc * kSubstreams; ++i) wr16(out + S + 2 * i, sync[i]);
+  for (uint64_t w = 0; w < total; ++w) wr32(out + P + 4 * w, payload[w]);
+  wr32(out + P + 4 * total, 0);
+  wr32(out + P + 4 * total + 4, 0);
+  *written = need;
+  return 0;
+}
+
+int shn_decode(const Shn& t, const uint8_t* st, uint64_t bytes, uint8_t* out, uint64_t n_expected) {
+  if (bytes < 64) return kErrCorrupt;
+  if (rd32(st) != kMagic || st[4] != kVersion || rd32(st + 8) != kChunk ||
+      rd32(st + 12) != kSubstreams)
+    return kErrCorrupt;
+  if (st[5] != kKindShannonic || st[6] != kShR || rd64(st + 40) != shn_hash(t)) return kErrCodebook;
+  const uint64_t n = rd64(st + 16);
+  if (n != n_expected || rd64(st + 24) != n_chunks_of(n)) return kErrCorrupt;
+  const uint64_t nc = n_chunks_of(n), S = sync_offset(n), P = payload_offset(n);
+  const uint64_t total = rd64(st + 32);
+  if (P > bytes || (bytes - P) / 4 < 2 || total > (bytes - P) / 4 - 2 || total >= (1ull << 32))
+    return kErrCorrupt;
+  int status = 0;
+  for (uint64_t c = 0; c < nc; ++c) {
+    const uint64_t lo = c * kChunk, hi = std::min(n, lo + kChunk);
+    const uint32_t w0 = rd32(st + 64 + 4 * c), w1 = rd32(st + 64 + 4 * (c + 1));
+    const uint8_t* sy = st + S + 16 * c;
+    const uint64_t nbits = rd16(sy);
+    if (w0 > w1 || w1 > total || nbits > 32ull * (w1 - w0) || (nbits + 31) / 32 != w1 - w0) {
+      status |= kErrCorrupt;
+      continue;
+    }
+    const uint64_t nsub = (hi - lo + kSubLen - 1) / kSubLen;
+    bool bad = false;
+    for (uint64_t k = 0; k < kSubstreams && !bad; ++k) {
+      const uint64_t a = k == 0 ? 0 : rd16(sy + 2 * k);
+      if (k >= nsub) {
+        if (k > 0 && a != nbits) bad = true;
+        continue;
+      }
+      const uint64_t b = k + 1 < nsub ? rd16(sy + 2 * (k + 1)) : nbits;
+      const uint64_t s0 = lo + k * kSubLen, s1 = std::min(hi, s0 + kSubLen);
+      if (a > b || b > nbits ||
+          !shn_decode_substream(t, st + P + 4ull * w0, a, b, out + s0, s1 - s0))
+        bad = true;
+    }
+    if (bad) status |= kErrCorrupt;
+  }
+  return status;
+}
+
+bool shn_from(int nr, const int* lo, const int* f, Shn& t) {
+  if (nr < 1 || nr > kShK || lo[0] != 0 || lo[nr] != 256) return false;
+  int sum = 0;
+  for (int r = 0; r < nr; ++r) {
+    if (lo[r + 1] <= lo[r] || f[r] < 1) return false;
+    sum += f[r];
+  }
+  if (sum != kShL) return false;
+  t.nr = nr;
+  for (int r = 0; r <= nr; ++r) t.lo[r] = lo[r];
+  for (int r = 0; r < nr; ++r) t.f[r] = f[r];
+  shn_tables(t);
+  return true;
+}
+
 }  // namespace
 
 // ================================ C entry points (ctypes) ====================================
@@ -500,6 +800,46 @@ double orc_mean_length(const uint64_t* counts, const uint8_t* len) {
     bits += (double)counts[s] * len[s];
   }
   return total ? bits / total : 0;
+}
+
+// [SHN] builder, partition (for any alphabet size, so tests can search small ones exhaustively),
+// hash, bound, encode and decode. lo: nr + 1 boundaries, f: nr frequencies (sum 128).
+int orc_shannonic_build(const uint64_t* counts, int K, int cover_all, int* nr, int* lo, int* f) {
+  Shn t;
+  if (!counts || !nr || !lo || !f || !shn_build(counts, K, cover_all != 0, t)) return kErrArg;
+  *nr = t.nr;
+  for (int r = 0; r <= t.nr; ++r) lo[r] = t.lo[r];
+  for (int r = 0; r < t.nr; ++r) f[r] = t.f[r];
+  return 0;
+}
+int orc_shannonic_partition(const uint64_t* w, int n, int K, int* lo) {
+  if (!w || !lo || n < 1 || K < 1) return -1;
+  return partition(w, n, K, lo);
+}
+int orc_shannonic_normalise(const uint64_t* wr, int nr, int* f) {
+  if (!wr || !f || nr < 1 || nr > kShL) return kErrArg;
+  normalise(wr, nr, f);
+  return 0;
+}
+uint64_t orc_hash_shannonic(int nr, const int* lo, const int* f) {
+  Shn t;
+  return shn_from(nr, lo, f, t) ? shn_hash(t) : 0;
+}
+uint64_t orc_shannonic_encode_bound(uint64_t n) {
+  // per sub-stream at most 512 * (8 offset + 7 state) + 7 bits: 1922 words per chunk
+  return payload_offset(n) + 4 * (n_chunks_of(n) * 1922 + 2);
+}
+int orc_encode_shannonic(int nr, const int* lo, const int* f, const uint8_t* x, uint64_t n,
+                         uint8_t* out, uint64_t cap, uint64_t* written) {
+  Shn t;
+  if (!shn_from(nr, lo, f, t)) return kErrArg;
+  return shn_encode(t, x, n, out, cap, written);
+}
+int orc_decode_shannonic(int nr, const int* lo, const int* f, const uint8_t* stream,
+                         uint64_t bytes, uint8_t* out, uint64_t n) {
+  Shn t;
+  if (!shn_from(nr, lo, f, t)) return kErrArg;
+  return shn_decode(t, stream, bytes, out, n);
 }
 
 }  // extern "C"
