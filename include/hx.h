@@ -58,7 +58,8 @@ typedef enum {
   HX_ERR_CAPACITY = 64   /* encode: out_cap is too small; header.total_words holds the need */
 } hx_status;
 
-enum { HX_KIND_HUFFMAN = 0, HX_KIND_QLC = 1 };
+enum { HX_KIND_HUFFMAN = 0, HX_KIND_QLC = 1, HX_KIND_SHANNONIC = 2 };
+enum { HX_SHN_K = 16, HX_SHN_L = 128, HX_SHN_R = 7 }; /* Shannonic: ranges, tANS states, log2 L */
 enum { HX_CHUNK = 4096, HX_SUBSTREAMS = 8, HX_LMAX_MAX = 12, HX_QLC_LMAX = 11 };
 enum { HX_CB_SEEN_ONLY = 1 }; /* hx_build_codebook flag: no code for bytes with count 0 */
 
@@ -77,8 +78,12 @@ typedef struct {
   uint16_t qlc_start[9]; /* QLC only                                                      */
   uint8_t rank2sym[256]; /* QLC only                                                      */
   uint64_t hash;         /* FNV-1a-64 of [kind, lmax, len[256]] (Huffman) or of
-                            [kind, 11, qlc_bits[8], rank2sym[256]] (QLC); the stream header
-                            carries it in place of the codebook                            */
+                            [kind, 11, qlc_bits[8], rank2sym[256]] (QLC) or of
+                            [kind, 7, nr, lo[1..nr-1], f[0..nr)] (Shannonic, bytes); the stream
+                            header carries it in place of the codebook                     */
+  uint8_t sh_nr;         /* Shannonic only: number of ranges (1..16)                     */
+  uint16_t sh_lo[HX_SHN_K + 1]; /* range r holds byte values sh_lo[r] .. sh_lo[r+1]-1       */
+  uint8_t sh_f[HX_SHN_K]; /* tANS frequency of each range, summing to 128                 */
 } hx_codebook;
 
 /* Length-limited canonical Huffman codebook from summed counts.
@@ -98,6 +103,17 @@ int hx_build_codebook(const uint64_t* counts, int lmax, uint32_t flags, hx_codeb
  * distinct values (4 = "quad"; 1..8), and minimise the mean code length; ties go to the
  * lexicographically smallest width vector. flags must be 0. */
 int hx_qlc_build(const uint64_t* counts, int max_distinct, uint32_t flags, hx_codebook* out);
+
+/* Shannonic codebook from counts: the review page's range-partitioned coder. The 256 byte values
+ * are split by dynamic programming into at most K (1..16) contiguous ranges minimising the sum
+ * over ranges of W_r log2(W / W_r) + W_r ceil(log2 size_r) (range entropy plus fixed-width
+ * offset bits; weights max(count, 1)); ties go to the smallest split point, then the fewest
+ * ranges. The range index is coded by tANS with 128 states: frequencies
+ * f_r = max(1, floor(128 W_r / W)), a shortfall given +1 at a time to the largest remainders
+ * (ties to the lower range, cycling), an excess taken -1 at a time from the largest f_r > 1
+ * (ties to the lower range); states spread with step 83. The offset inside the range takes
+ * ceil(log2 size_r) bits. flags must be 0. */
+int hx_shannonic_build(const uint64_t* counts, int K, uint32_t flags, hx_codebook* out);
 
 /* Pack a codebook into the HX_TABLES_BYTES table block in host memory (host_tables). */
 int hx_codebook_tables(const hx_codebook* cb, void* host_tables);
@@ -180,6 +196,21 @@ int hx_encode_measure(uint32_t kind, const void* d_tables, const uint8_t* d_in, 
 int hx_encode_pack(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                    void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_status,
                    void* stream);
+
+/* Shannonic encode and decode (kind 2 tables): the same chunked stream, sub-stream framing and
+ * index as hx_encode; inside a sub-stream the bits come from tANS run from its last symbol to
+ * its first, starting in state 128: per symbol the offset (ceil(log2 size) bits), then the low
+ * nb bits of the state (nb making state >> nb fall in [f_r, 2 f_r)), then the range's next
+ * state; after the first symbol the final state minus 128 in 7 bits. The decoder reads each
+ * sub-stream backwards from its end and must finish in state 128 exactly at its first bit (else
+ * HX_ERR_CORRUPT). A sub-stream can take up to 15 bits per symbol: size d_out with
+ * hx_shannonic_encode_bound(n). Arguments, scratch, histogram and status as hx_encode. */
+uint64_t hx_shannonic_encode_bound(uint64_t n); /* P + 4*(1922*chunks + 2)                   */
+int hx_shannonic_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                        uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
+                        void* stream);
+int hx_shannonic_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
+                        uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream);
 
 /* Allocation-free encode. The pages have no counterpart to this call: it exists for callers
  * that cannot allocate device memory when they encode -- for example code that runs under a
@@ -268,7 +299,8 @@ void hx_session_destroy(hx_session* s);
 
 /* Measurement helpers (host, fp64). Shannon entropy -sum p log2 p of counts[256] in bits per
  * symbol ("Single-Stage Huffman Encoder for ML Compression", abstract: the ideal the fixed code
- * is compared with), and the mean code length sum count*len / sum count of a codebook. Both
+ * is compared with), and the mean code length sum count*len / sum count of a codebook (for a
+ * Shannonic codebook the tANS ideal, log2(128 / f_r) + offset bits per symbol of range r). Both
  * return 0 for an all-zero histogram and -1 for a null pointer. */
 double hx_entropy(const uint64_t* counts);
 double hx_mean_length(const uint64_t* counts, const hx_codebook* cb);

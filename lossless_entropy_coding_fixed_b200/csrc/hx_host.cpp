@@ -176,6 +176,146 @@ int fill_qlc(const uint64_t counts[256], int max_distinct, hx_codebook* out) {
   return HX_OK;
 }
 
+// ---- Shannonic: range partition + 128-state tANS (the review page's method) ------------------
+constexpr int kShR = HX_SHN_R, kShL = HX_SHN_L, kShK = HX_SHN_K;
+constexpr int kShStep = kShL / 2 + kShL / 8 + 3;  // 83: odd, so it visits every state
+
+int bits_for(int size) {  // ceil(log2 size)
+  int b = 0;
+  while ((1 << b) < size) ++b;
+  return b;
+}
+
+// Minimal sum over ranges of W_r log2(W / W_r) + W_r ceil(log2 size_r), over partitions of the
+// 256 values into at most K contiguous ranges. best[k][b]: the first b values in k ranges; the
+// split point and range count are the smallest reaching the strict minimum.
+int shannonic_partition(const uint64_t w[256], int K, uint16_t lo[kShK + 1]) {
+  uint64_t pre[257];
+  pre[0] = 0;
+  for (int v = 0; v < 256; ++v) pre[v + 1] = pre[v] + w[v];
+  const double W = (double)pre[256];
+  auto cost = [&](int a, int b) -> double {
+    const uint64_t wab = pre[b] - pre[a];
+    if (wab == 0) return 0.0;
+    return (double)wab * std::log2(W / (double)wab) + (double)wab * (double)bits_for(b - a);
+  };
+  static thread_local double best[kShK + 1][257];
+  static thread_local int split[kShK + 1][257];
+  for (int b = 1; b <= 256; ++b) {
+    best[1][b] = cost(0, b);
+    split[1][b] = 0;
+  }
+  for (int k = 2; k <= K; ++k)
+    for (int b = k; b <= 256; ++b) {
+      best[k][b] = 1e300;
+      split[k][b] = -1;
+      for (int a = k - 1; a < b; ++a) {
+        const double c = best[k - 1][a] + cost(a, b);
+        if (c < best[k][b]) {
+          best[k][b] = c;
+          split[k][b] = a;
+        }
+      }
+    }
+  int kk = 1;
+  for (int k = 2; k <= K; ++k)
+    if (best[k][256] < best[kk][256]) kk = k;
+  int b = 256;
+  for (int k = kk; k >= 1; --k) {
+    lo[k] = (uint16_t)b;
+    b = split[k][b];
+  }
+  lo[0] = 0;
+  return kk;
+}
+
+// tANS frequencies summing to 128 from the ranges' weights.
+void shannonic_frequencies(const uint64_t* wr, int nr, uint8_t* f) {
+  uint64_t W = 0;
+  for (int r = 0; r < nr; ++r) W += wr[r];
+  int fi[kShK], sum = 0;
+  uint64_t rem[kShK];
+  for (int r = 0; r < nr; ++r) {
+    const uint64_t q = wr[r] * (uint64_t)kShL / W;
+    rem[r] = wr[r] * (uint64_t)kShL - q * W;
+    fi[r] = q > 0 ? (int)q : 1;
+    sum += fi[r];
+  }
+  if (sum < kShL) {
+    int order[kShK];
+    for (int r = 0; r < nr; ++r) order[r] = r;
+    std::stable_sort(order, order + nr, [&](int a, int b) { return rem[a] > rem[b]; });
+    for (int i = 0; sum < kShL; i = (i + 1) % nr, ++sum) ++fi[order[i]];
+  }
+  while (sum > kShL) {
+    int big = -1;
+    for (int r = 0; r < nr; ++r)
+      if (fi[r] > 1 && (big < 0 || fi[r] > fi[big])) big = r;
+    --fi[big];
+    --sum;
+  }
+  for (int r = 0; r < nr; ++r) f[r] = (uint8_t)fi[r];
+}
+
+uint64_t shannonic_hash(const hx_codebook& cb) {
+  uint8_t bytes[3 + 2 * kShK];
+  size_t n = 0;
+  bytes[n++] = HX_KIND_SHANNONIC;
+  bytes[n++] = (uint8_t)kShR;
+  bytes[n++] = cb.sh_nr;
+  for (int r = 1; r < cb.sh_nr; ++r) bytes[n++] = (uint8_t)cb.sh_lo[r];
+  for (int r = 0; r < cb.sh_nr; ++r) bytes[n++] = cb.sh_f[r];
+  return fnv1a_update(kFnvBasis, bytes, n);
+}
+
+bool shannonic_valid(const hx_codebook& cb) {
+  if (cb.sh_nr < 1 || cb.sh_nr > kShK || cb.sh_lo[0] != 0 || cb.sh_lo[cb.sh_nr] != 256)
+    return false;
+  int sum = 0;
+  for (int r = 0; r < cb.sh_nr; ++r) {
+    if (cb.sh_lo[r + 1] <= cb.sh_lo[r] || cb.sh_f[r] < 1) return false;
+    sum += cb.sh_f[r];
+  }
+  return sum == kShL;
+}
+
+int shannonic_tables(const hx_codebook& cb, hx::Tables* t) {
+  if (!shannonic_valid(cb)) return HX_ERR_ARG;
+  const int nr = cb.sh_nr;
+  int spread[kShL];
+  for (int r = 0, pos = 0; r < nr; ++r)
+    for (int j = 0; j < cb.sh_f[r]; ++j) {
+      spread[pos] = r;
+      pos = (pos + kShStep) % kShL;
+    }
+  int cum[kShK + 1];
+  cum[0] = 0;
+  for (int r = 0; r < nr; ++r) cum[r + 1] = cum[r] + cb.sh_f[r];
+  int seen[kShK] = {0};
+  for (int u = 0; u < kShL; ++u) {
+    const int r = spread[u];
+    const int xs = cb.sh_f[r] + seen[r];  // the seen[r]-th state of range r
+    t->sh_enc[cum[r] + seen[r]] = (uint8_t)u;
+    ++seen[r];
+    int lg = 0;
+    while ((2 << lg) <= xs) ++lg;
+    const int nb = kShR - lg;
+    const int size = cb.sh_lo[r + 1] - cb.sh_lo[r];
+    t->sh_dec[u] = (uint32_t)(xs << nb) | ((uint32_t)nb << 8) | ((uint32_t)bits_for(size) << 12) |
+                   ((uint32_t)cb.sh_lo[r] << 16) | ((uint32_t)(size - 1) << 24);
+  }
+  for (int r = 0; r < nr; ++r) {
+    int lg = 0;
+    while ((2 << lg) <= cb.sh_f[r]) ++lg;
+    const int size = cb.sh_lo[r + 1] - cb.sh_lo[r];
+    for (int v = cb.sh_lo[r]; v < cb.sh_lo[r + 1]; ++v)
+      t->sh_sym[v] = (uint32_t)cb.sh_f[r] | ((uint32_t)cum[r] << 8) |
+                     ((uint32_t)bits_for(size) << 16) | ((uint32_t)(v - cb.sh_lo[r]) << 20) |
+                     ((uint32_t)(kShR - lg) << 28);
+  }
+  return HX_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -202,11 +342,47 @@ int hx_qlc_build(const uint64_t* counts, int max_distinct, uint32_t flags, hx_co
   return fill_qlc(counts, max_distinct, out);
 }
 
+int hx_shannonic_build(const uint64_t* counts, int K, uint32_t flags, hx_codebook* out) {
+  if (!counts || !out || flags || K < 1 || K > kShK) return HX_ERR_ARG;
+  uint64_t w[256];
+  for (int v = 0; v < 256; ++v) w[v] = std::max<uint64_t>(counts[v], 1);
+  hx_codebook cb;
+  std::memset(&cb, 0, sizeof cb);
+  cb.kind = HX_KIND_SHANNONIC;
+  cb.lmax = (uint8_t)kShR;
+  cb.sh_nr = (uint8_t)shannonic_partition(w, K, cb.sh_lo);
+  uint64_t wr[kShK] = {0};
+  for (int r = 0; r < cb.sh_nr; ++r)
+    for (int v = cb.sh_lo[r]; v < cb.sh_lo[r + 1]; ++v) wr[r] += w[v];
+  shannonic_frequencies(wr, cb.sh_nr, cb.sh_f);
+  cb.hash = shannonic_hash(cb);
+  *out = cb;
+  return HX_OK;
+}
+
+uint64_t hx_shannonic_encode_bound(uint64_t n) {
+  const uint64_t chunks = (n + HX_CHUNK - 1) / HX_CHUNK;
+  // a sub-stream: at most 512 symbols of 8 offset + 7 state bits, then 7 bits of final state
+  const uint64_t words = (HX_SUBSTREAMS * (512 * 15 + 7) + 31) / 32;
+  return hx_payload_offset(n) + 4 * (chunks * words + 2);
+}
+
 int hx_codebook_tables(const hx_codebook* cb, void* host_tables) {
   if (!cb || !host_tables) return HX_ERR_ARG;
-  if (cb->kind != HX_KIND_HUFFMAN && cb->kind != HX_KIND_QLC) return HX_ERR_ARG;
+  if (cb->kind != HX_KIND_HUFFMAN && cb->kind != HX_KIND_QLC && cb->kind != HX_KIND_SHANNONIC)
+    return HX_ERR_ARG;
   std::memset(host_tables, 0, HX_TABLES_BYTES);
   hx::Tables* t = static_cast<hx::Tables*>(host_tables);
+  if (cb->kind == HX_KIND_SHANNONIC) {
+    const int rc = shannonic_tables(*cb, t);
+    if (rc) return rc;
+    t->complete = 0;
+    t->kind = cb->kind;
+    t->lmax = cb->lmax;
+    t->magic = hx::kTablesMagic;
+    t->hash = cb->hash;
+    return HX_OK;
+  }
   for (int s = 0; s < 256; ++s) {
     const int l = cb->len[s];
     if (l > HX_LMAX_MAX || (l && (cb->code[s] >> l))) return HX_ERR_ARG;
@@ -271,6 +447,18 @@ double hx_entropy(const uint64_t* counts) {
 double hx_mean_length(const uint64_t* counts, const hx_codebook* cb) {
   if (!counts || !cb) return -1;
   long double total = 0, bits = 0;
+  if (cb->kind == HX_KIND_SHANNONIC) {  // tANS codes range r in log2(128 / f_r) bits on average
+    if (!shannonic_valid(*cb)) return -1;
+    for (int r = 0; r < cb->sh_nr; ++r) {
+      const double len = std::log2((double)kShL / cb->sh_f[r]) +
+                         bits_for(cb->sh_lo[r + 1] - cb->sh_lo[r]);
+      for (int s = cb->sh_lo[r]; s < cb->sh_lo[r + 1]; ++s) {
+        total += counts[s];
+        bits += (long double)counts[s] * len;
+      }
+    }
+    return total == 0 ? 0 : (double)(bits / total);
+  }
   for (int s = 0; s < 256; ++s) {
     total += counts[s];
     bits += (long double)counts[s] * cb->len[s];

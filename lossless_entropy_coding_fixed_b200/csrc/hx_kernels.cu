@@ -752,10 +752,345 @@ __global__ void __launch_bounds__(kDecThreads, KIND == HX_KIND_QLC ? 4 : 5)
     decode_chunks<false>(a, lut, (uint32_t)total);
 }
 
+// ---------------------------------------------------------------------------------- shannonic
+// The review page's range-partitioned coder: a byte's range index is coded by tANS with 128
+// states (the table variant of asymmetric numeral systems), its offset inside the range in
+// ceil(log2 size) bits. tANS runs from a sub-stream's last symbol to its first, so its bit count
+// is known only after the whole sub-stream has been run: the encoder's first pass runs it to
+// count (k_sh_measure), the second runs it again and writes (k_sh_pack); one thread per
+// sub-stream in both, as in the decoder (k_sh_decode), which reads each sub-stream backwards.
+
+constexpr int kShThreads = 256;  // 8 threads per chunk, 32 chunks per block
+constexpr int kShCopies = 8;     // symbol table copies: lane l reads copy l % 8
+
+// Encoder tables in shared memory.
+struct ShEnc {
+  uint32_t sym[256 * kShCopies];  // [byte][copy]: per-byte fields of hx::Tables::sh_sym
+  uint8_t enc[128];               // the ranges' states minus 128
+};
+
+__device__ __forceinline__ void sh_load_tables(const hx::Tables* t, ShEnc& s) {
+  for (int i = threadIdx.x; i < 256 * kShCopies; i += blockDim.x) s.sym[i] = t->sh_sym[i / kShCopies];
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) s.enc[i] = t->sh_enc[i];
+}
+
+// One tANS step for byte `sym` from `state` (in [128, 256)): the bits it writes (the offset,
+// then the state's low nb bits) as (value, count), and the next state.
+__device__ __forceinline__ uint32_t sh_step(const ShEnc& s, const uint32_t* sym_lane,
+                                            uint32_t sym, uint32_t& state, uint32_t& nbits) {
+  const uint32_t e = sym_lane[sym * kShCopies];
+  const uint32_t f = e & 0xffu, kshift = e >> 28, ob = (e >> 16) & 15u;
+  const uint32_t nb = kshift - ((state >> kshift) < f ? 1u : 0u);  // state >> nb in [f, 2f)
+  const uint32_t value = (((e >> 20) & 0xffu) << nb) | (state & ((1u << nb) - 1u));
+  state = 128u + s.enc[((e >> 8) & 0x7fu) + (state >> nb) - f];
+  nbits = ob + nb;
+  return value;
+}
+
+// Bytes of sub-stream k of chunk c, last first: calls fn(byte) for each.
+template <class Fn>
+__device__ __forceinline__ void sh_reverse(const EncodeArgs& a, uint32_t c, uint32_t k,
+                                           uint32_t m, Fn&& fn) {
+  const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
+  if (m == kSubLen) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.in + first);
+#pragma unroll 1
+    for (int g = kSubLen / 16 - 1; g >= 0; --g) {
+      const uint4 v = __ldg(src + g);
+      const uint32_t w[4] = {v.w, v.z, v.y, v.x};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        fn(w[q] >> 24);
+        fn((w[q] >> 16) & 0xffu);
+        fn((w[q] >> 8) & 0xffu);
+        fn(w[q] & 0xffu);
+      }
+    }
+  } else {
+    for (uint32_t i = m; i-- > 0;) fn((uint32_t)a.in[first + i]);
+  }
+}
+
+// Symbols in sub-stream k of chunk c (0 past the end of the input).
+__device__ __forceinline__ uint32_t sh_count(uint64_t n, uint32_t c, uint32_t k) {
+  const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
+  return first < n ? (uint32_t)min((uint64_t)kSubLen, n - first) : 0u;
+}
+
+struct ShMeasureSmem {
+  ShEnc t;
+  uint32_t cnt[kMaxChunksPerBlock];
+  uint32_t red[kShThreads / 32];
+  uint32_t hist[kShThreads / 32][256];
+};
+
+__global__ void __launch_bounds__(kShThreads) k_sh_measure(EncodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ShMeasureSmem& sm = *reinterpret_cast<ShMeasureSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
+    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+    return;
+  }
+  sh_load_tables(a.tables, sm.t);
+  const bool hist = a.hist != nullptr;
+  if (hist)
+    for (int i = tid; i < (kShThreads / 32) * 256; i += kShThreads) (&sm.hist[0][0])[i] = 0;
+  __syncthreads();
+  const uint32_t* sym_lane = sm.t.sym + (lane % kShCopies);
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
+  const uint32_t c0 = blockIdx.x * a.cpb;
+  const uint32_t m_chunks = c0 < nchunks ? min(a.cpb, nchunks - c0) : 0u;
+  uint16_t* sync = reinterpret_cast<uint16_t*>(a.out + sync_offset(n));
+  const uint32_t k = tid & 7, slot = tid >> 3;
+  const uint32_t rounds = (m_chunks + 31) / 32;
+  for (uint32_t r = 0; r < rounds; ++r) {
+    const uint32_t i = r * 32 + slot;
+    const bool live = i < m_chunks;
+    const uint32_t c = c0 + (live ? i : 0);
+    const uint32_t m = live ? sh_count(n, c, k) : 0u;
+    uint32_t bits = 0;
+    if (m) {
+      uint32_t state = 128;
+      sh_reverse(a, c, k, m, [&](uint32_t s) {
+        uint32_t nb;
+        sh_step(sm.t, sym_lane, s, state, nb);
+        bits += nb;
+        if (hist) atomicAdd(&sm.hist[warp][s], 1u);
+      });
+      bits += HX_SHN_R;  // the final state
+    }
+    // the chunk's 8 sub-streams: sync offsets by a prefix sum over its 8 threads
+    uint32_t incl = bits;
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d, 8);
+      if (k >= (uint32_t)d) incl += t;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 7, 8);
+    if (live) {
+      sync[(uint64_t)c * HX_SUBSTREAMS + k] = (uint16_t)(k == 0 ? total : incl - bits);
+      if (k == 0) sm.cnt[i] = (total + 31) >> 5;
+    }
+  }
+  __syncthreads();
+  const uint32_t total = block_exclusive_scan<kShThreads>(sm.cnt, m_chunks, sm.red);
+  for (uint32_t i = tid; i < m_chunks; i += kShThreads) a.local[c0 + i] = sm.cnt[i];
+  if (tid == 0) a.btotal[blockIdx.x] = total;
+  if (hist) {
+    __syncthreads();
+    uint32_t sum = 0;
+#pragma unroll
+    for (int w = 0; w < kShThreads / 32; ++w) sum += sm.hist[w][tid];
+    if (sum) atomicAdd(&a.hist[tid], sum);
+  }
+}
+
+struct ShPackSmem {
+  ShEnc t;
+  uint32_t bpre[kMaxMeasureBlocks];
+  uint32_t red[kShThreads / 32];
+};
+
+__global__ void __launch_bounds__(kShThreads) k_sh_pack(EncodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ShPackSmem& sm = *reinterpret_cast<ShPackSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) return;  // measure said so
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
+  const uint64_t P = payload_offset(n);
+  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
+  const uint16_t* sync = reinterpret_cast<const uint16_t*>(a.out + sync_offset(n));
+  uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
+  sh_load_tables(a.tables, sm.t);
+  for (uint32_t i = tid; i < a.mblocks; i += kShThreads) sm.bpre[i] = a.btotal[i];
+  __syncthreads();
+  const uint32_t total = block_exclusive_scan<kShThreads>(sm.bpre, a.mblocks, sm.red);
+  const bool fits = P + 4ull * ((uint64_t)total + 2) <= a.cap;
+  if (blockIdx.x == 0 && tid == 0) {
+    write_header(a);
+    reinterpret_cast<uint64_t*>(a.out)[4] = total;
+    word_off[nchunks] = total;
+    if (fits) {
+      payload[total] = 0;
+      payload[total + 1] = 0;
+    } else {
+      atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
+    }
+  }
+  const uint32_t limit = fits ? total : 0u;
+  const uint32_t* sym_lane = sm.t.sym + (lane % kShCopies);
+  const uint32_t k = tid & 7;
+  const uint32_t groups = (nchunks + 31) / 32;
+  for (uint32_t gi = blockIdx.x; gi < groups; gi += gridDim.x) {
+    const uint32_t c = gi * 32 + (tid >> 3);
+    const bool live = c < nchunks;
+    const uint32_t m = live ? sh_count(n, c, k) : 0u;
+    uint32_t widx = 0, nacc = 0, tail = 0;
+    bool last = false;
+    if (live) {
+      const uint32_t woff = sm.bpre[c / a.cpb] + a.local[c];
+      if (k == 0) word_off[c] = woff;
+      const uint16_t* row = sync + (uint64_t)c * HX_SUBSTREAMS;
+      const uint32_t chunk_bits = row[0];
+      const uint32_t s = k == 0 ? 0u : row[k];
+      const uint32_t e = k + 1 < HX_SUBSTREAMS ? row[k + 1] : chunk_bits;
+      last = m != 0 && e == chunk_bits;
+      widx = woff + (s >> 5);
+      nacc = s & 31;  // the first bits belong to earlier sub-streams (zeros here)
+      uint32_t hi = 0, lo = 0;
+      auto put = [&](uint32_t value, uint32_t len) {
+        hi = __funnelshift_l(lo, hi, len);
+        lo = (lo << len) | value;
+        nacc += len;
+        if (nacc >= 32) {
+          nacc -= 32;
+          if (widx < limit) payload[widx] = __funnelshift_r(lo, hi, nacc);
+          ++widx;
+        }
+      };
+      if (m) {
+        uint32_t state = 128;
+        sh_reverse(a, c, k, m, [&](uint32_t sym) {
+          uint32_t nb;
+          const uint32_t v = sh_step(sm.t, sym_lane, sym, state, nb);
+          put(v, nb);
+        });
+        put(state - 128u, HX_SHN_R);
+      }
+      tail = nacc ? lo << (32 - nacc) : 0u;
+      // the chunk's last word is stored whole (zero padding)
+      if (last && nacc && widx < limit) payload[widx] = tail;
+    }
+    __syncwarp();
+    // any other unfinished word is OR-ed into the word the next sub-stream stored whole
+    if (live && m && !last && nacc && widx < limit) atomicOr(payload + widx, tail);
+  }
+}
+
+// Reads a sub-stream backwards: the unread bits end at bit 32 * j + t of the payload (t in
+// 1..32 unread bits in word j, MSB first); cur = word j, prv = word j - 1, two more below
+// already requested. Words outside the caller's buffer read as 0.
+// (j is signed: a reader that runs off the front of the payload must not wrap around; a payload
+// holds fewer than 2^31 words, since n < 2^32 bytes at no more than 15 bits each.)
+struct BackBits {
+  const uint32_t* words;
+  uint32_t wlimit;
+  int32_t j;
+  uint32_t t, cur, prv, pf0, pf1;
+  __device__ __forceinline__ uint32_t word(int32_t i) const {
+    return (uint32_t)i < wlimit ? __ldg(words + (uint32_t)i) : 0u;
+  }
+  __device__ __forceinline__ void start(uint64_t end_bit) {
+    const uint64_t last = end_bit - 1;  // the first bit to read (backwards)
+    j = (int32_t)(last >> 5);
+    t = (uint32_t)(last & 31) + 1;
+    cur = word(j);
+    prv = word(j - 1);
+    pf0 = word(j - 2);
+    pf1 = word(j - 3);
+  }
+  // the `len` (<= 15) bits before the read position, MSB first
+  __device__ __forceinline__ uint32_t read(uint32_t len) {
+    const uint32_t v = __funnelshift_r(cur, prv, 32 - t) & ((1u << len) - 1u);
+    if (t > len) {
+      t -= len;
+    } else {
+      t += 32 - len;
+      --j;
+      cur = prv;
+      prv = pf0;
+      pf0 = pf1;
+      pf1 = word(j - 3);
+    }
+    return v;
+  }
+  __device__ __forceinline__ int64_t position() const { return 32ll * j + t; }
+};
+
+__global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
+  __shared__ uint32_t s_dec[128];
+  __shared__ int64_t s_total;
+  __shared__ const hx::Tables* s_tables;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_total = check_header(a, &s_tables);
+  __syncthreads();
+  const int64_t total = s_total;
+  if (total < 0) {
+    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)(-total));
+    return;
+  }
+  if (tid < 128) s_dec[tid] = s_tables->sh_dec[tid];
+  __syncthreads();
+  const uint64_t n = a.n;
+  const uint64_t nchunks = n_chunks_of(n);
+  const uint64_t P = payload_offset(n);
+  const uint32_t* word_off = reinterpret_cast<const uint32_t*>(a.st + 64);
+  const uint4* sync = reinterpret_cast<const uint4*>(a.st + sync_offset(n));
+  BackBits rd;
+  rd.words = reinterpret_cast<const uint32_t*>(a.st + P);
+  rd.wlimit = (uint32_t)min((a.bytes - P) / 4, (uint64_t)0xffffffffull);
+  const uint32_t k = tid & 7;
+  for (uint64_t c = (uint64_t)blockIdx.x * (kDecThreads / 8) + (tid >> 3); c < nchunks;
+       c += (uint64_t)gridDim.x * (kDecThreads / 8)) {
+    const uint32_t w0 = __ldg(word_off + c), w1 = __ldg(word_off + c + 1);
+    const uint4 sy = __ldg(sync + c);
+    auto sync_at = [&](uint32_t i) -> uint32_t {
+      const uint32_t w = i < 2 ? sy.x : i < 4 ? sy.y : i < 6 ? sy.z : sy.w;
+      return (w >> (16 * (i & 1))) & 0xffffu;
+    };
+    const uint32_t nbits = sy.x & 0xffffu;
+    const uint32_t count = n - c * kChunk < kChunk ? (uint32_t)(n - c * kChunk) : kChunk;
+    const uint32_t nsub = (count + kSubLen - 1) / kSubLen;
+    bool bad = w0 > w1 || w1 > (uint32_t)total || nbits > 32u * (w1 - w0) ||
+               (nbits + 31) / 32 != w1 - w0;
+    const uint32_t mine = k < nsub ? min(kSubLen, count - k * kSubLen) : 0u;
+    if (mine == 0) {
+      bad |= k > 0 && sync_at(k) != nbits;
+    } else if (!bad) {
+      const uint32_t start = k == 0 ? 0u : sync_at(k);
+      const uint32_t end = k + 1 < nsub ? sync_at(k + 1) : nbits;
+      bad |= start >= end || end > nbits;
+      if (!bad) {
+        rd.start(32ull * w0 + end);
+        uint32_t state = 128u + rd.read(HX_SHN_R);
+        bool invalid = false;
+        uint8_t* dst = a.out + c * kChunk + (uint64_t)k * kSubLen;
+        auto one = [&]() -> uint32_t {
+          const uint32_t d = s_dec[(state - 128u) & 127u];
+          const uint32_t nb = (d >> 8) & 15u, ob = (d >> 12) & 15u;
+          const uint32_t v = rd.read(nb + ob);
+          const uint32_t off = v >> nb;
+          invalid |= off > (d >> 24);
+          state = (d & 0xffu) + (v & ((1u << nb) - 1u));
+          return ((d >> 16) & 0xffu) + off;
+        };
+        const uint32_t groups = mine / 16;
+        for (uint32_t g = 0; g < groups; ++g) {
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t b0 = one(), b1 = one(), b2 = one(), b3 = one();
+            o[q] = (b0 & 0xffu) | ((b1 & 0xffu) << 8) | ((b2 & 0xffu) << 16) | (b3 << 24);
+          }
+          __stcs(reinterpret_cast<uint4*>(dst + 16 * g), make_uint4(o[0], o[1], o[2], o[3]));
+        }
+        for (uint32_t i = groups * 16; i < mine; ++i) dst[i] = (uint8_t)one();
+        // the chain must end in state 128 exactly at the sub-stream's first bit
+        bad |= invalid || state != 128u || rd.position() != (int64_t)(32ull * w0 + start);
+      }
+    }
+    if (bad) atomicOr(a.status, (uint32_t)HX_ERR_CORRUPT);
+  }
+}
+
 // ---------------------------------------------------------------------------------- launch
 struct DeviceInfo {
   int sms = 0;
   int measure_per_sm = 0, pack_per_sm = 0, huff_per_sm = 0, qlc_per_sm = 0, hist_per_sm = 0;
+  int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0;
 };
 
 // Sets the shared-memory carveout of `fn` to the smallest share that still holds `per_sm` blocks,
@@ -808,8 +1143,20 @@ bool device_info(DeviceInfo* out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qlc_per_sm, k_decode<HX_KIND_QLC>,
                                                       kDecThreads, 0) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
-                                                      0) != cudaSuccess)
+                                                      0) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sh_measure, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(ShMeasureSmem)) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sh_pack, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(ShPackSmem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_measure_per_sm, k_sh_measure,
+                                                      kShThreads,
+                                                      sizeof(ShMeasureSmem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_pack_per_sm, k_sh_pack, kShThreads,
+                                                      sizeof(ShPackSmem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_decode_per_sm, k_sh_decode,
+                                                      kDecThreads, 0) != cudaSuccess)
       return false;
+    if (d.sh_measure_per_sm < 1 || d.sh_pack_per_sm < 1 || d.sh_decode_per_sm < 1) return false;
     if (d.measure_per_sm < 1 || d.pack_per_sm < 1 || d.huff_per_sm < 1 || d.qlc_per_sm < 1 ||
         d.hist_per_sm < 1)
       return false;
@@ -836,7 +1183,8 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
                 uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
                 EncodeArgs* a, DeviceInfo* info) {
   if (!d_tables || !d_out || !d_scratch || !d_status || (n && !d_in)) return HX_ERR_ARG;
-  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC) return HX_ERR_ARG;
+  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC && kind != HX_KIND_SHANNONIC)
+    return HX_ERR_ARG;
   if (n >= (1ull << 32) || out_cap < payload_offset(n) + 8) return HX_ERR_ARG;
   if (!aligned16(d_in) || !aligned16(d_out) || !aligned16(d_scratch) || !aligned16(d_tables))
     return HX_ERR_ARG;
@@ -859,12 +1207,23 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
 }
 
 int launch_measure(const EncodeArgs& a, cudaStream_t s) {
-  if (a.mblocks) k_measure<<<a.mblocks, kMeasureThreads, sizeof(MeasureSmem), s>>>(a);
+  if (a.mblocks) {
+    if (a.kind == HX_KIND_SHANNONIC)
+      k_sh_measure<<<a.mblocks, kShThreads, sizeof(ShMeasureSmem), s>>>(a);
+    else
+      k_measure<<<a.mblocks, kMeasureThreads, sizeof(MeasureSmem), s>>>(a);
+  }
   return launched();
 }
 
 int launch_pack(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
   const uint32_t nchunks = (uint32_t)n_chunks_of(a.n);
+  if (a.kind == HX_KIND_SHANNONIC) {  // 32 chunks per block and round
+    const uint32_t grid = (uint32_t)std::max<uint64_t>(
+        1, std::min<uint64_t>((nchunks + 31) / 32, (uint64_t)info.sms * info.sh_pack_per_sm));
+    k_sh_pack<<<grid, kShThreads, sizeof(ShPackSmem), s>>>(a);
+    return launched();
+  }
   const uint32_t grid = (uint32_t)std::max<uint64_t>(
       1, std::min<uint64_t>((nchunks + kPackThreads / 32 - 1) / (kPackThreads / 32),
                             (uint64_t)info.sms * info.pack_per_sm));
@@ -900,7 +1259,9 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint64_t nchunks = n_chunks_of(n);
   const uint64_t per_block = kDecThreads / 8;
-  const int per_sm = kind == HX_KIND_HUFFMAN ? info.huff_per_sm : info.qlc_per_sm;
+  const int per_sm = kind == HX_KIND_HUFFMAN ? info.huff_per_sm
+                     : kind == HX_KIND_QLC   ? info.qlc_per_sm
+                                             : info.sh_decode_per_sm;
   const uint64_t want = (nchunks + per_block - 1) / per_block;
   const uint32_t grid =
       (uint32_t)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)info.sms * per_sm));
@@ -915,8 +1276,10 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   a.kind = kind;
   if (kind == HX_KIND_HUFFMAN)
     k_decode<HX_KIND_HUFFMAN><<<grid, kDecThreads, 0, s>>>(a);
-  else
+  else if (kind == HX_KIND_QLC)
     k_decode<HX_KIND_QLC><<<grid, kDecThreads, 0, s>>>(a);
+  else
+    k_sh_decode<<<grid, kDecThreads, 0, s>>>(a);
   return launched();
 }
 
@@ -1033,10 +1396,24 @@ int hx_qlc_decode(const void* d_tables, const void* d_stream, uint64_t stream_by
                        d_status, stream);
 }
 
+int hx_shannonic_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                        uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
+                        void* stream) {
+  return encode_common(HX_KIND_SHANNONIC, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist,
+                       d_status, stream);
+}
+
+int hx_shannonic_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
+                        uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream) {
+  return decode_common(HX_KIND_SHANNONIC, &d_tables, 1, d_stream, stream_bytes, d_out, n_expected,
+                       d_status, stream);
+}
+
 int hx_decode_set(uint32_t kind, const void* const* d_tables, uint32_t n_tables,
                   const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
                   uint64_t n_expected, uint32_t* d_status, void* stream) {
-  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC) return HX_ERR_ARG;
+  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC && kind != HX_KIND_SHANNONIC)
+    return HX_ERR_ARG;
   return decode_common(kind, d_tables, n_tables, d_stream, stream_bytes, d_out, n_expected,
                        d_status, stream);
 }

@@ -12,9 +12,22 @@ constexpr uint32_t kTablesMagic = 0x42545848u;  // "HXTB"
 struct Tables {
   // Encoder: per byte value (code << 4) | len; len 0 = no code word.
   uint32_t enc[256];
-  // Decoder: for every 12-bit window w, (sym << 8) | len of the code word that w starts with;
-  // 0 when no code word is a prefix of w. (Filled for QLC codebooks as well.)
-  uint16_t dec[4096];
+  union {
+    // Decoder: for every 12-bit window w, (sym << 8) | len of the code word that w starts with;
+    // 0 when no code word is a prefix of w. (Filled for QLC codebooks as well.)
+    uint16_t dec[4096];
+    // Shannonic (kind 2) instead:
+    struct {
+      // per decoding state 128 + u: base (xs << nb, bits 0-7) | nb (8-11) | offset bits (12-15)
+      // | first byte value of the range (16-23) | range size - 1 (24-31)
+      uint32_t sh_dec[128];
+      // per byte value: f_r (bits 0-7) | first index of the range's states in sh_enc (8-14) |
+      // offset bits (16-19) | offset in the range (20-27) | 7 - floor(log2 f_r) (28-30)
+      uint32_t sh_sym[256];
+      // the range's decoding states in increasing order, minus 128, ranges one after another
+      uint8_t sh_enc[128];
+    };
+  };
   // QLC: byte value of each rank.
   uint8_t rank2sym[256];
   // QLC area a: first rank (bits 0-8) | number of ranks it holds (bits 9-17) | index bits (18-21).

@@ -18,7 +18,7 @@ from . import build as _build
 
 HX_OK, HX_ERR_ARG, HX_ERR_CUDA = 0, 1, 2
 HX_ERR_UNCODABLE, HX_ERR_CORRUPT, HX_ERR_CODEBOOK, HX_ERR_TIMEOUT, HX_ERR_CAPACITY = 4, 8, 16, 32, 64
-KIND_HUFFMAN, KIND_QLC = 0, 1
+KIND_HUFFMAN, KIND_QLC, KIND_SHANNONIC = 0, 1, 2
 CHUNK, SUBSTREAMS, LMAX_MAX, QLC_LMAX = 4096, 8, 12, 11
 CB_SEEN_ONLY = 1
 TABLES_BYTES = 10240
@@ -36,7 +36,9 @@ class _Codebook(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_uint8), ("lmax", ctypes.c_uint8),
                 ("len", ctypes.c_uint8 * 256), ("code", ctypes.c_uint16 * 256),
                 ("qlc_bits", ctypes.c_uint8 * 8), ("qlc_start", ctypes.c_uint16 * 9),
-                ("rank2sym", ctypes.c_uint8 * 256), ("hash", ctypes.c_uint64)]
+                ("rank2sym", ctypes.c_uint8 * 256), ("hash", ctypes.c_uint64),
+                ("sh_nr", ctypes.c_uint8), ("sh_lo", ctypes.c_uint16 * 17),
+                ("sh_f", ctypes.c_uint8 * 16)]
 
 
 _lib = None
@@ -74,6 +76,10 @@ def lib():
             "hx_qlc_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
             "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_encode_noalloc": (i32, [P, P, u64, P, u64, P, P, P]),
+            "hx_shannonic_build": (i32, [P, i32, u32, CB]),
+            "hx_shannonic_encode_bound": (u64, [u64]),
+            "hx_shannonic_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
+            "hx_shannonic_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_encode_measure": (i32, [u32, P, P, u64, P, u64, P, P, P, P]),
             "hx_decode_set": (i32, [u32, P, u32, P, u64, P, u64, P, P]),
             "hx_planner_create": (i32, [ctypes.POINTER(_SessionConfig), P, P]),
@@ -158,6 +164,14 @@ class Codebook:
     def hash(self) -> int:
         return int(self.raw.hash)
 
+    @property
+    def sh_lo(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.raw.sh_lo), np.uint16)[: self.raw.sh_nr + 1].copy()
+
+    @property
+    def sh_f(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.raw.sh_f), np.uint8)[: self.raw.sh_nr].copy()
+
     def tables(self) -> bytes:
         buf = (ctypes.c_uint8 * TABLES_BYTES)()
         _check(lib().hx_codebook_tables(ctypes.byref(self.raw), buf), "hx_codebook_tables")
@@ -195,6 +209,15 @@ def qlc_build(counts, max_distinct: int = 4) -> Codebook:
     return Codebook(raw)
 
 
+def shannonic_build(counts, K: int = 16) -> Codebook:
+    """hx_shannonic_build: range partition (at most K ranges) and 128-state tANS frequencies."""
+    c = _counts(counts)
+    raw = _Codebook()
+    _check(lib().hx_shannonic_build(c.ctypes.data, int(K), 0, ctypes.byref(raw)),
+           "hx_shannonic_build")
+    return Codebook(raw)
+
+
 def entropy(counts) -> float:
     """Shannon entropy of a 256-bin histogram, bits per symbol."""
     c = _counts(counts)
@@ -216,7 +239,9 @@ def sync_offset(n: int) -> int:
     return int(lib().hx_sync_offset(n))
 
 
-def encode_bound(n: int) -> int:
+def encode_bound(n: int, kind: int = KIND_HUFFMAN) -> int:
+    if kind == KIND_SHANNONIC:
+        return int(lib().hx_shannonic_encode_bound(n))
     return int(lib().hx_encode_bound(n))
 
 
@@ -265,12 +290,13 @@ def encode(tables, x, out=None, scratch=None, hist=None, status=None, kind: int 
     x = _dev_u8(x, "x")
     n = x.numel()
     if out is None:
-        out = torch.empty(encode_bound(n), dtype=torch.uint8, device=x.device)
+        out = torch.empty(encode_bound(n, kind), dtype=torch.uint8, device=x.device)
     if scratch is None:
         scratch = torch.empty(scratch_bytes(n), dtype=torch.uint8, device=x.device)
     if status is None:
         status = new_status(x.device)
-    fn = lib().hx_encode if kind == KIND_HUFFMAN else lib().hx_qlc_encode
+    fn = {KIND_HUFFMAN: lib().hx_encode, KIND_QLC: lib().hx_qlc_encode,
+          KIND_SHANNONIC: lib().hx_shannonic_encode}[kind]
     _check(fn(tables.data_ptr(), x.data_ptr(), n, out.data_ptr(), out.numel(), scratch.data_ptr(),
               hist.data_ptr() if hist is not None else None, status.data_ptr(), _stream(x)),
            "hx_encode")
@@ -324,7 +350,8 @@ def decode(tables, stream, n: int, out=None, status=None, kind: int = KIND_HUFFM
         out = torch.empty(max(n, 1), dtype=torch.uint8, device=stream.device)[:n]
     if status is None:
         status = new_status(stream.device)
-    fn = lib().hx_decode if kind == KIND_HUFFMAN else lib().hx_qlc_decode
+    fn = {KIND_HUFFMAN: lib().hx_decode, KIND_QLC: lib().hx_qlc_decode,
+          KIND_SHANNONIC: lib().hx_shannonic_decode}[kind]
     _check(fn(tables.data_ptr(), stream.data_ptr(), int(nbytes or stream.numel()),
               out.data_ptr() if n else stream.data_ptr(), n, status.data_ptr(), _stream(stream)),
            "hx_decode")
