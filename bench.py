@@ -50,6 +50,7 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-online", action="store_true")
+    p.add_argument("--no-shannonic", action="store_true")
     return p.parse_args()
 
 
@@ -202,6 +203,37 @@ def cpu_baseline_leg(counts):
     return {"value": 4 * sample / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"first {sample >> 20} MiB of the batch through the same 4 codec calls "
                       f"({dt:.1f} s, single-thread bit-serial C++)"}
+
+
+def shannonic_leg(dev, hx, torch, x, prior, h, scratch, y, status, steps):
+    """The Shannonic coder (range partition + 128-state tANS) on the same batch and prior:
+    encode and decode device time per call (CUDA events, inputs resident), bits per symbol."""
+    n = x.numel()
+    cb = hx.shannonic_build(prior)
+    t = cb.upload(dev)
+    out = torch.empty(hx.encode_bound(n, hx.KIND_SHANNONIC), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for name, fn in (("encode", lambda: hx.encode(t, x, out=out, scratch=scratch, status=status,
+                                                  kind=hx.KIND_SHANNONIC)),
+                     ("decode", lambda: hx.decode(t, out, n, out=y, status=status,
+                                                  kind=hx.KIND_SHANNONIC))):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = a.elapsed_time(b) / steps
+    assert int(status.item()) == 0 and torch.equal(x, y)
+    size = hx.stream_size(out, n)
+    return {"encode_ms": res["encode"], "decode_ms": res["decode"],
+            "encode_GB_per_s_uncompressed": n / (res["encode"] * 1e-3) / 1e9,
+            "decode_GB_per_s_uncompressed": n / (res["decode"] * 1e-3) / 1e9,
+            "ranges": int(cb.raw.sh_nr),
+            "bits_per_symbol": {"framed": size * 8 / n, "tans_ideal": hx.mean_length(h, cb)}}
 
 
 def online_leg(dev, hx, datagen, torch):
@@ -443,6 +475,11 @@ def main():
                "h2d_bytes_per_step": n, "d2h_bytes_per_step": d2h, "steps": k_e2e,
                "path": "pinned host batch -> H2D -> 4 codec calls -> D2H of both streams"}
 
+    shannonic = None
+    if not args.no_shannonic:
+        shannonic = shannonic_leg(dev, hx, torch, x, prior, h, scratch, y, status,
+                                  max(3, min(args.steps, 10)))
+
     online = None
     if not args.no_online:
         online = online_leg(dev, hx, datagen, torch)
@@ -481,6 +518,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": e2e,
             "online": online,
+            "shannonic": shannonic,
             "gpu_launches": 6 * args.steps,
             "clocks": clocks.summary(),
         }
