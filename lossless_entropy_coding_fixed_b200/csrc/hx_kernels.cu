@@ -760,6 +760,13 @@ __global__ void __launch_bounds__(kDecThreads, KIND == HX_KIND_QLC ? 4 : 5)
 // count (k_sh_measure), the second runs it again and writes (k_sh_pack); one thread per
 // sub-stream in both, as in the decoder (k_sh_decode), which reads each sub-stream backwards.
 
+// Bits [pos, pos + len) of x (len < 32; an empty field reads 0).
+__device__ __forceinline__ uint32_t bfe(uint32_t x, uint32_t pos, uint32_t len) {
+  uint32_t r;
+  asm("bfe.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(pos), "r"(len));
+  return r;
+}
+
 constexpr int kShThreads = 256;  // 8 threads per chunk, 32 chunks per block
 constexpr int kShCopies = 8;     // symbol table copies: lane l reads copy l % 8
 
@@ -992,6 +999,22 @@ struct BackBits {
     pf0 = word(j - 2);
     pf1 = word(j - 3);
   }
+  // the 32 bits before the read position, the last of them in bit 0 (bits before the payload's
+  // first word read as 0)
+  __device__ __forceinline__ uint32_t peek() const { return __funnelshift_r(cur, prv, 32 - t); }
+  // moves the read position back by len (<= 31) bits
+  __device__ __forceinline__ void skip(uint32_t len) {
+    if (t > len) {
+      t -= len;
+    } else {
+      t += 32 - len;
+      --j;
+      cur = prv;
+      prv = pf0;
+      pf0 = pf1;
+      pf1 = word(j - 3);
+    }
+  }
   // the `len` (<= 15) bits before the read position, MSB first
   __device__ __forceinline__ uint32_t read(uint32_t len) {
     const uint32_t v = __funnelshift_r(cur, prv, 32 - t) & ((1u << len) - 1u);
@@ -1058,26 +1081,42 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
         uint32_t state = 128u + rd.read(HX_SHN_R);
         bool invalid = false;
         uint8_t* dst = a.out + c * kChunk + (uint64_t)k * kSubLen;
-        auto one = [&]() -> uint32_t {
+        // One symbol from x, the bits before the read position (the last in bit 0): the
+        // state's low nb bits, before them the offset. Returns the byte, moves the state, and
+        // drops the symbol's bits from x, counting them in `used`.
+        auto one = [&](uint32_t& x, uint32_t& used) -> uint32_t {
           const uint32_t d = s_dec[(state - 128u) & 127u];
-          const uint32_t nb = (d >> 8) & 15u, ob = (d >> 12) & 15u;
-          const uint32_t v = rd.read(nb + ob);
-          const uint32_t off = v >> nb;
+          const uint32_t nb = bfe(d, 8, 4), ob = bfe(d, 12, 4);
+          const uint32_t off = bfe(x, nb, ob);
           invalid |= off > (d >> 24);
-          state = (d & 0xffu) + (v & ((1u << nb) - 1u));
-          return ((d >> 16) & 0xffu) + off;
+          state = (d & 0xffu) + bfe(x, 0, nb);
+          x >>= nb + ob;
+          used += nb + ob;
+          return bfe(d, 16, 8) + off;
         };
         const uint32_t groups = mine / 16;
         for (uint32_t g = 0; g < groups; ++g) {
           uint32_t o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint32_t b0 = one(), b1 = one(), b2 = one(), b3 = one();
-            o[q] = (b0 & 0xffu) | ((b1 & 0xffu) << 8) | ((b2 & 0xffu) << 16) | (b3 << 24);
+            uint32_t pair[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // two symbols take at most 30 of the 32 bits looked at
+              uint32_t x = rd.peek(), used = 0;
+              const uint32_t b0 = one(x, used);
+              const uint32_t b1 = one(x, used);
+              rd.skip(used);
+              pair[h] = __byte_perm(b0, b1, 0x0040);
+            }
+            o[q] = __byte_perm(pair[0], pair[1], 0x5410);
           }
           __stcs(reinterpret_cast<uint4*>(dst + 16 * g), make_uint4(o[0], o[1], o[2], o[3]));
         }
-        for (uint32_t i = groups * 16; i < mine; ++i) dst[i] = (uint8_t)one();
+        for (uint32_t i = groups * 16; i < mine; ++i) {
+          uint32_t x = rd.peek(), used = 0;
+          dst[i] = (uint8_t)one(x, used);
+          rd.skip(used);
+        }
         // the chain must end in state 128 exactly at the sub-stream's first bit
         bad |= invalid || state != 128u || rd.position() != (int64_t)(32ull * w0 + start);
       }
