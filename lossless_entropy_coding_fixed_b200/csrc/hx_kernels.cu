@@ -344,7 +344,9 @@ __global__ void __launch_bounds__(kMeasureThreads, 3) k_measure(EncodeArgs a) {
   }
 }
 
-constexpr int kPackThreads = 256;  // a warp per chunk; lane p codes piece p (128 bytes)
+// a warp per chunk; lane p codes piece p (128 bytes). One block of 24 warps per SM shares one
+// copy of the code table (measured best: more warps starve L1, fewer leave issue slots idle)
+constexpr int kPackThreads = 768;
 constexpr int kPackCopies = 32;    // lane l reads copy l: no bank conflicts
 constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
 constexpr uint32_t kMaxPieceBits = 128 * HX_LMAX_MAX;
@@ -420,7 +422,7 @@ __device__ __forceinline__ uint32_t pack_piece(const uint8_t* src, uint32_t m, c
   return lo;
 }
 
-__global__ void __launch_bounds__(kPackThreads, 2) k_pack(EncodeArgs a) {
+__global__ void __launch_bounds__(kPackThreads, 1) k_pack(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   PackSmem& sm = *reinterpret_cast<PackSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
