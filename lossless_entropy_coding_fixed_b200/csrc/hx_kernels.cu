@@ -57,6 +57,7 @@ __host__ __device__ inline uint64_t payload_offset(uint64_t n) {
 }
 
 // ---------------------------------------------------------------------------------- histogram
+static_assert(kHistThreads == 256, "k_histogram sums bin `tid` of every warp's table");
 __global__ void __launch_bounds__(kHistThreads) k_histogram(const uint8_t* __restrict__ in,
                                                             uint64_t n, uint32_t* counts) {
   __shared__ uint32_t bins[kHistThreads / 32][256];
@@ -288,20 +289,23 @@ __device__ void measure_chunks(const EncodeArgs& a, MeasureSmem& sm) {
 
   auto flush_hist = [&]() {  // counts of the table copies -> global, then clear them
     __syncthreads();
-    uint32_t sum = 0;
-    for (int l = 0; l < kMeasureCopies; ++l) {
-      const uint32_t e = sm.lut[tid * kMeasureCopies + l];
-      sum += e >> 16;
-      sm.lut[tid * kMeasureCopies + l] = e & 0xffffu;
+    for (int sym = tid; sym < 256; sym += kMeasureThreads) {
+      uint32_t sum = 0;
+      for (int l = 0; l < kMeasureCopies; ++l) {
+        const uint32_t e = sm.lut[sym * kMeasureCopies + l];
+        sum += e >> 16;
+        sm.lut[sym * kMeasureCopies + l] = e & 0xffffu;
+      }
+      if (sum) atomicAdd(&a.hist[sym], sum);
     }
-    if (sum) atomicAdd(&a.hist[tid], sum);
     __syncthreads();
   };
 
-  // round r: warp w measures the block's chunk 8r + w
-  const uint32_t rounds = (m + 7) / 8;
+  // round r: warp w measures the block's chunk kWarps * r + w
+  constexpr uint32_t kWarps = kMeasureThreads / 32;
+  const uint32_t rounds = (m + kWarps - 1) / kWarps;
   for (uint32_t r = 0; r < rounds; ++r) {
-    const uint32_t i = r * 8 + warp;
+    const uint32_t i = r * kWarps + warp;
     if (i < m) {
       const uint32_t c = c0 + i;
       const uint32_t bits =
@@ -889,10 +893,12 @@ __global__ void __launch_bounds__(kShThreads) k_sh_measure(EncodeArgs a) {
   if (tid == 0) a.btotal[blockIdx.x] = total;
   if (hist) {
     __syncthreads();
-    uint32_t sum = 0;
+    for (int sym = tid; sym < 256; sym += kShThreads) {
+      uint32_t sum = 0;
 #pragma unroll
-    for (int w = 0; w < kShThreads / 32; ++w) sum += sm.hist[w][tid];
-    if (sum) atomicAdd(&a.hist[tid], sum);
+      for (int w = 0; w < kShThreads / 32; ++w) sum += sm.hist[w][sym];
+      if (sum) atomicAdd(&a.hist[sym], sum);
+    }
   }
 }
 
