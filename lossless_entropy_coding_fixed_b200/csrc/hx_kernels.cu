@@ -195,7 +195,7 @@ __device__ uint32_t block_exclusive_scan(uint32_t* cnt, uint32_t m, uint32_t* re
   return total;
 }
 
-constexpr int kMeasureThreads = 256;
+constexpr int kMeasureThreads = 768;  // one block of 24 warps per SM, one table for all
 constexpr int kMeasureCopies = 32;            // lane l reads copy l: no bank conflicts
 constexpr uint32_t kMaxChunksPerBlock = 4096;  // chunks of one measure block
 constexpr uint32_t kMaxMeasureBlocks = 2048;
@@ -323,7 +323,7 @@ __device__ void measure_chunks(const EncodeArgs& a, MeasureSmem& sm) {
   if (HIST) flush_hist();
 }
 
-__global__ void __launch_bounds__(kMeasureThreads, 3) k_measure(EncodeArgs a) {
+__global__ void __launch_bounds__(kMeasureThreads, 1) k_measure(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   MeasureSmem& sm = *reinterpret_cast<MeasureSmem*>(smem_raw);
   const int tid = threadIdx.x;
