@@ -58,7 +58,7 @@ typedef enum {
   HX_ERR_CAPACITY = 64   /* encode: out_cap is too small; header.total_words holds the need */
 } hx_status;
 
-enum { HX_KIND_HUFFMAN = 0, HX_KIND_QLC = 1, HX_KIND_SHANNONIC = 2 };
+enum { HX_KIND_HUFFMAN = 0, HX_KIND_QLC = 1, HX_KIND_SHANNONIC = 2, HX_KIND_EXPGOLOMB = 3 };
 enum { HX_SHN_K = 16, HX_SHN_L = 128, HX_SHN_R = 7 }; /* Shannonic: ranges, tANS states, log2 L */
 enum { HX_CHUNK = 4096, HX_SUBSTREAMS = 8, HX_LMAX_MAX = 12, HX_QLC_LMAX = 11 };
 enum { HX_CB_SEEN_ONLY = 1 }; /* hx_build_codebook flag: no code for bytes with count 0 */
@@ -114,6 +114,16 @@ int hx_qlc_build(const uint64_t* counts, int max_distinct, uint32_t flags, hx_co
  * (ties to the lower range); states spread with step 83. The offset inside the range takes
  * ceil(log2 size_r) bits. flags must be 0. */
 int hx_shannonic_build(const uint64_t* counts, int K, uint32_t flags, hx_codebook* out);
+
+/* Exp-Golomb codebook: the universal code the QLC page contrasts QLC with ("faster to decode
+ * but [not exploiting] the symbol frequency distributions"), as a no-table reference point. A
+ * byte b maps to an index v -- map 0 (sign-magnitude bytes such as e4m3): v = ((b & 0x7f) << 1)
+ * | (b >> 7); map 1 (two's complement bytes such as INT8): zigzag, v = 2x for x >= 0, -2x - 1 for
+ * x < 0 -- and v is coded by Exp-Golomb of order k: floor(log2(v / 2^k + 1)) zeros, then v + 2^k
+ * in binary (ITU-T H.264 section 9.1 is order 0). order 5..8 keeps every code within 12 bits.
+ * The codebook is a prefix code like a Huffman one (len/code filled, lmax = order); hash =
+ * FNV-1a-64 of [3, order, map]. */
+int hx_expgolomb_build(int order, int map, hx_codebook* out);
 
 /* Pack a codebook into the HX_TABLES_BYTES table block in host memory (host_tables). */
 int hx_codebook_tables(const hx_codebook* cb, void* host_tables);
@@ -210,6 +220,14 @@ int hx_shannonic_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, v
                         uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
                         void* stream);
 int hx_shannonic_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
+                        uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream);
+
+/* Exp-Golomb encode and decode (kind 3 tables from hx_expgolomb_build): the prefix-code path of
+ * hx_encode / hx_decode with the universal code; same stream, arguments and errors. */
+int hx_expgolomb_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                        uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
+                        void* stream);
+int hx_expgolomb_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
                         uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream);
 
 /* Allocation-free encode. The pages have no counterpart to this call: it exists for callers

@@ -342,6 +342,32 @@ int hx_qlc_build(const uint64_t* counts, int max_distinct, uint32_t flags, hx_co
   return fill_qlc(counts, max_distinct, out);
 }
 
+int hx_expgolomb_build(int order, int map, hx_codebook* out) {
+  if (!out || order < 5 || order > 8 || (map != 0 && map != 1)) return HX_ERR_ARG;
+  hx_codebook cb;
+  std::memset(&cb, 0, sizeof cb);
+  cb.kind = HX_KIND_EXPGOLOMB;
+  cb.lmax = (uint8_t)order;
+  for (int b = 0; b < 256; ++b) {
+    int v;
+    if (map == 0) {
+      v = ((b & 0x7f) << 1) | (b >> 7);
+    } else {
+      const int x = (int)(int8_t)(uint8_t)b;
+      v = x >= 0 ? 2 * x : -2 * x - 1;
+    }
+    const uint32_t w = (uint32_t)v + (1u << order);  // written after (bits of w) - order - 1 zeros
+    int top = 0;
+    while ((w >> (top + 1)) != 0) ++top;
+    cb.len[b] = (uint8_t)(2 * top - order + 1);
+    cb.code[b] = (uint16_t)w;
+  }
+  const uint8_t bytes[3] = {HX_KIND_EXPGOLOMB, (uint8_t)order, (uint8_t)map};
+  cb.hash = fnv1a_update(kFnvBasis, bytes, 3);
+  *out = cb;
+  return HX_OK;
+}
+
 int hx_shannonic_build(const uint64_t* counts, int K, uint32_t flags, hx_codebook* out) {
   if (!counts || !out || flags || K < 1 || K > kShK) return HX_ERR_ARG;
   uint64_t w[256];
@@ -369,7 +395,8 @@ uint64_t hx_shannonic_encode_bound(uint64_t n) {
 
 int hx_codebook_tables(const hx_codebook* cb, void* host_tables) {
   if (!cb || !host_tables) return HX_ERR_ARG;
-  if (cb->kind != HX_KIND_HUFFMAN && cb->kind != HX_KIND_QLC && cb->kind != HX_KIND_SHANNONIC)
+  if (cb->kind != HX_KIND_HUFFMAN && cb->kind != HX_KIND_QLC && cb->kind != HX_KIND_SHANNONIC &&
+      cb->kind != HX_KIND_EXPGOLOMB)
     return HX_ERR_ARG;
   std::memset(host_tables, 0, HX_TABLES_BYTES);
   hx::Tables* t = static_cast<hx::Tables*>(host_tables);

@@ -1137,7 +1137,7 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
 struct DeviceInfo {
   int sms = 0;
   int measure_per_sm = 0, pack_per_sm = 0, huff_per_sm = 0, qlc_per_sm = 0, hist_per_sm = 0;
-  int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0;
+  int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0, eg_per_sm = 0;
 };
 
 // Sets the shared-memory carveout of `fn` to the smallest share that still holds `per_sm` blocks,
@@ -1201,6 +1201,8 @@ bool device_info(DeviceInfo* out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_pack_per_sm, k_sh_pack, kShThreads,
                                                       sizeof(ShPackSmem)) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_decode_per_sm, k_sh_decode,
+                                                      kDecThreads, 0) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.eg_per_sm, k_decode<HX_KIND_EXPGOLOMB>,
                                                       kDecThreads, 0) != cudaSuccess)
       return false;
     if (d.sh_measure_per_sm < 1 || d.sh_pack_per_sm < 1 || d.sh_decode_per_sm < 1) return false;
@@ -1212,6 +1214,8 @@ bool device_info(DeviceInfo* out) {
     if (!prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_HUFFMAN>), d.huff_per_sm,
                    kDecThreads) ||
         !prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_QLC>), d.qlc_per_sm,
+                   kDecThreads) ||
+        !prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_EXPGOLOMB>), d.eg_per_sm,
                    kDecThreads))
       return false;
     d.sms = sms;
@@ -1230,7 +1234,8 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
                 uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
                 EncodeArgs* a, DeviceInfo* info) {
   if (!d_tables || !d_out || !d_scratch || !d_status || (n && !d_in)) return HX_ERR_ARG;
-  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC && kind != HX_KIND_SHANNONIC)
+  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC && kind != HX_KIND_SHANNONIC &&
+      kind != HX_KIND_EXPGOLOMB)
     return HX_ERR_ARG;
   if (n >= (1ull << 32) || out_cap < payload_offset(n) + 8) return HX_ERR_ARG;
   if (!aligned16(d_in) || !aligned16(d_out) || !aligned16(d_scratch) || !aligned16(d_tables))
@@ -1308,6 +1313,7 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   const uint64_t per_block = kDecThreads / 8;
   const int per_sm = kind == HX_KIND_HUFFMAN ? info.huff_per_sm
                      : kind == HX_KIND_QLC   ? info.qlc_per_sm
+                     : kind == HX_KIND_EXPGOLOMB ? info.eg_per_sm
                                              : info.sh_decode_per_sm;
   const uint64_t want = (nchunks + per_block - 1) / per_block;
   const uint32_t grid =
@@ -1325,6 +1331,8 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
     k_decode<HX_KIND_HUFFMAN><<<grid, kDecThreads, 0, s>>>(a);
   else if (kind == HX_KIND_QLC)
     k_decode<HX_KIND_QLC><<<grid, kDecThreads, 0, s>>>(a);
+  else if (kind == HX_KIND_EXPGOLOMB)
+    k_decode<HX_KIND_EXPGOLOMB><<<grid, kDecThreads, 0, s>>>(a);
   else
     k_sh_decode<<<grid, kDecThreads, 0, s>>>(a);
   return launched();
@@ -1456,10 +1464,24 @@ int hx_shannonic_decode(const void* d_tables, const void* d_stream, uint64_t str
                        d_status, stream);
 }
 
+int hx_expgolomb_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
+                        uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
+                        void* stream) {
+  return encode_common(HX_KIND_EXPGOLOMB, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist,
+                       d_status, stream);
+}
+
+int hx_expgolomb_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes,
+                        uint8_t* d_out, uint64_t n_expected, uint32_t* d_status, void* stream) {
+  return decode_common(HX_KIND_EXPGOLOMB, &d_tables, 1, d_stream, stream_bytes, d_out,
+                       n_expected, d_status, stream);
+}
+
 int hx_decode_set(uint32_t kind, const void* const* d_tables, uint32_t n_tables,
                   const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
                   uint64_t n_expected, uint32_t* d_status, void* stream) {
-  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC && kind != HX_KIND_SHANNONIC)
+  if (kind != HX_KIND_HUFFMAN && kind != HX_KIND_QLC && kind != HX_KIND_SHANNONIC &&
+      kind != HX_KIND_EXPGOLOMB)
     return HX_ERR_ARG;
   return decode_common(kind, d_tables, n_tables, d_stream, stream_bytes, d_out, n_expected,
                        d_status, stream);

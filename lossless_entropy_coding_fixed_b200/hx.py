@@ -18,7 +18,7 @@ from . import build as _build
 
 HX_OK, HX_ERR_ARG, HX_ERR_CUDA = 0, 1, 2
 HX_ERR_UNCODABLE, HX_ERR_CORRUPT, HX_ERR_CODEBOOK, HX_ERR_TIMEOUT, HX_ERR_CAPACITY = 4, 8, 16, 32, 64
-KIND_HUFFMAN, KIND_QLC, KIND_SHANNONIC = 0, 1, 2
+KIND_HUFFMAN, KIND_QLC, KIND_SHANNONIC, KIND_EXPGOLOMB = 0, 1, 2, 3
 CHUNK, SUBSTREAMS, LMAX_MAX, QLC_LMAX = 4096, 8, 12, 11
 CB_SEEN_ONLY = 1
 TABLES_BYTES = 10240
@@ -77,6 +77,9 @@ def lib():
             "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_encode_noalloc": (i32, [P, P, u64, P, u64, P, P, P]),
             "hx_shannonic_build": (i32, [P, i32, u32, CB]),
+            "hx_expgolomb_build": (i32, [i32, i32, CB]),
+            "hx_expgolomb_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
+            "hx_expgolomb_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_shannonic_encode_bound": (u64, [u64]),
             "hx_shannonic_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
             "hx_shannonic_decode": (i32, [P, P, u64, P, u64, P, P]),
@@ -218,6 +221,14 @@ def shannonic_build(counts, K: int = 16) -> Codebook:
     return Codebook(raw)
 
 
+def expgolomb_build(order: int = 5, map: int = 0) -> Codebook:
+    """hx_expgolomb_build: Exp-Golomb of order 5..8 over a sign/magnitude (map 0) or zigzag
+    (map 1) index of the byte."""
+    raw = _Codebook()
+    _check(lib().hx_expgolomb_build(int(order), int(map), ctypes.byref(raw)), "hx_expgolomb_build")
+    return Codebook(raw)
+
+
 def entropy(counts) -> float:
     """Shannon entropy of a 256-bin histogram, bits per symbol."""
     c = _counts(counts)
@@ -296,7 +307,7 @@ def encode(tables, x, out=None, scratch=None, hist=None, status=None, kind: int 
     if status is None:
         status = new_status(x.device)
     fn = {KIND_HUFFMAN: lib().hx_encode, KIND_QLC: lib().hx_qlc_encode,
-          KIND_SHANNONIC: lib().hx_shannonic_encode}[kind]
+          KIND_SHANNONIC: lib().hx_shannonic_encode, KIND_EXPGOLOMB: lib().hx_expgolomb_encode}[kind]
     _check(fn(tables.data_ptr(), x.data_ptr(), n, out.data_ptr(), out.numel(), scratch.data_ptr(),
               hist.data_ptr() if hist is not None else None, status.data_ptr(), _stream(x)),
            "hx_encode")
@@ -351,7 +362,7 @@ def decode(tables, stream, n: int, out=None, status=None, kind: int = KIND_HUFFM
     if status is None:
         status = new_status(stream.device)
     fn = {KIND_HUFFMAN: lib().hx_decode, KIND_QLC: lib().hx_qlc_decode,
-          KIND_SHANNONIC: lib().hx_shannonic_decode}[kind]
+          KIND_SHANNONIC: lib().hx_shannonic_decode, KIND_EXPGOLOMB: lib().hx_expgolomb_decode}[kind]
     _check(fn(tables.data_ptr(), stream.data_ptr(), int(nbytes or stream.numel()),
               out.data_ptr() if n else stream.data_ptr(), n, status.data_ptr(), _stream(stream)),
            "hx_decode")

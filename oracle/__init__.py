@@ -18,7 +18,7 @@ SRC = os.path.join(HERE, "oracle.cpp")
 LIB = os.path.join(HERE, "liboracle.so")
 
 ERR_ARG, ERR_UNCODABLE, ERR_CORRUPT, ERR_CODEBOOK, ERR_CAPACITY = 1, 4, 8, 16, 64
-KIND_HUFFMAN, KIND_QLC, KIND_SHANNONIC = 0, 1, 2
+KIND_HUFFMAN, KIND_QLC, KIND_SHANNONIC, KIND_EXPGOLOMB = 0, 1, 2, 3
 SHN_K, SHN_L, SHN_R = 16, 128, 7
 QLC_LMAX = 11
 
@@ -65,6 +65,10 @@ def lib():
             "orc_shannonic_encode_bound": (u64, [u64]),
             "orc_encode_shannonic": (i32, [i32, P, P, P, u64, P, u64, P]),
             "orc_decode_shannonic": (i32, [i32, P, P, P, u64, P, u64]),
+            "orc_expgolomb_codes": (i32, [i32, i32, P, P]),
+            "orc_hash_expgolomb": (u64, [i32, i32]),
+            "orc_encode_expgolomb": (i32, [i32, i32, P, u64, P, u64, P]),
+            "orc_decode_expgolomb": (i32, [i32, i32, P, u64, P, u64]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -197,6 +201,30 @@ def shannonic_normalise(range_weights) -> np.ndarray:
     return f
 
 
+@dataclass
+class ExpGolombBook:
+    """[EG] order and byte-to-index map (0 sign-magnitude, 1 two's complement zigzag)."""
+    order: int
+    map: int
+    kind: int = KIND_EXPGOLOMB
+
+    @property
+    def hash(self) -> int:
+        return int(lib().orc_hash_expgolomb(self.order, self.map))
+
+    @property
+    def codes(self) -> tuple[np.ndarray, np.ndarray]:
+        ln = np.zeros(256, np.uint8)
+        code = np.zeros(256, np.uint32)
+        if lib().orc_expgolomb_codes(self.order, self.map, _p(ln), _p(code)):
+            raise ValueError("bad Exp-Golomb order or map")
+        return ln, code
+
+    @property
+    def len(self) -> np.ndarray:
+        return self.codes[0]
+
+
 def shannonic_encode_bound(n: int) -> int:
     return int(lib().orc_shannonic_encode_bound(n))
 
@@ -204,6 +232,13 @@ def shannonic_encode_bound(n: int) -> int:
 def encode(cb, x, cap: int | None = None) -> tuple[int, np.ndarray]:
     """Bit-serial encode into the chunked stream; returns (status, stream bytes)."""
     x = _u8(x)
+    if cb.kind == KIND_EXPGOLOMB:
+        cap = encode_bound(x.size) if cap is None else int(cap)
+        out = np.zeros(max(cap, 1), dtype=np.uint8)
+        written = ctypes.c_uint64(0)
+        st = lib().orc_encode_expgolomb(cb.order, cb.map, _p(x), x.size, _p(out), cap,
+                                        ctypes.byref(written))
+        return int(st), out[: written.value] if written.value else out[: min(cap, 64)]
     if cb.kind == KIND_SHANNONIC:
         cap = shannonic_encode_bound(x.size) if cap is None else int(cap)
         out = np.zeros(max(cap, 1), dtype=np.uint8)
@@ -227,7 +262,9 @@ def decode(cb, stream, n: int) -> tuple[int, np.ndarray]:
     """Bit-serial decode; returns (status, n bytes)."""
     s = _u8(stream)
     out = np.zeros(max(n, 1), dtype=np.uint8)
-    if cb.kind == KIND_SHANNONIC:
+    if cb.kind == KIND_EXPGOLOMB:
+        st = lib().orc_decode_expgolomb(cb.order, cb.map, _p(s), s.size, _p(out), n)
+    elif cb.kind == KIND_SHANNONIC:
         st = lib().orc_decode_shannonic(cb.nr, _p(cb.lo), _p(cb.f), _p(s), s.size, _p(out), n)
     elif cb.kind == KIND_HUFFMAN:
         st = lib().orc_decode_huffman(cb.lmax, _p(cb.len), _p(s), s.size, _p(out), n)

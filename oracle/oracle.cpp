@@ -19,6 +19,9 @@
 //         entropy plus the fixed-width offset bits; the range index is coded by 128-state tANS
 //         (J. Duda, asymmetric numeral systems, table variant), the offset in ceil(log2 size)
 //         bits.
+//   [EG]  the QLC page's contrast case, universal Exp-Golomb codes: order k codes v >= 0 as
+//         floor(log2(v / 2^k + 1)) zeros, then v + 2^k in binary (ITU-T H.264 section 9.1
+//         is the order-0 case); a byte is first mapped to v by its sign and magnitude.
 //
 // Readings where the pages are silent (all stated once more in the design notes):
 //   - averaging over equal-size batches == summing their counts; every byte gets a code
@@ -684,6 +687,52 @@ bool shn_from(int nr, const int* lo, const int* f, Shn& t) {
   return true;
 }
 
+// ---- [EG] Exp-Golomb over a sign/magnitude index ----------------------------------------------
+// map 0 (sign-magnitude bytes, e4m3): v = (magnitude << 1) | sign; map 1 (two's complement,
+// INT8): v = 2x for x >= 0 and -2x - 1 for x < 0 (zigzag).
+constexpr uint8_t kKindExpGolomb = 3;
+
+int eg_index(int byte, int map) {
+  if (map == 0) return ((byte & 0x7f) << 1) | (byte >> 7);
+  const int x = byte >= 128 ? byte - 256 : byte;
+  return x >= 0 ? 2 * x : -2 * x - 1;
+}
+
+void eg_codes(int order, int map, uint8_t* len, uint32_t* code) {
+  for (int b = 0; b < 256; ++b) {
+    const uint32_t v = (uint32_t)eg_index(b, map) + (1u << order);
+    int top = 0;  // bits of v + 2^k
+    while ((v >> top) > 1) ++top;
+    len[b] = (uint8_t)(2 * top - order + 1);  // (top - order) zeros, then top + 1 bits
+    code[b] = v;
+  }
+}
+
+uint64_t eg_hash(int order, int map) {
+  return fnv1a({kKindExpGolomb, (uint8_t)order, (uint8_t)map});
+}
+
+struct EgDecoder {  // [EG]: count zeros, then read that many + order + 1 bits
+  int order;
+  int byte_of[512];  // index v -> byte (-1: no byte has it)
+  EgDecoder(int order_, int map) : order(order_) {
+    for (int v = 0; v < 512; ++v) byte_of[v] = -1;
+    for (int b = 0; b < 256; ++b) byte_of[eg_index(b, map)] = b;
+  }
+  int next(BitReader& br) const {
+    int zeros = 0;
+    while (br.get() == 0) {
+      if (br.past_end || ++zeros > 16) return -1;
+    }
+    if (br.past_end) return -1;
+    uint32_t v = 1;
+    for (int i = 0; i < zeros + order; ++i) v = (v << 1) | (uint32_t)br.get();
+    if (br.past_end) return -1;
+    v -= 1u << order;
+    return v < 512 ? byte_of[v] : -1;
+  }
+};
+
 }  // namespace
 
 // ================================ C entry points (ctypes) ====================================
@@ -840,6 +889,29 @@ int orc_decode_shannonic(int nr, const int* lo, const int* f, const uint8_t* str
   Shn t;
   if (!shn_from(nr, lo, f, t)) return kErrArg;
   return shn_decode(t, stream, bytes, out, n);
+}
+
+// [EG] per-byte code words, hash, encode and decode.
+int orc_expgolomb_codes(int order, int map, uint8_t* len, uint32_t* code) {
+  if (order < 0 || order > 8 || (map != 0 && map != 1) || !len || !code) return kErrArg;
+  eg_codes(order, map, len, code);
+  return 0;
+}
+uint64_t orc_hash_expgolomb(int order, int map) { return eg_hash(order, map); }
+int orc_encode_expgolomb(int order, int map, const uint8_t* x, uint64_t n, uint8_t* out,
+                         uint64_t cap, uint64_t* written) {
+  uint8_t len[256];
+  uint32_t code[256];
+  if (orc_expgolomb_codes(order, map, len, code)) return kErrArg;
+  Header h{kKindExpGolomb, (uint8_t)order, eg_hash(order, map)};
+  return encode(h, len, code, x, n, out, cap, written);
+}
+int orc_decode_expgolomb(int order, int map, const uint8_t* stream, uint64_t bytes, uint8_t* out,
+                         uint64_t n) {
+  if (order < 0 || order > 8 || (map != 0 && map != 1)) return kErrArg;
+  Header h{kKindExpGolomb, (uint8_t)order, eg_hash(order, map)};
+  EgDecoder dec(order, map);
+  return decode(h, dec, stream, bytes, out, n);
 }
 
 }  // extern "C"
