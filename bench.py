@@ -51,6 +51,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-online", action="store_true")
     p.add_argument("--no-shannonic", action="store_true")
+    p.add_argument("--no-expgolomb", action="store_true")
     return p.parse_args()
 
 
@@ -234,6 +235,36 @@ def shannonic_leg(dev, hx, torch, x, prior, h, scratch, y, status, steps):
             "decode_GB_per_s_uncompressed": n / (res["decode"] * 1e-3) / 1e9,
             "ranges": int(cb.raw.sh_nr),
             "bits_per_symbol": {"framed": size * 8 / n, "tans_ideal": hx.mean_length(h, cb)}}
+
+
+def expgolomb_leg(dev, hx, torch, x, h, scratch, y, status, steps):
+    """Exp-Golomb (the QLC page's universal-code contrast) on the same batch: the order 5..8 with
+    the shortest mean length on the batch's own histogram (sign-magnitude index, e4m3), encode and
+    decode device time per call, bits per symbol."""
+    n = x.numel()
+    books = {k: hx.expgolomb_build(k, 0) for k in (5, 6, 7, 8)}
+    order = min(books, key=lambda k: hx.mean_length(h, books[k]))
+    t = books[order].upload(dev)
+    out = torch.empty(hx.encode_bound(n), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for name, fn in (("encode", lambda: hx.encode(t, x, out=out, scratch=scratch, status=status,
+                                                  kind=hx.KIND_EXPGOLOMB)),
+                     ("decode", lambda: hx.decode(t, out, n, out=y, status=status,
+                                                  kind=hx.KIND_EXPGOLOMB))):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = a.elapsed_time(b) / steps
+    assert int(status.item()) == 0 and torch.equal(x, y)
+    return {"order": order, "encode_ms": res["encode"], "decode_ms": res["decode"],
+            "bits_per_symbol": {"framed": hx.stream_size(out, n) * 8 / n,
+                                "payload": hx.mean_length(h, books[order])}}
 
 
 def online_leg(dev, hx, datagen, torch):
@@ -480,6 +511,11 @@ def main():
         shannonic = shannonic_leg(dev, hx, torch, x, prior, h, scratch, y, status,
                                   max(3, min(args.steps, 10)))
 
+    expgolomb = None
+    if not args.no_expgolomb:
+        expgolomb = expgolomb_leg(dev, hx, torch, x, h, scratch, y, status,
+                                  max(3, min(args.steps, 10)))
+
     online = None
     if not args.no_online:
         online = online_leg(dev, hx, datagen, torch)
@@ -519,6 +555,7 @@ def main():
             "e2e": e2e,
             "online": online,
             "shannonic": shannonic,
+            "expgolomb": expgolomb,
             "gpu_launches": 6 * args.steps,
             "clocks": clocks.summary(),
         }
