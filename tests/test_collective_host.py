@@ -1,0 +1,77 @@
+"""The compressed all-gather's exchange on CPU ranks (gloo, world size 2), with a stand-in coder:
+the real one needs a GPU. Checks the size exchange, the padding to the longest stream, the
+reassembly in rank order and the refusal of unequal shards."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from lossless_entropy_coding_fixed_b200 import collective, hx
+
+
+class StandInCodec(collective.Codec):
+    """A 'stream' in the library's layout with the shard's bytes as payload: header with
+    total_words, then the bytes at the payload offset (the length depends on the shard)."""
+
+    def bound(self, n):
+        return hx.payload_offset(n) + n + 64
+
+    def encode(self, tables, x, out):
+        n = x.numel()
+        keep = n - int(x[0]) % 7  # streams of different lengths on different ranks
+        words = (keep + 3) // 4
+        out.zero_()
+        out[32:40] = torch.tensor([words], dtype=torch.int64).view(torch.uint8)
+        P = hx.payload_offset(n)
+        out[P:P + n] = x
+
+    def decode(self, tables, stream, n, out):
+        P = hx.payload_offset(n)
+        assert stream.numel() == hx.stream_bytes(n, int(stream[32:40].view(torch.int64)[0]))
+        out.copy_(stream[P:P + n]) if stream.numel() >= P + n else out.copy_(torch.cat(
+            [stream[P:], torch.zeros(P + n - stream.numel(), dtype=torch.uint8)]))
+
+
+def _run(rank, world, port, n, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        x = torch.from_numpy(np.random.default_rng(rank).integers(0, 256, n, dtype=np.uint8))
+        out, sizes = collective.compressed_all_gather(x, None, codec=StandInCodec())
+        results[rank] = (out.numpy().copy(), sizes)
+    finally:
+        dist.destroy_process_group()
+
+
+def _port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_two_ranks_gather_in_rank_order():
+    n, world = 10000, 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        results = m.dict()
+        port = _port()
+        procs = [ctx.Process(target=_run, args=(r, world, port, n, results)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0
+        expect = np.concatenate([np.random.default_rng(r).integers(0, 256, n, dtype=np.uint8)
+                                 for r in range(world)])
+        keep = [n - int(expect[r * n]) % 7 for r in range(world)]
+        for r in range(world):
+            out, sizes = results[r]
+            assert sizes == [hx.stream_bytes(n, (k + 3) // 4) for k in keep]
+            for q in range(world):
+                got = out[q * n:(q + 1) * n]
+                # the stand-in keeps the whole shard whenever the stream holds it
+                assert (got[:keep[q] - 3] == expect[q * n:q * n + keep[q] - 3]).all()

@@ -1,0 +1,62 @@
+"""The compressed all-gather on a GPU with NCCL and the real coder. Runs as one rank (this pool
+gives one GPU per run; the exchange logic for two ranks is covered on CPU ranks), in a child
+process so the process group does not outlive the test."""
+import os
+import socket
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+
+def _port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(port, q):
+    import datetime
+
+    import torch.distributed as dist
+
+    import datagen
+    from lossless_entropy_coding_fixed_b200 import collective, hx
+    import oracle
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda:0"))
+    try:
+        res = {}
+        for kind in (hx.KIND_HUFFMAN, hx.KIND_QLC):
+            x = datagen.data(1, n=(1 << 20) - 77)
+            prior = sum(oracle.histogram(b) for b in datagen.prior_batches(1))
+            cb = hx.build_codebook(prior) if kind == hx.KIND_HUFFMAN else hx.qlc_build(prior)
+            ocb = oracle.huffman_codebook(prior) if kind == hx.KIND_HUFFMAN else oracle.qlc_codebook(prior)
+            out, sizes = collective.compressed_all_gather(torch.from_numpy(x).cuda(), cb.upload("cuda"),
+                                                          codec=collective.Codec(kind))
+            torch.cuda.synchronize()
+            res[kind] = (bool((out.cpu().numpy() == x).all()), sizes, int(oracle.encode(ocb, x)[1].size))
+        q.put(res)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_one_rank_round_trip():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_rank, args=(_port(), q))
+    p.start()
+    res = q.get(timeout=300)
+    p.join(120)
+    assert p.exitcode == 0
+    for kind, (ok, sizes, ref_size) in res.items():
+        assert ok and sizes == [ref_size], kind
