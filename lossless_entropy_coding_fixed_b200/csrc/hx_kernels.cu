@@ -355,11 +355,23 @@ constexpr int kPackCopies = 32;    // lane l reads copy l: no bank conflicts
 constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
 constexpr uint32_t kMaxPieceBits = 128 * HX_LMAX_MAX;
 
+// Two layouts of a warp's chunk buffer, chosen per chunk:
+//   plain   chunk word w at w + (the chunk's word offset & 3), so that 16-byte aligned runs of the
+//           payload are 16-byte aligned here too and leave as uint4;
+//   spread  chunk word w at w + w / 32 (one unused word after every 32), copied out word by word.
+// Lanes store the words their pieces finish at about the same pace, so pieces that start in the
+// same bank keep colliding; a warp takes spread when kCrowded or more of its 32 pieces start in
+// one bank (pieces a multiple of 32 words long, as when every code has 8 bits), where the plain
+// layout would serialise most of its stores.
+constexpr uint32_t kCrowded = 8;
+template <bool SPREAD>
+__device__ __forceinline__ uint32_t buf_slot(uint32_t w) { return SPREAD ? w + (w >> 5) : w; }
+constexpr uint32_t kBufWords = (kMaxChunkWords + kMaxChunkWords / 32 + 3) & ~3u;  // both fit
+static_assert(kBufWords >= kMaxChunkWords + 4, "the plain layout needs 3 words of offset");
+
 struct PackSmem {
   uint32_t lut[256 * kPackCopies];                  // [symbol][copy]: (code << 20) | len
-  // one chunk per warp; word w of the chunk sits at w + (its offset & 3), so that 16-byte
-  // aligned runs of the payload are 16-byte aligned here too
-  alignas(16) uint32_t out[kPackThreads / 32][kMaxChunkWords + 4];
+  alignas(16) uint32_t out[kPackThreads / 32][kBufWords];  // one chunk per warp
   uint32_t bpre[kMaxMeasureBlocks];                  // word offset of each measure block
   uint32_t red[kPackThreads / 32];
 };
@@ -373,9 +385,9 @@ __device__ __forceinline__ uint32_t lut_entry(const char* lut, uint32_t w, uint3
 // Codes m (<= 128) bytes at src as the bits [s, s + its length) of the chunk's word buffer:
 // two codes are joined in a 32-bit register (<= 24 bits), appended to a 64-bit accumulator
 // (hi:lo) with funnel shifts, and every word this piece finishes is stored whole (bits of earlier
-// pieces in it as zeros). Returns the unfinished last word's bits in the low *nacc bits; *widx
-// is its index.
-template <bool WHOLE>
+// pieces in it as zeros) at its buf_slot. Returns the unfinished last word's bits in the low
+// *nacc bits; *widx is its index.
+template <bool WHOLE, bool SPREAD>
 __device__ __forceinline__ uint32_t pack_piece(const uint8_t* src, uint32_t m, const char* lut,
                                                uint32_t lane4, uint32_t* buf, uint32_t s,
                                                uint32_t* widx_out, uint32_t* nacc_out) {
@@ -389,7 +401,7 @@ __device__ __forceinline__ uint32_t pack_piece(const uint8_t* src, uint32_t m, c
     nacc += pl;
     const bool full = nacc >= 32;
     nacc -= full ? 32u : 0u;
-    if (full) buf[widx] = __funnelshift_r(lo, hi, nacc);
+    if (full) buf[buf_slot<SPREAD>(widx)] = __funnelshift_r(lo, hi, nacc);
     widx += full ? 1u : 0u;
   };
   auto put_word = [&](uint32_t w, uint32_t count) {  // bytes 0..count-1 of w
@@ -424,6 +436,52 @@ __device__ __forceinline__ uint32_t pack_piece(const uint8_t* src, uint32_t m, c
   *widx_out = widx;
   *nacc_out = nacc;
   return lo;
+}
+
+// One chunk by one warp: lane p codes piece p from bit s of the chunk into the warp's buffer
+// (layout SPREAD), then the warp copies the chunk's words out to the payload at woff (none at or
+// past `limit`).
+template <bool SPREAD>
+__device__ __forceinline__ void pack_chunk(const EncodeArgs& a, uint32_t c, const char* lut,
+                                           uint32_t lane4, uint32_t* wbuf, uint32_t s,
+                                           uint32_t mine, bool last_piece, uint32_t woff,
+                                           uint32_t words, uint32_t limit, bool whole) {
+  const uint32_t lane = lane4 >> 2;
+  uint32_t* const payload = reinterpret_cast<uint32_t*>(a.out + payload_offset(a.n));
+  uint32_t* const buf = SPREAD ? wbuf : wbuf + (woff & 3);
+  uint32_t widx = 0, nacc = 0, tail = 0;
+  const uint8_t* src = a.in + (uint64_t)c * kChunk + lane * 128;
+  if (whole) {
+    tail = pack_piece<true, SPREAD>(src, 128, lut, lane4, buf, s, &widx, &nacc);
+  } else {
+    const uint64_t first = (uint64_t)c * kChunk + lane * 128;
+    const uint32_t m = first < a.n ? (uint32_t)min((uint64_t)128, a.n - first) : 0u;
+    tail = pack_piece<false, SPREAD>(src, m, lut, lane4, buf, s, &widx, &nacc);
+  }
+  // The piece's unfinished word: the chunk's last word is stored whole (zero padding); any
+  // other is OR-ed, after a warp barrier, into the word that a later piece stored whole.
+  const bool has_tail = mine != 0 && nacc != 0;
+  const bool last = mine != 0 && last_piece;
+  tail = has_tail ? tail << (32 - nacc) : 0u;
+  uint32_t* const tail_word = buf + buf_slot<SPREAD>(widx);
+  if (has_tail && last) *tail_word = tail;
+  __syncwarp();
+  if (has_tail && !last) atomicOr(tail_word, tail);
+  __syncwarp();
+  const uint32_t end = min(woff + words, limit);
+  if (SPREAD) {
+    // word by word, each warp store 128 contiguous bytes
+    for (uint32_t i = lane; woff + i < end; i += 32) payload[woff + i] = buf[buf_slot<true>(i)];
+  } else {
+    // a ragged head and tail word by word, the 16-byte aligned middle as uint4
+    const uint32_t g0 = min((woff + 3) & ~3u, end), g1 = max(end & ~3u, g0);
+    if (woff + lane < g0) payload[woff + lane] = buf[lane];
+    if (g1 + lane < end) payload[g1 + lane] = buf[g1 - woff + lane];
+    const uint4* b4 = reinterpret_cast<const uint4*>(buf + (g0 - woff));
+    uint4* p4 = reinterpret_cast<uint4*>(payload + g0);
+    for (uint32_t q = lane; q < (g1 - g0) / 4; q += 32) p4[q] = b4[q];
+  }
+  __syncwarp();
 }
 
 __global__ void __launch_bounds__(kPackThreads, 1) k_pack(EncodeArgs a) {
@@ -468,7 +526,6 @@ __global__ void __launch_bounds__(kPackThreads, 1) k_pack(EncodeArgs a) {
   for (uint32_t c = blockIdx.x * (kPackThreads / 32) + warp; c < nchunks; c += stride) {
     const uint32_t woff = sm.bpre[c / a.cpb] + a.local[c];
     if (lane == 0) word_off[c] = woff;
-    uint32_t* buf = wbuf + (woff & 3);
     // this piece's first bit: a warp prefix sum of the piece bit counts
     const uint32_t mine = min((uint32_t)a.pieces[(uint64_t)c * 32 + lane], kMaxPieceBits);
     uint32_t incl = mine;
@@ -485,33 +542,13 @@ __global__ void __launch_bounds__(kPackThreads, 1) k_pack(EncodeArgs a) {
       if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
       continue;
     }
-    uint32_t widx = 0, nacc = 0, tail = 0;
-    const uint8_t* src = a.in + (uint64_t)c * kChunk + lane * 128;
-    if (c < full_chunks) {
-      tail = pack_piece<true>(src, 128, lut, lane4, buf, s, &widx, &nacc);
-    } else {
-      const uint64_t first = (uint64_t)c * kChunk + lane * 128;
-      const uint32_t m = first < n ? (uint32_t)min((uint64_t)128, n - first) : 0u;
-      tail = pack_piece<false>(src, m, lut, lane4, buf, s, &widx, &nacc);
-    }
-    // The piece's unfinished word: the chunk's last word is stored whole (zero padding); any
-    // other is OR-ed, after a warp barrier, into the word that a later piece stored whole.
-    const bool has_tail = mine != 0 && nacc != 0;
-    const bool last = mine != 0 && incl == chunk_bits;
-    tail = has_tail ? tail << (32 - nacc) : 0u;
-    if (has_tail && last) buf[widx] = tail;
-    __syncwarp();
-    if (has_tail && !last) atomicOr(buf + widx, tail);
-    __syncwarp();
-    // out: a ragged head and tail word by word, the 16-byte aligned middle as uint4
-    const uint32_t end = min(woff + words, limit);
-    const uint32_t g0 = min((woff + 3) & ~3u, end), g1 = max(end & ~3u, g0);
-    if (woff + lane < g0) payload[woff + lane] = buf[lane];
-    if (g1 + lane < end) payload[g1 + lane] = buf[g1 - woff + lane];
-    const uint4* b4 = reinterpret_cast<const uint4*>(buf + (g0 - woff));
-    uint4* p4 = reinterpret_cast<uint4*>(payload + g0);
-    for (uint32_t q = lane; q < (g1 - g0) / 4; q += 32) p4[q] = b4[q];
-    __syncwarp();
+    const uint32_t peers = __popc(__match_any_sync(0xffffffffu, (s >> 5) & 31u));
+    if (__any_sync(0xffffffffu, peers >= kCrowded))
+      pack_chunk<true>(a, c, lut, lane4, wbuf, s, mine, incl == chunk_bits, woff, words, limit,
+                       c < full_chunks);
+    else
+      pack_chunk<false>(a, c, lut, lane4, wbuf, s, mine, incl == chunk_bits, woff, words, limit,
+                        c < full_chunks);
   }
 }
 
@@ -774,7 +811,7 @@ __device__ __forceinline__ uint32_t bfe(uint32_t x, uint32_t pos, uint32_t len) 
 }
 
 constexpr int kShThreads = 256;  // 8 threads per chunk, 32 chunks per block
-constexpr int kShCopies = 8;     // symbol table copies: lane l reads copy l % 8
+constexpr int kShCopies = 16;    // symbol table copies: lane l reads copy l % 16 (<= 2-way)
 
 // Encoder tables in shared memory.
 struct ShEnc {
@@ -807,9 +844,11 @@ __device__ __forceinline__ void sh_reverse(const EncodeArgs& a, uint32_t c, uint
   const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
   if (m == kSubLen) {
     const uint4* src = reinterpret_cast<const uint4*>(a.in + first);
+    uint4 nxt = __ldg(src + kSubLen / 16 - 1);
 #pragma unroll 1
     for (int g = kSubLen / 16 - 1; g >= 0; --g) {
-      const uint4 v = __ldg(src + g);
+      const uint4 v = nxt;
+      if (g > 0) nxt = __ldg(src + g - 1);
       const uint32_t w[4] = {v.w, v.z, v.y, v.x};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -1242,11 +1281,13 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
     return HX_ERR_ARG;
   if (!device_info(info)) return HX_ERR_CUDA;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  // measure blocks: at least one wave of resident blocks, at most kMaxChunksPerBlock chunks each
-  // (n < 2^32 gives at most 2^20 chunks, so 256 blocks always suffice)
+  // measure blocks: at least one wave of resident blocks of the kind's measure kernel, at most
+  // kMaxChunksPerBlock chunks each (n < 2^32 gives at most 2^20 chunks, so 256 blocks always
+  // suffice)
+  const int per_sm = kind == HX_KIND_SHANNONIC ? info->sh_measure_per_sm : info->measure_per_sm;
   uint32_t mblocks = (uint32_t)std::min<uint64_t>(
       {(uint64_t)nchunks, (uint64_t)kMaxMeasureBlocks,
-       std::max<uint64_t>((uint64_t)info->sms * info->measure_per_sm,
+       std::max<uint64_t>((uint64_t)info->sms * per_sm,
                           (nchunks + kMaxChunksPerBlock - 1) / kMaxChunksPerBlock)});
   const uint32_t cpb = mblocks ? (nchunks + mblocks - 1) / mblocks : 1;
   if (mblocks) mblocks = (nchunks + cpb - 1) / cpb;  // no block without chunks

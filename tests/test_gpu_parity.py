@@ -279,3 +279,35 @@ def test_other_codebook_rejected(orc, damaged_setup, cuda):
     other = hx.build_codebook(datagen.random_counts(99)).upload(cuda)
     st, _ = gpu_decode(other, s, x.size, 0)
     assert st == hx.HX_ERR_CODEBOOK == orc.decode(orc.huffman_codebook(datagen.random_counts(99)), s, x.size)[0]
+
+
+@pytest.mark.parametrize("n", [4096, 5 * 4096 + 77, 1 << 20])
+def test_flat_8bit_codes(orc, cuda, n):
+    """Every code 8 bits long (a code built from uniform counts): each 128-byte piece packs to
+    exactly 32 words, so all 32 pieces of a chunk start in one shared-memory bank and the encoder
+    takes its spread buffer layout for every chunk."""
+    counts = np.ones(256, np.uint64)
+    cb, ocb = hx.build_codebook(counts), orc.huffman_codebook(counts)
+    assert (ocb.len == 8).all()
+    tables = cb.upload(cuda)
+    x = datagen.uniform_bytes(n, 9)
+    ref = orc.encode(ocb, x)[1]
+    got, st, _ = gpu_encode(tables, x, cb.kind)
+    assert st == 0 and (got == ref).all()
+    st, y = gpu_decode(tables, ref, n, cb.kind)
+    assert st == 0 and (y == x).all()
+
+
+def test_mixed_buffer_layouts(orc, books):
+    """Chunks of bytes whose codes are all 8 bits long (spread layout) between chunks of the
+    workload's law (plain layout), in one stream."""
+    cb, tables, ocb, k = books["huffman"]
+    eight = np.flatnonzero(ocb.len == 8).astype(np.uint8)
+    assert eight.size > 0
+    rng = np.random.default_rng(31)
+    law = datagen.data(1, n=6 * 4096)
+    parts = [rng.choice(eight, 4096) if i % 2 else law[i * 4096:(i + 1) * 4096] for i in range(6)]
+    x = np.concatenate(parts + [rng.choice(eight, 1500)]).astype(np.uint8)
+    ref = orc.encode(ocb, x)[1]
+    got, st, _ = gpu_encode(tables, x, k)
+    assert st == 0 and (got == ref).all()
