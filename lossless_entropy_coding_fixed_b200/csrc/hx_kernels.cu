@@ -649,6 +649,77 @@ struct SubstreamBits {
 // most kSubLen codes of at most 15 bits (the table's length field).
 constexpr uint32_t kReaderReach = 4 + (kSubLen * 15 + 31) / 32;
 
+// The same w0:w1 window fed from 16-byte loads: a queue of the next `left` words (q0..q3, 1 to 4
+// of them), refilled with one 16-byte block when it runs dry, so a lane requests a block every
+// fourth word.
+// The decoder uses it for warps whose lanes all read the same bank of their lines (sub-streams a
+// multiple of 128 bytes apart advancing in step, as when every code has 8 bits), where it makes
+// a quarter of the conflicted load requests. Unchecked only: the caller guarantees that every
+// block it may request lies inside the buffer (kReaderReach16).
+struct SubstreamBits16 {
+  const uint4* blocks;  // the payload as 16-byte blocks (its base is 16-byte aligned)
+  uint32_t bi;          // index of the next block to request
+  uint32_t w0, w1, q0, q1, q2, q3, left;
+  uint32_t bo;
+
+  __device__ __forceinline__ static uint4 load(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+  }
+  __device__ __forceinline__ uint32_t pull() {
+    const uint32_t v = q0;
+    q0 = q1;
+    q1 = q2;
+    q2 = q3;
+    if (--left == 0) {
+      const uint4 v = load(blocks + bi++);
+      q0 = v.x;
+      q1 = v.y;
+      q2 = v.z;
+      q3 = v.w;
+      left = 4;
+    }
+    return v;
+  }
+  __device__ __forceinline__ void start(uint32_t fw, uint32_t first_bo) {
+    bi = fw >> 2;
+    const uint4 v = load(blocks + bi);
+    bi += 1;
+    q0 = v.x;
+    q1 = v.y;
+    q2 = v.z;
+    q3 = v.w;
+    left = 4;
+    for (uint32_t r = fw & 3u; r > 0; --r) pull();
+    w0 = pull();
+    w1 = pull();
+    bo = first_bo;
+  }
+  __device__ __forceinline__ uint32_t peek() const { return __funnelshift_l(w1, w0, bo); }
+  __device__ __forceinline__ void advance(uint32_t nbits) {
+    bo += nbits;
+    if (bo >= 32) {
+      bo -= 32;
+      w0 = w1;
+      w1 = pull();
+    }
+  }
+  // the queue holds words 4 * bi - left .. 4 * bi - 1, so w0 is word 4 * bi - 2 - left
+  __device__ __forceinline__ uint64_t position() const {
+    return 32ull * (4ull * bi - 2 - left) + bo;
+  }
+};
+// Words the 16-byte reader may request for a sub-stream whose first word is fw, counted from
+// 4 * (fw / 4): one block at the start and one per 4 words taken, of at most 3 + 2 + one per 32
+// bits of at most kSubLen codes of at most 15 bits.
+constexpr uint32_t kReaderPulls16 = 3 + 2 + (31 + kSubLen * 15) / 32;
+constexpr uint32_t kReaderReach16 = 4 * (1 + kReaderPulls16 / 4);
+// a warp reads with 16-byte blocks when this many of its lanes start in one bank
+constexpr uint32_t kCrowdedReaders = 16;
+
 // The decode table in shared memory: for every 12-bit window, (symbol << 8) | length of the code
 // word it starts with; 0 when none does (an incomplete code).
 struct DecLut {
@@ -659,9 +730,9 @@ struct DecLut {
 // Two symbols from the reader: table entries (symbol << 8) | length for either kind (for a QLC
 // table the length is 3 + the width of the area in the top 3 bits; the table holds it already).
 // An entry of 0 (no code word starts the window) only occurs for an incomplete code.
-template <bool COMPLETE, bool CHECKED>
-__device__ __forceinline__ void decode_pair(SubstreamBits<CHECKED>& rd, bool& invalid,
-                                            const DecLut& lut, uint32_t& e1, uint32_t& e2) {
+template <bool COMPLETE, class Reader>
+__device__ __forceinline__ void decode_pair(Reader& rd, bool& invalid, const DecLut& lut,
+                                            uint32_t& e1, uint32_t& e2) {
   const uint32_t x = rd.peek();
   e1 = lut(x);
   const uint32_t l1 = e1 & 15u;
@@ -673,9 +744,9 @@ __device__ __forceinline__ void decode_pair(SubstreamBits<CHECKED>& rd, bool& in
 
 // 32 symbols -> 32 output bytes, one 32-byte streaming store (a whole sector) when the output is
 // 32-byte aligned, else two 16-byte stores. The symbol bytes are gathered with byte permutes.
-template <bool COMPLETE, bool CHECKED>
-__device__ __forceinline__ void decode_group32(SubstreamBits<CHECKED>& rd, bool& invalid,
-                                               uint8_t* dst, bool out32, const DecLut& lut) {
+template <bool COMPLETE, class Reader>
+__device__ __forceinline__ void decode_group32(Reader& rd, bool& invalid, uint8_t* dst,
+                                               bool out32, const DecLut& lut) {
   uint32_t o[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -695,16 +766,12 @@ __device__ __forceinline__ void decode_group32(SubstreamBits<CHECKED>& rd, bool&
   }
 }
 
-// Decodes `mine` symbols of one sub-stream to dst; returns the reader's final bit position.
-template <bool COMPLETE, bool CHECKED>
-__device__ __forceinline__ uint64_t decode_substream(const uint32_t* words, uint32_t wlimit,
-                                                     uint64_t first_bit, uint32_t mine,
-                                                     uint8_t* dst, bool out32, bool& invalid,
+// Decodes `mine` symbols of one sub-stream from a started reader to dst; returns the reader's
+// final bit position.
+template <bool COMPLETE, class Reader>
+__device__ __forceinline__ uint64_t decode_substream(Reader& rd, uint32_t mine, uint8_t* dst,
+                                                     bool out32, bool& invalid,
                                                      const DecLut& lut) {
-  SubstreamBits<CHECKED> rd;
-  rd.words = words;
-  rd.wlimit = wlimit;
-  rd.start((uint32_t)(first_bit >> 5), (uint32_t)(first_bit & 31));
   const uint32_t groups = mine / 32;
   for (uint32_t g = 0; g < groups; ++g)
     decode_group32<COMPLETE>(rd, invalid, dst + 32 * g, out32, lut);
@@ -717,7 +784,7 @@ __device__ __forceinline__ uint64_t decode_substream(const uint32_t* words, uint
   return rd.position();
 }
 
-template <bool COMPLETE>
+template <bool COMPLETE, bool VOTE>
 __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut& lut,
                                               uint32_t total) {
   const int tid = threadIdx.x;
@@ -730,6 +797,7 @@ __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut&
   // payload words inside the buffer, capped at 2^32 - 1 (no payload word lies beyond 2^32 - 2)
   const uint32_t wlimit = (uint32_t)min((a.bytes - P) / 4, (uint64_t)0xffffffffull);
   const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;
+  const bool blocks16 = (reinterpret_cast<uintptr_t>(words) & 15) == 0;
   const int k = tid & 7;
 
   for (uint64_t c = (uint64_t)blockIdx.x * (kDecThreads / 8) + (tid >> 3); c < nchunks;
@@ -754,17 +822,57 @@ __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut&
       bool invalid = false;
       uint8_t* dst = a.out + c * kChunk + (uint64_t)k * kSubLen;
       uint64_t pos;
-      if ((first_bit >> 5) + kReaderReach <= wlimit)
-        pos = decode_substream<COMPLETE, false>(words, wlimit, first_bit, mine, dst, out32,
-                                                invalid, lut);
-      else
-        pos = decode_substream<COMPLETE, true>(words, wlimit, first_bit, mine, dst, out32,
-                                               invalid, lut);
+      const uint32_t fw = (uint32_t)(first_bit >> 5), fbo = (uint32_t)(first_bit & 31);
+      // VOTE: the lanes decoding now vote, and read 16-byte blocks when many of them start on
+      // one bank
+      bool crowded = false;
+      if (VOTE) {
+        const uint32_t voters = __activemask();
+        crowded = __any_sync(voters,
+                             __popc(__match_any_sync(voters, fw & 31u)) >= kCrowdedReaders);
+      }
+      if (VOTE && crowded && blocks16 && (uint64_t)(fw & ~3u) + kReaderReach16 <= wlimit) {
+        SubstreamBits16 rd;
+        rd.blocks = reinterpret_cast<const uint4*>(words);
+        rd.start(fw, fbo);
+        pos = decode_substream<COMPLETE>(rd, mine, dst, out32, invalid, lut);
+      } else if ((uint64_t)fw + kReaderReach <= wlimit) {
+        SubstreamBits<false> rd;
+        rd.words = words;
+        rd.wlimit = wlimit;
+        rd.start(fw, fbo);
+        pos = decode_substream<COMPLETE>(rd, mine, dst, out32, invalid, lut);
+      } else {
+        SubstreamBits<true> rd;
+        rd.words = words;
+        rd.wlimit = wlimit;
+        rd.start(fw, fbo);
+        pos = decode_substream<COMPLETE>(rd, mine, dst, out32, invalid, lut);
+      }
       // the sub-stream must end exactly where the next one starts
       bad |= invalid || pos != 32ull * w0 + end;
     }
     if (bad) atomicOr(a.status, (uint32_t)HX_ERR_CORRUPT);
   }
+}
+
+// Whether the sub-streams of chunk c start crowded on one bank of their lines: 4 or more of its
+// 8 first words equal modulo 32 (any flat code length does it: a sub-stream of 512 codes of L
+// bits is 16 L words long; codes of mixed lengths do it by chance for about 1 chunk in 500).
+// Read by one thread after the header checks.
+__device__ bool crowded_chunk(const DecodeArgs& a, uint64_t c) {
+  if (c >= n_chunks_of(a.n)) return false;
+  const uint32_t w0 = reinterpret_cast<const uint32_t*>(a.st + 64)[c];
+  const uint16_t* row = reinterpret_cast<const uint16_t*>(a.st + sync_offset(a.n)) + 8 * c;
+  uint32_t bank[HX_SUBSTREAMS];
+  for (int k = 0; k < HX_SUBSTREAMS; ++k)
+    bank[k] = (w0 + ((k == 0 ? 0u : (uint32_t)row[k]) >> 5)) & 31u;
+  for (int k = 0; k < HX_SUBSTREAMS; ++k) {
+    int same = 0;
+    for (int q = 0; q < HX_SUBSTREAMS; ++q) same += bank[q] == bank[k];
+    if (same >= 4) return true;
+  }
+  return false;
 }
 
 // KIND is checked against the stream header and the tables; the symbol loop is the same. (The
@@ -775,8 +883,14 @@ __global__ void __launch_bounds__(kDecThreads, KIND == HX_KIND_QLC ? 4 : 5)
   __shared__ __align__(16) uint16_t s_lut[4096];
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
+  __shared__ bool s_crowded;
   const int tid = threadIdx.x;
-  if (tid == 0) s_total = check_header(a, &s_tables);
+  if (tid == 0) {
+    s_total = check_header(a, &s_tables);
+    // the block's first chunk stands for the rest: a block whose chunks look crowded takes the
+    // voting loop (the word-by-word loop alone runs faster elsewhere)
+    s_crowded = s_total >= 0 && crowded_chunk(a, (uint64_t)blockIdx.x * (kDecThreads / 8));
+  }
   __syncthreads();
   const int64_t total = s_total;
   if (total < 0) {
@@ -789,10 +903,14 @@ __global__ void __launch_bounds__(kDecThreads, KIND == HX_KIND_QLC ? 4 : 5)
   for (int i = tid; i < 4096 * 2 / 16; i += kDecThreads) dst[i] = src[i];
   __syncthreads();
   const DecLut lut{s_lut};
-  if (tables->complete)
-    decode_chunks<true>(a, lut, (uint32_t)total);
-  else
-    decode_chunks<false>(a, lut, (uint32_t)total);
+  const bool crowded = s_crowded;
+  if (tables->complete) {
+    if (crowded) decode_chunks<true, true>(a, lut, (uint32_t)total);
+    else decode_chunks<true, false>(a, lut, (uint32_t)total);
+  } else {
+    if (crowded) decode_chunks<false, true>(a, lut, (uint32_t)total);
+    else decode_chunks<false, false>(a, lut, (uint32_t)total);
+  }
 }
 
 // ---------------------------------------------------------------------------------- shannonic
@@ -1084,8 +1202,14 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
   __shared__ uint32_t s_dec[128];
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
+  __shared__ bool s_crowded;
   const int tid = threadIdx.x;
-  if (tid == 0) s_total = check_header(a, &s_tables);
+  if (tid == 0) {
+    s_total = check_header(a, &s_tables);
+    // the block's first chunk stands for the rest: a block whose chunks look crowded takes the
+    // voting loop (the word-by-word loop alone runs faster elsewhere)
+    s_crowded = s_total >= 0 && crowded_chunk(a, (uint64_t)blockIdx.x * (kDecThreads / 8));
+  }
   __syncthreads();
   const int64_t total = s_total;
   if (total < 0) {
