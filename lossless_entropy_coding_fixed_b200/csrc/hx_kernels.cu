@@ -875,10 +875,10 @@ __device__ bool crowded_chunk(const DecodeArgs& a, uint64_t c) {
   return false;
 }
 
-// KIND is checked against the stream header and the tables; the symbol loop is the same. (The
-// register budgets are the measured best per kind: 48 for Huffman, 64 for QLC.)
+// KIND is checked against the stream header and the tables; the symbol loop is the same. (64
+// registers and 4 blocks per SM measured best for every kind.)
 template <int KIND>
-__global__ void __launch_bounds__(kDecThreads, KIND == HX_KIND_QLC ? 4 : 5)
+__global__ void __launch_bounds__(kDecThreads, 4)
     k_decode(DecodeArgs a) {
   __shared__ __align__(16) uint16_t s_lut[4096];
   __shared__ int64_t s_total;
@@ -1202,14 +1202,8 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
   __shared__ uint32_t s_dec[128];
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
-  __shared__ bool s_crowded;
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    s_total = check_header(a, &s_tables);
-    // the block's first chunk stands for the rest: a block whose chunks look crowded takes the
-    // voting loop (the word-by-word loop alone runs faster elsewhere)
-    s_crowded = s_total >= 0 && crowded_chunk(a, (uint64_t)blockIdx.x * (kDecThreads / 8));
-  }
+  if (tid == 0) s_total = check_header(a, &s_tables);
   __syncthreads();
   const int64_t total = s_total;
   if (total < 0) {
