@@ -51,3 +51,38 @@ def test_damage_matches_oracle(orc, cuda):
         assert int(st.item()) == ost
         if ost == 0:
             assert (y.cpu().numpy() == oy).all()
+
+
+def test_crowded_reader_damage_matches_oracle(orc, cuda):
+    """Order 7 on e4m3 bytes: almost every code is 8 bits, so sub-streams start on one bank of
+    their lines and the decoder's blocks take the voting loop with its 16-byte reader. Flipped
+    payload bits and damaged sync entries must raise the oracle's statuses there too."""
+    x = datagen.data(1, n=40 * 4096 + 333)
+    cb, ocb = hx.expgolomb_build(7, 0), orc.ExpGolombBook(7, 0)
+    tables = cb.upload(cuda)
+    _, s = orc.encode(ocb, x)
+    S, P = orc.sync_offset(x.size), orc.payload_offset(x.size)
+    first = [0] + [int(v) for v in s[S + 2:S + 16].view(np.uint16)]
+    banks = [(b >> 5) & 31 for b in first]
+    assert max(banks.count(b) for b in banks) >= 4  # the first chunk looks crowded
+    rng = np.random.default_rng(12)
+    cases = []
+    for _ in range(30):
+        t = s.copy()
+        t[int(rng.integers(P, s.size - 8))] ^= np.uint8(1 << int(rng.integers(0, 8)))
+        cases.append(t)
+    for c, k, v in [(0, 3, 4100), (5, 1, 0), (9, 7, 30000), (33, 4, 16385)]:
+        t = s.copy()
+        o = S + 16 * c + 2 * k
+        t[o:o + 2] = np.array([v], np.uint16).view(np.uint8)
+        cases.append(t)
+    flagged = 0
+    for t in cases:
+        ost, oy = orc.decode(ocb, t, x.size)
+        y, st = hx.decode(tables, torch.from_numpy(t).cuda(), x.size, kind=K)
+        torch.cuda.synchronize()
+        assert int(st.item()) == ost
+        flagged += ost != 0
+        if ost == 0:
+            assert (y.cpu().numpy() == oy).all()
+    assert flagged >= 4  # at least the sync damages
