@@ -419,7 +419,7 @@ int hx_codebook_tables(const hx_codebook* cb, void* host_tables) {
     const uint32_t hi = lo + (1u << (HX_LMAX_MAX - l));
     for (uint32_t wv = lo; wv < hi; ++wv) {
       if (t->dec[wv]) return HX_ERR_ARG;  // not a prefix code
-      t->dec[wv] = (uint16_t)((s << 8) | l);
+      t->dec[wv] = (uint16_t)((s << 8) | hx::kDecValid | l);
     }
   }
   if (cb->kind == HX_KIND_QLC) {

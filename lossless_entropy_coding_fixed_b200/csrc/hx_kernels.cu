@@ -720,39 +720,40 @@ constexpr uint32_t kReaderReach16 = 4 * (1 + kReaderPulls16 / 4);
 // a warp reads with 16-byte blocks when this many of its lanes start in one bank
 constexpr uint32_t kCrowdedReaders = 16;
 
-// The decode table in shared memory: for every 12-bit window, (symbol << 8) | length of the code
-// word it starts with; 0 when none does (an incomplete code).
+// The decode table in shared memory: for every 12-bit window, (symbol << 8) | hx::kDecValid |
+// length of the code word it starts with; 0 when none does (an incomplete code).
 struct DecLut {
   const uint16_t* full;
   __device__ __forceinline__ uint32_t operator()(uint32_t x) const { return full[x >> 20]; }
 };
 
-// Two symbols from the reader: table entries (symbol << 8) | length for either kind (for a QLC
-// table the length is 3 + the width of the area in the top 3 bits; the table holds it already).
-// An entry of 0 (no code word starts the window) only occurs for an incomplete code.
+// Two symbols from the reader: table entries (symbol << 8) | kDecValid | length for either kind
+// (for a QLC table the length is 3 + the width of the area in the top 3 bits; the table holds it
+// already). An entry of 0 (no code word starts the window) only occurs for an incomplete code:
+// `valid` is the AND of the entries used, so its kDecValid bit ends up clear if any was 0.
 template <bool COMPLETE, class Reader>
-__device__ __forceinline__ void decode_pair(Reader& rd, bool& invalid, const DecLut& lut,
+__device__ __forceinline__ void decode_pair(Reader& rd, uint32_t& valid, const DecLut& lut,
                                             uint32_t& e1, uint32_t& e2) {
   const uint32_t x = rd.peek();
   e1 = lut(x);
   const uint32_t l1 = e1 & 15u;
   e2 = lut(x << l1);
   const uint32_t l2 = e2 & 15u;
-  if (!COMPLETE) invalid |= l1 == 0 || l2 == 0;
+  if (!COMPLETE) valid &= e1 & e2;
   rd.advance(l1 + l2);
 }
 
 // 32 symbols -> 32 output bytes, one 32-byte streaming store (a whole sector) when the output is
 // 32-byte aligned, else two 16-byte stores. The symbol bytes are gathered with byte permutes.
 template <bool COMPLETE, class Reader>
-__device__ __forceinline__ void decode_group32(Reader& rd, bool& invalid, uint8_t* dst,
+__device__ __forceinline__ void decode_group32(Reader& rd, uint32_t& valid, uint8_t* dst,
                                                bool out32, const DecLut& lut) {
   uint32_t o[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     uint32_t e1, e2, e3, e4;
-    decode_pair<COMPLETE>(rd, invalid, lut, e1, e2);
-    decode_pair<COMPLETE>(rd, invalid, lut, e3, e4);
+    decode_pair<COMPLETE>(rd, valid, lut, e1, e2);
+    decode_pair<COMPLETE>(rd, valid, lut, e3, e4);
     o[q] = __byte_perm(__byte_perm(e1, e2, 0x0051), __byte_perm(e3, e4, 0x0051), 0x5410);
   }
   if (out32) {
@@ -767,20 +768,22 @@ __device__ __forceinline__ void decode_group32(Reader& rd, bool& invalid, uint8_
 }
 
 // Decodes `mine` symbols of one sub-stream from a started reader to dst; returns the reader's
-// final bit position.
+// final bit position. Sets *invalid when a window started no code word.
 template <bool COMPLETE, class Reader>
 __device__ __forceinline__ uint64_t decode_substream(Reader& rd, uint32_t mine, uint8_t* dst,
                                                      bool out32, bool& invalid,
                                                      const DecLut& lut) {
+  uint32_t valid = hx::kDecValid;
   const uint32_t groups = mine / 32;
   for (uint32_t g = 0; g < groups; ++g)
-    decode_group32<COMPLETE>(rd, invalid, dst + 32 * g, out32, lut);
+    decode_group32<COMPLETE>(rd, valid, dst + 32 * g, out32, lut);
   for (uint32_t i = groups * 32; i < mine; ++i) {
     const uint32_t e = lut(rd.peek());
-    if (!COMPLETE) invalid |= (e & 15u) == 0;
+    if (!COMPLETE) valid &= e;
     rd.advance(e & 15u);
     dst[i] = (uint8_t)(e >> 8);
   }
+  invalid = !COMPLETE && (valid & hx::kDecValid) == 0;
   return rd.position();
 }
 

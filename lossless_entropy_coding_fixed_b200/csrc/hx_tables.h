@@ -8,13 +8,16 @@
 namespace hx {
 
 constexpr uint32_t kTablesMagic = 0x42545848u;  // "HXTB"
+// Set in every decode table entry that holds a code word: a decoder ANDs the entries it uses and
+// finds an unused window (entry 0) from one bit at the end.
+constexpr uint32_t kDecValid = 0x10u;
 
 struct Tables {
   // Encoder: per byte value (code << 4) | len; len 0 = no code word.
   uint32_t enc[256];
   union {
-    // Decoder: for every 12-bit window w, (sym << 8) | len of the code word that w starts with;
-    // 0 when no code word is a prefix of w. (Filled for QLC codebooks as well.)
+    // Decoder: for every 12-bit window w, (sym << 8) | kDecValid | len of the code word that w
+    // starts with; 0 when no code word is a prefix of w. (Filled for QLC codebooks as well.)
     uint16_t dec[4096];
     // Shannonic (kind 2) instead:
     struct {

@@ -104,11 +104,11 @@ def test_table_block_consistent(orc, kind):
     coded = np.nonzero(ln)[0]
     for w in range(4096):
         e = int(dec[w])
-        s, l = e >> 8, e & 0xff
+        s, flag, l = e >> 8, (e >> 4) & 15, e & 15
         if e == 0:  # no code word starts this window (only possible for an incomplete code)
             assert not any((w >> (12 - ln[t])) == code[t] for t in coded)
-        else:
-            assert l == ln[s] and (w >> (12 - l)) == code[s]
+        else:  # (symbol << 8) | valid flag (bit 4) | length
+            assert flag == 1 and l == ln[s] and (w >> (12 - l)) == code[s]
     if kind == "qlc":
         assert (r2s == cb.rank2sym).all()
         for a in range(8):
