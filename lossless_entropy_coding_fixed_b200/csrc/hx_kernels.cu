@@ -21,7 +21,9 @@
 //                register and appended to a 64-bit accumulator, each finished word stored in the
 //                warp's shared buffer (a word two pieces share is stored by the piece that
 //                finishes it and the other ORs its bits in after a warp barrier). The chunk then
-//                leaves with coalesced stores at its final offset.
+//                leaves with coalesced stores at its final offset. A warp whose pieces start
+//                crowded in one shared-memory bank (every code 8 bits long) uses a spread buffer
+//                layout for that chunk.
 //
 //   k_decode     one thread per sub-stream (8 per chunk, 32 chunks per 256-thread block). The
 //                two payload words in use and a bit offset into them give the next 32 bits with
@@ -30,7 +32,12 @@
 //                the 4096-entry shared table gives symbol and length for either kind (for a QLC
 //                code it is precomputed from the area widths and the rank table). 32 decoded
 //                bytes leave as one 32-byte store (a whole sector). Every sub-stream must end
-//                exactly where the next one starts.
+//                exactly where the next one starts. Blocks whose sub-streams start crowded in one
+//                bank of their lines (codes of one length) vote per warp and may read 16-byte
+//                blocks instead.
+//
+//   k_sh_*       the Shannonic range coder: tANS over range indices, one thread per sub-stream
+//                in its measure, pack and (backward) decode kernels.
 #include <cuda_runtime.h>
 
 #include <algorithm>

@@ -62,3 +62,12 @@ def test_reference_arm_runs_oracle_on_rank0_only():
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["higher_is_better"] is True
+
+
+def test_code_only_ignores_comments_and_layout():
+    src = 'int f(int a) {  // the sum\n  /* two\n lines */ return a + 1;\n}\nconst char* s = "a // b";\n'
+    same = 'int f(int a) { return a + 1; }\n// another note\nconst char* s = "a // b";'
+    changed = 'int f(int a) { return a + 2; }\nconst char* s = "a // b";'
+    assert bench.code_only(src) == bench.code_only(same)
+    assert bench.code_only(src) != bench.code_only(changed)
+    assert '"a // b"' in bench.code_only(src)
