@@ -5,8 +5,9 @@ share a fixed codebook, so only coded data travels).
 
 Every rank encodes its shard with the shared table block, the ranks exchange stream sizes and
 then the streams themselves (one NCCL all-gather of buffers padded to the largest stream), and
-every rank decodes every stream. The coding runs in libhx.so; the exchange is torch.distributed
-(NCCL on GPUs).
+every rank decodes every stream. With several parts per shard the three stages overlap: one
+part's exchange runs while the next part is encoded and the previous one decoded. The coding
+runs in libhx.so; the exchange is torch.distributed (NCCL on GPUs).
 """
 from __future__ import annotations
 
@@ -40,34 +41,100 @@ def _round16(v: int) -> int:
     return (v + 15) // 16 * 16
 
 
-def compressed_all_gather(x, tables, group=None, codec: Codec | None = None):
+def part_bounds(n: int, parts: int) -> list[tuple[int, int]]:
+    """[lo, hi) byte ranges of at most `parts` contiguous parts of n bytes, each a whole number of
+    chunks (HX_CHUNK symbols) but the last."""
+    chunks = -(-n // hx.CHUNK)
+    if chunks == 0:
+        return [(0, 0)]
+    parts = max(1, min(parts, chunks))
+    per = -(-chunks // parts) * hx.CHUNK
+    return [(lo, min(n, lo + per)) for lo in range(0, n, per)]
+
+
+def _host_ints(tensors, work, side):
+    """The values of one-element int64 tensors that an async collective fills, on the host. On a
+    GPU a side stream waits for the collective and copies them, so the host does not wait for
+    the codec work queued on the current stream after it."""
+    import torch
+    if side is None:
+        work.wait()
+        return [int(t.item()) for t in tensors]
+    host = torch.empty(len(tensors), dtype=torch.int64, pin_memory=True)
+    with torch.cuda.stream(side):
+        work.wait()
+        for i, t in enumerate(tensors):
+            t.record_stream(side)
+            host[i:i + 1].copy_(t, non_blocking=True)
+        done = torch.cuda.Event()
+        done.record(side)
+    done.synchronize()
+    return host.tolist()
+
+
+def compressed_all_gather(x, tables, group=None, codec: Codec | None = None, parts: int = 1):
     """All-gather of equal-size uint8 shards through the coder.
 
     x: this rank's shard (contiguous uint8 tensor, the same size on every rank); tables: the
     shared table block (device uint8 tensor). Returns (gathered, sizes): gathered holds
-    world_size * n bytes in rank order, sizes the stream bytes each rank sent. One host sync
-    reads the stream sizes, to size the exchange."""
+    world_size * n bytes in rank order, sizes the stream bytes each rank sent.
+
+    With parts > 1 the shard is coded as that many chunk-aligned parts, each its own stream, in a
+    three-stage pipeline: part p is encoded while part p - 1 is exchanged and part p - 2 decoded.
+    A part's exchange is sized by the ranks' stream sizes (one small all-gather, read on the host)
+    and moves every stream padded to the longest. Every rank takes the same collective steps."""
     import torch
     import torch.distributed as dist
 
     codec = codec or Codec()
     world = dist.get_world_size(group)
     n = x.numel()
-    stream = torch.empty(_round16(codec.bound(n)), dtype=torch.uint8, device=x.device)
-    codec.encode(tables, x, stream)
-    # the stream size, from its header's total_words (on the device)
-    total = stream[HEADER_TOTAL_WORDS].view(torch.int64)
-    mine = torch.stack([torch.tensor(n, device=x.device, dtype=torch.int64), total[0]])
-    sizes = [torch.empty_like(mine) for _ in range(world)]
-    dist.all_gather(sizes, mine, group=group)
-    host = [tuple(int(v) for v in s.tolist()) for s in sizes]
-    if any(hn != n for hn, _ in host):
+    dev = x.device
+    # the shard sizes first: every rank sees them all, so unequal shards stop every rank here
+    ns = [torch.empty(1, dtype=torch.int64, device=dev) for _ in range(world)]
+    dist.all_gather(ns, torch.tensor([n], dtype=torch.int64, device=dev), group=group)
+    if any(int(v.item()) != n for v in ns):
         raise ValueError("compressed_all_gather needs the same shard size on every rank")
-    nbytes = [codec.stream_bytes(n, tw) for _, tw in host]
-    span = _round16(max(nbytes))  # every rank sends the same length: the longest stream
-    recv = [torch.empty(span, dtype=torch.uint8, device=x.device) for _ in range(world)]
-    dist.all_gather(recv, stream[:span], group=group)
-    out = torch.empty(world * n, dtype=torch.uint8, device=x.device)
-    for r in range(world):
-        codec.decode(tables, recv[r][:nbytes[r]], n, out[r * n:(r + 1) * n])
-    return out, nbytes
+    bounds = part_bounds(n, parts)
+    # decoded shards go to rows of a multiple of 16 bytes (the decoder's output alignment)
+    row = _round16(n)
+    rows = torch.empty(world * row, dtype=torch.uint8, device=dev)
+    sent = [0] * world
+    side = torch.cuda.Stream(dev) if x.is_cuda else None
+    live = {}
+
+    def code(p):  # encode part p, then start the exchange of its stream sizes
+        lo, hi = bounds[p]
+        stream = torch.empty(_round16(codec.bound(hi - lo)), dtype=torch.uint8, device=dev)
+        codec.encode(tables, x[lo:hi], stream)
+        total = stream[HEADER_TOTAL_WORDS].view(torch.int64).clone()
+        sizes = [torch.empty(1, dtype=torch.int64, device=dev) for _ in range(world)]
+        live[p] = {"stream": stream, "sizes": sizes,
+                   "work": dist.all_gather(sizes, total, group=group, async_op=True)}
+
+    def send(p):  # start the exchange of part p's streams, padded to the longest
+        st, (lo, hi) = live[p], bounds[p]
+        totals = _host_ints(st["sizes"], st["work"], side)
+        st["bytes"] = [codec.stream_bytes(hi - lo, t) for t in totals]
+        span = _round16(max(st["bytes"]))
+        st["recv"] = [torch.empty(span, dtype=torch.uint8, device=dev) for _ in range(world)]
+        st["work"] = dist.all_gather(st["recv"], st["stream"][:span], group=group,
+                                     async_op=True)
+
+    def unpack(p):  # decode every rank's stream of part p into its place
+        st, (lo, hi) = live.pop(p), bounds[p]
+        st["work"].wait()
+        for r in range(world):
+            codec.decode(tables, st["recv"][r][:st["bytes"][r]], hi - lo,
+                         rows[r * row + lo:r * row + hi])
+            sent[r] += st["bytes"][r]
+
+    for p in range(len(bounds) + 2):
+        if p < len(bounds):
+            code(p)
+        if 0 <= p - 1 < len(bounds):
+            send(p - 1)
+        if 0 <= p - 2 < len(bounds):
+            unpack(p - 2)
+    out = rows if row == n else rows.view(world, row)[:, :n].reshape(-1)
+    return out, sent

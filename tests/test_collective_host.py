@@ -75,3 +75,79 @@ def test_two_ranks_gather_in_rank_order():
                 got = out[q * n:(q + 1) * n]
                 # the stand-in keeps the whole shard whenever the stream holds it
                 assert (got[:keep[q] - 3] == expect[q * n:q * n + keep[q] - 3]).all()
+
+
+class LosslessStandIn(collective.Codec):
+    """A lossless stand-in: the header's total_words covers the bytes plus 0..2 spare words that
+    depend on the first byte, so streams differ in length across ranks and parts."""
+
+    def bound(self, n):
+        return hx.stream_bytes(n, (n + 3) // 4 + 2)
+
+    def words(self, x):
+        return (x.numel() + 3) // 4 + (int(x[0]) % 3 if x.numel() else 0)
+
+    def encode(self, tables, x, out):
+        n = x.numel()
+        out.zero_()
+        out[32:40] = torch.tensor([self.words(x)], dtype=torch.int64).view(torch.uint8)
+        P = hx.payload_offset(n)
+        out[P:P + n] = x
+
+    def decode(self, tables, stream, n, out):
+        assert stream.numel() == hx.stream_bytes(n, int(stream[32:40].view(torch.int64)[0]))
+        P = hx.payload_offset(n)
+        out.copy_(stream[P:P + n])
+
+
+CASES = [(10000, 1), (10000, 3), (10000, 6), (3 * 4096, 2), (0, 3), (1, 4)]
+
+
+def _shard(rank, n):
+    return torch.from_numpy(np.random.default_rng(100 + rank).integers(0, 256, n, dtype=np.uint8))
+
+
+def _run_parts(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        res = []
+        for n, parts in CASES:
+            out, sent = collective.compressed_all_gather(_shard(rank, n), None,
+                                                         codec=LosslessStandIn(), parts=parts)
+            res.append((out.numpy().copy(), sent))
+        try:  # unequal shards: every rank must refuse, none may hang
+            collective.compressed_all_gather(_shard(rank, 4096 + rank), None,
+                                             codec=LosslessStandIn(), parts=2)
+            res.append("accepted")
+        except ValueError:
+            res.append("refused")
+        results[rank] = res
+    finally:
+        dist.destroy_process_group()
+
+
+def test_parts_pipeline_two_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        results = m.dict()
+        port = _port()
+        procs = [ctx.Process(target=_run_parts, args=(r, world, port, results))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(180)
+            assert p.exitcode == 0
+        codec = LosslessStandIn()
+        for r in range(world):
+            res = results[r]
+            assert res[-1] == "refused"
+            for (n, parts), (out, sent) in zip(CASES, res[:-1]):
+                shards = [_shard(q, n) for q in range(world)]
+                assert (out == np.concatenate([s.numpy() for s in shards])).all(), (n, parts)
+                bounds = collective.part_bounds(n, parts)
+                assert len(bounds) == max(1, min(parts, -(-n // 4096)))
+                assert sent == [sum(hx.stream_bytes(hi - lo, codec.words(s[lo:hi]))
+                                    for lo, hi in bounds) for s in shards], (n, parts)

@@ -34,14 +34,19 @@ def _rank(port, q):
     try:
         res = {}
         for kind in (hx.KIND_HUFFMAN, hx.KIND_QLC):
-            x = datagen.data(1, n=(1 << 20) - 77)
-            prior = sum(oracle.histogram(b) for b in datagen.prior_batches(1))
-            cb = hx.build_codebook(prior) if kind == hx.KIND_HUFFMAN else hx.qlc_build(prior)
-            ocb = oracle.huffman_codebook(prior) if kind == hx.KIND_HUFFMAN else oracle.qlc_codebook(prior)
-            out, sizes = collective.compressed_all_gather(torch.from_numpy(x).cuda(), cb.upload("cuda"),
-                                                          codec=collective.Codec(kind))
-            torch.cuda.synchronize()
-            res[kind] = (bool((out.cpu().numpy() == x).all()), sizes, int(oracle.encode(ocb, x)[1].size))
+            for parts in (1, 3):
+                x = datagen.data(1, n=(1 << 20) - 77)
+                prior = sum(oracle.histogram(b) for b in datagen.prior_batches(1))
+                cb = hx.build_codebook(prior) if kind == hx.KIND_HUFFMAN else hx.qlc_build(prior)
+                ocb = (oracle.huffman_codebook(prior) if kind == hx.KIND_HUFFMAN
+                       else oracle.qlc_codebook(prior))
+                out, sizes = collective.compressed_all_gather(
+                    torch.from_numpy(x).cuda(), cb.upload("cuda"), codec=collective.Codec(kind),
+                    parts=parts)
+                torch.cuda.synchronize()
+                ref = sum(int(oracle.encode(ocb, x[lo:hi])[1].size)
+                          for lo, hi in collective.part_bounds(x.size, parts))
+                res[(kind, parts)] = (bool((out.cpu().numpy() == x).all()), sizes, ref)
         q.put(res)
     finally:
         dist.destroy_process_group()
@@ -58,5 +63,6 @@ def test_one_rank_round_trip():
     res = q.get(timeout=300)
     p.join(120)
     assert p.exitcode == 0
-    for kind, (ok, sizes, ref_size) in res.items():
-        assert ok and sizes == [ref_size], kind
+    assert len(res) == 4
+    for case, (ok, sizes, ref_size) in res.items():
+        assert ok and sizes == [ref_size], case
