@@ -794,6 +794,9 @@ __device__ __forceinline__ uint64_t decode_substream(Reader& rd, uint32_t mine, 
   return rd.position();
 }
 
+// The block's chunks in a grid-stride loop, 8 lanes per chunk (one per sub-stream). COMPLETE:
+// every window starts a code word, so no entry is checked. VOTE: the block's first chunk looked
+// crowded (crowded_chunk), so the lanes about to decode vote on the 16-byte reader.
 template <bool COMPLETE, bool VOTE>
 __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut& lut,
                                               uint32_t total) {
