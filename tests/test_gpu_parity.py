@@ -281,13 +281,19 @@ def test_other_codebook_rejected(orc, damaged_setup, cuda):
     assert st == hx.HX_ERR_CODEBOOK == orc.decode(orc.huffman_codebook(datagen.random_counts(99)), s, x.size)[0]
 
 
+@pytest.mark.parametrize("kind", ["huffman", "qlc"])
 @pytest.mark.parametrize("n", [4096, 5 * 4096 + 77, 1 << 20])
-def test_flat_8bit_codes(orc, cuda, n):
-    """Every code 8 bits long (a code built from uniform counts): each 128-byte piece packs to
-    exactly 32 words, so all 32 pieces of a chunk start in one shared-memory bank and the encoder
-    takes its spread buffer layout for every chunk."""
+def test_flat_8bit_codes(orc, cuda, n, kind):
+    """Every code 8 bits long (uniform counts: Huffman, or QLC with eight areas of 5 index bits):
+    each 128-byte piece packs to exactly 32 words, so all 32 pieces of a chunk start in one
+    shared-memory bank and the encoder takes its spread buffer layout for every chunk; every
+    sub-stream is 128 words long, so the decoder's blocks take the voting loop and its 16-byte
+    reader."""
     counts = np.ones(256, np.uint64)
-    cb, ocb = hx.build_codebook(counts), orc.huffman_codebook(counts)
+    if kind == "huffman":
+        cb, ocb = hx.build_codebook(counts), orc.huffman_codebook(counts)
+    else:
+        cb, ocb = hx.qlc_build(counts), orc.qlc_codebook(counts)
     assert (ocb.len == 8).all()
     tables = cb.upload(cuda)
     x = datagen.uniform_bytes(n, 9)
