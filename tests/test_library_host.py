@@ -93,10 +93,11 @@ def _tables(cb):
     return enc, dec, r2s, area
 
 
-@pytest.mark.parametrize("kind", ["huffman", "qlc"])
+@pytest.mark.parametrize("kind", ["huffman", "qlc", "expgolomb"])
 def test_table_block_consistent(orc, kind):
     counts = datagen.random_counts(5, zeros=0.4)
-    cb = hx.build_codebook(counts) if kind == "huffman" else hx.qlc_build(counts)
+    cb = (hx.build_codebook(counts) if kind == "huffman" else hx.qlc_build(counts)
+          if kind == "qlc" else hx.expgolomb_build(6, 0))
     enc, dec, r2s, area = _tables(cb)
     ln, code = cb.len.astype(np.int64), cb.code.astype(np.int64)
     assert (enc == (code << 4) | ln).all()
