@@ -1,6 +1,6 @@
-"""The compressed all-gather on a GPU with NCCL and the real coder. Runs as one rank (this pool
-gives one GPU per run; the exchange logic for two ranks is covered on CPU ranks), in a child
-process so the process group does not outlive the test."""
+"""The compressed all-gather on a GPU with NCCL and the real coder, as one rank (the exchange
+between two ranks is covered on CPU ranks), in a child process so the process group does not
+outlive the test."""
 import os
 import socket
 
