@@ -72,12 +72,54 @@ def _host_ints(tensors, work, side):
     return host.tolist()
 
 
-def compressed_all_gather(x, tables, group=None, codec: Codec | None = None, parts: int = 1):
+def merge_streams(streams, ns):
+    """One stream of sum(ns) bytes from the streams of consecutive pieces of it, each piece but the
+    last a whole number of chunks. The headers must agree on version, kind, lmax and codebook
+    hash; the word offsets are rebased by the payload words before each piece, and the sync rows
+    and payload words are concatenated. The result is the stream the encoder writes for the whole
+    input (its chunks code the same bytes from the same word boundaries)."""
+    import torch
+
+    if not streams or len(streams) != len(ns):
+        raise ValueError("merge_streams needs one size per stream")
+    if any(n % hx.CHUNK for n in ns[:-1]):
+        raise ValueError("every piece but the last must be a whole number of chunks")
+    head = streams[0][:64]
+    for st in streams[1:]:
+        if not (torch.equal(st[:8], head[:8]) and torch.equal(st[40:48], head[40:48])):
+            raise ValueError("the streams were not coded with the same codebook")
+    totals = [int(st[32:40].view(torch.int64)[0]) for st in streams]
+    chunks = [-(-n // hx.CHUNK) for n in ns]
+    n_all, words = sum(ns), sum(totals)
+    if words >= 1 << 32:
+        raise ValueError("the merged payload exceeds 2^32 words")
+    out = torch.zeros(hx.stream_bytes(n_all, words), dtype=torch.uint8, device=head.device)
+    out[:64] = head
+    out[16:40] = torch.tensor([n_all, sum(chunks), words], dtype=torch.int64).view(torch.uint8)
+    woff = out[64:64 + 4 * (sum(chunks) + 1)].view(torch.int32)
+    S, P = hx.sync_offset(n_all), hx.payload_offset(n_all)
+    c0 = w0 = 0
+    for st, n, nc, tw in zip(streams, ns, chunks, totals):
+        own = st[64:64 + 4 * nc].view(torch.int32).to(torch.int64) & 0xFFFFFFFF
+        woff[c0:c0 + nc] = (own + w0).to(torch.int32)  # u32 bits, below 2^32
+        s_i, p_i = hx.sync_offset(n), hx.payload_offset(n)
+        out[S + 16 * c0:S + 16 * (c0 + nc)] = st[s_i:s_i + 16 * nc]
+        out[P + 4 * w0:P + 4 * (w0 + tw)] = st[p_i:p_i + 4 * tw]
+        c0, w0 = c0 + nc, w0 + tw
+    woff[c0:c0 + 1] = torch.tensor([words], dtype=torch.int64).to(torch.int32)
+    return out
+
+
+def compressed_all_gather(x, tables, group=None, codec: Codec | None = None, parts: int = 1,
+                          decode: bool = True):
     """All-gather of equal-size uint8 shards through the coder.
 
     x: this rank's shard (contiguous uint8 tensor, the same size on every rank); tables: the
     shared table block (device uint8 tensor). Returns (gathered, sizes): gathered holds
-    world_size * n bytes in rank order, sizes the stream bytes each rank sent.
+    world_size * n bytes in rank order, sizes the stream bytes each rank sent. With
+    decode=False, gathered is instead the one stream of all ranks' bytes in rank order
+    (merge_streams of the received streams; with 2 or more ranks n must be a whole number of
+    chunks), for a receiver that keeps the data coded.
 
     With parts > 1 the shard is coded as that many chunk-aligned parts, each its own stream, in a
     three-stage pipeline: part p is encoded while part p - 1 is exchanged and part p - 2 decoded.
@@ -95,10 +137,12 @@ def compressed_all_gather(x, tables, group=None, codec: Codec | None = None, par
     dist.all_gather(ns, torch.tensor([n], dtype=torch.int64, device=dev), group=group)
     if any(int(v.item()) != n for v in ns):
         raise ValueError("compressed_all_gather needs the same shard size on every rank")
+    if not decode and world > 1 and n % hx.CHUNK:
+        raise ValueError("a merged stream needs shards of whole chunks")
     bounds = part_bounds(n, parts)
     # decoded shards go to rows of a multiple of 16 bytes (the decoder's output alignment)
     row = _round16(n)
-    rows = torch.empty(world * row, dtype=torch.uint8, device=dev)
+    rows = torch.empty(world * row if decode else 0, dtype=torch.uint8, device=dev)
     sent = [0] * world
     side = torch.cuda.Stream(dev) if x.is_cuda else None
     live = {}
@@ -121,12 +165,17 @@ def compressed_all_gather(x, tables, group=None, codec: Codec | None = None, par
         st["work"] = dist.all_gather(st["recv"], st["stream"][:span], group=group,
                                      async_op=True)
 
-    def unpack(p):  # decode every rank's stream of part p into its place
+    kept = {}
+
+    def unpack(p):  # decode every rank's stream of part p into its place (or keep it)
         st, (lo, hi) = live.pop(p), bounds[p]
         st["work"].wait()
         for r in range(world):
-            codec.decode(tables, st["recv"][r][:st["bytes"][r]], hi - lo,
-                         rows[r * row + lo:r * row + hi])
+            if decode:
+                codec.decode(tables, st["recv"][r][:st["bytes"][r]], hi - lo,
+                             rows[r * row + lo:r * row + hi])
+            else:
+                kept[(r, p)] = st["recv"][r][:st["bytes"][r]]
             sent[r] += st["bytes"][r]
 
     for p in range(len(bounds) + 2):
@@ -136,5 +185,9 @@ def compressed_all_gather(x, tables, group=None, codec: Codec | None = None, par
             send(p - 1)
         if 0 <= p - 2 < len(bounds):
             unpack(p - 2)
+    if not decode:
+        order = [(r, p) for r in range(world) for p in range(len(bounds))]
+        return merge_streams([kept[k] for k in order],
+                             [bounds[p][1] - bounds[p][0] for _, p in order]), sent
     out = rows if row == n else rows.view(world, row)[:, :n].reshape(-1)
     return out, sent

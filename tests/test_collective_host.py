@@ -101,6 +101,7 @@ class LosslessStandIn(collective.Codec):
 
 
 CASES = [(10000, 1), (10000, 3), (10000, 6), (3 * 4096, 2), (0, 3), (1, 4)]
+MERGED = [(3 * 4096, 1), (3 * 4096, 2)]
 
 
 def _shard(rank, n):
@@ -116,6 +117,17 @@ def _run_parts(rank, world, port, results):
             out, sent = collective.compressed_all_gather(_shard(rank, n), None,
                                                          codec=LosslessStandIn(), parts=parts)
             res.append((out.numpy().copy(), sent))
+        for n, parts in MERGED:  # one global stream instead of the decoded bytes
+            st, sent = collective.compressed_all_gather(_shard(rank, n), None,
+                                                        codec=LosslessStandIn(), parts=parts,
+                                                        decode=False)
+            res.append((st.numpy().copy(), sent))
+        try:  # a merged stream of shards that are not whole chunks: every rank refuses
+            collective.compressed_all_gather(_shard(rank, 5000), None, codec=LosslessStandIn(),
+                                             decode=False)
+            res.append("accepted")
+        except ValueError:
+            res.append("refused")
         try:  # unequal shards: every rank must refuse, none may hang
             collective.compressed_all_gather(_shard(rank, 4096 + rank), None,
                                              codec=LosslessStandIn(), parts=2)
@@ -143,11 +155,59 @@ def test_parts_pipeline_two_ranks():
         codec = LosslessStandIn()
         for r in range(world):
             res = results[r]
-            assert res[-1] == "refused"
-            for (n, parts), (out, sent) in zip(CASES, res[:-1]):
+            assert res[-2:] == ["refused", "refused"]
+            merged = res[len(CASES):len(CASES) + len(MERGED)]
+            for (n, parts), (st, sent) in zip(MERGED, merged):
+                streams, sizes = [], []
+                for q in range(world):
+                    shard = _shard(q, n)
+                    for lo, hi in collective.part_bounds(n, parts):
+                        buf = torch.empty(codec.bound(hi - lo), dtype=torch.uint8)
+                        codec.encode(None, shard[lo:hi], buf)
+                        streams.append(buf[:hx.stream_bytes(hi - lo, codec.words(shard[lo:hi]))])
+                        sizes.append(hi - lo)
+                expect = collective.merge_streams(streams, sizes).numpy()
+                assert st.size == expect.size and (st == expect).all(), (n, parts)
+            for (n, parts), (out, sent) in zip(CASES, res[:len(CASES)]):
                 shards = [_shard(q, n) for q in range(world)]
                 assert (out == np.concatenate([s.numpy() for s in shards])).all(), (n, parts)
                 bounds = collective.part_bounds(n, parts)
                 assert len(bounds) == max(1, min(parts, -(-n // 4096)))
                 assert sent == [sum(hx.stream_bytes(hi - lo, codec.words(s[lo:hi]))
                                     for lo, hi in bounds) for s in shards], (n, parts)
+
+
+# ------------------------------------------------------------------ one global stream
+@pytest.fixture(scope="module")
+def orc_books():
+    import datagen
+    import oracle
+    counts = sum(oracle.histogram(b) for b in datagen.prior_batches(1))
+    return oracle, datagen, [oracle.huffman_codebook(counts), oracle.qlc_codebook(counts),
+                             oracle.shannonic_codebook(counts), oracle.ExpGolombBook(6, 0)]
+
+
+@pytest.mark.parametrize("cuts", [[0, 5 * 4096 + 777], [0, 8192, 16384, 5 * 4096 + 777],
+                                  [0, 4096, 4096, 12288, 5 * 4096 + 777], [0, 4096, 8192]])
+def test_merge_streams_equals_stream_of_whole(orc_books, cuts):
+    """Streams of consecutive chunk-aligned pieces, merged, are byte for byte the oracle's
+    stream of the whole input (every chunk codes the same bytes from a word boundary)."""
+    oracle, datagen, books = orc_books
+    x = datagen.data(1, n=cuts[-1])
+    for cb in books:
+        pieces = [torch.from_numpy(oracle.encode(cb, x[a:b])[1]) for a, b in zip(cuts, cuts[1:])]
+        merged = collective.merge_streams(pieces, [b - a for a, b in zip(cuts, cuts[1:])])
+        assert (merged.numpy() == oracle.encode(cb, x)[1]).all()
+
+
+def test_merge_streams_refusals(orc_books):
+    oracle, datagen, books = orc_books
+    x = datagen.data(1, n=3 * 4096)
+    a = torch.from_numpy(oracle.encode(books[0], x[:4096])[1])
+    b = torch.from_numpy(oracle.encode(books[1], x[4096:])[1])
+    with pytest.raises(ValueError):  # another codebook
+        collective.merge_streams([a, b], [4096, 8192])
+    c = torch.from_numpy(oracle.encode(books[0], x[:4000])[1])
+    d = torch.from_numpy(oracle.encode(books[0], x[4000:])[1])
+    with pytest.raises(ValueError):  # a piece that is not whole chunks
+        collective.merge_streams([c, d], [4000, 8288])
