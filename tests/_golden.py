@@ -63,3 +63,13 @@ def abc_counts():
     c = np.zeros(256, dtype=np.uint64)
     c[0x41], c[0x42], c[0x43] = 2, 1, 1
     return c
+
+
+def histograms():
+    """(bytes, {value: count}) from histogram_hand.txt."""
+    out = []
+    for ln in _lines("histogram_hand.txt"):
+        data, bins = (t.strip() for t in ln.split("|"))
+        raw = b"" if data == "-" else bytes.fromhex(data)
+        out.append((raw, {int(v): int(c) for v, c in (b.split(":") for b in bins.split())}))
+    return out

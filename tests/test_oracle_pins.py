@@ -272,3 +272,35 @@ def test_codebook_hash_serialisation(orc):
     assert cb.hash == orc.fnv1a(bytes([0, 12]) + cb.len.tobytes())
     q = orc.qlc_codebook(np.ones(256, np.uint64))
     assert q.hash == orc.fnv1a(bytes([1, 11]) + q.bits.tobytes() + q.rank2sym.tobytes())
+
+
+# --------------------------------------------------------------------------- histogram
+def test_histogram_hand_counted(orc):
+    """Small inputs counted by hand, the empty input and a last byte that differs included."""
+    for raw, bins in G.histograms():
+        want = np.zeros(256, np.uint64)
+        for v, c in bins.items():
+            want[v] = c
+        got = orc.histogram(np.frombuffer(raw, dtype=np.uint8))
+        assert got.dtype == np.uint64 and (got == want).all(), raw.hex()
+
+
+@pytest.mark.parametrize("n", [0, 1, 15, 16, 17, 4095, 4096, 4097, 3 * 4096 + 100])
+def test_histogram_closed_form_ramp(orc, n):
+    """x[i] = i mod 256: every bin holds floor(n/256), and the first n mod 256 bins one more,
+    so a dropped or doubled byte at any ragged length changes a bin."""
+    x = (np.arange(n) % 256).astype(np.uint8)
+    want = np.full(256, n // 256, np.uint64)
+    want[: n % 256] += 1
+    assert (orc.histogram(x) == want).all()
+    assert int(orc.histogram(x).sum()) == n
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_histogram_equals_bincount(orc, seed):
+    """Against numpy's bincount on random and skewed inputs of ragged sizes."""
+    rng = np.random.default_rng(seed)
+    for n in (0, 1, 17, 4097, 65537):
+        x = rng.integers(0, 256, n, dtype=np.uint8) if seed % 2 else \
+            np.minimum(rng.geometric(0.1, n), 255).astype(np.uint8)
+        assert (orc.histogram(x) == np.bincount(x, minlength=256).astype(np.uint64)).all()
