@@ -84,10 +84,16 @@ def merge_streams(streams, ns):
         raise ValueError("merge_streams needs one size per stream")
     if any(n % hx.CHUNK for n in ns[:-1]):
         raise ValueError("every piece but the last must be a whole number of chunks")
+    if sum(ns) >= 1 << 32:
+        raise ValueError("a stream codes fewer than 2^32 bytes; the merged input is larger")
     head = streams[0][:64]
     for st in streams[1:]:
         if not (torch.equal(st[:8], head[:8]) and torch.equal(st[40:48], head[40:48])):
             raise ValueError("the streams were not coded with the same codebook")
+    for st, n in zip(streams, ns):
+        hn, hc = (int(v) for v in st[16:32].view(torch.int64).tolist())
+        if hn != n or hc != -(-n // hx.CHUNK):
+            raise ValueError(f"a stream's header codes {hn} bytes, not the {n} given for it")
     totals = [int(st[32:40].view(torch.int64)[0]) for st in streams]
     chunks = [-(-n // hx.CHUNK) for n in ns]
     n_all, words = sum(ns), sum(totals)
@@ -139,6 +145,8 @@ def compressed_all_gather(x, tables, group=None, codec: Codec | None = None, par
         raise ValueError("compressed_all_gather needs the same shard size on every rank")
     if not decode and world > 1 and n % hx.CHUNK:
         raise ValueError("a merged stream needs shards of whole chunks")
+    if not decode and world * n >= 1 << 32:
+        raise ValueError("a merged stream codes fewer than 2^32 bytes; world * n is larger")
     bounds = part_bounds(n, parts)
     # decoded shards go to rows of a multiple of 16 bytes (the decoder's output alignment)
     row = _round16(n)

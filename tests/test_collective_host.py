@@ -100,6 +100,30 @@ class LosslessStandIn(collective.Codec):
         out.copy_(stream[P:P + n])
 
 
+class OracleCodec(collective.Codec):
+    """The CPU oracle as the coder: real streams in the library's format, so a merged stream can
+    be checked against the oracle's stream of all ranks' bytes (not against merge_streams)."""
+
+    def __init__(self):
+        import datagen
+        import oracle
+        self.oracle = oracle
+        self.cb = oracle.huffman_codebook(sum(oracle.histogram(b)
+                                              for b in datagen.prior_batches(1)))
+
+    def bound(self, n):
+        return self.oracle.encode_bound(n)
+
+    def encode(self, tables, x, out):
+        st = self.oracle.encode(self.cb, x.numpy())[1]
+        out[:st.size] = torch.from_numpy(st)
+
+    def decode(self, tables, stream, n, out):
+        status, y = self.oracle.decode(self.cb, stream.numpy(), n)
+        assert status == 0
+        out.copy_(torch.from_numpy(y))
+
+
 CASES = [(10000, 1), (10000, 3), (10000, 6), (3 * 4096, 2), (0, 3), (1, 4)]
 MERGED = [(3 * 4096, 1), (3 * 4096, 2)]
 
@@ -119,12 +143,19 @@ def _run_parts(rank, world, port, results):
             res.append((out.numpy().copy(), sent))
         for n, parts in MERGED:  # one global stream instead of the decoded bytes
             st, sent = collective.compressed_all_gather(_shard(rank, n), None,
-                                                        codec=LosslessStandIn(), parts=parts,
+                                                        codec=OracleCodec(), parts=parts,
                                                         decode=False)
             res.append((st.numpy().copy(), sent))
         try:  # a merged stream of shards that are not whole chunks: every rank refuses
             collective.compressed_all_gather(_shard(rank, 5000), None, codec=LosslessStandIn(),
                                              decode=False)
+            res.append("accepted")
+        except ValueError:
+            res.append("refused")
+        try:  # a merged stream of 2^32 bytes or more: refused before any coding (the shard is
+            # never touched, so its pages are never committed)
+            collective.compressed_all_gather(torch.empty(1 << 31, dtype=torch.uint8), None,
+                                             codec=LosslessStandIn(), decode=False)
             res.append("accepted")
         except ValueError:
             res.append("refused")
@@ -155,18 +186,13 @@ def test_parts_pipeline_two_ranks():
         codec = LosslessStandIn()
         for r in range(world):
             res = results[r]
-            assert res[-2:] == ["refused", "refused"]
+            assert res[-3:] == ["refused", "refused", "refused"]
             merged = res[len(CASES):len(CASES) + len(MERGED)]
+            oc = OracleCodec()
             for (n, parts), (st, sent) in zip(MERGED, merged):
-                streams, sizes = [], []
-                for q in range(world):
-                    shard = _shard(q, n)
-                    for lo, hi in collective.part_bounds(n, parts):
-                        buf = torch.empty(codec.bound(hi - lo), dtype=torch.uint8)
-                        codec.encode(None, shard[lo:hi], buf)
-                        streams.append(buf[:hx.stream_bytes(hi - lo, codec.words(shard[lo:hi]))])
-                        sizes.append(hi - lo)
-                expect = collective.merge_streams(streams, sizes).numpy()
+                # the oracle's stream of every rank's bytes in rank order
+                whole = np.concatenate([_shard(q, n).numpy() for q in range(world)])
+                expect = oc.oracle.encode(oc.cb, whole)[1]
                 assert st.size == expect.size and (st == expect).all(), (n, parts)
             for (n, parts), (out, sent) in zip(CASES, res[:len(CASES)]):
                 shards = [_shard(q, n) for q in range(world)]
@@ -211,3 +237,8 @@ def test_merge_streams_refusals(orc_books):
     d = torch.from_numpy(oracle.encode(books[0], x[4000:])[1])
     with pytest.raises(ValueError):  # a piece that is not whole chunks
         collective.merge_streams([c, d], [4000, 8288])
+    e = torch.from_numpy(oracle.encode(books[0], x[4096:])[1])
+    with pytest.raises(ValueError):  # a size that its stream's header does not code
+        collective.merge_streams([a, e], [4096, 4096])
+    with pytest.raises(ValueError):  # 2^32 bytes or more cannot be one stream
+        collective.merge_streams([a, e], [1 << 31, 1 << 31])
