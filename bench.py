@@ -36,6 +36,7 @@ WORKLOAD = ("cfg4: 1 GiB e4m3 bytes of N(0,1)*0.5; fixed Huffman (Lmax 12) and Q
             "QLC encode + decode")
 METRIC = "encode & decode GB/s (uncompressed) at 1 B200, % of HBM roofline; bits/symbol"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0  # the B200's HBM3e specification (DGX figure)
 KERNEL_SOURCES = ["lossless_entropy_coding_fixed_b200/csrc/hx_kernels.cu",
                   "lossless_entropy_coding_fixed_b200/csrc/hx_tables.h"]
 
@@ -52,7 +53,17 @@ def parse():
     p.add_argument("--no-online", action="store_true")
     p.add_argument("--no-shannonic", action="store_true")
     p.add_argument("--no-expgolomb", action="store_true")
-    return p.parse_args()
+    p.add_argument("--no-configs", action="store_true")
+    p.add_argument("--no-cfg5", action="store_true")
+    p.add_argument("--no-collective", action="store_true")
+    p.add_argument("--quick", action="store_true",
+                   help="the headline step only (no e2e, legs, configs or CPU baseline)")
+    a = p.parse_args()
+    if a.quick:
+        for k in ("no_e2e", "no_cpu_baseline", "no_online", "no_shannonic", "no_expgolomb",
+                  "no_configs", "no_cfg5", "no_collective"):
+            setattr(a, k, True)
+    return a
 
 
 def dist_env():
@@ -176,29 +187,52 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------------------
+def _oracle_slices(x, threads):
+    """Chunk-aligned slices of x, one per thread."""
+    per = -(-x.size // threads)
+    per = -(-per // 4096) * 4096
+    return [x[i:i + per] for i in range(0, x.size, per)]
+
+
+def oracle_codec_pass(books, x, threads: int) -> float:
+    """The oracle as it stands, encoding and decoding x with each codebook: x is cut into
+    chunk-aligned slices, each coded as its own stream on its own thread (ctypes releases the
+    interpreter lock). Returns the seconds taken."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    slices = _oracle_slices(x, threads)
+
+    def one(sl):
+        for cb in books:
+            st, s = oracle.encode(cb, sl)
+            assert st == 0
+            st, y = oracle.decode(cb, s, sl.size)
+            assert st == 0 and (y == sl).all()
+
+    t0 = time.perf_counter()
+    if threads == 1:
+        for sl in slices:
+            one(sl)
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(one, slices))
+    return time.perf_counter() - t0
+
+
 def cpu_reference(args, rank, ws):
-    """The oracle on a bounded sample of the workload (rank 0 only)."""
+    """The oracle on a bounded sample of the workload, on all host cores (rank 0 only)."""
     if rank != 0:
         return 0
     import oracle
     import datagen
-    sample = 1 << 20
+    cores = os.cpu_count() or 1
+    sample = 4 << 20
     counts = sum(oracle.histogram(b) for b in datagen.prior_batches(4))
-    hb, qb = oracle.huffman_codebook(counts), oracle.qlc_codebook(counts)
+    books = (oracle.huffman_codebook(counts), oracle.qlc_codebook(counts))
     x = datagen.data(4, n=sample)
-
-    def step():
-        _, sh = oracle.encode(hb, x)
-        oracle.decode(hb, sh, x.size)
-        _, sq = oracle.encode(qb, x)
-        oracle.decode(qb, sq, x.size)
-
     for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    dt = time.perf_counter() - t0
+        oracle_codec_pass(books, x, cores)
+    dt = sum(oracle_codec_pass(books, x, cores) for _ in range(args.steps))
     value = 4 * sample * args.steps / dt / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
@@ -206,9 +240,10 @@ def cpu_reference(args, rank, ws):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "sample_bytes_per_step": sample},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {sample} bytes of the 1 GiB batch per step, "
-                                   "single-thread bit-serial C++"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {sample >> 20} MiB of the 1 GiB batch per step, in "
+                                   f"{cores} chunk-aligned slices on {cores} threads: Huffman and "
+                                   "QLC encode + decode, bit-serial C++"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -216,21 +251,344 @@ def cpu_reference(args, rank, ws):
 
 
 def cpu_baseline_leg(counts):
-    """Time the oracle as it stands on a 64 MiB slice of the workload (~10-30 s, one core)."""
+    """Time the oracle as it stands on a slice of the workload: one thread on 16 MiB, and all host
+    cores on 64 MiB in chunk-aligned slices (~10-30 s in all)."""
     import oracle
     import datagen
-    sample = 64 << 20
-    x = datagen.data(4, n=sample)
-    hb, qb = oracle.huffman_codebook(counts), oracle.qlc_codebook(counts)
-    t0 = time.perf_counter()
-    _, sh = oracle.encode(hb, x)
-    oracle.decode(hb, sh, x.size)
-    _, sq = oracle.encode(qb, x)
-    oracle.decode(qb, sq, x.size)
-    dt = time.perf_counter() - t0
-    return {"value": 4 * sample / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {sample >> 20} MiB of the batch through the same 4 codec calls "
-                      f"({dt:.1f} s, single-thread bit-serial C++)"}
+    cores = os.cpu_count() or 1
+    books = (oracle.huffman_codebook(counts), oracle.qlc_codebook(counts))
+    x1 = datagen.data(4, n=16 << 20)
+    dt1 = oracle_codec_pass(books, x1, 1)
+    xa = datagen.data(4, n=64 << 20)
+    dta = oracle_codec_pass(books, xa, cores)
+    return {"value": 4 * xa.size / dta / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"first 64 MiB of the batch through the same 4 codec calls, cut into {cores} "
+                      f"chunk-aligned slices on {cores} threads ({dta:.1f} s, bit-serial C++)",
+            "single_thread": {"value": 4 * x1.size / dt1 / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"first 16 MiB, one thread ({dt1:.1f} s)"}}
+
+
+def roofline_entry(kernel, launches, peak, peak_kind):
+    """HBM roofline of one kernel from its launches in a step: [(algorithmic bytes, ms)]."""
+    b = sum(x for x, _ in launches) / len(launches)
+    ms = sum(t for _, t in launches) / len(launches)
+    achieved = b / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peak,
+            "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+            "frac_spec": achieved / SPEC_HBM_GBS, "peak_spec": SPEC_HBM_GBS,
+            "algorithmic_bytes_per_launch": b, "launches_per_step": len(launches),
+            "ms_per_launch": ms}
+
+
+def graph_ms(torch, fn, reps: int) -> float:
+    """Device time of one fn() call: reps calls captured in a CUDA graph, replayed (no launch
+    gaps; for inputs too small to hide the host's launch time)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / reps
+
+
+def config_numbers(dev, hx, torch, x, prior, peak, kinds=("huffman", "qlc"), reps=20, graph=False):
+    """Encode and decode of one input with the fixed codebooks from `prior`: time per call
+    (inputs resident), GB/s, roofline fraction, bits per symbol against per-shard Huffman and
+    the entropy. Checks the round trip."""
+    n = x.numel()
+    h = np.bincount(x.cpu().numpy(), minlength=256).astype(np.uint64)
+    per_shard = hx.mean_length(h, hx.build_codebook(h, seen_only=True))
+    H = hx.entropy(h)
+    out = torch.empty(hx.encode_bound(n), dtype=torch.uint8, device=dev)
+    scratch = torch.empty(hx.scratch_bytes(n), dtype=torch.uint8, device=dev)
+    y = torch.empty(n, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    res = {"n": n, "entropy": H, "per_shard_huffman": per_shard}
+    for name in kinds:
+        cb = hx.build_codebook(prior) if name == "huffman" else hx.qlc_build(prior)
+        t = cb.upload(dev)
+        enc = lambda: hx.encode(t, x, out=out, scratch=scratch, status=status, kind=cb.kind)
+        dec = lambda: hx.decode(t, out, n, out=y, status=status, kind=cb.kind)
+        enc()
+        dec()
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0 and torch.equal(x, y)
+        size = hx.stream_size(out, n)
+        r = {}
+        for op, fn in (("encode", enc), ("decode", dec)):
+            if graph:
+                ms = graph_ms(torch, fn, reps)
+            else:
+                for _ in range(3):
+                    fn()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                for _ in range(reps):
+                    fn()
+                b.record()
+                torch.cuda.synchronize()
+                ms = a.elapsed_time(b) / reps
+            alg = (n + size) / (ms * 1e-3) / 1e9
+            r[op] = {"ms": ms, "GB_per_s_uncompressed": n / (ms * 1e-3) / 1e9,
+                     "hbm_frac_algorithmic": alg / peak, "hbm_frac_spec": alg / SPEC_HBM_GBS}
+        assert int(status.item()) == 0
+        bits = hx.mean_length(h, cb)
+        r["bits_per_symbol"] = {"payload": bits, "framed": size * 8 / n,
+                                "vs_per_shard": bits / per_shard - 1, "vs_entropy": bits / H - 1}
+        res[name] = r
+    return res
+
+
+def configs_leg(dev, hx, datagen, torch, peak):
+    """cfg 1 (1 MiB, timed through CUDA graphs of 200 calls), cfg 2 (256 MiB FFN mixture, codebook
+    from 8 prior 256 MiB batches) and cfg 3 (64 MiB INT8 weights, per-tensor codebook)."""
+    out = {}
+    for cfg in (1, 2, 3):
+        prior = sum(np.bincount(b, minlength=256) for b in datagen.prior_batches(cfg))
+        x = torch.from_numpy(datagen.data(cfg)).to(dev)
+        out[f"cfg{cfg}"] = config_numbers(dev, hx, torch, x, prior.astype(np.uint64), peak,
+                                          reps=200 if cfg == 1 else 20, graph=cfg == 1)
+        del x
+    return out
+
+
+def cfg5_leg(dev, hx, datagen, torch):
+    """cfg 5: 64 tensors of 64 MiB (16 layers x 4 shards, e4m3 and INT8, laws and scales per
+    layer); each shard coded with its layer's fixed Huffman codebook (4 prior batches). Per
+    shard: fixed-codebook bits per symbol against a per-shard Huffman code and the entropy (the
+    drift); the whole batch's encode and decode time on the device (inputs resident)."""
+    rows = []
+    enc_ms = dec_ms = 0.0
+    total = 0
+    out = torch.empty(hx.encode_bound(datagen.CFG5_TENSOR), dtype=torch.uint8, device=dev)
+    scratch = torch.empty(hx.scratch_bytes(datagen.CFG5_TENSOR), dtype=torch.uint8, device=dev)
+    y = torch.empty(datagen.CFG5_TENSOR, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for layer in range(16):
+        prior = sum(np.bincount(b, minlength=256) for b in datagen.prior_batches(5, layer))
+        cb = hx.build_codebook(prior.astype(np.uint64))
+        t = cb.upload(dev)
+        law = datagen.cfg5_layer(layer)
+        for j in range(datagen.CFG5_SHARDS):
+            shard = layer * datagen.CFG5_SHARDS + j
+            xh = datagen.data(5, shard=shard)
+            x = torch.from_numpy(xh).to(dev)
+            n = x.numel()
+            h = np.bincount(xh, minlength=256).astype(np.uint64)
+            ms = {}
+            for op, fn in (("enc", lambda: hx.encode(t, x, out=out, scratch=scratch,
+                                                      status=status)),
+                           ("dec", lambda: hx.decode(t, out, n, out=y, status=status))):
+                fn()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                ms[op] = a.elapsed_time(b)
+            assert int(status.item()) == 0 and torch.equal(x, y)
+            enc_ms += ms["enc"]
+            dec_ms += ms["dec"]
+            total += n
+            fixed = hx.mean_length(h, cb)
+            own = hx.mean_length(h, hx.build_codebook(h, seen_only=True))
+            rows.append({"shard": shard, "layer": layer, "dtype": law["dtype"],
+                         "family": law["family"], "scale": round(law["scale"], 4),
+                         "fixed_bits": round(fixed, 4), "per_shard_bits": round(own, 4),
+                         "entropy": round(hx.entropy(h), 4),
+                         "drift": round(fixed / own - 1, 5),
+                         "framed_bits": round(hx.stream_size(out, n) * 8 / n, 4)})
+    drifts = [r["drift"] for r in rows]
+    return {"shards": len(rows), "bytes": total,
+            "encode_GB_per_s": total / (enc_ms * 1e-3) / 1e9,
+            "decode_GB_per_s": total / (dec_ms * 1e-3) / 1e9,
+            "drift_mean": float(np.mean(drifts)), "drift_max": float(np.max(drifts)),
+            "drift_min": float(np.min(drifts)),
+            "fixed_bits_mean": float(np.mean([r["fixed_bits"] for r in rows])),
+            "per_shard_bits_mean": float(np.mean([r["per_shard_bits"] for r in rows])),
+            "rows": rows}
+
+
+def collective_leg(dev, hx, datagen, torch, tables, prior):
+    """The compressed all-gather on one rank (NCCL, a process group of one): ms per GiB through
+    compressed_all_gather with 1 and 4 parts, against Huffman encode + decode alone. No figure
+    exists for 2 or more GPUs (every run here has one)."""
+    import datetime
+    import torch.distributed as dist
+    from lossless_entropy_coding_fixed_b200 import collective
+    n = 1 << 28
+    x = torch.from_numpy(datagen.data(4, n=n)).to(dev)
+    own = not dist.is_initialized()
+    if own:
+        store = dist.TCPStore("127.0.0.1", 0, 1, True, timeout=datetime.timedelta(seconds=60))
+        dist.init_process_group("nccl", store=store, rank=0, world_size=1, device_id=dev,
+                                timeout=datetime.timedelta(seconds=60))
+    try:
+        res = {"n": n}
+        for parts in (1, 4):
+            out, sent = collective.compressed_all_gather(x, tables, parts=parts)
+            torch.cuda.synchronize()
+            assert torch.equal(out, x)
+            t0 = time.perf_counter()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(5):
+                collective.compressed_all_gather(x, tables, parts=parts)
+            b.record()
+            torch.cuda.synchronize()
+            res[f"parts{parts}_ms_per_GiB"] = a.elapsed_time(b) / 5 * (1 << 30) / n
+            res[f"parts{parts}_wall_ms_per_GiB"] = (time.perf_counter() - t0) / 5 * 1e3 * (1 << 30) / n
+        st = hx.new_status(dev)
+        out = torch.empty(hx.encode_bound(n), dtype=torch.uint8, device=dev)
+        y = torch.empty_like(x)
+        scratch = torch.empty(hx.scratch_bytes(n), dtype=torch.uint8, device=dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(5):
+            hx.encode(tables, x, out=out, scratch=scratch, status=st)
+            hx.decode(tables, out, n, out=y, status=st)
+        b.record()
+        torch.cuda.synchronize()
+        res["codec_alone_ms_per_GiB"] = a.elapsed_time(b) / 5 * (1 << 30) / n
+        res["note"] = "one rank: the exchange is a local NCCL all-gather; no NVLink figure"
+        return res
+    finally:
+        if own:
+            dist.destroy_process_group()
+
+
+def e2e_leg(args, dev, hx, torch, pg, ws, x_host, ht, qt, n, bound, scratch, status):
+    """End to end through the public API with host buffers, both directions of a link: every step
+    uploads its batch from pinned memory, encodes it with both codebooks and downloads the two
+    streams (sender), then uploads the two streams, decodes them and downloads both decoded
+    batches (receiver). Steps are pipelined over two buffer slots on upload / codec / download
+    streams; every step's copies are inside the timed region."""
+    x_pin = torch.from_numpy(x_host).pin_memory()
+    host_st = [torch.empty(bound, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    host_y = [torch.empty(n, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    st_host = torch.empty(1, dtype=torch.int32).pin_memory()
+    hdr = torch.empty(2, 64, dtype=torch.uint8).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    s_in, s_out, s_hdr = (torch.cuda.Stream(dev) for _ in range(3))
+    slots = []
+    for _ in range(2):
+        sl = {"x": torch.empty(n, dtype=torch.uint8, device=dev),
+              "st": [torch.empty(bound, dtype=torch.uint8, device=dev) for _ in range(2)],
+              "rx": [torch.empty(bound, dtype=torch.uint8, device=dev) for _ in range(2)],
+              "y": [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(2)],
+              "used": torch.cuda.Event(), "free": torch.cuda.Event()}
+        sl["used"].record(stream)
+        sl["free"].record(s_out)
+        slots.append(sl)
+    books = ((ht, hx.KIND_HUFFMAN), (qt, hx.KIND_QLC))
+    counted = {"h2d": 0, "d2h": 0}
+    host_free = [torch.cuda.Event()]
+    host_free[0].record(s_in)
+
+    def sender(sl):
+        s_in.wait_event(sl["used"])
+        s_in.wait_event(sl["free"])
+        with torch.cuda.stream(s_in):
+            sl["x"].copy_(x_pin, non_blocking=True)
+        up = torch.cuda.Event()
+        up.record(s_in)
+        stream.wait_event(up)
+        done = []
+        for j, (t, kind) in enumerate(books):
+            hx.encode(t, sl["x"], out=sl["st"][j], scratch=scratch, status=status, kind=kind)
+            e = torch.cuda.Event()
+            e.record(stream)
+            done.append(e)
+        sl["enc"] = done
+        return n
+
+    def link(sl):
+        # the streams' sizes (their headers), then stream bytes down and back up
+        for j, e in enumerate(sl["enc"]):
+            s_hdr.wait_event(e)
+            with torch.cuda.stream(s_hdr):
+                hdr[j].copy_(sl["st"][j][:64], non_blocking=True)
+        got = torch.cuda.Event()
+        got.record(s_hdr)
+        got.synchronize()
+        sizes = [hx.stream_bytes(n, int(hdr[j][32:40].numpy().view(np.uint64)[0]))
+                 for j in range(2)]
+        # the host stream buffers are free once the previous step's upload has read them
+        s_out.wait_event(host_free[0])
+        for j in range(2):
+            s_out.wait_event(sl["enc"][j])
+            with torch.cuda.stream(s_out):
+                host_st[j][:sizes[j]].copy_(sl["st"][j][:sizes[j]], non_blocking=True)
+        down = torch.cuda.Event()
+        down.record(s_out)
+        s_in.wait_event(down)
+        with torch.cuda.stream(s_in):
+            for j in range(2):
+                sl["rx"][j][:sizes[j]].copy_(host_st[j][:sizes[j]], non_blocking=True)
+        up = torch.cuda.Event()
+        up.record(s_in)
+        host_free[0] = up
+        stream.wait_event(up)
+        for j, (t, kind) in enumerate(books):
+            hx.decode(t, sl["rx"][j], n, out=sl["y"][j], status=status, kind=kind,
+                      nbytes=sizes[j])
+        sl["used"].record(stream)
+        s_out.wait_event(sl["used"])
+        with torch.cuda.stream(s_out):
+            for j in range(2):
+                host_y[j].copy_(sl["y"][j], non_blocking=True)
+            st_host.copy_(status, non_blocking=True)
+        sl["free"].record(s_out)
+        # (bytes up, bytes down): the streams up; headers, streams, decoded batches, status down
+        return sum(sizes), 64 * 2 + sum(sizes) + 2 * n + 4
+
+    def run(k):
+        counted["h2d"] = counted["d2h"] = 0
+        pending = None
+        for t in range(k):
+            sl = slots[t % 2]
+            counted["h2d"] += sender(sl)
+            if pending is not None:
+                up, down = link(pending)
+                counted["h2d"] += up
+                counted["d2h"] += down
+            pending = sl
+        up, down = link(pending)
+        counted["h2d"] += up
+        counted["d2h"] += down
+        end = torch.cuda.Event()
+        end.record(s_out)
+        stream.wait_event(end)
+
+    run(2)  # untimed: both slots once
+    torch.cuda.synchronize(dev)
+    k = max(3, min(args.steps, 10))
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    run(k)
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    assert int(st_host.item()) == 0
+    assert torch.equal(host_y[0], x_pin) and torch.equal(host_y[1], x_pin)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / k, pg, dev)
+    return {"value": job_gbs(ws, 4 * n, e2e_ms), "unit": "GB/s",
+            "h2d_bytes_per_step": counted["h2d"] // k, "d2h_bytes_per_step": counted["d2h"] // k,
+            "steps": k,
+            "path": "pinned host batch -> H2D -> Huffman and QLC encode -> D2H of both streams "
+                    "-> H2D of both streams -> decode -> D2H of both decoded batches; steps "
+                    "pipelined over 2 buffer slots on upload / codec / download streams"}
 
 
 def shannonic_leg(dev, hx, torch, x, prior, h, scratch, y, status, steps):
@@ -403,28 +761,24 @@ def main():
     hist = torch.zeros(args.steps + 1, 256, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     ops = ["huffman_encode", "huffman_decode", "qlc_encode", "qlc_decode"]
-    # one event pair per kernel launch: an encode is two launches (measure, then pack)
-    kern = ["huffman_measure", "huffman_pack", "huffman_decode",
-            "qlc_measure", "qlc_pack", "qlc_decode"]
-    ev = {k: [] for k in kern}
+    ev = {o: [] for o in ops}
 
     def step(record: bool, row: int = 0):
-        marks = [torch.cuda.Event(enable_timing=True) for _ in range(7)] if record else None
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
         mark = (lambda i: marks[i].record(stream)) if record else (lambda i: None)
         mark(0)
-        hx.encode_passes(ht, x, sh, scratch, hist=hist[row], status=status,
-                         kind=hx.KIND_HUFFMAN, between=lambda: mark(1))
-        mark(2)
+        hx.encode(ht, x, out=sh, scratch=scratch, hist=hist[row], status=status,
+                  kind=hx.KIND_HUFFMAN)
+        mark(1)
         hx.decode(ht, sh, n, out=y, status=status, kind=hx.KIND_HUFFMAN)
+        mark(2)
+        hx.encode(qt, x, out=sq, scratch=scratch, status=status, kind=hx.KIND_QLC)
         mark(3)
-        hx.encode_passes(qt, x, sq, scratch, status=status, kind=hx.KIND_QLC,
-                         between=lambda: mark(4))
-        mark(5)
         hx.decode(qt, sq, n, out=y, status=status, kind=hx.KIND_QLC)
-        mark(6)
+        mark(4)
         if record:
-            for i, k in enumerate(kern):
-                ev[k].append((marks[i], marks[i + 1]))
+            for i, o in enumerate(ops):
+                ev[o].append((marks[i], marks[i + 1]))
 
     for _ in range(max(3, args.warmup)):
         step(False, args.steps)
@@ -451,11 +805,7 @@ def main():
         pg.barrier()
     elapsed_ms = max_over_ranks(start.elapsed_time(end), pg, dev)
     assert int(status.item()) == 0, f"status {int(status.item())}"
-    per_kernel_ms = {k: sum(a.elapsed_time(b) for a, b in ev[k]) / args.steps for k in kern}
-    per_op_ms = {"huffman_encode": per_kernel_ms["huffman_measure"] + per_kernel_ms["huffman_pack"],
-                 "huffman_decode": per_kernel_ms["huffman_decode"],
-                 "qlc_encode": per_kernel_ms["qlc_measure"] + per_kernel_ms["qlc_pack"],
-                 "qlc_decode": per_kernel_ms["qlc_decode"]}
+    per_op_ms = {o: sum(a.elapsed_time(b) for a, b in ev[o]) / args.steps for o in ops}
 
     # sizes and bits per symbol
     rows = hist[: args.steps].cpu().numpy().astype(np.uint64)
@@ -471,117 +821,19 @@ def main():
     ms_per_step = elapsed_ms / args.steps
     value = job_gbs(ws, 4 * n, ms_per_step)
     peak, peak_kind = hbm_peak()
-    # Algorithmic bytes of each kernel launch: measure reads the batch and writes the sync rows;
-    # pack reads the batch and writes the stream; decode reads the stream and writes the batch.
-    index = 16 * ((n + 4095) // 4096)
-    kernels = {  # kernel name -> [(algorithmic bytes, ms) per launch in a step]
-        "k_measure": [(n + index, per_kernel_ms["huffman_measure"]),
-                      (n + index, per_kernel_ms["qlc_measure"])],
-        "k_pack": [(n + size_h, per_kernel_ms["huffman_pack"]),
-                   (n + size_q, per_kernel_ms["qlc_pack"])],
-        "k_decode<0>": [(size_h + n, per_kernel_ms["huffman_decode"])],
-        "k_decode<1>": [(size_q + n, per_kernel_ms["qlc_decode"])],
-    }
+    # Each op is one launch of the library's kernel (an encode also clears its look-back words
+    # first, inside the op's time): k_encode reads the batch and writes the stream, k_decode reads
+    # the stream and writes the batch.
+    kernels = {"k_encode": ["huffman_encode", "qlc_encode"],
+               "k_decode": ["huffman_decode", "qlc_decode"]}
+    roof = {k: roofline_entry(k, [(alg_bytes[o], per_op_ms[o]) for o in v], peak, peak_kind)
+            for k, v in kernels.items()}
     # the dominant kernel: the largest share of the step
-    kernel_name = max(kernels, key=lambda k: sum(ms for _, ms in kernels[k]))
-    launches = kernels[kernel_name]
-    bytes_per_launch = sum(b for b, _ in launches) / len(launches)
-    ms_per_launch = sum(ms for _, ms in launches) / len(launches)
-    achieved = bytes_per_launch / (ms_per_launch * 1e-3) / 1e9
+    kernel_name = max(roof, key=lambda k: roof[k]["ms_per_launch"] * roof[k]["launches_per_step"])
 
-    # end to end through the public API with host buffers: every step uploads its batch from
-    # pinned memory, runs the four codec calls and downloads both streams (their sizes read from
-    # the headers). Steps are pipelined over two buffer slots and three streams (upload, codec,
-    # download), so one step's upload and the previous step's download overlap each other and
-    # the codec calls, as a caller streaming batches through the library would run them.
     e2e = None
     if not args.no_e2e:
-        x_pin = torch.from_numpy(x_host).pin_memory()
-        out_h = torch.empty(bound, dtype=torch.uint8).pin_memory()
-        out_q = torch.empty(bound, dtype=torch.uint8).pin_memory()
-        st_host = torch.empty(1, dtype=torch.int32).pin_memory()
-        hdr = torch.empty(2, 64, dtype=torch.uint8).pin_memory()
-        s_in, s_out, s_hdr = (torch.cuda.Stream(dev) for _ in range(3))
-        slots = [{"x": x, "sh": sh, "sq": sq},
-                 {"x": torch.empty_like(x), "sh": torch.empty_like(sh),
-                  "sq": torch.empty_like(sq)}]
-        for sl in slots:
-            sl["used"] = torch.cuda.Event()  # the codec calls are done with the slot's input
-            sl["free"] = torch.cuda.Event()  # the slot's streams have been downloaded
-            sl["used"].record(stream)
-            sl["free"].record(s_out)
-
-        def upload_and_code(sl):
-            s_in.wait_event(sl["used"])
-            with torch.cuda.stream(s_in):
-                sl["x"].copy_(x_pin, non_blocking=True)
-            up = torch.cuda.Event()
-            up.record(s_in)
-            stream.wait_event(up)
-            stream.wait_event(sl["free"])
-            done = []
-            for t, kind, key in ((ht, hx.KIND_HUFFMAN, "sh"), (qt, hx.KIND_QLC, "sq")):
-                hx.encode(t, sl["x"], out=sl[key], scratch=scratch, status=status, kind=kind)
-                e = torch.cuda.Event()
-                e.record(stream)
-                done.append(e)
-                hx.decode(t, sl[key], n, out=y, status=status, kind=kind)
-            sl["used"].record(stream)
-            return sl, done
-
-        def download(sl, done):
-            for j, (e, key) in enumerate(zip(done, ("sh", "sq"))):
-                s_hdr.wait_event(e)
-                with torch.cuda.stream(s_hdr):
-                    hdr[j].copy_(sl[key][:64], non_blocking=True)
-            got = torch.cuda.Event()
-            got.record(s_hdr)
-            got.synchronize()  # the host needs both stream sizes to copy them
-            d2h = 0
-            for j, (key, host) in enumerate((("sh", out_h), ("sq", out_q))):
-                size = hx.stream_bytes(n, int(hdr[j][32:40].numpy().view(np.uint64)[0]))
-                s_out.wait_event(done[j])
-                with torch.cuda.stream(s_out):
-                    host[:size].copy_(sl[key][:size], non_blocking=True)
-                d2h += size + 64
-            s_out.wait_event(sl["used"])
-            with torch.cuda.stream(s_out):
-                st_host.copy_(status, non_blocking=True)  # the step's status word
-            sl["free"].record(s_out)
-            return d2h + 4
-
-        def run(k, start=None):
-            if start is not None:
-                s_in.wait_event(start)
-            pending, d2h = None, 0
-            for t in range(k):
-                nxt = upload_and_code(slots[t % 2])
-                if pending:
-                    d2h = download(*pending)
-                pending = nxt
-            d2h = download(*pending)
-            end = torch.cuda.Event()
-            end.record(s_out)
-            stream.wait_event(end)
-            return d2h
-
-        run(2)  # untimed: both slots once
-        torch.cuda.synchronize(dev)
-        k_e2e = max(3, min(args.steps, 10))
-        if pg:
-            pg.barrier()
-        torch.cuda.synchronize(dev)
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        d2h = run(k_e2e, start=s0)
-        s1.record(stream)
-        torch.cuda.synchronize(dev)
-        assert int(st_host.item()) == 0
-        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / k_e2e, pg, dev)
-        e2e = {"value": job_gbs(ws, 4 * n, e2e_ms), "unit": "GB/s",
-               "h2d_bytes_per_step": n, "d2h_bytes_per_step": d2h, "steps": k_e2e,
-               "path": "pinned host batch -> H2D -> 4 codec calls -> D2H of both streams; steps "
-                       "pipelined over 2 buffer slots on upload / codec / download streams"}
+        e2e = e2e_leg(args, dev, hx, torch, pg, ws, x_host, ht, qt, n, bound, scratch, status)
 
     shannonic = None
     if not args.no_shannonic:
@@ -592,16 +844,32 @@ def main():
     if not args.no_expgolomb:
         expgolomb = expgolomb_leg(dev, hx, torch, x, h, scratch, y, status,
                                   max(3, min(args.steps, 10)))
+    del x, y, sh, sq, scratch
+    torch.cuda.empty_cache()
 
     online = None
     if not args.no_online:
         online = online_leg(dev, hx, datagen, torch)
+
+    configs = None
+    if not args.no_configs:
+        configs = configs_leg(dev, hx, datagen, torch, peak)
+
+    cfg5 = None
+    if not args.no_cfg5:
+        cfg5 = cfg5_leg(dev, hx, datagen, torch)
+
+    collective = None
+    if ws == 1 and not args.no_collective:
+        collective = collective_leg(dev, hx, datagen, torch, ht, prior)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_leg(prior)
 
     if rank == 0:
+        main_roof = dict(roof[kernel_name])
+        main_roof["traffic"] = recorded_traffic(kernel_name)
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -612,9 +880,9 @@ def main():
                        "parallelism": f"replicas x{ws} (independent batches, no collective)"},
             "ops": {o: {"ms": per_op_ms[o], "GB_per_s_uncompressed": n / (per_op_ms[o] * 1e-3) / 1e9,
                         "hbm_GB_per_s_algorithmic": alg_bytes[o] / (per_op_ms[o] * 1e-3) / 1e9,
-                        "hbm_frac_algorithmic": alg_bytes[o] / (per_op_ms[o] * 1e-3) / 1e9 / peak}
+                        "hbm_frac_algorithmic": alg_bytes[o] / (per_op_ms[o] * 1e-3) / 1e9 / peak,
+                        "hbm_frac_spec": alg_bytes[o] / (per_op_ms[o] * 1e-3) / 1e9 / SPEC_HBM_GBS}
                     for o in ops},
-            "kernels_ms": per_kernel_ms,
             "bits_per_symbol": {"huffman_payload": payload_bits_h,
                                 "huffman_framed": size_h * 8 / n,
                                 "qlc_payload": payload_bits_q, "qlc_framed": size_q * 8 / n,
@@ -622,18 +890,18 @@ def main():
                                 "fixed_vs_per_shard": payload_bits_h / per_shard - 1,
                                 "fixed_vs_entropy": payload_bits_h / H - 1},
             "host_codebook_build_us": {"huffman": (t1 - t0) * 1e6, "qlc": (t2 - t1) * 1e6},
-            "roofline": {"bound": "hbm", "kernel": kernel_name,
-                         "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                         "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": recorded_traffic(kernel_name),
-                         "algorithmic_bytes_per_launch": bytes_per_launch,
-                         "launches_per_step": len(launches), "ms_per_launch": ms_per_launch},
+            "roofline": main_roof,
+            "roofline_kernels": {k: dict(v, traffic=recorded_traffic(k)) for k, v in roof.items()},
             "cpu_baseline": cpu,
             "e2e": e2e,
+            "configs": configs,
+            "cfg5_drift": cfg5,
+            "collective": collective,
             "online": online,
             "shannonic": shannonic,
             "expgolomb": expgolomb,
-            "gpu_launches": 6 * args.steps,
+            # the library's kernels in the timed region: per step two k_encode, two k_decode
+            "gpu_launches": 4 * args.steps,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -54,7 +54,7 @@ typedef enum {
   HX_ERR_UNCODABLE = 4,  /* encode: an input byte has no code word (seen-only codebook)      */
   HX_ERR_CORRUPT = 8,    /* decode: the stream is malformed or does not decode exactly      */
   HX_ERR_CODEBOOK = 16,  /* decode: the stream was written with another codebook or kind    */
-  HX_ERR_TIMEOUT = 32,   /* reserved: a bounded device wait ran out (no current kernel waits) */
+  HX_ERR_TIMEOUT = 32,   /* encode: a bounded wait for the chunks before one ran out          */
   HX_ERR_CAPACITY = 64   /* encode: out_cap is too small; header.total_words holds the need */
 } hx_status;
 
@@ -125,11 +125,16 @@ int hx_shannonic_build(const uint64_t* counts, int K, uint32_t flags, hx_codeboo
  * FNV-1a-64 of [3, order, map]. */
 int hx_expgolomb_build(int order, int map, hx_codebook* out);
 
-/* Pack a codebook into the HX_TABLES_BYTES table block in host memory (host_tables). */
+/* Pack a codebook into the HX_TABLES_BYTES table block in host memory (host_tables): the
+ * encoder's code/length entry per byte value and the decoder's window table (for a QLC code the
+ * window table is computed from the area widths and the rank table), plus the codebook's kind,
+ * limit and hash. "Single-Stage Huffman Encoder for ML Compression", abstract: the sender and
+ * the receiver hold the same fixed codebook, so this block is built once per codebook, never per
+ * batch. The block's layout is private to the library. */
 int hx_codebook_tables(const hx_codebook* cb, void* host_tables);
 
 /* Pack and copy the table block to d_tables (HX_TABLES_BYTES of device memory) on `stream`.
- * cb may be released when the call returns. */
+ * cb may be released when the call returns. Same source as hx_codebook_tables. */
 int hx_codebook_upload(const hx_codebook* cb, void* d_tables, void* stream);
 
 /* Histogram of byte values: d_counts[v] += occurrences of v in d_in[0..n). d_counts is a
@@ -138,19 +143,23 @@ int hx_codebook_upload(const hx_codebook* cb, void* d_tables, void* stream);
  * running average defines the next fixed codebook). */
 int hx_histogram(const uint8_t* d_in, uint64_t n, uint32_t* d_counts, void* stream);
 
-/* Layout helpers (pure functions of n). */
+/* Layout helpers (pure functions of n): offsets and sizes of the stream format above. The pages
+ * fix no format; this one follows from decoding every chunk and sub-stream in parallel with no
+ * codebook shipped (the stream format, no passage). */
 uint64_t hx_payload_offset(uint64_t n);   /* P above                                         */
 uint64_t hx_sync_offset(uint64_t n);      /* S above                                         */
 uint64_t hx_encode_bound(uint64_t n);     /* largest stream for n bytes: P + 4*(1536*chunks+2) */
-uint64_t hx_scratch_bytes(uint64_t n);    /* device scratch that hx_encode needs             */
+uint64_t hx_scratch_bytes(uint64_t n);    /* device scratch of an encode: 8*chunks + 16       */
 
 /* Encode d_in[0..n) with the fixed Huffman codebook in d_tables into the stream d_out.
  * "Single-Stage Huffman Encoder for ML Compression", abstract (fixed codebook, nothing sent
- * but the coded data and a hash of the codebook).
+ * but the coded data and a hash of the codebook). One pass over the input: each chunk's word
+ * offset comes from the chunks before it through a bounded wait (see hx_encode_bounded).
  * d_out: out_cap bytes, at least hx_payload_offset(n) + 8. If the coded stream does not fit,
  * HX_ERR_CAPACITY is raised in *d_status, the header (with total_words) and the index are
- * still written, and the payload is not. d_scratch: hx_scratch_bytes(n) bytes of device memory,
- * contents ignored on entry and clobbered. d_hist: NULL, or a device u32[256] that accumulates
+ * still written, and no payload word is written at or past the space that out_cap leaves (the
+ * chunks that fit may have written theirs). d_scratch: hx_scratch_bytes(n) bytes of device
+ * memory, contents ignored on entry and clobbered (the call clears what it needs first). d_hist: NULL, or a device u32[256] that accumulates
  * the histogram of d_in (as hx_histogram) in the same pass. d_status: device u32.
  * Bytes with no code word raise HX_ERR_UNCODABLE and emit no bits. Tables of the wrong kind
  * raise HX_ERR_ARG in *d_status. */
@@ -158,6 +167,10 @@ int hx_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out
               void* d_scratch, uint32_t* d_hist, uint32_t* d_status, void* stream);
 
 /* Decode the stream d_stream (stream_bytes bytes) into d_out[0..n_expected).
+ * "Single-Stage Huffman Encoder for ML Compression", abstract: the receiver decodes with the
+ * same fixed codebook the sender used, identified by the hash in the header; "Quad Length Codes
+ * for Lossless Compression of e4m3", abstract: Huffman decoding is bit-sequential, which the
+ * stream's 8 sub-streams per 4096-symbol chunk turn into independent runs.
  * The header must match: magic, version, chunk, sub-streams, n == n_expected (else
  * HX_ERR_CORRUPT), kind, lmax and hash == the tables' (else HX_ERR_CODEBOOK). Every chunk's
  * index entries are checked, and each of its 8 sub-streams must decode to exactly the bit
@@ -190,22 +203,18 @@ int hx_decode_set(uint32_t kind, const void* const* d_tables, uint32_t n_tables,
                   const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
                   uint64_t n_expected, uint32_t* d_status, void* stream);
 
-/* The two passes of an encode, for callers that schedule or time them apart; hx_encode (kind 0)
- * and hx_qlc_encode (kind 1) are exactly hx_encode_measure followed by hx_encode_pack. The pages
- * do not split the encoder: the split is this library's way to give every chunk its offset with
- * no block waiting for another. kind: 0 Huffman, 1 QLC (must match the tables).
- *  - hx_encode_measure: code lengths only. Writes the index's sync rows into d_out, per-chunk
- *    word counts and per-piece bit counts into d_scratch, and (d_hist non-NULL) accumulates the
- *    histogram of d_in.
- *  - hx_encode_pack: from those, the header, the word offsets and the payload.
- * Give both the same arguments, in this order, on one stream; d_in, d_scratch and d_out must not
- * change in between. Errors as for hx_encode. */
-int hx_encode_measure(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
+/* hx_encode (and hx_qlc_encode, hx_expgolomb_encode) with its bounded wait exposed, for
+ * failure-detection tests; the pages have no counterpart (they describe no GPU encoder). The
+ * encoder reads its input once: each chunk publishes its word count as soon as it has measured
+ * it, and learns its word offset from the chunks before it (they are always running, so the wait
+ * ends). Every such wait is still bounded: after wait_ns nanoseconds (hx_encode uses 2 s) the
+ * chunk raises HX_ERR_TIMEOUT in *d_status and writes no payload, and every chunk still waiting
+ * gives up at once; the kernel completes and the context stays usable. withhold: a chunk that
+ * never publishes its count (UINT64_MAX: none), so that the chunks after it time out. kind 0, 1
+ * or 3 (HX_ERR_ARG for kind 2); other arguments and errors as hx_encode. */
+int hx_encode_bounded(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                       void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
-                      uint32_t* d_status, void* stream);
-int hx_encode_pack(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
-                   void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_status,
-                   void* stream);
+                      uint32_t* d_status, uint64_t wait_ns, uint64_t withhold, void* stream);
 
 /* Shannonic encode and decode (kind 2 tables): the same chunked stream, sub-stream framing and
  * index as hx_encode; inside a sub-stream the bits come from tANS run from its last symbol to

@@ -7,25 +7,17 @@
 //   k_histogram  byte histogram: 16-byte loads, one private 256-bin table per warp in shared
 //                memory, one global atomic per non-empty bin and block.
 //
-//   k_measure    code lengths only (the first of two passes over the input): a warp measures one
-//                4096-symbol chunk -- lane l looks up 16 bytes of each sub-stream in its own copy
-//                of the length table (no bank conflicts) -- and writes the chunk's sync row; a
-//                block owns a contiguous run of chunks and scans their word counts into
-//                block-local offsets. The fused histogram rides on the same lookups (a shared
-//                atomic that returns the length adds to a per-copy count).
+//   k_encode     one pass over the input. A warp takes the next chunk from a counter and loads it
+//                with coalesced 16-byte loads (16 bytes of each sub-stream per lane); the length
+//                pass (one lookup per symbol in the lane's own copy of the length table, a shared
+//                atomic that also counts the fused histogram) and a warp scan give the sync row
+//                and the chunk's word count, which it publishes at once; the coding pass joins two
+//                codes per 32-bit register, appends them to a 64-bit accumulator and ORs each
+//                finished word into the warp's chunk buffer; a decoupled look-back over the
+//                chunks before it (bounded wait) gives the chunk's word offset, and the chunk
+//                leaves with coalesced stores.
 //
-//   k_pack       every block scans the measure blocks' totals into offsets, so no block waits
-//                for another. A warp codes a whole chunk, lane p its piece p (128 bytes, a
-//                quarter sub-stream) starting at the bit that a warp prefix sum of the measured
-//                piece bit counts gives: one table lookup per symbol, two codes joined per 32-bit
-//                register and appended to a 64-bit accumulator, each finished word stored in the
-//                warp's shared buffer (a word two pieces share is stored by the piece that
-//                finishes it and the other ORs its bits in after a warp barrier). The chunk then
-//                leaves with coalesced stores at its final offset. A warp whose pieces start
-//                crowded in one shared-memory bank (every code 8 bits long) uses a spread buffer
-//                layout for that chunk.
-//
-//   k_decode     one thread per sub-stream (8 per chunk, 32 chunks per 256-thread block). The
+//   k_decode     one thread per sub-stream (8 per chunk, 128 chunks per 1024-thread block). The
 //                two payload words in use and a bit offset into them give the next 32 bits with
 //                one funnel shift, enough for two codes; two more words are already requested
 //                (predicated 4-byte loads, no lane-dependent branch). One lookup per symbol in
@@ -37,7 +29,8 @@
 //                blocks instead.
 //
 //   k_sh_*       the Shannonic range coder: tANS over range indices, one thread per sub-stream
-//                in its measure, pack and (backward) decode kernels.
+//                in its measure, pack and (backward) decode kernels (two encode passes: a tANS
+//                sub-stream's length is known only once it has been run).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -52,7 +45,8 @@ namespace {
 constexpr uint32_t kMagic = 0x31305848u;  // "HX01"
 constexpr uint32_t kChunk = HX_CHUNK;
 constexpr uint32_t kSubLen = HX_CHUNK / HX_SUBSTREAMS;
-constexpr int kDecThreads = 256;  // 8 threads per chunk, 32 chunks per block
+constexpr int kDecThreads = 256;  // Shannonic decode: 8 threads per chunk, 32 chunks per block
+constexpr int kPfxThreads = 1024;  // prefix-code decode: 8 threads per chunk, 128 chunks per block
 constexpr int kHistThreads = 256;
 
 __host__ __device__ inline uint64_t n_chunks_of(uint64_t n) { return (n + kChunk - 1) / kChunk; }
@@ -96,28 +90,26 @@ __global__ void __launch_bounds__(kHistThreads) k_histogram(const uint8_t* __res
 }
 
 // ---------------------------------------------------------------------------------- encode
-// Two passes over the input, with no block waiting for another:
-//   k_measure  code lengths only. Every chunk's sub-stream bit counts become its sync row (the
-//              stream's index) and its word count; a measure block owns a contiguous run of
-//              chunks, scans their word counts into block-local offsets (scratch) and records
-//              its total. The fused histogram is counted here.
-//   k_pack     every block scans the measure blocks' totals (a few thousand at most) into their
-//              offsets; then one warp codes one whole chunk, sub-stream by sub-stream, into a
-//              shared-memory buffer and stores it at its final place in the payload.
+// The arguments of an encode: k_encode (kinds 0, 1, 3) reads the look-back fields, the Shannonic
+// passes (kind 2) the measure-block fields.
 struct EncodeArgs {
   const hx::Tables* tables;
   const uint8_t* in;
   uint64_t n;
   uint8_t* out;
   uint64_t cap;
-  uint32_t* local;   // scratch: block-local word offset of every chunk
-  uint32_t* btotal;  // scratch: words of each measure block
-  uint16_t* pieces;  // scratch: bit count of each 128-byte piece, 32 per chunk
-  uint32_t mblocks;  // measure blocks
-  uint32_t cpb;      // chunks per measure block
+  uint32_t* local;   // Shannonic scratch: block-local word offset of every chunk
+  uint32_t* btotal;  // Shannonic scratch: words of each measure block
+  uint32_t mblocks;  // Shannonic measure blocks
+  uint32_t cpb;      // chunks per Shannonic measure block
   uint32_t* hist;    // optional fused histogram
   uint32_t* status;
   uint32_t kind;
+  // single-pass encoder (k_encode)
+  uint64_t* look;     // scratch: each chunk's published word count or word offset (zeroed)
+  uint32_t* counter;  // scratch: next chunk to take (zeroed)
+  uint64_t wait_ns;   // limit of one chunk's wait for its predecessors
+  uint64_t withhold;  // a chunk that publishes nothing (failure tests), else ~0
 };
 
 // Every header field but total_words.
@@ -202,45 +194,93 @@ __device__ uint32_t block_exclusive_scan(uint32_t* cnt, uint32_t m, uint32_t* re
   return total;
 }
 
-constexpr int kMeasureThreads = 768;  // one block of 24 warps per SM, one table for all
-constexpr int kMeasureCopies = 32;            // lane l reads copy l: no bank conflicts
+// Limits of the Shannonic coder's measure blocks (the two-pass encoder of kind 2).
 constexpr uint32_t kMaxChunksPerBlock = 4096;  // chunks of one measure block
 constexpr uint32_t kMaxMeasureBlocks = 2048;
-// 16-bit counters; a round (one chunk per warp) adds at most 8 * 128 to a copy
-constexpr uint32_t kMeasureFlushRounds = 65535 / ((kMeasureThreads / 32) * 128);
+constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536: a chunk's largest size
 
-struct MeasureSmem {
-  uint32_t lut[256 * kMeasureCopies];  // [symbol][copy]: (count << 16) | len
-  uint32_t cnt[kMaxChunksPerBlock];    // words per chunk, then block-local word offsets
-  uint32_t red[kMeasureThreads / 32];
+// ---------------------------------------------------------------------------------- encode, one pass
+// k_encode reads the input once. A warp takes the next chunk from a counter, loads it (16 bytes
+// of each sub-stream per lane: every load instruction reads 512 contiguous bytes), sums the code
+// lengths of its 16-symbol segments (with the fused histogram), scans them into the sync row, and
+// publishes the chunk's word count at once. It then codes the chunk into its shared-memory buffer
+// while the chunks before it finish, learns its word offset from them (a decoupled look-back:
+// the nearest published offset plus the word counts in between), and copies the chunk out.
+// Chunks are taken in order by running warps, each of which publishes its count before it waits,
+// so every wait ends; each is still bounded (wait_ns), after which the chunk raises HX_ERR_TIMEOUT
+// and writes no payload, and every later wait gives up at once.
+constexpr int kEncThreads = 768;  // one block of 24 warps per SM sharing the two tables
+constexpr uint32_t kEncWarps = kEncThreads / 32;
+// 16-bit counts in the length table: a round of chunks adds at most kEncWarps * 128 to an entry
+constexpr uint32_t kEncFlushRounds = 65535 / (kEncWarps * 128);
+static_assert(kEncFlushRounds >= 1, "16-bit counts overflow within one round");
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kLookAgg = 1ull << 62;   // word count of the chunk alone
+constexpr uint64_t kLookPre = 2ull << 62;   // word offset of the chunk's end (inclusive prefix)
+constexpr uint64_t kLookValue = (1ull << 62) - 1;
+
+// Two tables, entries [symbol][copy] with lane l using copy l (no bank conflicts): `len` =
+// (count << 16) | len for the length pass (with the fused histogram the lookup is a shared atomic
+// that adds 1 << 16), `code` = (code << 20) | len for the coding pass.
+struct EncSmem {
+  uint32_t len[256 * 32];
+  uint32_t code[256 * 32];
+  alignas(16) uint32_t buf[kEncWarps][kMaxChunkWords];  // each warp's chunk, zero between chunks
+  uint32_t sink[kEncWarps][32];  // a word per lane for the stores a pair does not make
 };
 
-// Byte offset of table entry sym * 32 + lane in a [symbol][32] u32 table, for byte J (0..3) of w:
-// one shift and one AND-OR (lane4 = lane * 4 < 128).
-template <int J>
-__device__ __forceinline__ uint32_t lut_off(uint32_t w, uint32_t lane4) {
-  return ((J == 0 ? (w << 7) : (w >> (8 * J - 7))) & 0x7f80u) | lane4;
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
 
-// Sum of the table entries of the 16 bytes in v (count of them: `valid`); the low 16 bits of the
-// sum are the bit count (<= 16 * 12). With HIST each lookup is a shared atomic that also adds 1
-// to the entry's count (bits 16..31).
+// 32-bit shared-memory addresses for the encoder's tables and buffers (no generic 64-bit address
+// arithmetic): byte J of w picks the row of a [symbol][32] table with one byte permute and one
+// multiply-add; `base` is the table's shared address plus 4 * lane.
+template <int J>
+__device__ __forceinline__ uint32_t row_addr(uint32_t w, uint32_t base) {
+  return __byte_perm(w, 0u, 0x4440u + J) * 128u + base;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t atoms_add_u32(uint32_t a, uint32_t x) {
+  uint32_t v;
+  asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(v) : "r"(a), "r"(x) : "memory");
+  return v;
+}
+__device__ __forceinline__ void reds_or_u32(uint32_t a, uint32_t x) {
+  asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(x) : "memory");
+}
+
+// Sum of the length-table entries of the 16 bytes in v (count of them exist); as measure16, on
+// 32-bit shared addresses.
 template <bool HIST, bool COMPLETE, bool WHOLE>
-__device__ __forceinline__ uint32_t measure16(char* lut, uint32_t lane4, const uint4& v,
-                                              uint32_t valid, bool& uncodable) {
+__device__ __forceinline__ uint32_t lengths16(uint32_t base, const uint4& v, uint32_t count,
+                                              bool& uncodable) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t sum = 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      if (WHOLE || (uint32_t)(4 * q + j) < valid) {
-        const uint32_t off = j == 0   ? lut_off<0>(w[q], lane4)
-                             : j == 1 ? lut_off<1>(w[q], lane4)
-                             : j == 2 ? lut_off<2>(w[q], lane4)
-                                      : lut_off<3>(w[q], lane4);
-        uint32_t* slot = reinterpret_cast<uint32_t*>(lut + off);
-        const uint32_t e = HIST ? atomicAdd(slot, 1u << 16) : *slot;
+      if (WHOLE || (uint32_t)(4 * q + j) < count) {
+        const uint32_t a = j == 0   ? row_addr<0>(w[q], base)
+                           : j == 1 ? row_addr<1>(w[q], base)
+                           : j == 2 ? row_addr<2>(w[q], base)
+                                    : row_addr<3>(w[q], base);
+        const uint32_t e = HIST ? atoms_add_u32(a, 1u << 16) : lds_u32(a);
         sum += e;
         if (!COMPLETE) uncodable |= (e & 0xffu) == 0;
       }
@@ -249,313 +289,261 @@ __device__ __forceinline__ uint32_t measure16(char* lut, uint32_t lane4, const u
   return sum & 0xffffu;
 }
 
-// One chunk's sync row (lane 0 writes it) and the bit counts of its 32 pieces of 128 bytes
-// (piece p = bytes 128p .. 128p + 127: a quarter of sub-stream p / 4); returns its bit count.
-// WHOLE: all 4096 bytes exist.
-template <bool HIST, bool COMPLETE, bool WHOLE>
-__device__ __forceinline__ uint32_t measure_chunk(const EncodeArgs& a, uint32_t c, char* lut,
-                                                  uint4* sync, bool& uncodable) {
-  const uint32_t lane = threadIdx.x & 31, lane4 = lane * 4;
-  uint4 v[HX_SUBSTREAMS];
-  uint32_t valid[HX_SUBSTREAMS];
+// Word offset of chunk c (c > 0) from the chunks before it, read 32 at a time by the warp: the
+// sum of the counts back to (and including) the nearest published offset. ~0 when the wait ran
+// out or another chunk's did.
+__device__ uint64_t lookback(const EncodeArgs& a, uint32_t c, uint32_t lane) {
+  uint64_t excl = 0;
+  const uint64_t t0 = global_ns();
+  for (int64_t base = (int64_t)c - 1; base >= 0; base -= 32) {
+    const int64_t i = base - (int64_t)lane;
+    uint64_t v = i >= 0 ? ld_relaxed_u64(a.look + i) : kLookPre;  // before chunk 0: offset 0
+    uint32_t pmask, need;
+    for (;;) {
+      pmask = __ballot_sync(0xffffffffu, (v >> 62) == 2);
+      const uint32_t zmask = __ballot_sync(0xffffffffu, (v >> 62) == 0);
+      // lanes up to the nearest published offset, or all of them
+      need = pmask ? ((pmask & (0u - pmask)) << 1) - 1u : 0xffffffffu;
+      if ((zmask & need) == 0) break;
+      const bool out = global_ns() - t0 > a.wait_ns ||
+                       (*reinterpret_cast<volatile uint32_t*>(a.status) & HX_ERR_TIMEOUT);
+      if (__any_sync(0xffffffffu, out)) return ~0ull;
+      __nanosleep(64);
+      if ((v >> 62) == 0) v = ld_relaxed_u64(a.look + i);
+    }
+    uint64_t val = (need >> lane) & 1u ? (v & kLookValue) : 0ull;
 #pragma unroll
-  for (int k = 0; k < HX_SUBSTREAMS; ++k) valid[k] = load16(a, c, k, lane, WHOLE, v[k]);
-  uint32_t row[HX_SUBSTREAMS];  // bit offset of each sub-stream in the chunk
-  uint32_t run = 0, piece = 0;
-#pragma unroll
-  for (int k = 0; k < HX_SUBSTREAMS; ++k) {
-    row[k] = run;
-    // lanes 8q .. 8q + 7 hold quarter q of sub-stream k: three steps sum each quarter
-    uint32_t x = measure16<HIST, COMPLETE, WHOLE>(lut, lane4, v[k], valid[k], uncodable);
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 4);
-    if ((lane & 7) == (uint32_t)k) piece = x;  // lane 8q + k keeps piece 4k + q
-    x += __shfl_xor_sync(0xffffffffu, x, 8);
-    x += __shfl_xor_sync(0xffffffffu, x, 16);
-    run += x;
+    for (int d = 16; d > 0; d >>= 1) val += __shfl_xor_sync(0xffffffffu, val, d);
+    excl += val;
+    if (pmask) break;
   }
-  a.pieces[(uint64_t)c * 32 + (lane & 7) * 4 + (lane >> 3)] = (uint16_t)piece;
-  if (lane == 0)
+  return excl;
+}
+
+// Codes the lane's 16 symbols of one sub-stream (bytes of v, `count` of them) as the bits
+// [s, s + their length) of the chunk buffer, which is zero there: two codes are joined in a
+// 32-bit register (at most 24 bits) and appended to a 64-bit accumulator; each finished word,
+// and the unfinished last one, is OR-ed into the buffer (the pieces of neighbouring lanes share
+// the first and the last word). Every pair makes one OR, into the lane's sink word when it
+// finishes no word, so the loop has no branch.
+template <bool WHOLE>
+__device__ __forceinline__ void pack_segment(uint32_t base, const uint4& v, uint32_t count,
+                                             uint32_t buf, uint32_t sink, uint32_t s) {
+  uint32_t wa = buf + 4 * (s >> 5), nacc = s & 31, hi = 0, lo = 0;
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t e[4];
+    e[0] = (WHOLE || 4 * q + 0 < (int)count) ? lds_u32(row_addr<0>(w[q], base)) : 0u;
+    e[1] = (WHOLE || 4 * q + 1 < (int)count) ? lds_u32(row_addr<1>(w[q], base)) : 0u;
+    e[2] = (WHOLE || 4 * q + 2 < (int)count) ? lds_u32(row_addr<2>(w[q], base)) : 0u;
+    e[3] = (WHOLE || 4 * q + 3 < (int)count) ? lds_u32(row_addr<3>(w[q], base)) : 0u;
+#pragma unroll
+    for (int h = 0; h < 4; h += 2) {
+      const uint32_t l1 = e[h + 1] & 0xffu;
+      const uint32_t pl = (e[h] & 0xffu) + l1;
+      const uint32_t pc = ((e[h] >> 20) << l1) | (e[h + 1] >> 20);
+      hi = __funnelshift_l(lo, hi, pl);
+      lo = (lo << pl) | pc;
+      nacc += pl;
+      const bool full = nacc >= 32;
+      nacc -= full ? 32u : 0u;
+      reds_or_u32(full ? wa : sink, __funnelshift_r(lo, hi, nacc));
+      wa += full ? 4u : 0u;
+    }
+  }
+  reds_or_u32(nacc ? wa : sink, lo << (32 - nacc));
+}
+
+// One chunk by one warp (see k_encode).
+template <bool HIST, bool COMPLETE, bool WHOLE>
+__device__ __forceinline__ void encode_chunk(const EncodeArgs& a, EncSmem& sm, uint32_t c,
+                                             uint32_t* buf, uint32_t* sink, bool& uncodable) {
+  const uint32_t lane = threadIdx.x & 31, lane4 = lane * 4;
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
+  uint32_t first[HX_SUBSTREAMS], row[HX_SUBSTREAMS];
+  uint32_t run = 0;
+  {
+    // the length pass: 16 bytes of each sub-stream per lane (coalesced 512-byte loads)
+    uint4 v[HX_SUBSTREAMS];
+    uint32_t valid[HX_SUBSTREAMS];
+#pragma unroll
+    for (int k = 0; k < HX_SUBSTREAMS; ++k) valid[k] = load16(a, c, k, lane, WHOLE, v[k]);
+    const uint32_t lenbase = (uint32_t)__cvta_generic_to_shared(sm.len) + lane4;
+#pragma unroll
+    for (int k = 0; k < HX_SUBSTREAMS; k += 2) {
+      // two sub-streams per scan: bit counts < 2^16 in the two halves of a word
+      const uint32_t b0 = lengths16<HIST, COMPLETE, WHOLE>(lenbase, v[k], valid[k], uncodable);
+      const uint32_t b1 = lengths16<HIST, COMPLETE, WHOLE>(lenbase, v[k + 1], valid[k + 1],
+                                                           uncodable);
+      uint32_t incl = b0 | (b1 << 16);
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= (uint32_t)d) incl += t;
+      }
+      const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+      row[k] = run;
+      first[k] = run + (incl & 0xffffu) - b0;
+      run += tot & 0xffffu;
+      row[k + 1] = run;
+      first[k + 1] = run + (incl >> 16) - b1;
+      run += tot >> 16;
+    }
+  }
+  const uint32_t words = (run + 31) >> 5;
+  // publish the word count before anything waits
+  if (lane == 0 && c != a.withhold)
+    st_relaxed_u64(a.look + c, (c == 0 ? kLookPre : kLookAgg) | words);
+  if (lane == 0) {
+    uint4* sync = reinterpret_cast<uint4*>(a.out + sync_offset(n));
     sync[c] = make_uint4(run | (row[1] << 16), row[2] | (row[3] << 16), row[4] | (row[5] << 16),
                          row[6] | (row[7] << 16));
-  return run;
+  }
+  // the coding pass, sub-stream by sub-stream; the lane's bytes again (from L2, where the first
+  // load left them), one sub-stream ahead of the coding
+  const uint32_t f01 = first[0] | (first[1] << 16), f23 = first[2] | (first[3] << 16);
+  const uint32_t f45 = first[4] | (first[5] << 16), f67 = first[6] | (first[7] << 16);
+  const uint32_t codebase = (uint32_t)__cvta_generic_to_shared(sm.code) + lane4;
+  const uint32_t buf32 = (uint32_t)__cvta_generic_to_shared(buf);
+  const uint32_t sink32 = (uint32_t)__cvta_generic_to_shared(sink);
+  uint4 vn;
+  uint32_t cn = load16(a, c, 0, lane, WHOLE, vn);
+#pragma unroll 1
+  for (uint32_t k = 0; k < HX_SUBSTREAMS; ++k) {
+    const uint4 vk = vn;
+    const uint32_t ck = cn;
+    if (k + 1 < HX_SUBSTREAMS) cn = load16(a, c, k + 1, lane, WHOLE, vn);
+    const uint32_t fw = k < 2 ? f01 : k < 4 ? f23 : k < 6 ? f45 : f67;
+    pack_segment<WHOLE>(codebase, vk, ck, buf32, sink32, (fw >> (16 * (k & 1))) & 0xffffu);
+  }
+  __syncwarp();
+  // the chunk's word offset
+  uint64_t off = 0;
+  bool copy = true;
+  if (c > 0) {
+    off = lookback(a, c, lane);
+    if (off == ~0ull) {
+      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
+      copy = false;
+    } else if (lane == 0 && c != a.withhold) {
+      st_relaxed_u64(a.look + c, kLookPre | (off + words));
+    }
+  }
+  if (copy) {
+    const uint64_t P = payload_offset(n);
+    uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
+    uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
+    const uint64_t end = off + words;
+    if (lane == 0) word_off[c] = (uint32_t)off;
+    if (c + 1 == nchunks && lane == 0) {
+      reinterpret_cast<uint64_t*>(a.out)[4] = end;
+      word_off[nchunks] = (uint32_t)end;
+    }
+    // payload words that fit before the 2 guard words at the end of the caller's buffer
+    const uint64_t room = a.cap >= P + 8 ? (a.cap - P - 8) / 4 : 0;
+    if (end > room) {
+      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
+    } else {
+      for (uint32_t i = lane; i < words; i += 32) payload[off + i] = buf[i];
+      if (c + 1 == nchunks && lane < 2) payload[end + lane] = 0;
+    }
+  }
+  __syncwarp();
+  // leave the buffer zero for the next chunk
+  uint4* b4 = reinterpret_cast<uint4*>(buf);
+  for (uint32_t q = lane; q < (words + 3) / 4; q += 32) b4[q] = make_uint4(0, 0, 0, 0);
+  __syncwarp();
 }
 
 template <bool HIST, bool COMPLETE>
-__device__ void measure_chunks(const EncodeArgs& a, MeasureSmem& sm) {
+__device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint64_t n = a.n;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  const uint32_t full_chunks = (uint32_t)(n / kChunk);
-  const uint32_t c0 = blockIdx.x * a.cpb;
-  const uint32_t m = c0 < nchunks ? min(a.cpb, nchunks - c0) : 0u;
-  uint4* sync = reinterpret_cast<uint4*>(a.out + sync_offset(n));
-  char* lut = reinterpret_cast<char*>(sm.lut);
+  const uint32_t nchunks = (uint32_t)n_chunks_of(a.n);
+  const uint32_t full_chunks = (uint32_t)(a.n / kChunk);
+  uint32_t* buf = sm.buf[warp];
+  uint32_t* sink = &sm.sink[warp][lane];
+  for (uint32_t q = lane; q < kMaxChunkWords / 4; q += 32)
+    reinterpret_cast<uint4*>(buf)[q] = make_uint4(0, 0, 0, 0);
+  __syncwarp();
   bool uncodable = false;
-
-  auto flush_hist = [&]() {  // counts of the table copies -> global, then clear them
-    __syncthreads();
-    for (int sym = tid; sym < 256; sym += kMeasureThreads) {
-      uint32_t sum = 0;
-      for (int l = 0; l < kMeasureCopies; ++l) {
-        const uint32_t e = sm.lut[sym * kMeasureCopies + l];
-        sum += e >> 16;
-        sm.lut[sym * kMeasureCopies + l] = e & 0xffffu;
+  bool more = true;
+  for (uint32_t r = 0;; ++r) {
+    if (more) {
+      uint32_t c = 0;
+      if (lane == 0) c = atomicAdd(a.counter, 1u);
+      c = __shfl_sync(0xffffffffu, c, 0);
+      more = c < nchunks;
+      if (more) {
+        // the chunk a warp will most likely take one round from now, into L2
+        const uint64_t ahead = (uint64_t)c + gridDim.x * kEncWarps;
+        if (lane == 0 && ahead < full_chunks)
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.in + ahead * kChunk),
+                       "r"(kChunk)
+                       : "memory");
+        if (c < full_chunks) encode_chunk<HIST, COMPLETE, true>(a, sm, c, buf, sink, uncodable);
+        else encode_chunk<HIST, COMPLETE, false>(a, sm, c, buf, sink, uncodable);
       }
-      if (sum) atomicAdd(&a.hist[sym], sum);
     }
-    __syncthreads();
-  };
-
-  // round r: warp w measures the block's chunk kWarps * r + w
-  constexpr uint32_t kWarps = kMeasureThreads / 32;
-  const uint32_t rounds = (m + kWarps - 1) / kWarps;
-  for (uint32_t r = 0; r < rounds; ++r) {
-    const uint32_t i = r * kWarps + warp;
-    if (i < m) {
-      const uint32_t c = c0 + i;
-      const uint32_t bits =
-          c < full_chunks ? measure_chunk<HIST, COMPLETE, true>(a, c, lut, sync, uncodable)
-                          : measure_chunk<HIST, COMPLETE, false>(a, c, lut, sync, uncodable);
-      if (lane == 0) sm.cnt[i] = (bits + 31) >> 5;
+    if (HIST) {
+      // the 16-bit counts go to the histogram every kEncFlushRounds rounds (a warp without a
+      // chunk left just counts rounds); the block leaves together once no warp has one
+      if ((r + 1) % kEncFlushRounds == 0) {
+        __syncthreads();
+        for (int sym = tid; sym < 256; sym += kEncThreads) {
+          uint32_t sum = 0;
+          for (int l = 0; l < 32; ++l) {
+            const uint32_t e = sm.len[sym * 32 + l];
+            sum += e >> 16;
+            sm.len[sym * 32 + l] = e & 0xffffu;
+          }
+          if (sum) atomicAdd(&a.hist[sym], sum);
+        }
+        if (!__syncthreads_or(more)) break;
+      }
+    } else if (!more) {
+      break;
     }
-    if (HIST && (r + 1) % kMeasureFlushRounds == 0) flush_hist();
   }
-  __syncthreads();
-  const uint32_t total = block_exclusive_scan<kMeasureThreads>(sm.cnt, m, sm.red);
-  for (uint32_t i = tid; i < m; i += kMeasureThreads) a.local[c0 + i] = sm.cnt[i];
-  if (tid == 0) a.btotal[blockIdx.x] = total;
-  if (!COMPLETE && uncodable) atomicOr(a.status, (uint32_t)HX_ERR_UNCODABLE);
-  if (HIST) flush_hist();
+  if (!COMPLETE && __any_sync(0xffffffffu, uncodable) && lane == 0)
+    atomicOr(a.status, (uint32_t)HX_ERR_UNCODABLE);
 }
 
-__global__ void __launch_bounds__(kMeasureThreads, 1) k_measure(EncodeArgs a) {
+__global__ void __launch_bounds__(kEncThreads, 1) k_encode(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  MeasureSmem& sm = *reinterpret_cast<MeasureSmem*>(smem_raw);
+  EncSmem& sm = *reinterpret_cast<EncSmem*>(smem_raw);
   const int tid = threadIdx.x;
   if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
     return;
   }
   bool complete = true;
-  for (int i = tid; i < 256 * kMeasureCopies; i += kMeasureThreads) {
+  for (int i = tid; i < 256 * 32; i += kEncThreads) {
     uint32_t code;
-    const uint32_t len = checked_code(a, i / kMeasureCopies, &code);
+    const uint32_t len = checked_code(a, i / 32, &code);
     complete &= len != 0;
-    sm.lut[i] = len;
+    sm.len[i] = len;
+    sm.code[i] = (code << 20) | len;
   }
   complete = __syncthreads_and(complete);
-  if (a.hist) {
-    if (complete) measure_chunks<true, true>(a, sm);
-    else measure_chunks<true, false>(a, sm);
-  } else {
-    if (complete) measure_chunks<false, true>(a, sm);
-    else measure_chunks<false, false>(a, sm);
-  }
-}
-
-// a warp per chunk; lane p codes piece p (128 bytes). One block of 24 warps per SM shares one
-// copy of the code table (measured best: more warps starve L1, fewer leave issue slots idle)
-constexpr int kPackThreads = 768;
-constexpr int kPackCopies = 32;    // lane l reads copy l: no bank conflicts
-constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536
-constexpr uint32_t kMaxPieceBits = 128 * HX_LMAX_MAX;
-
-// Two layouts of a warp's chunk buffer, chosen per chunk:
-//   plain   chunk word w at w + (the chunk's word offset & 3), so that 16-byte aligned runs of the
-//           payload are 16-byte aligned here too and leave as uint4;
-//   spread  chunk word w at w + w / 32 (one unused word after every 32), copied out word by word.
-// Lanes store the words their pieces finish at about the same pace, so pieces that start in the
-// same bank keep colliding; a warp takes spread when kCrowded or more of its 32 pieces start in
-// one bank (pieces a multiple of 32 words long, as when every code has 8 bits), where the plain
-// layout would serialise most of its stores.
-constexpr uint32_t kCrowded = 8;
-template <bool SPREAD>
-__device__ __forceinline__ uint32_t buf_slot(uint32_t w) { return SPREAD ? w + (w >> 5) : w; }
-constexpr uint32_t kBufWords = (kMaxChunkWords + kMaxChunkWords / 32 + 3) & ~3u;  // both fit
-static_assert(kBufWords >= kMaxChunkWords + 4, "the plain layout needs 3 words of offset");
-
-struct PackSmem {
-  uint32_t lut[256 * kPackCopies];                  // [symbol][copy]: (code << 20) | len
-  alignas(16) uint32_t out[kPackThreads / 32][kBufWords];  // one chunk per warp
-  uint32_t bpre[kMaxMeasureBlocks];                  // word offset of each measure block
-  uint32_t red[kPackThreads / 32];
-};
-
-// Table entry of byte J (0..3) of w for this lane (copy `lane` of the [symbol][32] table).
-template <int J>
-__device__ __forceinline__ uint32_t lut_entry(const char* lut, uint32_t w, uint32_t lane4) {
-  return *reinterpret_cast<const uint32_t*>(lut + lut_off<J>(w, lane4));
-}
-
-// Codes m (<= 128) bytes at src as the bits [s, s + its length) of the chunk's word buffer:
-// two codes are joined in a 32-bit register (<= 24 bits), appended to a 64-bit accumulator
-// (hi:lo) with funnel shifts, and every word this piece finishes is stored whole (bits of earlier
-// pieces in it as zeros) at its buf_slot. Returns the unfinished last word's bits in the low
-// *nacc bits; *widx is its index.
-template <bool WHOLE, bool SPREAD>
-__device__ __forceinline__ uint32_t pack_piece(const uint8_t* src, uint32_t m, const char* lut,
-                                               uint32_t lane4, uint32_t* buf, uint32_t s,
-                                               uint32_t* widx_out, uint32_t* nacc_out) {
-  uint32_t widx = s >> 5, nacc = s & 31, hi = 0, lo = 0;
-  auto put2 = [&](uint32_t e0, uint32_t e1) {
-    const uint32_t l1 = e1 & 0xffu;
-    const uint32_t pl = (e0 & 0xffu) + l1;
-    const uint32_t pc = ((e0 >> 20) << l1) | (e1 >> 20);
-    hi = __funnelshift_l(lo, hi, pl);
-    lo = (lo << pl) | pc;
-    nacc += pl;
-    const bool full = nacc >= 32;
-    nacc -= full ? 32u : 0u;
-    if (full) buf[buf_slot<SPREAD>(widx)] = __funnelshift_r(lo, hi, nacc);
-    widx += full ? 1u : 0u;
-  };
-  auto put_word = [&](uint32_t w, uint32_t count) {  // bytes 0..count-1 of w
-    uint32_t e[4];
-    e[0] = (WHOLE || count > 0) ? lut_entry<0>(lut, w, lane4) : 0u;
-    e[1] = (WHOLE || count > 1) ? lut_entry<1>(lut, w, lane4) : 0u;
-    e[2] = (WHOLE || count > 2) ? lut_entry<2>(lut, w, lane4) : 0u;
-    e[3] = (WHOLE || count > 3) ? lut_entry<3>(lut, w, lane4) : 0u;
-    put2(e[0], e[1]);
-    put2(e[2], e[3]);
-  };
-  if (WHOLE) {
-    const uint4* s4 = reinterpret_cast<const uint4*>(src);
-    uint4 v = __ldg(s4);
-#pragma unroll 1
-    for (uint32_t g = 0; g < 8; ++g) {
-      const uint4 cur = v;
-      if (g + 1 < 8) v = __ldg(s4 + g + 1);
-      put_word(cur.x, 4);
-      put_word(cur.y, 4);
-      put_word(cur.z, 4);
-      put_word(cur.w, 4);
-    }
-  } else {
-    for (uint32_t i = 0; i < m; i += 4) {
-      const uint32_t cnt = min(4u, m - i);
-      uint32_t w = 0;
-      for (uint32_t j = 0; j < cnt; ++j) w |= (uint32_t)src[i + j] << (8 * j);
-      put_word(w, cnt);
-    }
-  }
-  *widx_out = widx;
-  *nacc_out = nacc;
-  return lo;
-}
-
-// One chunk by one warp: lane p codes piece p from bit s of the chunk into the warp's buffer
-// (layout SPREAD), then the warp copies the chunk's words out to the payload at woff (none at or
-// past `limit`).
-template <bool SPREAD>
-__device__ __forceinline__ void pack_chunk(const EncodeArgs& a, uint32_t c, const char* lut,
-                                           uint32_t lane4, uint32_t* wbuf, uint32_t s,
-                                           uint32_t mine, bool last_piece, uint32_t woff,
-                                           uint32_t words, uint32_t limit, bool whole) {
-  const uint32_t lane = lane4 >> 2;
-  uint32_t* const payload = reinterpret_cast<uint32_t*>(a.out + payload_offset(a.n));
-  uint32_t* const buf = SPREAD ? wbuf : wbuf + (woff & 3);
-  uint32_t widx = 0, nacc = 0, tail = 0;
-  const uint8_t* src = a.in + (uint64_t)c * kChunk + lane * 128;
-  if (whole) {
-    tail = pack_piece<true, SPREAD>(src, 128, lut, lane4, buf, s, &widx, &nacc);
-  } else {
-    const uint64_t first = (uint64_t)c * kChunk + lane * 128;
-    const uint32_t m = first < a.n ? (uint32_t)min((uint64_t)128, a.n - first) : 0u;
-    tail = pack_piece<false, SPREAD>(src, m, lut, lane4, buf, s, &widx, &nacc);
-  }
-  // The piece's unfinished word: the chunk's last word is stored whole (zero padding); any
-  // other is OR-ed, after a warp barrier, into the word that a later piece stored whole.
-  const bool has_tail = mine != 0 && nacc != 0;
-  const bool last = mine != 0 && last_piece;
-  tail = has_tail ? tail << (32 - nacc) : 0u;
-  uint32_t* const tail_word = buf + buf_slot<SPREAD>(widx);
-  if (has_tail && last) *tail_word = tail;
-  __syncwarp();
-  if (has_tail && !last) atomicOr(tail_word, tail);
-  __syncwarp();
-  const uint32_t end = min(woff + words, limit);
-  if (SPREAD) {
-    // word by word, each warp store 128 contiguous bytes
-    for (uint32_t i = lane; woff + i < end; i += 32) payload[woff + i] = buf[buf_slot<true>(i)];
-  } else {
-    // a ragged head and tail word by word, the 16-byte aligned middle as uint4
-    const uint32_t g0 = min((woff + 3) & ~3u, end), g1 = max(end & ~3u, g0);
-    if (woff + lane < g0) payload[woff + lane] = buf[lane];
-    if (g1 + lane < end) payload[g1 + lane] = buf[g1 - woff + lane];
-    const uint4* b4 = reinterpret_cast<const uint4*>(buf + (g0 - woff));
-    uint4* p4 = reinterpret_cast<uint4*>(payload + g0);
-    for (uint32_t q = lane; q < (g1 - g0) / 4; q += 32) p4[q] = b4[q];
-  }
-  __syncwarp();
-}
-
-__global__ void __launch_bounds__(kPackThreads, 1) k_pack(EncodeArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  PackSmem& sm = *reinterpret_cast<PackSmem*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lane4 = lane * 4;
-  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) return;  // k_measure said so
-  const uint64_t n = a.n;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  const uint32_t full_chunks = (uint32_t)(n / kChunk);
-  const uint64_t P = payload_offset(n);
-  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
-  const uint4* sync = reinterpret_cast<const uint4*>(a.out + sync_offset(n));
-  uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
-  const char* lut = reinterpret_cast<const char*>(sm.lut);
-
-  for (int i = tid; i < 256 * kPackCopies; i += kPackThreads) {
-    uint32_t code;
-    const uint32_t len = checked_code(a, i / kPackCopies, &code);
-    sm.lut[i] = (code << 20) | len;
-  }
-  for (uint32_t i = tid; i < a.mblocks; i += kPackThreads) sm.bpre[i] = a.btotal[i];
-  __syncthreads();
-  const uint32_t total = block_exclusive_scan<kPackThreads>(sm.bpre, a.mblocks, sm.red);
-  const bool fits = P + 4ull * ((uint64_t)total + 2) <= a.cap;
   if (blockIdx.x == 0 && tid == 0) {
     write_header(a);
-    reinterpret_cast<uint64_t*>(a.out)[4] = total;
-    word_off[nchunks] = total;
-    if (fits) {
-      payload[total] = 0;
-      payload[total + 1] = 0;
-    } else {
-      atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
+    if (a.n == 0) {  // no chunk writes the totals
+      reinterpret_cast<uint64_t*>(a.out)[4] = 0;
+      reinterpret_cast<uint32_t*>(a.out + 64)[0] = 0;
+      if (a.cap >= payload_offset(0) + 8) {
+        uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + payload_offset(0));
+        payload[0] = payload[1] = 0;
+      }
     }
   }
-  const uint32_t limit = fits ? total : 0u;  // no payload store at all when it does not fit
-
-  uint32_t* const wbuf = sm.out[warp];
-  const uint32_t stride = gridDim.x * (kPackThreads / 32);
-  for (uint32_t c = blockIdx.x * (kPackThreads / 32) + warp; c < nchunks; c += stride) {
-    const uint32_t woff = sm.bpre[c / a.cpb] + a.local[c];
-    if (lane == 0) word_off[c] = woff;
-    // this piece's first bit: a warp prefix sum of the piece bit counts
-    const uint32_t mine = min((uint32_t)a.pieces[(uint64_t)c * 32 + lane], kMaxPieceBits);
-    uint32_t incl = mine;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += t;
-    }
-    const uint32_t chunk_bits = __shfl_sync(0xffffffffu, incl, 31);
-    const uint32_t s = incl - mine;
-    const uint32_t words = (chunk_bits + 31) >> 5;
-    if (chunk_bits != (__ldg(reinterpret_cast<const uint32_t*>(sync + c)) & 0xffffu)) {
-      // the scratch disagrees with the index k_measure wrote: leave the chunk's words unwritten
-      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
-      continue;
-    }
-    const uint32_t peers = __popc(__match_any_sync(0xffffffffu, (s >> 5) & 31u));
-    if (__any_sync(0xffffffffu, peers >= kCrowded))
-      pack_chunk<true>(a, c, lut, lane4, wbuf, s, mine, incl == chunk_bits, woff, words, limit,
-                       c < full_chunks);
-    else
-      pack_chunk<false>(a, c, lut, lane4, wbuf, s, mine, incl == chunk_bits, woff, words, limit,
-                        c < full_chunks);
+  if (a.hist) {
+    if (complete) encode_chunks<true, true>(a, sm);
+    else encode_chunks<true, false>(a, sm);
+  } else {
+    if (complete) encode_chunks<false, true>(a, sm);
+    else encode_chunks<false, false>(a, sm);
   }
 }
 
@@ -813,8 +801,8 @@ __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut&
   const bool blocks16 = (reinterpret_cast<uintptr_t>(words) & 15) == 0;
   const int k = tid & 7;
 
-  for (uint64_t c = (uint64_t)blockIdx.x * (kDecThreads / 8) + (tid >> 3); c < nchunks;
-       c += (uint64_t)gridDim.x * (kDecThreads / 8)) {
+  for (uint64_t c = (uint64_t)blockIdx.x * (kPfxThreads / 8) + (tid >> 3); c < nchunks;
+       c += (uint64_t)gridDim.x * (kPfxThreads / 8)) {
     const uint32_t w0 = __ldg(word_off + c), w1 = __ldg(word_off + c + 1);
     const uint4 sy = __ldg(sync + c);
     auto sync_at = [&](uint32_t i) -> uint32_t {  // u16 entry i of the chunk's sync row
@@ -844,7 +832,8 @@ __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut&
         crowded = __any_sync(voters,
                              __popc(__match_any_sync(voters, fw & 31u)) >= kCrowdedReaders);
       }
-      if (VOTE && crowded && blocks16 && (uint64_t)(fw & ~3u) + kReaderReach16 <= wlimit) {
+      if (VOTE && crowded && blocks16 &&
+                 (uint64_t)(fw & ~3u) + kReaderReach16 <= wlimit) {
         SubstreamBits16 rd;
         rd.blocks = reinterpret_cast<const uint4*>(words);
         rd.start(fw, fbo);
@@ -888,11 +877,11 @@ __device__ bool crowded_chunk(const DecodeArgs& a, uint64_t c) {
   return false;
 }
 
-// KIND is checked against the stream header and the tables; the symbol loop is the same. (64
-// registers and 4 blocks per SM measured best for every kind.)
+// KIND is checked against the stream header and the tables; the symbol loop is the same. One
+// block of kPfxThreads per SM with one copy of the table: the rest of the on-chip memory serves as
+// L1 for the payload words (a block of 1024 measured 1 % faster than four of 256).
 template <int KIND>
-__global__ void __launch_bounds__(kDecThreads, 4)
-    k_decode(DecodeArgs a) {
+__global__ void __launch_bounds__(kPfxThreads, 1) k_decode(DecodeArgs a) {
   __shared__ __align__(16) uint16_t s_lut[4096];
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
@@ -902,7 +891,7 @@ __global__ void __launch_bounds__(kDecThreads, 4)
     s_total = check_header(a, &s_tables);
     // the block's first chunk stands for the rest: a block whose chunks look crowded takes the
     // voting loop (the word-by-word loop alone runs faster elsewhere)
-    s_crowded = s_total >= 0 && crowded_chunk(a, (uint64_t)blockIdx.x * (kDecThreads / 8));
+    s_crowded = s_total >= 0 && crowded_chunk(a, (uint64_t)blockIdx.x * (kPfxThreads / 8));
   }
   __syncthreads();
   const int64_t total = s_total;
@@ -913,7 +902,7 @@ __global__ void __launch_bounds__(kDecThreads, 4)
   const hx::Tables* tables = s_tables;
   const uint4* src = reinterpret_cast<const uint4*>(tables->dec);
   uint4* dst = reinterpret_cast<uint4*>(s_lut);
-  for (int i = tid; i < 4096 * 2 / 16; i += kDecThreads) dst[i] = src[i];
+  for (int i = tid; i < 4096 * 2 / 16; i += kPfxThreads) dst[i] = src[i];
   __syncthreads();
   const DecLut lut{s_lut};
   const bool crowded = s_crowded;
@@ -1306,13 +1295,14 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
 // ---------------------------------------------------------------------------------- launch
 struct DeviceInfo {
   int sms = 0;
-  int measure_per_sm = 0, pack_per_sm = 0, huff_per_sm = 0, qlc_per_sm = 0, hist_per_sm = 0;
+  int huff_per_sm = 0, qlc_per_sm = 0, hist_per_sm = 0;
   int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0, eg_per_sm = 0;
+  int enc_per_sm = 0;
 };
 
 // Sets the shared-memory carveout of `fn` to the smallest share that still holds `per_sm` blocks,
 // the rest going to L1; keeps the default if that would lower the occupancy.
-bool prefer_l1(int dev, const void* fn, int per_sm, int threads) {
+bool prefer_l1(int dev, const void* fn, int per_sm, int threads, size_t dyn_smem) {
   cudaFuncAttributes fa;
   int max_smem = 0;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
@@ -1320,12 +1310,13 @@ bool prefer_l1(int dev, const void* fn, int per_sm, int threads) {
           cudaSuccess ||
       max_smem <= 0)
     return false;
-  const long need = (long)per_sm * (long)(fa.sharedSizeBytes + 1024);  // + the per-block reserve
+  // + the per-block reserve
+  const long need = (long)per_sm * (long)(fa.sharedSizeBytes + dyn_smem + 1024);
   const int pct = (int)std::min<long>(100, (need * 100 + max_smem - 1) / max_smem + 1);
   if (cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, pct) != cudaSuccess)
     return false;
   int now = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&now, fn, threads, 0) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&now, fn, threads, dyn_smem) != cudaSuccess)
     return false;
   if (now < per_sm)
     return cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -1345,20 +1336,10 @@ bool device_info(DeviceInfo* out) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return false;
-    if (cudaFuncSetAttribute(k_measure, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(MeasureSmem)) != cudaSuccess ||
-        cudaFuncSetAttribute(k_pack, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(PackSmem)) != cudaSuccess)
-      return false;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.measure_per_sm, k_measure,
-                                                      kMeasureThreads,
-                                                      sizeof(MeasureSmem)) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.pack_per_sm, k_pack, kPackThreads,
-                                                      sizeof(PackSmem)) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.huff_per_sm, k_decode<HX_KIND_HUFFMAN>,
-                                                      kDecThreads, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.huff_per_sm, k_decode<HX_KIND_HUFFMAN>,
+                                                      kPfxThreads, 0) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qlc_per_sm, k_decode<HX_KIND_QLC>,
-                                                      kDecThreads, 0) != cudaSuccess ||
+                                                      kPfxThreads, 0) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
                                                       0) != cudaSuccess ||
         cudaFuncSetAttribute(k_sh_measure, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1373,20 +1354,25 @@ bool device_info(DeviceInfo* out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_decode_per_sm, k_sh_decode,
                                                       kDecThreads, 0) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.eg_per_sm, k_decode<HX_KIND_EXPGOLOMB>,
-                                                      kDecThreads, 0) != cudaSuccess)
+                                                      kPfxThreads, 0) != cudaSuccess)
+      return false;
+    if (cudaFuncSetAttribute(k_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(EncSmem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.enc_per_sm, k_encode, kEncThreads,
+                                                      sizeof(EncSmem)) != cudaSuccess ||
+        d.enc_per_sm < 1)
       return false;
     if (d.sh_measure_per_sm < 1 || d.sh_pack_per_sm < 1 || d.sh_decode_per_sm < 1) return false;
-    if (d.measure_per_sm < 1 || d.pack_per_sm < 1 || d.huff_per_sm < 1 || d.qlc_per_sm < 1 ||
-        d.hist_per_sm < 1)
+    if (d.huff_per_sm < 1 || d.qlc_per_sm < 1 || d.eg_per_sm < 1 || d.hist_per_sm < 1)
       return false;
-    // The decoder's payload reads hit L1 about half the time: give L1 all the on-chip memory
-    // that the resident decode blocks do not need for their tables.
+    // The decoders' payload reads hit L1 most of the time: give L1 all the on-chip memory that
+    // the resident decode blocks do not need for their tables.
     if (!prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_HUFFMAN>), d.huff_per_sm,
-                   kDecThreads) ||
+                   kPfxThreads, 0) ||
         !prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_QLC>), d.qlc_per_sm,
-                   kDecThreads) ||
+                   kPfxThreads, 0) ||
         !prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_EXPGOLOMB>), d.eg_per_sm,
-                   kDecThreads))
+                   kPfxThreads, 0))
       return false;
     d.sms = sms;
   }
@@ -1398,8 +1384,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 int launched() { return cudaGetLastError() == cudaSuccess ? HX_OK : HX_ERR_CUDA; }
 
-// Checks the arguments and fills the kernel arguments of one encode (both passes compute the same
-// from the same call arguments). Returns HX_OK or a host error.
+// Checks the arguments and fills the kernel arguments of one encode. Returns HX_OK or a host
+// error.
 int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
                 uint64_t out_cap, void* d_scratch, uint32_t* d_hist, uint32_t* d_status,
                 EncodeArgs* a, DeviceInfo* info) {
@@ -1412,61 +1398,67 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
     return HX_ERR_ARG;
   if (!device_info(info)) return HX_ERR_CUDA;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  // measure blocks: at least one wave of resident blocks of the kind's measure kernel, at most
+  // the Shannonic coder's measure blocks: at least one wave of resident blocks, at most
   // kMaxChunksPerBlock chunks each (n < 2^32 gives at most 2^20 chunks, so 256 blocks always
   // suffice)
-  const int per_sm = kind == HX_KIND_SHANNONIC ? info->sh_measure_per_sm : info->measure_per_sm;
+  const int per_sm = info->sh_measure_per_sm;
   uint32_t mblocks = (uint32_t)std::min<uint64_t>(
       {(uint64_t)nchunks, (uint64_t)kMaxMeasureBlocks,
        std::max<uint64_t>((uint64_t)info->sms * per_sm,
                           (nchunks + kMaxChunksPerBlock - 1) / kMaxChunksPerBlock)});
   const uint32_t cpb = mblocks ? (nchunks + mblocks - 1) / mblocks : 1;
   if (mblocks) mblocks = (nchunks + cpb - 1) / cpb;  // no block without chunks
-  // scratch: u32 local[nchunks], u32 btotal[mblocks] (mblocks <= nchunks), u16 pieces[32 nchunks]
+  // scratch (hx_scratch_bytes): Shannonic u32 local[nchunks], u32 btotal[mblocks] (mblocks <=
+  // nchunks); or the single pass's u64 look[nchunks] and u32 counter
   auto* local = static_cast<uint32_t*>(d_scratch);
-  auto* pieces = reinterpret_cast<uint16_t*>(local + 2 * (uint64_t)nchunks);
   *a = EncodeArgs{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
-                  out_cap, local, local + nchunks, pieces, mblocks, cpb, d_hist, d_status, kind};
+                  out_cap, local, local + nchunks, mblocks, cpb, d_hist, d_status, kind,
+                  // the single pass: u64 look[nchunks], then the u32 chunk counter
+                  static_cast<uint64_t*>(d_scratch),
+                  reinterpret_cast<uint32_t*>(static_cast<uint64_t*>(d_scratch) + nchunks),
+                  kDefaultWaitNs, ~0ull};
   return HX_OK;
 }
 
-int launch_measure(const EncodeArgs& a, cudaStream_t s) {
-  if (a.mblocks) {
-    if (a.kind == HX_KIND_SHANNONIC)
-      k_sh_measure<<<a.mblocks, kShThreads, sizeof(ShMeasureSmem), s>>>(a);
-    else
-      k_measure<<<a.mblocks, kMeasureThreads, sizeof(MeasureSmem), s>>>(a);
-  }
+// The single-pass encode: zero the look-back words and the counter, then one block per SM.
+int launch_encode(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
+  const uint64_t nchunks = n_chunks_of(a.n);
+  if (cudaMemsetAsync(a.look, 0, 8 * nchunks + 4, s) != cudaSuccess) return HX_ERR_CUDA;
+  const uint32_t grid = (uint32_t)std::max<uint64_t>(
+      1, std::min<uint64_t>((nchunks + kEncWarps - 1) / kEncWarps,
+                            (uint64_t)info.sms * info.enc_per_sm));
+  k_encode<<<grid, kEncThreads, sizeof(EncSmem), s>>>(a);
   return launched();
 }
 
-int launch_pack(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
+// The Shannonic coder's two passes (tANS runs backwards, so a sub-stream's length is known only
+// once it has been run): measure, then pack.
+int launch_shannonic(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
+  if (a.mblocks) k_sh_measure<<<a.mblocks, kShThreads, sizeof(ShMeasureSmem), s>>>(a);
+  if (launched()) return HX_ERR_CUDA;
   const uint32_t nchunks = (uint32_t)n_chunks_of(a.n);
-  if (a.kind == HX_KIND_SHANNONIC) {  // 32 chunks per block and round
-    const uint32_t grid = (uint32_t)std::max<uint64_t>(
-        1, std::min<uint64_t>((nchunks + 31) / 32, (uint64_t)info.sms * info.sh_pack_per_sm));
-    k_sh_pack<<<grid, kShThreads, sizeof(ShPackSmem), s>>>(a);
-    return launched();
-  }
-  const uint32_t grid = (uint32_t)std::max<uint64_t>(
-      1, std::min<uint64_t>((nchunks + kPackThreads / 32 - 1) / (kPackThreads / 32),
-                            (uint64_t)info.sms * info.pack_per_sm));
-  k_pack<<<grid, kPackThreads, sizeof(PackSmem), s>>>(a);
+  const uint32_t grid = (uint32_t)std::max<uint64_t>(  // 32 chunks per block and round
+      1, std::min<uint64_t>((nchunks + 31) / 32, (uint64_t)info.sms * info.sh_pack_per_sm));
+  k_sh_pack<<<grid, kShThreads, sizeof(ShPackSmem), s>>>(a);
   return launched();
 }
 
 int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                   void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
-                  uint32_t* d_status, void* stream) {
+                  uint32_t* d_status, void* stream, uint64_t wait_ns = kDefaultWaitNs,
+                  uint64_t withhold = ~0ull) {
   EncodeArgs a;
   DeviceInfo info;
   const int rc = encode_args(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
                              &a, &info);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int m = launch_measure(a, s);
-  if (m) return m;
-  return launch_pack(a, info, s);
+  if (kind != HX_KIND_SHANNONIC) {
+    a.wait_ns = wait_ns;
+    a.withhold = withhold;
+    return launch_encode(a, info, s);
+  }
+  return launch_shannonic(a, info, s);
 }
 
 int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const void* d_stream,
@@ -1482,7 +1474,7 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   if (!device_info(&info)) return HX_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint64_t nchunks = n_chunks_of(n);
-  const uint64_t per_block = kDecThreads / 8;
+  const uint64_t per_block = (kind == HX_KIND_SHANNONIC ? kDecThreads : kPfxThreads) / 8;
   const int per_sm = kind == HX_KIND_HUFFMAN ? info.huff_per_sm
                      : kind == HX_KIND_QLC   ? info.qlc_per_sm
                      : kind == HX_KIND_EXPGOLOMB ? info.eg_per_sm
@@ -1500,11 +1492,11 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   a.status = d_status;
   a.kind = kind;
   if (kind == HX_KIND_HUFFMAN)
-    k_decode<HX_KIND_HUFFMAN><<<grid, kDecThreads, 0, s>>>(a);
+    k_decode<HX_KIND_HUFFMAN><<<grid, kPfxThreads, 0, s>>>(a);
   else if (kind == HX_KIND_QLC)
-    k_decode<HX_KIND_QLC><<<grid, kDecThreads, 0, s>>>(a);
+    k_decode<HX_KIND_QLC><<<grid, kPfxThreads, 0, s>>>(a);
   else if (kind == HX_KIND_EXPGOLOMB)
-    k_decode<HX_KIND_EXPGOLOMB><<<grid, kDecThreads, 0, s>>>(a);
+    k_decode<HX_KIND_EXPGOLOMB><<<grid, kPfxThreads, 0, s>>>(a);
   else
     k_sh_decode<<<grid, kDecThreads, 0, s>>>(a);
   return launched();
@@ -1512,12 +1504,12 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
 
 }  // namespace
 
-// Scratch of hx_encode_noalloc: hx_scratch_bytes(HX_NOALLOC_MAX_BYTES) bytes (per chunk a
-// block-local word offset and 32 piece bit counts; the measure blocks' totals). Host code must not pass this name to a kernel
-// (on the host it is only a stand-in); its device address comes from cudaGetSymbolAddress, once
-// per device.
-static __device__ __align__(256) unsigned char
-    g_noalloc_scratch[72 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16];
+// Scratch of hx_encode_noalloc: the single-pass encoder's look-back words (8 bytes per chunk)
+// and its chunk counter, for HX_NOALLOC_MAX_BYTES of input. Host code must not pass this name to
+// a kernel (on the host it is only a stand-in); its device address comes from
+// cudaGetSymbolAddress, once per device.
+constexpr uint64_t kNoallocScratch = 8 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratch];
 
 namespace {
 std::mutex g_noalloc_mutex;
@@ -1526,18 +1518,19 @@ void* g_noalloc_ptr[64];  // device address of g_noalloc_scratch, per device
 
 extern "C" {
 
-uint64_t hx_scratch_bytes(uint64_t n) { return 72 * n_chunks_of(n) + 16; }
+uint64_t hx_scratch_bytes(uint64_t n) { return 8 * n_chunks_of(n) + 16; }
 
 // For callers that cannot allocate device memory at encode time (a framework's caching
 // allocator owns the device memory, or a path that cannot take cudaMalloc's implicit
 // synchronisation): hx_encode with Huffman tables, its scratch in g_noalloc_scratch. The first
-// call on a device fetches that array's address with the device current; every call writes each
-// scratch word before reading it, and calls that overlap on the GPU race on the shared array.
+// call on a device fetches that array's address with the device current; every call clears the
+// words it uses there first (a cudaMemsetAsync, which allocates nothing), and calls that overlap
+// on the GPU race on the shared array.
 int hx_encode_noalloc(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d_out,
                       uint64_t out_cap, uint32_t* d_hist, uint32_t* d_status, void* stream) {
   if (n > HX_NOALLOC_MAX_BYTES) return HX_ERR_ARG;
-  static_assert(sizeof(g_noalloc_scratch) >= 72 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 16,
-                "scratch array smaller than hx_scratch_bytes(HX_NOALLOC_MAX_BYTES)");
+  static_assert(sizeof(g_noalloc_scratch) >= 8 * (HX_NOALLOC_MAX_BYTES / HX_CHUNK) + 4,
+                "scratch array smaller than the look-back words and counter of the limit");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HX_ERR_CUDA;
   void* scratch = nullptr;
@@ -1591,24 +1584,12 @@ int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d
                        d_status, stream);
 }
 
-int hx_encode_measure(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
+int hx_encode_bounded(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                       void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
-                      uint32_t* d_status, void* stream) {
-  EncodeArgs a;
-  DeviceInfo info;
-  const int rc = encode_args(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
-                             &a, &info);
-  return rc ? rc : launch_measure(a, static_cast<cudaStream_t>(stream));
-}
-
-int hx_encode_pack(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
-                   void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_status,
-                   void* stream) {
-  EncodeArgs a;
-  DeviceInfo info;
-  const int rc = encode_args(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, nullptr,
-                             d_status, &a, &info);
-  return rc ? rc : launch_pack(a, info, static_cast<cudaStream_t>(stream));
+                      uint32_t* d_status, uint64_t wait_ns, uint64_t withhold, void* stream) {
+  if (kind == HX_KIND_SHANNONIC) return HX_ERR_ARG;
+  return encode_common(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
+                       stream, wait_ns, withhold);
 }
 
 int hx_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,

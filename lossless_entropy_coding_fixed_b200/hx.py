@@ -76,6 +76,7 @@ def lib():
             "hx_qlc_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
             "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_encode_noalloc": (i32, [P, P, u64, P, u64, P, P, P]),
+            "hx_encode_bounded": (i32, [u32, P, P, u64, P, u64, P, P, P, u64, u64, P]),
             "hx_shannonic_build": (i32, [P, i32, u32, CB]),
             "hx_expgolomb_build": (i32, [i32, i32, CB]),
             "hx_expgolomb_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
@@ -83,7 +84,6 @@ def lib():
             "hx_shannonic_encode_bound": (u64, [u64]),
             "hx_shannonic_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
             "hx_shannonic_decode": (i32, [P, P, u64, P, u64, P, P]),
-            "hx_encode_measure": (i32, [u32, P, P, u64, P, u64, P, P, P, P]),
             "hx_decode_set": (i32, [u32, P, u32, P, u64, P, u64, P, P]),
             "hx_planner_create": (i32, [ctypes.POINTER(_SessionConfig), P, P]),
             "hx_planner_codebook": (i32, [P, u64, CB]),
@@ -95,7 +95,6 @@ def lib():
             "hx_session_drain": (i32, [P]),
             "hx_session_batch_info": (i32, [P, u64, ctypes.POINTER(_BatchInfo)]),
             "hx_session_destroy": (None, [P]),
-            "hx_encode_pack": (i32, [u32, P, P, u64, P, u64, P, P, P]),
             "hx_entropy": (ctypes.c_double, [P]),
             "hx_mean_length": (ctypes.c_double, [P, CB]),
             "hx_version": (i32, []),
@@ -314,25 +313,19 @@ def encode(tables, x, out=None, scratch=None, hist=None, status=None, kind: int 
     return out, status
 
 
-def encode_passes(tables, x, out, scratch, hist=None, status=None, kind: int = KIND_HUFFMAN,
-                  between=None):
-    """The same encode as encode(), as its two calls: hx_encode_measure, then hx_encode_pack.
-    `between`, if given, is called (host side) after the first is enqueued -- e.g. to record an
-    event. Returns (out, status)."""
+def encode_bounded(tables, x, out, scratch, wait_ns: int, withhold: int = (1 << 64) - 1,
+                   hist=None, status=None, kind: int = KIND_HUFFMAN):
+    """hx_encode_bounded: encode() with the chunks' wait limit in nanoseconds and, for failure
+    tests, one chunk (`withhold`) that never publishes its word count. Returns (out, status)."""
     x = _dev_u8(x, "x")
     out = _dev_u8(out, "out")
     if status is None:
         status = new_status(x.device)
-    n, s = x.numel(), _stream(x)
-    _check(lib().hx_encode_measure(kind, tables.data_ptr(), x.data_ptr(), n, out.data_ptr(),
-                                   out.numel(), scratch.data_ptr(),
+    _check(lib().hx_encode_bounded(kind, tables.data_ptr(), x.data_ptr(), x.numel(),
+                                   out.data_ptr(), out.numel(), scratch.data_ptr(),
                                    hist.data_ptr() if hist is not None else None,
-                                   status.data_ptr(), s), "hx_encode_measure")
-    if between is not None:
-        between()
-    _check(lib().hx_encode_pack(kind, tables.data_ptr(), x.data_ptr(), n, out.data_ptr(),
-                                out.numel(), scratch.data_ptr(), status.data_ptr(), s),
-           "hx_encode_pack")
+                                   status.data_ptr(), int(wait_ns), int(withhold), _stream(x)),
+           "hx_encode_bounded")
     return out, status
 
 

@@ -60,8 +60,27 @@ def test_reference_arm_runs_oracle_on_rank0_only():
         assert bench.cpu_reference(args, rank=0, ws=1) == 0
     line = json.loads(buf.getvalue().strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["cores"] == (os.cpu_count() or 1)
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["higher_is_better"] is True
+
+
+def test_oracle_slices_are_chunk_aligned_and_cover_the_input():
+    import numpy as np
+    x = np.arange(5 * 4096 + 77, dtype=np.uint64).astype(np.uint8)
+    for threads in (1, 2, 3, 8, 64):
+        sl = bench._oracle_slices(x, threads)
+        assert len(sl) <= threads and all(s.size % 4096 == 0 for s in sl[:-1])
+        assert (np.concatenate(sl) == x).all()
+
+
+def test_roofline_entry_arithmetic():
+    r = bench.roofline_entry("k", [(2e9, 1.0), (1e9, 0.5)], 6000.0, "measured")
+    assert r["algorithmic_bytes_per_launch"] == 1.5e9 and r["ms_per_launch"] == 0.75
+    assert r["achieved"] == pytest.approx(1.5e9 / 0.75e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6000.0)
+    assert r["frac_spec"] == pytest.approx(r["achieved"] / bench.SPEC_HBM_GBS)
+    assert r["launches_per_step"] == 2
 
 
 def test_code_only_ignores_comments_and_layout():

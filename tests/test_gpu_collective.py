@@ -46,7 +46,15 @@ def _rank(port, q):
                 torch.cuda.synchronize()
                 ref = sum(int(oracle.encode(ocb, x[lo:hi])[1].size)
                           for lo, hi in collective.part_bounds(x.size, parts))
-                res[(kind, parts)] = (bool((out.cpu().numpy() == x).all()), sizes, ref)
+                # the stream bytes themselves: kept coded, the parts merge into the oracle's
+                # stream of the whole shard
+                xs = x[:(x.size // 4096) * 4096]
+                st, _ = collective.compressed_all_gather(
+                    torch.from_numpy(xs).cuda(), cb.upload("cuda"), codec=collective.Codec(kind),
+                    parts=parts, decode=False)
+                torch.cuda.synchronize()
+                same = bool(np.array_equal(st.cpu().numpy(), oracle.encode(ocb, xs)[1]))
+                res[(kind, parts)] = (bool((out.cpu().numpy() == x).all()), sizes, ref, same)
         q.put(res)
     finally:
         dist.destroy_process_group()
@@ -64,5 +72,5 @@ def test_one_rank_round_trip():
     p.join(120)
     assert p.exitcode == 0
     assert len(res) == 4
-    for case, (ok, sizes, ref_size) in res.items():
-        assert ok and sizes == [ref_size], case
+    for case, (ok, sizes, ref_size, same_stream) in res.items():
+        assert ok and sizes == [ref_size] and same_stream, case

@@ -59,15 +59,17 @@ def check_workload(orc, x, counts, kind):
     return bits / x.size
 
 
-def test_cfg2_ffn_mix_256mib(orc):
+@pytest.mark.parametrize("kind", ["huffman", "qlc"])
+def test_cfg2_ffn_mix_256mib(orc, kind):
     x = datagen.data(2)
-    check_workload(orc, x, prior_counts(orc, 2), "huffman")
+    check_workload(orc, x, prior_counts(orc, 2), kind)
 
 
-def test_cfg3_int8_per_tensor_64mib(orc):
+@pytest.mark.parametrize("kind", ["huffman", "qlc"])
+def test_cfg3_int8_per_tensor_64mib(orc, kind):
     x = datagen.data(3)
     counts = orc.histogram(x)
-    check_workload(orc, x, counts, "huffman")
+    check_workload(orc, x, counts, kind)
 
 
 @pytest.mark.parametrize("kind", ["huffman", "qlc"])
@@ -83,8 +85,12 @@ def test_cfg4_e4m3_1gib(orc, kind):
 
 @pytest.mark.parametrize("layer", range(16))
 def test_cfg5_layer_shards(orc, layer):
-    shard = 4 * layer + layer % 4
-    x = datagen.data(5, shard=shard)
-    bps = check_workload(orc, x, prior_counts(orc, 5, layer), "huffman")
+    """Every layer (so every dtype and law of the batch): one shard with its layer's Huffman
+    codebook, another with its layer's QLC (32 of the 64 shards)."""
+    counts = prior_counts(orc, 5, layer)
+    x = datagen.data(5, shard=4 * layer + layer % 4)
+    bps = check_workload(orc, x, counts, "huffman")
     h = orc.histogram(x)
     assert bps >= orc.mean_length(h, orc.huffman_lengths(h, cover_all=False)) >= orc.entropy(h)
+    x = datagen.data(5, shard=4 * layer + (layer + 2) % 4)
+    check_workload(orc, x, counts, "qlc")

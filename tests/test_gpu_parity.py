@@ -193,24 +193,6 @@ def test_wrong_kind_tables(books):
     assert st == hx.HX_ERR_ARG
 
 
-@pytest.mark.parametrize("kind", ["huffman", "qlc"])
-@pytest.mark.parametrize("n", [4096 * 5 + 777, (1 << 20) - 5])
-def test_encode_passes_equal_oracle(orc, books, kind, n):
-    """hx_encode_measure then hx_encode_pack (timed apart by bench.py) write the oracle's stream."""
-    cb, tables, ocb, k = books[kind]
-    x = datagen.data(1, n=n)
-    ost, ref = orc.encode(ocb, x)
-    xd = dev(x)
-    out = torch.empty(hx.encode_bound(n), dtype=torch.uint8, device="cuda")
-    scratch = torch.empty(hx.scratch_bytes(n), dtype=torch.uint8, device="cuda")
-    hist = torch.zeros(256, dtype=torch.int32, device="cuda")
-    out, st = hx.encode_passes(tables, xd, out, scratch, hist=hist, kind=k)
-    torch.cuda.synchronize()
-    assert int(st.item()) == ost == 0
-    assert (out[:ref.size].cpu().numpy() == ref).all()
-    assert (hist.cpu().numpy().astype(np.uint64) == orc.histogram(x)).all()
-
-
 def test_deterministic_repeat(books):
     cb, tables, ocb, k = books["huffman"]
     x = datagen.data(4, n=(1 << 23) + 12345)

@@ -63,6 +63,28 @@ def test_noalloc_equals_encode_twice(setup, n):
         assert torch.equal(hist, hist_ref)
 
 
+@pytest.mark.parametrize("n", [128 << 20, (100 << 20) + 4095])
+def test_noalloc_equals_oracle_at_the_limit(setup, n):
+    """The largest input the library's array is sized for (HX_NOALLOC_MAX_BYTES exactly), and a
+    ragged size: the stream equals the oracle's byte for byte."""
+    import oracle
+    dev, tables = setup
+    assert n <= hx.NOALLOC_MAX_BYTES
+    counts = sum(oracle.histogram(b) for b in datagen.prior_batches(1))
+    xh = datagen.data(4, n=n)
+    x = torch.from_numpy(xh).to(dev)
+    out = torch.full((hx.encode_bound(n),), 0xA5, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    hist = torch.zeros(256, dtype=torch.int32, device=dev)
+    assert _raw_noalloc(tables, x, out, hist, status) == 0
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref = oracle.encode(oracle.huffman_codebook(counts), xh)[1]
+    assert hx.stream_size(out, n) == ref.size
+    assert (out[:ref.size].cpu().numpy() == ref).all()
+    assert (hist.cpu().numpy().astype(np.uint64) == oracle.histogram(xh)).all()
+
+
 def test_noalloc_refuses_oversize(setup):
     dev, tables = setup
     n = (128 << 20) + 1
