@@ -831,6 +831,22 @@ def main():
     # the dominant kernel: the largest share of the step
     kernel_name = max(roof, key=lambda k: roof[k]["ms_per_launch"] * roof[k]["launches_per_step"])
 
+    # the histogram on its own (the frequency analysis that defines the next codebook), over the
+    # same batch: device time per call, inputs resident
+    hc = torch.zeros(256, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        hx.histogram(x, hc)
+    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_.record(stream)
+    for _ in range(10):
+        hx.histogram(x, hc)
+    b_.record(stream)
+    torch.cuda.synchronize(dev)
+    hist_ms = a_.elapsed_time(b_) / 10
+    assert (hc.cpu().numpy().astype(np.uint64) == h * 13).all()
+    histogram = {"ms": hist_ms, "GB_per_s": n / (hist_ms * 1e-3) / 1e9,
+                 "hbm_frac": n / (hist_ms * 1e-3) / 1e9 / peak}
+
     e2e = None
     if not args.no_e2e:
         e2e = e2e_leg(args, dev, hx, torch, pg, ws, x_host, ht, qt, n, bound, scratch, status)
@@ -892,6 +908,7 @@ def main():
             "host_codebook_build_us": {"huffman": (t1 - t0) * 1e6, "qlc": (t2 - t1) * 1e6},
             "roofline": main_roof,
             "roofline_kernels": {k: dict(v, traffic=recorded_traffic(k)) for k, v in roof.items()},
+            "histogram": histogram,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "configs": configs,

@@ -46,7 +46,6 @@ constexpr uint32_t kMagic = 0x31305848u;  // "HX01"
 constexpr uint32_t kChunk = HX_CHUNK;
 constexpr uint32_t kSubLen = HX_CHUNK / HX_SUBSTREAMS;
 constexpr int kDecThreads = 256;  // Shannonic decode: 8 threads per chunk, 32 chunks per block
-constexpr int kPfxThreads = 1024;  // prefix-code decode: 8 threads per chunk, 128 chunks per block
 constexpr int kHistThreads = 256;
 
 __host__ __device__ inline uint64_t n_chunks_of(uint64_t n) { return (n + kChunk - 1) / kChunk; }
@@ -58,34 +57,39 @@ __host__ __device__ inline uint64_t payload_offset(uint64_t n) {
 }
 
 // ---------------------------------------------------------------------------------- histogram
-static_assert(kHistThreads == 256, "k_histogram sums bin `tid` of every warp's table");
+// One table of 32 copies per block: bin v of copy l at word 32 v + l, lane l counting into copy l,
+// so the 32 increments of a warp never share a bank; the copies are summed into the caller's
+// counts at the end (one global atomic per non-empty bin and block).
+static_assert(kHistThreads == 256, "k_histogram sums bin `tid` over the copies");
 __global__ void __launch_bounds__(kHistThreads) k_histogram(const uint8_t* __restrict__ in,
                                                             uint64_t n, uint32_t* counts) {
-  __shared__ uint32_t bins[kHistThreads / 32][256];
-  const int tid = threadIdx.x, warp = tid >> 5;
-  for (int i = tid; i < (kHistThreads / 32) * 256; i += kHistThreads) (&bins[0][0])[i] = 0;
+  __shared__ uint32_t bins[256 * 32];
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i < 256 * 32; i += kHistThreads) bins[i] = 0;
   __syncthreads();
-  uint32_t* mine = bins[warp];
+  const uint32_t base = (uint32_t)__cvta_generic_to_shared(bins) + 4 * lane;
+  auto count4 = [&](uint32_t w) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t a = __byte_perm(w, 0u, 0x4440u + j) * 128u + base;
+      asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(a) : "memory");
+    }
+  };
   const uint64_t nvec = n / 16;
   const uint4* v = reinterpret_cast<const uint4*>(in);
   for (uint64_t i = blockIdx.x * (uint64_t)kHistThreads + tid; i < nvec;
        i += (uint64_t)gridDim.x * kHistThreads) {
     const uint4 x = __ldcs(v + i);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      atomicAdd(&mine[w[j] & 0xff], 1u);
-      atomicAdd(&mine[(w[j] >> 8) & 0xff], 1u);
-      atomicAdd(&mine[(w[j] >> 16) & 0xff], 1u);
-      atomicAdd(&mine[w[j] >> 24], 1u);
-    }
+    count4(x.x);
+    count4(x.y);
+    count4(x.z);
+    count4(x.w);
   }
   if (blockIdx.x == 0)
-    for (uint64_t i = nvec * 16 + tid; i < n; i += kHistThreads) atomicAdd(&mine[in[i]], 1u);
+    for (uint64_t i = nvec * 16 + tid; i < n; i += kHistThreads) atomicAdd(&bins[in[i] * 32 + lane], 1u);
   __syncthreads();
   uint32_t sum = 0;
-#pragma unroll
-  for (int w = 0; w < kHistThreads / 32; ++w) sum += bins[w][tid];
+  for (int l = 0; l < 32; ++l) sum += bins[tid * 32 + ((l + tid) & 31)];
   if (sum) atomicAdd(&counts[tid], sum);
 }
 
@@ -785,7 +789,7 @@ __device__ __forceinline__ uint64_t decode_substream(Reader& rd, uint32_t mine, 
 // The block's chunks in a grid-stride loop, 8 lanes per chunk (one per sub-stream). COMPLETE:
 // every window starts a code word, so no entry is checked. VOTE: the block's first chunk looked
 // crowded (crowded_chunk), so the lanes about to decode vote on the 16-byte reader.
-template <bool COMPLETE, bool VOTE>
+template <int THREADS, bool COMPLETE, bool VOTE>
 __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut& lut,
                                               uint32_t total) {
   const int tid = threadIdx.x;
@@ -801,8 +805,8 @@ __device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut&
   const bool blocks16 = (reinterpret_cast<uintptr_t>(words) & 15) == 0;
   const int k = tid & 7;
 
-  for (uint64_t c = (uint64_t)blockIdx.x * (kPfxThreads / 8) + (tid >> 3); c < nchunks;
-       c += (uint64_t)gridDim.x * (kPfxThreads / 8)) {
+  for (uint64_t c = (uint64_t)blockIdx.x * (THREADS / 8) + (tid >> 3); c < nchunks;
+       c += (uint64_t)gridDim.x * (THREADS / 8)) {
     const uint32_t w0 = __ldg(word_off + c), w1 = __ldg(word_off + c + 1);
     const uint4 sy = __ldg(sync + c);
     auto sync_at = [&](uint32_t i) -> uint32_t {  // u16 entry i of the chunk's sync row
@@ -877,11 +881,12 @@ __device__ bool crowded_chunk(const DecodeArgs& a, uint64_t c) {
   return false;
 }
 
-// KIND is checked against the stream header and the tables; the symbol loop is the same. One
-// block of kPfxThreads per SM with one copy of the table: the rest of the on-chip memory serves as
-// L1 for the payload words (a block of 1024 measured 1 % faster than four of 256).
-template <int KIND>
-__global__ void __launch_bounds__(kPfxThreads, 1) k_decode(DecodeArgs a) {
+// KIND is checked against the stream header and the tables; the symbol loop is the same. THREADS:
+// one block of 1024 per SM for large inputs, with one copy of the table, the rest of the on-chip
+// memory serving as L1 for the payload words; smaller blocks spread smaller inputs over more SMs
+// (decode_common picks).
+template <int KIND, int THREADS>
+__global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a) {
   __shared__ __align__(16) uint16_t s_lut[4096];
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
@@ -891,7 +896,7 @@ __global__ void __launch_bounds__(kPfxThreads, 1) k_decode(DecodeArgs a) {
     s_total = check_header(a, &s_tables);
     // the block's first chunk stands for the rest: a block whose chunks look crowded takes the
     // voting loop (the word-by-word loop alone runs faster elsewhere)
-    s_crowded = s_total >= 0 && crowded_chunk(a, (uint64_t)blockIdx.x * (kPfxThreads / 8));
+    s_crowded = s_total >= 0 && crowded_chunk(a, (uint64_t)blockIdx.x * (THREADS / 8));
   }
   __syncthreads();
   const int64_t total = s_total;
@@ -902,16 +907,16 @@ __global__ void __launch_bounds__(kPfxThreads, 1) k_decode(DecodeArgs a) {
   const hx::Tables* tables = s_tables;
   const uint4* src = reinterpret_cast<const uint4*>(tables->dec);
   uint4* dst = reinterpret_cast<uint4*>(s_lut);
-  for (int i = tid; i < 4096 * 2 / 16; i += kPfxThreads) dst[i] = src[i];
+  for (int i = tid; i < 4096 * 2 / 16; i += THREADS) dst[i] = src[i];
   __syncthreads();
   const DecLut lut{s_lut};
   const bool crowded = s_crowded;
   if (tables->complete) {
-    if (crowded) decode_chunks<true, true>(a, lut, (uint32_t)total);
-    else decode_chunks<true, false>(a, lut, (uint32_t)total);
+    if (crowded) decode_chunks<THREADS, true, true>(a, lut, (uint32_t)total);
+    else decode_chunks<THREADS, true, false>(a, lut, (uint32_t)total);
   } else {
-    if (crowded) decode_chunks<false, true>(a, lut, (uint32_t)total);
-    else decode_chunks<false, false>(a, lut, (uint32_t)total);
+    if (crowded) decode_chunks<THREADS, false, true>(a, lut, (uint32_t)total);
+    else decode_chunks<THREADS, false, false>(a, lut, (uint32_t)total);
   }
 }
 
@@ -1293,10 +1298,24 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------------- launch
+// The prefix-code decoder's block sizes, and the kernel of a kind at size index i.
+constexpr int kDecodeBlock[3] = {1024, 256, 64};
+using DecodeKernel = void (*)(DecodeArgs);
+template <int KIND>
+DecodeKernel prefix_decoder_of(int i) {
+  return i == 0 ? k_decode<KIND, 1024> : i == 1 ? k_decode<KIND, 256> : k_decode<KIND, 64>;
+}
+DecodeKernel prefix_decoder(uint32_t kind, int i) {
+  return kind == HX_KIND_HUFFMAN ? prefix_decoder_of<HX_KIND_HUFFMAN>(i)
+         : kind == HX_KIND_QLC   ? prefix_decoder_of<HX_KIND_QLC>(i)
+                                 : prefix_decoder_of<HX_KIND_EXPGOLOMB>(i);
+}
+
 struct DeviceInfo {
   int sms = 0;
-  int huff_per_sm = 0, qlc_per_sm = 0, hist_per_sm = 0;
-  int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0, eg_per_sm = 0;
+  int hist_per_sm = 0;
+  int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0;
+  int dec_per_sm[3] = {0, 0, 0};  // prefix-code decode blocks per SM at 1024, 256, 64 threads
   int enc_per_sm = 0;
 };
 
@@ -1336,10 +1355,13 @@ bool device_info(DeviceInfo* out) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return false;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.huff_per_sm, k_decode<HX_KIND_HUFFMAN>,
-                                                      kPfxThreads, 0) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.qlc_per_sm, k_decode<HX_KIND_QLC>,
-                                                      kPfxThreads, 0) != cudaSuccess ||
+    for (int i = 0; i < 3; ++i)
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+              &d.dec_per_sm[i], reinterpret_cast<const void*>(prefix_decoder(HX_KIND_HUFFMAN, i)),
+              kDecodeBlock[i], 0) != cudaSuccess ||
+          d.dec_per_sm[i] < 1)
+        return false;
+    if (
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
                                                       0) != cudaSuccess ||
         cudaFuncSetAttribute(k_sh_measure, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1352,9 +1374,7 @@ bool device_info(DeviceInfo* out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_pack_per_sm, k_sh_pack, kShThreads,
                                                       sizeof(ShPackSmem)) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_decode_per_sm, k_sh_decode,
-                                                      kDecThreads, 0) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.eg_per_sm, k_decode<HX_KIND_EXPGOLOMB>,
-                                                      kPfxThreads, 0) != cudaSuccess)
+                                                      kDecThreads, 0) != cudaSuccess)
       return false;
     if (cudaFuncSetAttribute(k_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sizeof(EncSmem)) != cudaSuccess ||
@@ -1363,17 +1383,15 @@ bool device_info(DeviceInfo* out) {
         d.enc_per_sm < 1)
       return false;
     if (d.sh_measure_per_sm < 1 || d.sh_pack_per_sm < 1 || d.sh_decode_per_sm < 1) return false;
-    if (d.huff_per_sm < 1 || d.qlc_per_sm < 1 || d.eg_per_sm < 1 || d.hist_per_sm < 1)
+    if (d.hist_per_sm < 1)
       return false;
     // The decoders' payload reads hit L1 most of the time: give L1 all the on-chip memory that
     // the resident decode blocks do not need for their tables.
-    if (!prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_HUFFMAN>), d.huff_per_sm,
-                   kPfxThreads, 0) ||
-        !prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_QLC>), d.qlc_per_sm,
-                   kPfxThreads, 0) ||
-        !prefer_l1(dev, reinterpret_cast<const void*>(k_decode<HX_KIND_EXPGOLOMB>), d.eg_per_sm,
-                   kPfxThreads, 0))
-      return false;
+    for (uint32_t kind : {HX_KIND_HUFFMAN, HX_KIND_QLC, HX_KIND_EXPGOLOMB})
+      for (int i = 0; i < 3; ++i)
+        if (!prefer_l1(dev, reinterpret_cast<const void*>(prefix_decoder(kind, i)),
+                       d.dec_per_sm[i], kDecodeBlock[i], 0))
+          return false;
     d.sms = sms;
   }
   *out = d;
@@ -1474,11 +1492,15 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   if (!device_info(&info)) return HX_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint64_t nchunks = n_chunks_of(n);
-  const uint64_t per_block = (kind == HX_KIND_SHANNONIC ? kDecThreads : kPfxThreads) / 8;
-  const int per_sm = kind == HX_KIND_HUFFMAN ? info.huff_per_sm
-                     : kind == HX_KIND_QLC   ? info.qlc_per_sm
-                     : kind == HX_KIND_EXPGOLOMB ? info.eg_per_sm
-                                             : info.sh_decode_per_sm;
+  // prefix codes: blocks of 1024 from half a wave of them on (64 chunks per SM; the one table
+  // copy per SM leaves the most L1 for the payload words), else of 256 from 16 chunks per SM, else
+  // of 64 (small inputs over as many SMs as possible)
+  int bi = 2;
+  if (nchunks >= (uint64_t)info.sms * 64) bi = 0;
+  else if (nchunks >= (uint64_t)info.sms * 16) bi = 1;
+  const int threads = kind == HX_KIND_SHANNONIC ? kDecThreads : kDecodeBlock[bi];
+  const int per_sm = kind == HX_KIND_SHANNONIC ? info.sh_decode_per_sm : info.dec_per_sm[bi];
+  const uint64_t per_block = threads / 8;
   const uint64_t want = (nchunks + per_block - 1) / per_block;
   const uint32_t grid =
       (uint32_t)std::max<uint64_t>(1, std::min<uint64_t>(want, (uint64_t)info.sms * per_sm));
@@ -1491,14 +1513,10 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   a.n = n;
   a.status = d_status;
   a.kind = kind;
-  if (kind == HX_KIND_HUFFMAN)
-    k_decode<HX_KIND_HUFFMAN><<<grid, kPfxThreads, 0, s>>>(a);
-  else if (kind == HX_KIND_QLC)
-    k_decode<HX_KIND_QLC><<<grid, kPfxThreads, 0, s>>>(a);
-  else if (kind == HX_KIND_EXPGOLOMB)
-    k_decode<HX_KIND_EXPGOLOMB><<<grid, kPfxThreads, 0, s>>>(a);
-  else
+  if (kind == HX_KIND_SHANNONIC)
     k_sh_decode<<<grid, kDecThreads, 0, s>>>(a);
+  else
+    prefix_decoder(kind, bi)<<<grid, threads, 0, s>>>(a);
   return launched();
 }
 
