@@ -77,8 +77,22 @@ __global__ void __launch_bounds__(kHistThreads) k_histogram(const uint8_t* __res
   };
   const uint64_t nvec = n / 16;
   const uint4* v = reinterpret_cast<const uint4*>(in);
-  for (uint64_t i = blockIdx.x * (uint64_t)kHistThreads + tid; i < nvec;
-       i += (uint64_t)gridDim.x * kHistThreads) {
+  const uint64_t stride = (uint64_t)gridDim.x * kHistThreads;
+  uint64_t i = blockIdx.x * (uint64_t)kHistThreads + tid;
+  // four 16-byte loads in flight per thread, then their 64 bytes counted
+  for (; i + 3 * stride < nvec; i += 4 * stride) {
+    uint4 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = __ldcs(v + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      count4(x[u].x);
+      count4(x[u].y);
+      count4(x[u].z);
+      count4(x[u].w);
+    }
+  }
+  for (; i < nvec; i += stride) {
     const uint4 x = __ldcs(v + i);
     count4(x.x);
     count4(x.y);
