@@ -282,8 +282,9 @@ __device__ __forceinline__ void reds_or_u32(uint32_t a, uint32_t x) {
   asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(x) : "memory");
 }
 
-// Sum of the length-table entries of the 16 bytes in v (count of them exist); as measure16, on
-// 32-bit shared addresses.
+// The bit count of the 16 bytes in v (count of them exist): the sum of their length-table entries
+// ((count << 16) | len; the low 16 bits of the sum are the bit count, at most 16 * 12). With HIST
+// each lookup is a shared atomic that also adds 1 to the entry's count.
 template <bool HIST, bool COMPLETE, bool WHOLE>
 __device__ __forceinline__ uint32_t lengths16(uint32_t base, const uint4& v, uint32_t count,
                                               bool& uncodable) {
