@@ -348,7 +348,7 @@ __device__ uint64_t lookback(const EncodeArgs& a, uint32_t c, uint32_t lane) {
 template <bool WHOLE>
 __device__ __forceinline__ void pack_segment(uint32_t base, const uint4& v, uint32_t count,
                                              uint32_t buf, uint32_t sink, uint32_t s) {
-  uint32_t wa = buf + 4 * (s >> 5), nacc = s & 31, hi = 0, lo = 0;
+  uint32_t d = buf + 4 * (s >> 5) - sink, nacc = s & 31, hi = 0, lo = 0;
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -359,19 +359,22 @@ __device__ __forceinline__ void pack_segment(uint32_t base, const uint4& v, uint
     e[3] = (WHOLE || 4 * q + 3 < (int)count) ? lds_u32(row_addr<3>(w[q], base)) : 0u;
 #pragma unroll
     for (int h = 0; h < 4; h += 2) {
+      // the bookkeeping in multiply-adds where it can be (the integer logic pipe is the busy
+      // one): the word goes to sink + f * d, d = (its address) - sink, f = 1 when a word is
+      // finished; the codes' bits do not overlap, so the adds are ORs
       const uint32_t l1 = e[h + 1] & 0xffu;
       const uint32_t pl = (e[h] & 0xffu) + l1;
-      const uint32_t pc = ((e[h] >> 20) << l1) | (e[h + 1] >> 20);
+      const uint32_t pc = ((e[h] >> 20) << l1) + (e[h + 1] >> 20);
       hi = __funnelshift_l(lo, hi, pl);
-      lo = (lo << pl) | pc;
+      lo = (lo << pl) + pc;
       nacc += pl;
-      const bool full = nacc >= 32;
-      nacc -= full ? 32u : 0u;
-      reds_or_u32(full ? wa : sink, __funnelshift_r(lo, hi, nacc));
-      wa += full ? 4u : 0u;
+      const uint32_t f = nacc >> 5;  // 0 or 1: a pair adds at most 24 bits to at most 31
+      nacc &= 31u;
+      reds_or_u32(sink + f * d, __funnelshift_r(lo, hi, nacc));
+      d += f * 4u;
     }
   }
-  reds_or_u32(nacc ? wa : sink, lo << (32 - nacc));
+  reds_or_u32(nacc ? sink + d : sink, lo << (32 - nacc));
 }
 
 // One chunk by one warp (see k_encode).
