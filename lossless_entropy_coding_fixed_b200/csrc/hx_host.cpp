@@ -295,23 +295,29 @@ int shannonic_tables(const hx_codebook& cb, hx::Tables* t) {
   for (int u = 0; u < kShL; ++u) {
     const int r = spread[u];
     const int xs = cb.sh_f[r] + seen[r];  // the seen[r]-th state of range r
-    t->sh_enc[cum[r] + seen[r]] = (uint8_t)u;
+    t->sh_enc[cum[r] + seen[r]] = (uint8_t)(kShL + u);
     ++seen[r];
     int lg = 0;
     while ((2 << lg) <= xs) ++lg;
     const int nb = kShR - lg;
     const int size = cb.sh_lo[r + 1] - cb.sh_lo[r];
-    t->sh_dec[u] = (uint32_t)(xs << nb) | ((uint32_t)nb << 8) | ((uint32_t)bits_for(size) << 12) |
-                   ((uint32_t)cb.sh_lo[r] << 16) | ((uint32_t)(size - 1) << 24);
+    const int tot = nb + bits_for(size);
+    t->sh_dec[u][0] = (1u << tot) - 1u;
+    t->sh_dec[u][1] = (uint32_t)tot | ((uint32_t)(xs << nb) << 16);
+    t->sh_dec[u][2] = (uint32_t)nb;
+    t->sh_dec[u][3] = (uint32_t)cb.sh_lo[r] | ((uint32_t)(0x8000 - size) << 16);
   }
   for (int r = 0; r < nr; ++r) {
     int lg = 0;
     while ((2 << lg) <= cb.sh_f[r]) ++lg;
-    const int size = cb.sh_lo[r + 1] - cb.sh_lo[r];
-    for (int v = cb.sh_lo[r]; v < cb.sh_lo[r + 1]; ++v)
-      t->sh_sym[v] = (uint32_t)cb.sh_f[r] | ((uint32_t)cum[r] << 8) |
-                     ((uint32_t)bits_for(size) << 16) | ((uint32_t)(v - cb.sh_lo[r]) << 20) |
-                     ((uint32_t)(kShR - lg) << 28);
+    const int k = kShR - lg, f = cb.sh_f[r];
+    const int size = cb.sh_lo[r + 1] - cb.sh_lo[r], ob = bits_for(size);
+    // (k << 8) - (f << k) + 256 ob lies in [-255, 3840): stored as 12 bits, two's complement
+    const uint32_t key = (uint32_t)((k << 8) - (f << k) + 256 * ob) & 0xfffu;
+    for (int v = cb.sh_lo[r]; v < cb.sh_lo[r + 1]; ++v) {
+      t->sh_sym[v] = (uint32_t)ob | ((uint32_t)(cum[r] - f + 128) << 8) | (key << 20);
+      t->sh_off[v] = (uint8_t)(v - cb.sh_lo[r]);
+    }
   }
   return HX_OK;
 }

@@ -213,7 +213,7 @@ __device__ uint32_t block_exclusive_scan(uint32_t* cnt, uint32_t m, uint32_t* re
 }
 
 // Limits of the Shannonic coder's measure blocks (the two-pass encoder of kind 2).
-constexpr uint32_t kMaxChunksPerBlock = 4096;  // chunks of one measure block
+constexpr uint32_t kMaxChunksPerBlock = 1024;  // chunks of one measure block
 constexpr uint32_t kMaxMeasureBlocks = 2048;
 constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536: a chunk's largest size
 
@@ -377,6 +377,51 @@ __device__ __forceinline__ void pack_segment(uint32_t base, const uint4& v, uint
   reds_or_u32(nacc ? sink + d : sink, lo << (32 - nacc));
 }
 
+
+// A coded chunk's way out (see k_encode): its word offset, then its words.
+__device__ __forceinline__ void chunk_out(const EncodeArgs& a, uint32_t c, uint32_t words,
+                                          uint32_t* buf, uint32_t lane) {
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
+  __syncwarp();
+  // the chunk's word offset
+  uint64_t off = 0;
+  bool copy = true;
+  if (c > 0) {
+    off = lookback(a, c, lane);
+    if (off == ~0ull) {
+      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
+      copy = false;
+    } else if (lane == 0 && c != a.withhold) {
+      st_relaxed_u64(a.look + c, kLookPre | (off + words));
+    }
+  }
+  if (copy) {
+    const uint64_t P = payload_offset(n);
+    uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
+    uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
+    const uint64_t end = off + words;
+    if (lane == 0) word_off[c] = (uint32_t)off;
+    if (c + 1 == nchunks && lane == 0) {
+      reinterpret_cast<uint64_t*>(a.out)[4] = end;
+      word_off[nchunks] = (uint32_t)end;
+    }
+    // payload words that fit before the 2 guard words at the end of the caller's buffer
+    const uint64_t room = a.cap >= P + 8 ? (a.cap - P - 8) / 4 : 0;
+    if (end > room) {
+      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
+    } else {
+      for (uint32_t i = lane; i < words; i += 32) payload[off + i] = buf[i];
+      if (c + 1 == nchunks && lane < 2) payload[end + lane] = 0;
+    }
+  }
+  __syncwarp();
+  // leave the buffer zero for the next chunk
+  uint4* b4 = reinterpret_cast<uint4*>(buf);
+  for (uint32_t q = lane; q < (words + 3) / 4; q += 32) b4[q] = make_uint4(0, 0, 0, 0);
+  __syncwarp();
+}
+
 // One chunk by one warp (see k_encode).
 template <bool HIST, bool COMPLETE, bool WHOLE>
 __device__ __forceinline__ void encode_chunk(const EncodeArgs& a, EncSmem& sm, uint32_t c,
@@ -440,44 +485,9 @@ __device__ __forceinline__ void encode_chunk(const EncodeArgs& a, EncSmem& sm, u
     const uint32_t fw = k < 2 ? f01 : k < 4 ? f23 : k < 6 ? f45 : f67;
     pack_segment<WHOLE>(codebase, vk, ck, buf32, sink32, (fw >> (16 * (k & 1))) & 0xffffu);
   }
-  __syncwarp();
-  // the chunk's word offset
-  uint64_t off = 0;
-  bool copy = true;
-  if (c > 0) {
-    off = lookback(a, c, lane);
-    if (off == ~0ull) {
-      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_TIMEOUT);
-      copy = false;
-    } else if (lane == 0 && c != a.withhold) {
-      st_relaxed_u64(a.look + c, kLookPre | (off + words));
-    }
-  }
-  if (copy) {
-    const uint64_t P = payload_offset(n);
-    uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
-    uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
-    const uint64_t end = off + words;
-    if (lane == 0) word_off[c] = (uint32_t)off;
-    if (c + 1 == nchunks && lane == 0) {
-      reinterpret_cast<uint64_t*>(a.out)[4] = end;
-      word_off[nchunks] = (uint32_t)end;
-    }
-    // payload words that fit before the 2 guard words at the end of the caller's buffer
-    const uint64_t room = a.cap >= P + 8 ? (a.cap - P - 8) / 4 : 0;
-    if (end > room) {
-      if (lane == 0) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
-    } else {
-      for (uint32_t i = lane; i < words; i += 32) payload[off + i] = buf[i];
-      if (c + 1 == nchunks && lane < 2) payload[end + lane] = 0;
-    }
-  }
-  __syncwarp();
-  // leave the buffer zero for the next chunk
-  uint4* b4 = reinterpret_cast<uint4*>(buf);
-  for (uint32_t q = lane; q < (words + 3) / 4; q += 32) b4[q] = make_uint4(0, 0, 0, 0);
-  __syncwarp();
+  chunk_out(a, c, words, buf, lane);
 }
+
 
 template <bool HIST, bool COMPLETE>
 __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
@@ -946,38 +956,66 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a
 // count (k_sh_measure), the second runs it again and writes (k_sh_pack); one thread per
 // sub-stream in both, as in the decoder (k_sh_decode), which reads each sub-stream backwards.
 
-// Bits [pos, pos + len) of x (len < 32; an empty field reads 0).
-__device__ __forceinline__ uint32_t bfe(uint32_t x, uint32_t pos, uint32_t len) {
-  uint32_t r;
-  asm("bfe.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(pos), "r"(len));
-  return r;
-}
-
 constexpr int kShThreads = 256;  // 8 threads per chunk, 32 chunks per block
 constexpr int kShCopies = 16;    // symbol table copies: lane l reads copy l % 16 (<= 2-way)
 
-// Encoder tables in shared memory.
+// Encoder tables in shared memory: per byte value [byte][copy] the step's fields (sh_sym) and,
+// at a fixed distance, its offset in its range (sh_off); the ranges' states (sh_enc). The
+// measure pass needs no offsets (ShCount).
 struct ShEnc {
-  uint32_t sym[256 * kShCopies];  // [byte][copy]: per-byte fields of hx::Tables::sh_sym
-  uint8_t enc[128];               // the ranges' states minus 128
+  uint32_t sym[256 * kShCopies];
+  uint32_t off[256 * kShCopies];
+  uint8_t enc[128];
+};
+struct ShCount {
+  uint32_t sym[256 * kShCopies];
+  uint8_t enc[128];
 };
 
-__device__ __forceinline__ void sh_load_tables(const hx::Tables* t, ShEnc& s) {
-  for (int i = threadIdx.x; i < 256 * kShCopies; i += blockDim.x) s.sym[i] = t->sh_sym[i / kShCopies];
+template <class T>
+__device__ __forceinline__ void sh_load_tables(const hx::Tables* t, T& s) {
+  for (int i = threadIdx.x; i < 256 * kShCopies; i += blockDim.x) {
+    s.sym[i] = t->sh_sym[i / kShCopies];
+    if constexpr (sizeof(T) == sizeof(ShEnc)) s.off[i] = t->sh_off[i / kShCopies];
+  }
   for (int i = threadIdx.x; i < 128; i += blockDim.x) s.enc[i] = t->sh_enc[i];
 }
 
-// One tANS step for byte `sym` from `state` (in [128, 256)): the bits it writes (the offset,
-// then the state's low nb bits) as (value, count), and the next state.
-__device__ __forceinline__ uint32_t sh_step(const ShEnc& s, const uint32_t* sym_lane,
-                                            uint32_t sym, uint32_t& state, uint32_t& nbits) {
-  const uint32_t e = sym_lane[sym * kShCopies];
-  const uint32_t f = e & 0xffu, kshift = e >> 28, ob = (e >> 16) & 15u;
-  const uint32_t nb = kshift - ((state >> kshift) < f ? 1u : 0u);  // state >> nb in [f, 2f)
-  const uint32_t value = (((e >> 20) & 0xffu) << nb) | (state & ((1u << nb) - 1u));
-  state = 128u + s.enc[((e >> 8) & 0x7fu) + (state >> nb) - f];
-  nbits = ob + nb;
-  return value;
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+
+// Shared addresses of the encoder tables for this lane: its copy of byte b's entry is at
+// sym + 4 * kShCopies * b, b's offset kOffDist further; `enc` is sh_enc's address - 128.
+struct ShLane {
+  uint32_t sym, enc;
+};
+constexpr uint32_t kOffDist = 4 * 256 * kShCopies;
+template <class T>
+__device__ __forceinline__ ShLane sh_lane(const T& s, uint32_t lane) {
+  return {(uint32_t)__cvta_generic_to_shared(s.sym) + 4 * (lane % kShCopies),
+          (uint32_t)__cvta_generic_to_shared(s.enc) - 128u};
+}
+
+// One tANS step from state x (in [128, 256)) with the byte's entry e: returns the bit count
+// len = nb + ob it writes and moves x to the next state. The entry's key makes (x + key) >> 8 =
+// len; x >> nb is (x << ob) >> len, and the ob in e's low bits is all a wrapping shift reads.
+__device__ __forceinline__ uint32_t sh_next(uint32_t e, uint32_t& x, uint32_t enc, uint32_t& xo,
+                                            uint32_t& hi) {
+  const uint32_t len = (x * (1u << 20) + e) >> 28;
+  xo = __funnelshift_l(0u, x, e);  // x << ob
+  hi = xo >> len;                  // x >> nb, in [f, 2f)
+  x = lds_u8(enc + __byte_perm(e, 0u, 0x4441) + hi);  // sh_enc[cum - f + hi]
+  return len;
+}
+
+// The bits a step writes, (offset << nb) | (x mod 2^nb), from its entry e, the byte's offset,
+// x << ob (xo), x >> nb (hi) and len: ((offset - hi) << len) + xo is the same value times 2^ob.
+__device__ __forceinline__ uint32_t sh_value(uint32_t e, uint32_t off, uint32_t xo, uint32_t hi,
+                                             uint32_t len) {
+  return __funnelshift_r((((off - hi) << len) + xo), 0u, e);
 }
 
 // Bytes of sub-stream k of chunk c, last first: calls fn(byte) for each.
@@ -1013,7 +1051,7 @@ __device__ __forceinline__ uint32_t sh_count(uint64_t n, uint32_t c, uint32_t k)
 }
 
 struct ShMeasureSmem {
-  ShEnc t;
+  ShCount t;
   uint32_t cnt[kMaxChunksPerBlock];
   uint32_t red[kShThreads / 32];
   uint32_t hist[kShThreads / 32][256];
@@ -1032,7 +1070,7 @@ __global__ void __launch_bounds__(kShThreads) k_sh_measure(EncodeArgs a) {
   if (hist)
     for (int i = tid; i < (kShThreads / 32) * 256; i += kShThreads) (&sm.hist[0][0])[i] = 0;
   __syncthreads();
-  const uint32_t* sym_lane = sm.t.sym + (lane % kShCopies);
+  const ShLane tl = sh_lane(sm.t, lane);
   const uint64_t n = a.n;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
   const uint32_t c0 = blockIdx.x * a.cpb;
@@ -1049,9 +1087,8 @@ __global__ void __launch_bounds__(kShThreads) k_sh_measure(EncodeArgs a) {
     if (m) {
       uint32_t state = 128;
       sh_reverse(a, c, k, m, [&](uint32_t s) {
-        uint32_t nb;
-        sh_step(sm.t, sym_lane, s, state, nb);
-        bits += nb;
+        uint32_t xo, hi;
+        bits += sh_next(lds_u32(tl.sym + s * (4 * kShCopies)), state, tl.enc, xo, hi);
         if (hist) atomicAdd(&sm.hist[warp][s], 1u);
       });
       bits += HX_SHN_R;  // the final state
@@ -1082,6 +1119,17 @@ __global__ void __launch_bounds__(kShThreads) k_sh_measure(EncodeArgs a) {
       if (sum) atomicAdd(&a.hist[sym], sum);
     }
   }
+}
+
+// Predicated global stores (no branch around them).
+__device__ __forceinline__ void st_global_if(bool p, uint32_t* a, uint32_t v) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q st.global.u32 [%0], %1;\n}"
+               ::"l"(a), "r"(v), "r"((uint32_t)p) : "memory");
+}
+__device__ __forceinline__ void st_global_v4_if(bool p, uint32_t* a, uint4 v) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.u32 q, %5, 0;\n @q st.global.v4.u32 [%0], {%1, %2, %3, %4};\n}"
+      ::"l"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"((uint32_t)p) : "memory");
 }
 
 struct ShPackSmem {
@@ -1117,8 +1165,12 @@ __global__ void __launch_bounds__(kShThreads) k_sh_pack(EncodeArgs a) {
       atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
     }
   }
-  const uint32_t limit = fits ? total : 0u;
-  const uint32_t* sym_lane = sm.t.sym + (lane % kShCopies);
+  if (!fits) {  // the index still, but no payload word
+    for (uint32_t c = blockIdx.x * kShThreads + tid; c < nchunks; c += gridDim.x * kShThreads)
+      word_off[c] = sm.bpre[c / a.cpb] + a.local[c];
+    return;
+  }
+  const ShLane tl = sh_lane(sm.t, lane);
   const uint32_t k = tid & 7;
   const uint32_t groups = (nchunks + 31) / 32;
   for (uint32_t gi = blockIdx.x; gi < groups; gi += gridDim.x) {
@@ -1138,47 +1190,100 @@ __global__ void __launch_bounds__(kShThreads) k_sh_pack(EncodeArgs a) {
       widx = woff + (s >> 5);
       nacc = s & 31;  // the first bits belong to earlier sub-streams (zeros here)
       uint32_t hi = 0, lo = 0;
+      // Finished words leave in aligned groups of 4 (one 16-byte store; q0..q2 hold the three
+      // words before the current one), those before the sub-stream's first whole group one by one.
+      const uint32_t gfirst = (widx + 3) & ~3u;
+      uint32_t q0 = 0, q1 = 0, q2 = 0;
+      // appends len (<= 30) bits
       auto put = [&](uint32_t value, uint32_t len) {
         hi = __funnelshift_l(lo, hi, len);
         lo = (lo << len) | value;
         nacc += len;
-        if (nacc >= 32) {
-          nacc -= 32;
-          if (widx < limit) payload[widx] = __funnelshift_r(lo, hi, nacc);
-          ++widx;
-        }
+        const bool full = nacc >= 32;
+        nacc -= full ? 32u : 0u;
+        const uint32_t w = __funnelshift_r(lo, hi, nacc);
+        st_global_if(full && widx < gfirst, payload + widx, w);
+        st_global_v4_if(full && widx >= gfirst && (widx & 3) == 3, payload + widx - 3,
+                        make_uint4(q0, q1, q2, w));
+        q0 = full ? q1 : q0;
+        q1 = full ? q2 : q1;
+        q2 = full ? w : q2;
+        widx += full ? 1u : 0u;
       };
-      if (m) {
-        uint32_t state = 128;
-        sh_reverse(a, c, k, m, [&](uint32_t sym) {
-          uint32_t nb;
-          const uint32_t v = sh_step(sm.t, sym_lane, sym, state, nb);
-          put(v, nb);
-        });
-        put(state - 128u, HX_SHN_R);
+      uint32_t state = 128;
+      // the bits of byte `sym` (as sh_value) and their count
+      auto code = [&](uint32_t sym, uint32_t& len) -> uint32_t {
+        const uint32_t ea = tl.sym + sym * (4 * kShCopies);
+        const uint32_t e = lds_u32(ea), off = lds_u32(ea + kOffDist);
+        uint32_t xo, xh;
+        len = sh_next(e, state, tl.enc, xo, xh);
+        return sh_value(e, off, xo, xh, len);
+      };
+      if (m == kSubLen) {
+        // whole sub-stream: 16 bytes at a time from the end, two codes joined per append
+        const uint4* src = reinterpret_cast<const uint4*>(a.in + (uint64_t)c * kChunk +
+                                                          (uint64_t)k * kSubLen);
+        uint4 nxt = __ldg(src + kSubLen / 16 - 1);
+#pragma unroll 1
+        for (int g = kSubLen / 16 - 1; g >= 0; --g) {
+          const uint4 v = nxt;
+          if (g > 0) nxt = __ldg(src + g - 1);
+          const uint32_t w[4] = {v.w, v.z, v.y, v.x};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+#pragma unroll
+            for (int h = 3; h > 0; h -= 2) {
+              uint32_t l0, l1;
+              const uint32_t v0 = code(__byte_perm(w[q], 0u, 0x4440 + h), l0);
+              const uint32_t v1 = code(__byte_perm(w[q], 0u, 0x4440 + h - 1), l1);
+              put((v0 << l1) | v1, l0 + l1);
+            }
+          }
+        }
+      } else if (m) {
+        const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
+        for (uint32_t i = m; i-- > 0;) {
+          uint32_t l;
+          const uint32_t v = code((uint32_t)a.in[first + i], l);
+          put(v, l);
+        }
       }
+      if (m) put(state - 128u, HX_SHN_R);
+      // the finished words of the last, incomplete group
+      const uint32_t g = max(gfirst, widx & ~3u);
+      if (widx >= g + 1) payload[widx - 1] = q2;
+      if (widx >= g + 2) payload[widx - 2] = q1;
+      if (widx >= g + 3) payload[widx - 3] = q0;
       tail = nacc ? lo << (32 - nacc) : 0u;
       // the chunk's last word is stored whole (zero padding)
-      if (last && nacc && widx < limit) payload[widx] = tail;
+      if (last && nacc) payload[widx] = tail;
     }
     __syncwarp();
     // any other unfinished word is OR-ed into the word the next sub-stream stored whole
-    if (live && m && !last && nacc && widx < limit) atomicOr(payload + widx, tail);
+    if (live && m && !last && nacc) atomicOr(payload + widx, tail);
   }
 }
 
 // Reads a sub-stream backwards: the unread bits end at bit 32 * j + t of the payload (t in
-// 1..32 unread bits in word j, MSB first); cur = word j, prv = word j - 1, two more below
-// already requested. Words outside the caller's buffer read as 0.
+// 1..32 unread bits in word j, MSB first); cur = word j, prv = word j - 1. The words below come
+// in aligned 16-byte blocks: r is block rb, the one that holds the next word to come in, and the
+// block below it is already requested (nx), so a block is moved only once it has had a whole
+// block's worth of symbols to arrive. Words outside the caller's buffer read as 0.
 // (j is signed: a reader that runs off the front of the payload must not wrap around; a payload
 // holds fewer than 2^31 words, since n < 2^32 bytes at no more than 15 bits each.)
 struct BackBits {
-  const uint32_t* words;
+  const uint32_t* words;  // 16-byte aligned
   uint32_t wlimit;
-  int32_t j;
-  uint32_t t, cur, prv, pf0, pf1;
+  int32_t j, rb;
+  uint32_t t, cur, prv;
+  uint4 r, nx;
   __device__ __forceinline__ uint32_t word(int32_t i) const {
     return (uint32_t)i < wlimit ? __ldg(words + (uint32_t)i) : 0u;
+  }
+  __device__ __forceinline__ uint4 block(int32_t b) const {
+    if (b >= 0 && 4u * (uint32_t)b + 4u <= wlimit)
+      return __ldg(reinterpret_cast<const uint4*>(words) + b);
+    return make_uint4(word(4 * b), word(4 * b + 1), word(4 * b + 2), word(4 * b + 3));
   }
   __device__ __forceinline__ void start(uint64_t end_bit) {
     const uint64_t last = end_bit - 1;  // the first bit to read (backwards)
@@ -1186,45 +1291,59 @@ struct BackBits {
     t = (uint32_t)(last & 31) + 1;
     cur = word(j);
     prv = word(j - 1);
-    pf0 = word(j - 2);
-    pf1 = word(j - 3);
+    rb = (j - 2) >> 2;  // floor: the block of word j - 2
+    r = block(rb);
+    nx = block(rb - 1);
   }
   // the 32 bits before the read position, the last of them in bit 0 (bits before the payload's
   // first word read as 0)
   __device__ __forceinline__ uint32_t peek() const { return __funnelshift_r(cur, prv, 32 - t); }
+  __device__ __forceinline__ void advance() {
+    --j;
+    cur = prv;
+    const int32_t i = j - 1;  // the word that comes in
+    if ((i >> 2) != rb) {
+      --rb;
+      r = nx;
+      nx = block(rb - 1);
+    }
+    const uint32_t lo = (i & 1) ? r.y : r.x, hi = (i & 1) ? r.w : r.z;
+    prv = (i & 2) ? hi : lo;
+  }
   // moves the read position back by len (<= 31) bits
   __device__ __forceinline__ void skip(uint32_t len) {
     if (t > len) {
       t -= len;
     } else {
       t += 32 - len;
-      --j;
-      cur = prv;
-      prv = pf0;
-      pf0 = pf1;
-      pf1 = word(j - 3);
+      advance();
     }
   }
   // the `len` (<= 15) bits before the read position, MSB first
   __device__ __forceinline__ uint32_t read(uint32_t len) {
-    const uint32_t v = __funnelshift_r(cur, prv, 32 - t) & ((1u << len) - 1u);
-    if (t > len) {
-      t -= len;
-    } else {
-      t += 32 - len;
-      --j;
-      cur = prv;
-      prv = pf0;
-      pf0 = pf1;
-      pf1 = word(j - 3);
-    }
+    const uint32_t v = peek() & ((1u << len) - 1u);
+    skip(len);
     return v;
   }
   __device__ __forceinline__ int64_t position() const { return 32ll * j + t; }
 };
 
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+
+// Decoding states in shared memory, [state][copy] with 16-byte entries: lane l reads copy l % 8,
+// so the 8 lanes of each quarter of a warp read 8 different bank groups (no conflicts).
+constexpr int kShDecCopies = 8;
+
+// 5 resident blocks (48 registers): 6 would spill the reader's blocks
 __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
-  __shared__ uint32_t s_dec[128];
+  __shared__ __align__(16) uint4 s_dec[128 * kShDecCopies];
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
   const int tid = threadIdx.x;
@@ -1235,8 +1354,14 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)(-total));
     return;
   }
-  if (tid < 128) s_dec[tid] = s_tables->sh_dec[tid];
+  for (int i = tid; i < 128 * kShDecCopies; i += kDecThreads) {
+    const uint32_t* d = s_tables->sh_dec[i / kShDecCopies];
+    s_dec[i] = make_uint4(d[0], d[1], d[2], d[3]);
+  }
   __syncthreads();
+  // the entry of state x (in [128, 256)) is at tab + 16 * kShDecCopies * x
+  const uint32_t tab = (uint32_t)__cvta_generic_to_shared(s_dec) + 16u * (tid % kShDecCopies) -
+                       128u * 16u * kShDecCopies;
   const uint64_t n = a.n;
   const uint64_t nchunks = n_chunks_of(n);
   const uint64_t P = payload_offset(n);
@@ -1269,20 +1394,21 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
       if (!bad) {
         rd.start(32ull * w0 + end);
         uint32_t state = 128u + rd.read(HX_SHN_R);
-        bool invalid = false;
+        uint32_t over = 0;  // bit 31 set once an offset was not inside its range
         uint8_t* dst = a.out + c * kChunk + (uint64_t)k * kSubLen;
         // One symbol from x, the bits before the read position (the last in bit 0): the
-        // state's low nb bits, before them the offset. Returns the byte, moves the state, and
-        // drops the symbol's bits from x, counting them in `used`.
+        // state's low nb bits, before them the offset. Returns the byte (in the low 8 bits),
+        // moves the state, and drops the symbol's bits from x, counting them in `used`.
         auto one = [&](uint32_t& x, uint32_t& used) -> uint32_t {
-          const uint32_t d = s_dec[(state - 128u) & 127u];
-          const uint32_t nb = bfe(d, 8, 4), ob = bfe(d, 12, 4);
-          const uint32_t off = bfe(x, nb, ob);
-          invalid |= off > (d >> 24);
-          state = (d & 0xffu) + bfe(x, 0, nb);
-          x >>= nb + ob;
-          used += nb + ob;
-          return bfe(d, 16, 8) + off;
+          const uint4 d = lds_v4(tab + 16u * kShDecCopies * state);
+          const uint32_t v = x & d.x;       // offset and state bits
+          x = __funnelshift_r(x, 0u, d.y);  // x >> (nb + ob)
+          used += d.y;                      // (the count is its low 16 bits)
+          const uint32_t off = __funnelshift_r(v, 0u, d.z);                  // v >> nb
+          state = (d.y >> 16) + v - __funnelshift_l(0u, off, d.z);          // base + v mod 2^nb
+          const uint32_t r = off * 0x10001u + d.w;
+          over |= r;
+          return r;
         };
         const uint32_t groups = mine / 16;
         for (uint32_t g = 0; g < groups; ++g) {
@@ -1295,7 +1421,7 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
               uint32_t x = rd.peek(), used = 0;
               const uint32_t b0 = one(x, used);
               const uint32_t b1 = one(x, used);
-              rd.skip(used);
+              rd.skip(used & 0xffffu);
               pair[h] = __byte_perm(b0, b1, 0x0040);
             }
             o[q] = __byte_perm(pair[0], pair[1], 0x5410);
@@ -1305,10 +1431,11 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
         for (uint32_t i = groups * 16; i < mine; ++i) {
           uint32_t x = rd.peek(), used = 0;
           dst[i] = (uint8_t)one(x, used);
-          rd.skip(used);
+          rd.skip(used & 0xffffu);
         }
         // the chain must end in state 128 exactly at the sub-stream's first bit
-        bad |= invalid || state != 128u || rd.position() != (int64_t)(32ull * w0 + start);
+        bad |= (over >> 31) || state != 128u ||
+               rd.position() != (int64_t)(32ull * w0 + start);
       }
     }
     if (bad) atomicOr(a.status, (uint32_t)HX_ERR_CORRUPT);
@@ -1435,7 +1562,7 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
   if (!device_info(info)) return HX_ERR_CUDA;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
   // the Shannonic coder's measure blocks: at least one wave of resident blocks, at most
-  // kMaxChunksPerBlock chunks each (n < 2^32 gives at most 2^20 chunks, so 256 blocks always
+  // kMaxChunksPerBlock chunks each (n < 2^32 gives at most 2^20 chunks, so 1024 blocks always
   // suffice)
   const int per_sm = info->sh_measure_per_sm;
   uint32_t mblocks = (uint32_t)std::min<uint64_t>(

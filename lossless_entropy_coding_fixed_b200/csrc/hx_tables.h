@@ -21,13 +21,21 @@ struct Tables {
     uint16_t dec[4096];
     // Shannonic (kind 2) instead:
     struct {
-      // per decoding state 128 + u: base (xs << nb, bits 0-7) | nb (8-11) | offset bits (12-15)
-      // | first byte value of the range (16-23) | range size - 1 (24-31)
-      uint32_t sh_dec[128];
-      // per byte value: f_r (bits 0-7) | first index of the range's states in sh_enc (8-14) |
-      // offset bits (16-19) | offset in the range (20-27) | 7 - floor(log2 f_r) (28-30)
+      // per decoding state 128 + u, four words: the mask of the bits its symbol took (the
+      // offset and the state bits, 2^(nb + ob) - 1); their count nb + ob (bits 0-4) | the base of
+      // the next state (xs << nb, bits 16-23: the next state is base + the nb state bits); nb;
+      // first byte value of the range (bits 0-15) | 0x8000 - range size (16-31), so that
+      // offset * 0x10001 + this word holds the byte in bits 0-7 and sets bit 31 exactly when the
+      // offset is not inside the range
+      uint32_t sh_dec[128][4];
+      // per byte value: offset bits ob (bits 0-3) | cum_r - f_r + 128 (8-15) | the 12-bit key
+      // 256 * ob + (k << 8) - (f_r << k), k = 7 - floor(log2 f_r) (20-31): for a state x in
+      // [128, 256), (x + key) >> 8 = nb + ob, nb the state bits the step writes (x >> nb in
+      // [f_r, 2 f_r))
       uint32_t sh_sym[256];
-      // the range's decoding states in increasing order, minus 128, ranges one after another
+      // per byte value: its offset in its range
+      uint8_t sh_off[256];
+      // the ranges' decoding states in increasing order (128 + u), ranges one after another
       uint8_t sh_enc[128];
     };
   };
