@@ -953,10 +953,11 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a
 // states (the table variant of asymmetric numeral systems), its offset inside the range in
 // ceil(log2 size) bits. tANS runs from a sub-stream's last symbol to its first, so its bit count
 // is known only after the whole sub-stream has been run: the encoder's first pass runs it to
-// count (k_sh_measure), the second runs it again and writes (k_sh_pack); one thread per
-// sub-stream in both, as in the decoder (k_sh_decode), which reads each sub-stream backwards.
+// count (k_sh_measure, two sub-streams per thread), the second runs it again and writes
+// (k_sh_pack, one per thread, as in the decoder, k_sh_decode, which reads each sub-stream
+// backwards).
 
-constexpr int kShThreads = 256;  // 8 threads per chunk, 32 chunks per block
+constexpr int kShThreads = 256;  // pack and decode: 8 threads per chunk, 32 chunks per block
 constexpr int kShCopies = 16;    // symbol table copies: lane l reads copy l % 16 (<= 2-way)
 
 // Encoder tables in shared memory: per byte value [byte][copy] the step's fields (sh_sym) and,
@@ -1076,34 +1077,68 @@ __global__ void __launch_bounds__(kShThreads) k_sh_measure(EncodeArgs a) {
   const uint32_t c0 = blockIdx.x * a.cpb;
   const uint32_t m_chunks = c0 < nchunks ? min(a.cpb, nchunks - c0) : 0u;
   uint16_t* sync = reinterpret_cast<uint16_t*>(a.out + sync_offset(n));
-  const uint32_t k = tid & 7, slot = tid >> 3;
-  const uint32_t rounds = (m_chunks + 31) / 32;
+  // two sub-streams per thread, q and q + 4, their tANS chains interleaved (each step waits on
+  // the table load of the one before it)
+  const uint32_t q = tid & 3, slot = tid >> 2;
+  const uint32_t rounds = (m_chunks + 63) / 64;
   for (uint32_t r = 0; r < rounds; ++r) {
-    const uint32_t i = r * 32 + slot;
+    const uint32_t i = r * 64 + slot;
     const bool live = i < m_chunks;
     const uint32_t c = c0 + (live ? i : 0);
-    const uint32_t m = live ? sh_count(n, c, k) : 0u;
-    uint32_t bits = 0;
-    if (m) {
-      uint32_t state = 128;
-      sh_reverse(a, c, k, m, [&](uint32_t s) {
-        uint32_t xo, hi;
-        bits += sh_next(lds_u32(tl.sym + s * (4 * kShCopies)), state, tl.enc, xo, hi);
-        if (hist) atomicAdd(&sm.hist[warp][s], 1u);
-      });
-      bits += HX_SHN_R;  // the final state
-    }
-    // the chunk's 8 sub-streams: sync offsets by a prefix sum over its 8 threads
-    uint32_t incl = bits;
+    const uint32_t m0 = live ? sh_count(n, c, q) : 0u, m1 = live ? sh_count(n, c, q + 4) : 0u;
+    uint32_t b0 = 0, b1 = 0;
+    auto step = [&](uint32_t s, uint32_t& x) -> uint32_t {
+      uint32_t xo, hi;
+      if (hist) atomicAdd(&sm.hist[warp][s], 1u);
+      return sh_next(lds_u32(tl.sym + s * (4 * kShCopies)), x, tl.enc, xo, hi);
+    };
+    if (m1 == kSubLen) {  // both whole
+      const uint4* s0 =
+          reinterpret_cast<const uint4*>(a.in + (uint64_t)c * kChunk + (uint64_t)q * kSubLen);
+      const uint4* s1 = s0 + 4 * kSubLen / 16;
+      uint4 n0 = __ldg(s0 + kSubLen / 16 - 1), n1 = __ldg(s1 + kSubLen / 16 - 1);
+      uint32_t x0 = 128, x1 = 128;
+#pragma unroll 1
+      for (int g = kSubLen / 16 - 1; g >= 0; --g) {
+        const uint4 v0 = n0, v1 = n1;
+        if (g > 0) {
+          n0 = __ldg(s0 + g - 1);
+          n1 = __ldg(s1 + g - 1);
+        }
+        const uint32_t w0[4] = {v0.w, v0.z, v0.y, v0.x}, w1[4] = {v1.w, v1.z, v1.y, v1.x};
 #pragma unroll
-    for (int d = 1; d < 8; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d, 8);
-      if (k >= (uint32_t)d) incl += t;
+        for (int qq = 0; qq < 4; ++qq) {
+#pragma unroll
+          for (int h = 3; h >= 0; --h) {
+            b0 += step(__byte_perm(w0[qq], 0u, 0x4440 + h), x0);
+            b1 += step(__byte_perm(w1[qq], 0u, 0x4440 + h), x1);
+          }
+        }
+      }
+    } else {
+      uint32_t x0 = 128, x1 = 128;
+      if (m0) sh_reverse(a, c, q, m0, [&](uint32_t s) { b0 += step(s, x0); });
+      if (m1) sh_reverse(a, c, q + 4, m1, [&](uint32_t s) { b1 += step(s, x1); });
     }
-    const uint32_t total = __shfl_sync(0xffffffffu, incl, 7, 8);
+    if (m0) b0 += HX_SHN_R;  // the final states
+    if (m1) b1 += HX_SHN_R;
+    // the chunk's 8 sub-streams: sync offsets by prefix sums over its 4 threads
+    uint32_t i0 = b0, i1 = b1;
+#pragma unroll
+    for (int d = 1; d < 4; d <<= 1) {
+      const uint32_t t0 = __shfl_up_sync(0xffffffffu, i0, d, 4);
+      const uint32_t t1 = __shfl_up_sync(0xffffffffu, i1, d, 4);
+      if (q >= (uint32_t)d) {
+        i0 += t0;
+        i1 += t1;
+      }
+    }
+    const uint32_t tot0 = __shfl_sync(0xffffffffu, i0, 3, 4);
+    const uint32_t total = tot0 + __shfl_sync(0xffffffffu, i1, 3, 4);
     if (live) {
-      sync[(uint64_t)c * HX_SUBSTREAMS + k] = (uint16_t)(k == 0 ? total : incl - bits);
-      if (k == 0) sm.cnt[i] = (total + 31) >> 5;
+      sync[(uint64_t)c * HX_SUBSTREAMS + q] = (uint16_t)(q == 0 ? total : i0 - b0);
+      sync[(uint64_t)c * HX_SUBSTREAMS + q + 4] = (uint16_t)(tot0 + i1 - b1);
+      if (q == 0) sm.cnt[i] = (total + 31) >> 5;
     }
   }
   __syncthreads();

@@ -173,11 +173,16 @@ def test_capacity(orc, books):
     x = datagen.data(1, n=5 * 4096 + 3)
     ref = orc.encode(ocb, x)[1]
     need = ref.size
-    for cap in (need - 4, need // 2, hx.payload_offset(x.size) + 8):
+    P = hx.payload_offset(x.size)
+    for cap in (need - 4, need // 2, P + 8):
         got, st, total = gpu_encode(tables, x, k, cap=cap)
         assert st == hx.HX_ERR_CAPACITY
         assert hx.stream_bytes(x.size, total) == need
         assert orc.encode(ocb, x, cap=cap)[0] & orc.ERR_CAPACITY
+        # the header and the index are those of the whole stream; a payload word is either the
+        # stream's own (a chunk that fitted) or untouched (zero), and none lies past the buffer
+        assert got.size == cap and (got[:P] == ref[:P]).all()
+        assert ((got[P:] == ref[P:cap]) | (got[P:] == 0)).all()
     got, st, _ = gpu_encode(tables, x, k, cap=need)
     assert st == 0 and (got == ref).all()
 

@@ -89,9 +89,14 @@ def test_adversarial_inputs(orc, cuda):
 def test_capacity_and_wrong_tables(orc, cuda):
     x = datagen.data(1, n=5 * 4096 + 3)
     tables, ocb = _book(orc, orc.histogram(x), cuda)
-    need = orc.encode(ocb, x)[1].size
-    got, st, total = _enc(tables, x, cap=need - 4)
-    assert st == hx.HX_ERR_CAPACITY and hx.stream_bytes(x.size, total) == need
+    full = orc.encode(ocb, x)[1]
+    need = full.size
+    P = hx.payload_offset(x.size)
+    for cap in (need - 4, P + 8):
+        got, st, total = _enc(tables, x, cap=cap)
+        assert st == hx.HX_ERR_CAPACITY and hx.stream_bytes(x.size, total) == need
+        # the header and the index are those of the whole stream, and no payload word is written
+        assert got.size == cap and (got[:P] == full[:P]).all() and (got[P:] == 0).all()
     huff = hx.build_codebook(orc.histogram(x)).upload(cuda)
     _, st, _ = _enc(huff, x)
     assert st == hx.HX_ERR_ARG
