@@ -359,12 +359,13 @@ __device__ __forceinline__ void pack_segment(uint32_t base, const uint4& v, uint
     e[3] = (WHOLE || 4 * q + 3 < (int)count) ? lds_u32(row_addr<3>(w[q], base)) : 0u;
 #pragma unroll
     for (int h = 0; h < 4; h += 2) {
-      // the bookkeeping in multiply-adds where it can be (the integer logic pipe is the busy
-      // one): the word goes to sink + f * d, d = (its address) - sink, f = 1 when a word is
-      // finished; the codes' bits do not overlap, so the adds are ORs
-      const uint32_t l1 = e[h + 1] & 0xffu;
-      const uint32_t pl = (e[h] & 0xffu) + l1;
-      const uint32_t pc = ((e[h] >> 20) << l1) + (e[h + 1] >> 20);
+      // The integer logic pipe is the busy one, so: the pair's length comes from one add (the
+      // codes sit above bit 20), the shift by l1 is a wrapping funnel shift (it reads only
+      // e[h + 1]'s low 5 bits, the length), and the bookkeeping is in multiply-adds: the word
+      // goes to sink + f * d, d = (its address) - sink, f = 1 when a word is finished. The
+      // codes' bits do not overlap, so the adds are ORs.
+      const uint32_t pl = (e[h] + e[h + 1]) & 0xffu;
+      const uint32_t pc = __funnelshift_l(0u, e[h] >> 20, e[h + 1]) + (e[h + 1] >> 20);
       hi = __funnelshift_l(lo, hi, pl);
       lo = (lo << pl) + pc;
       nacc += pl;
