@@ -466,96 +466,99 @@ def collective_leg(dev, hx, datagen, torch, tables, prior):
             dist.destroy_process_group()
 
 
+E2E_SLOTS = 3  # buffer slots of the end-to-end pipeline (2: 50.6 GB/s, 3: 55.6, 4: 55.5)
+
+
 def e2e_leg(args, dev, hx, torch, pg, ws, x_host, ht, qt, n, bound, scratch, status):
     """End to end through the public API with host buffers, both directions of a link: every step
     uploads its batch from pinned memory, encodes it with both codebooks and downloads the two
     streams (sender), then uploads the two streams, decodes them and downloads both decoded
-    batches (receiver). Steps are pipelined over two buffer slots on upload / codec / download
-    streams; every step's copies are inside the timed region."""
+    batches (receiver). Steps are pipelined over E2E_SLOTS buffer slots. Each kind of transfer
+    has its own copy stream (batch up, streams down, streams up, decoded batches down) and encode
+    and decode their own compute streams, so one step's transfers overlap the next step's;
+    events order every reuse of a buffer. Every step's copies are inside the timed region."""
     x_pin = torch.from_numpy(x_host).pin_memory()
-    host_st = [torch.empty(bound, dtype=torch.uint8).pin_memory() for _ in range(2)]
     host_y = [torch.empty(n, dtype=torch.uint8).pin_memory() for _ in range(2)]
     st_host = torch.empty(1, dtype=torch.int32).pin_memory()
-    hdr = torch.empty(2, 64, dtype=torch.uint8).pin_memory()
     stream = torch.cuda.current_stream(dev)
-    s_in, s_out, s_hdr = (torch.cuda.Stream(dev) for _ in range(3))
+    up_x, down_st, up_st, down_y, s_hdr, s_enc, s_dec = (torch.cuda.Stream(dev) for _ in range(7))
+    books = ((ht, hx.KIND_HUFFMAN), (qt, hx.KIND_QLC))
     slots = []
-    for _ in range(2):
+    for _ in range(E2E_SLOTS):
         sl = {"x": torch.empty(n, dtype=torch.uint8, device=dev),
               "st": [torch.empty(bound, dtype=torch.uint8, device=dev) for _ in range(2)],
               "rx": [torch.empty(bound, dtype=torch.uint8, device=dev) for _ in range(2)],
               "y": [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(2)],
-              "used": torch.cuda.Event(), "free": torch.cuda.Event()}
-        sl["used"].record(stream)
-        sl["free"].record(s_out)
+              "host_st": [torch.empty(bound, dtype=torch.uint8).pin_memory() for _ in range(2)],
+              "hdr": torch.empty(2, 64, dtype=torch.uint8).pin_memory()}
+        # the slot's last encode, header read, stream download, stream upload, decode and
+        # decoded download
+        for name, s_ in (("enc", s_enc), ("hdr_ev", s_hdr), ("stdown", down_st),
+                         ("stup", up_st), ("dec", s_dec), ("ydown", down_y)):
+            sl[name] = torch.cuda.Event()
+            sl[name].record(s_)
         slots.append(sl)
-    books = ((ht, hx.KIND_HUFFMAN), (qt, hx.KIND_QLC))
     counted = {"h2d": 0, "d2h": 0}
-    host_free = [torch.cuda.Event()]
-    host_free[0].record(s_in)
 
     def sender(sl):
-        s_in.wait_event(sl["used"])
-        s_in.wait_event(sl["free"])
-        with torch.cuda.stream(s_in):
+        up_x.wait_event(sl["enc"])  # the slot's last encode has read its batch
+        with torch.cuda.stream(up_x):
             sl["x"].copy_(x_pin, non_blocking=True)
         up = torch.cuda.Event()
-        up.record(s_in)
-        stream.wait_event(up)
-        done = []
-        for j, (t, kind) in enumerate(books):
-            hx.encode(t, sl["x"], out=sl["st"][j], scratch=scratch, status=status, kind=kind)
-            e = torch.cuda.Event()
-            e.record(stream)
-            done.append(e)
-        sl["enc"] = done
+        up.record(up_x)
+        s_enc.wait_event(up)
+        s_enc.wait_event(sl["stdown"])  # the slot's last streams are downloaded
+        with torch.cuda.stream(s_enc):
+            for j, (t, kind) in enumerate(books):
+                hx.encode(t, sl["x"], out=sl["st"][j], scratch=scratch, status=status, kind=kind)
+        sl["enc"].record(s_enc)
+        s_hdr.wait_event(sl["enc"])
+        with torch.cuda.stream(s_hdr):
+            for j in range(2):
+                sl["hdr"][j].copy_(sl["st"][j][:64], non_blocking=True)
+        sl["hdr_ev"].record(s_hdr)
         return n
 
     def link(sl):
         # the streams' sizes (their headers), then stream bytes down and back up
-        for j, e in enumerate(sl["enc"]):
-            s_hdr.wait_event(e)
-            with torch.cuda.stream(s_hdr):
-                hdr[j].copy_(sl["st"][j][:64], non_blocking=True)
-        got = torch.cuda.Event()
-        got.record(s_hdr)
-        got.synchronize()
-        sizes = [hx.stream_bytes(n, int(hdr[j][32:40].numpy().view(np.uint64)[0]))
+        sl["hdr_ev"].synchronize()
+        sizes = [hx.stream_bytes(n, int(sl["hdr"][j][32:40].numpy().view(np.uint64)[0]))
                  for j in range(2)]
-        # the host stream buffers are free once the previous step's upload has read them
-        s_out.wait_event(host_free[0])
-        for j in range(2):
-            s_out.wait_event(sl["enc"][j])
-            with torch.cuda.stream(s_out):
-                host_st[j][:sizes[j]].copy_(sl["st"][j][:sizes[j]], non_blocking=True)
-        down = torch.cuda.Event()
-        down.record(s_out)
-        s_in.wait_event(down)
-        with torch.cuda.stream(s_in):
+        down_st.wait_event(sl["enc"])
+        down_st.wait_event(sl["stup"])  # the slot's host stream buffers were read
+        with torch.cuda.stream(down_st):
             for j in range(2):
-                sl["rx"][j][:sizes[j]].copy_(host_st[j][:sizes[j]], non_blocking=True)
-        up = torch.cuda.Event()
-        up.record(s_in)
-        host_free[0] = up
-        stream.wait_event(up)
-        for j, (t, kind) in enumerate(books):
-            hx.decode(t, sl["rx"][j], n, out=sl["y"][j], status=status, kind=kind,
-                      nbytes=sizes[j])
-        sl["used"].record(stream)
-        s_out.wait_event(sl["used"])
-        with torch.cuda.stream(s_out):
+                sl["host_st"][j][:sizes[j]].copy_(sl["st"][j][:sizes[j]], non_blocking=True)
+        sl["stdown"].record(down_st)
+        up_st.wait_event(sl["stdown"])
+        up_st.wait_event(sl["dec"])  # the slot's last decode has read its received streams
+        with torch.cuda.stream(up_st):
+            for j in range(2):
+                sl["rx"][j][:sizes[j]].copy_(sl["host_st"][j][:sizes[j]], non_blocking=True)
+        sl["stup"].record(up_st)
+        s_dec.wait_event(sl["stup"])
+        s_dec.wait_event(sl["ydown"])  # the slot's last decoded batches are downloaded
+        with torch.cuda.stream(s_dec):
+            for j, (t, kind) in enumerate(books):
+                hx.decode(t, sl["rx"][j], n, out=sl["y"][j], status=status, kind=kind,
+                          nbytes=sizes[j])
+        sl["dec"].record(s_dec)
+        down_y.wait_event(sl["dec"])
+        with torch.cuda.stream(down_y):
             for j in range(2):
                 host_y[j].copy_(sl["y"][j], non_blocking=True)
             st_host.copy_(status, non_blocking=True)
-        sl["free"].record(s_out)
+        sl["ydown"].record(down_y)
         # (bytes up, bytes down): the streams up; headers, streams, decoded batches, status down
         return sum(sizes), 64 * 2 + sum(sizes) + 2 * n + 4
 
     def run(k):
         counted["h2d"] = counted["d2h"] = 0
+        for s_ in (up_x, down_st, up_st, down_y, s_hdr, s_enc, s_dec):
+            s_.wait_stream(stream)
         pending = None
         for t in range(k):
-            sl = slots[t % 2]
+            sl = slots[t % E2E_SLOTS]
             counted["h2d"] += sender(sl)
             if pending is not None:
                 up, down = link(pending)
@@ -565,11 +568,10 @@ def e2e_leg(args, dev, hx, torch, pg, ws, x_host, ht, qt, n, bound, scratch, sta
         up, down = link(pending)
         counted["h2d"] += up
         counted["d2h"] += down
-        end = torch.cuda.Event()
-        end.record(s_out)
-        stream.wait_event(end)
+        for s_ in (up_x, down_st, up_st, down_y, s_hdr, s_enc, s_dec):
+            stream.wait_stream(s_)
 
-    run(2)  # untimed: both slots once
+    run(E2E_SLOTS)  # untimed: every slot once
     torch.cuda.synchronize(dev)
     k = max(3, min(args.steps, 10))
     if pg:
@@ -588,7 +590,8 @@ def e2e_leg(args, dev, hx, torch, pg, ws, x_host, ht, qt, n, bound, scratch, sta
             "steps": k,
             "path": "pinned host batch -> H2D -> Huffman and QLC encode -> D2H of both streams "
                     "-> H2D of both streams -> decode -> D2H of both decoded batches; steps "
-                    "pipelined over 2 buffer slots on upload / codec / download streams"}
+                    f"pipelined over {E2E_SLOTS} buffer slots, each transfer kind on its own "
+                    "copy stream, encode and decode on their own streams"}
 
 
 def shannonic_leg(dev, hx, torch, x, prior, h, scratch, y, status, steps):
