@@ -4,8 +4,9 @@
 // from earlier batches, so the coder runs with no frequency pass and ships no codebook; "Quad
 // Length Codes for Lossless Compression of e4m3" (abstract, Tables 1-2) -- the area code.
 //
-//   k_histogram  byte histogram: 16-byte loads, one private 256-bin table per warp in shared
-//                memory, one global atomic per non-empty bin and block.
+//   k_histogram  byte histogram: 16-byte loads, four in flight per thread; one table of 32
+//                copies per block in shared memory (lane l counts into copy l, so a warp's
+//                atomics never conflict), one global atomic per non-empty bin and block.
 //
 //   k_encode     one pass over the input. A warp takes the next chunk from a counter and loads it
 //                with coalesced 16-byte loads (16 bytes of each sub-stream per lane); the length
@@ -28,9 +29,10 @@
 //                bank of their lines (codes of one length) vote per warp and may read 16-byte
 //                blocks instead.
 //
-//   k_sh_*       the Shannonic range coder: tANS over range indices, one thread per sub-stream
-//                in its measure, pack and (backward) decode kernels (two encode passes: a tANS
-//                sub-stream's length is known only once it has been run).
+//   k_sh_*       the Shannonic range coder: tANS over range indices with one table entry per
+//                step; a measure pass (two sub-streams per thread) and a pack pass (one per
+//                thread, 16-byte stores), since a tANS sub-stream's length is known only once it
+//                has been run; the decoder reads each sub-stream backwards, one thread each.
 #include <cuda_runtime.h>
 
 #include <algorithm>
