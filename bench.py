@@ -854,36 +854,39 @@ def main():
     if not args.no_e2e:
         e2e = e2e_leg(args, dev, hx, torch, pg, ws, x_host, ht, qt, n, bound, scratch, status)
 
+    # the side legs run on one GPU only: their figures are per-GPU and rank 0 alone reports them,
+    # and cfg5 alone builds 8 GiB of input on the host
+    side = ws == 1
     shannonic = None
-    if not args.no_shannonic:
+    if side and not args.no_shannonic:
         shannonic = shannonic_leg(dev, hx, torch, x, prior, h, scratch, y, status,
                                   max(3, min(args.steps, 10)))
 
     expgolomb = None
-    if not args.no_expgolomb:
+    if side and not args.no_expgolomb:
         expgolomb = expgolomb_leg(dev, hx, torch, x, h, scratch, y, status,
                                   max(3, min(args.steps, 10)))
     del x, y, sh, sq, scratch
     torch.cuda.empty_cache()
 
     online = None
-    if not args.no_online:
+    if side and not args.no_online:
         online = online_leg(dev, hx, datagen, torch)
 
     configs = None
-    if not args.no_configs:
+    if side and not args.no_configs:
         configs = configs_leg(dev, hx, datagen, torch, peak)
 
     cfg5 = None
-    if not args.no_cfg5:
+    if side and not args.no_cfg5:
         cfg5 = cfg5_leg(dev, hx, datagen, torch)
 
     collective = None
-    if ws == 1 and not args.no_collective:
+    if side and not args.no_collective:
         collective = collective_leg(dev, hx, datagen, torch, ht, prior)
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and side and not args.no_cpu_baseline:
         cpu = cpu_baseline_leg(prior)
 
     if rank == 0:
