@@ -210,11 +210,15 @@ int hx_decode_set(uint32_t kind, const void* const* d_tables, uint32_t n_tables,
  * ends). Every such wait is still bounded: after wait_ns nanoseconds (hx_encode uses 2 s) the
  * chunk raises HX_ERR_TIMEOUT in *d_status and writes no payload, and every chunk still waiting
  * gives up at once; the kernel completes and the context stays usable. withhold: a chunk that
- * never publishes its count (UINT64_MAX: none), so that the chunks after it time out. kind 0, 1
- * or 3 (HX_ERR_ARG for kind 2); other arguments and errors as hx_encode. */
+ * never publishes its count (UINT64_MAX: none), so that the chunks after it time out.
+ * flush_rounds: with d_hist, the chunks a warp codes between its flushes of the fused counts into
+ * d_hist (0: the 128 of hx_encode; at most 4096, else HX_ERR_ARG), so that a test can make the
+ * flush run often. kind 0, 1 or 3 (HX_ERR_ARG for kind 2); other arguments and errors as
+ * hx_encode. */
 int hx_encode_bounded(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                       void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
-                      uint32_t* d_status, uint64_t wait_ns, uint64_t withhold, void* stream);
+                      uint32_t* d_status, uint64_t wait_ns, uint64_t withhold,
+                      uint32_t flush_rounds, void* stream);
 
 /* Shannonic encode and decode (kind 2 tables): the same chunked stream, sub-stream framing and
  * index as hx_encode; inside a sub-stream the bits come from tANS run from its last symbol to

@@ -130,6 +130,7 @@ struct EncodeArgs {
   uint32_t* counter;  // scratch: next chunk to take (zeroed)
   uint64_t wait_ns;   // limit of one chunk's wait for its predecessors
   uint64_t withhold;  // a chunk that publishes nothing (failure tests), else ~0
+  uint32_t flush;     // fused histogram: a warp's chunks between its flushes of the counts
 };
 
 // Every header field but total_words.
@@ -231,9 +232,16 @@ constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536: a chu
 // and writes no payload, and every later wait gives up at once.
 constexpr int kEncThreads = 768;  // one block of 24 warps per SM sharing the two tables
 constexpr uint32_t kEncWarps = kEncThreads / 32;
-// 16-bit counts in the length table: a round of chunks adds at most kEncWarps * 128 to an entry
-constexpr uint32_t kEncFlushRounds = 65535 / (kEncWarps * 128);
-static_assert(kEncFlushRounds >= 1, "16-bit counts overflow within one round");
+// 24-bit counts in the length table (bits 8-31; the length in bits 0-7, so 16 summed entries keep
+// their bit count, at most 16 * 12, in the low byte). A warp that has taken `flush` chunks since
+// its last flush clears the whole table into the histogram by itself (atomic ANDs beside the
+// other warps' atomic adds), so between two flushes every warp takes fewer than `flush` chunks
+// of 128 symbols per lane, and no entry grows by 2^24. The block's last counts go out once all
+// its warps are done; no warp waits at a block barrier while chunks are left.
+constexpr uint32_t kEncCountShift = 8;
+constexpr uint32_t kEncFlushRounds = 128;     // `flush` of hx_encode (0.4 % of the work)
+constexpr uint32_t kEncFlushRoundsMax = 4096;  // the largest `flush` hx_encode_bounded takes
+static_assert(uint64_t(kEncWarps) * kEncFlushRoundsMax * 128 < (1ull << 24), "24-bit counts");
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
 constexpr uint64_t kLookAgg = 1ull << 62;   // word count of the chunk alone
 constexpr uint64_t kLookPre = 2ull << 62;   // word offset of the chunk's end (inclusive prefix)
@@ -241,8 +249,8 @@ constexpr uint64_t kLookValue = (1ull << 62) - 1;
 constexpr int kLookLoads = 2;  // look-back loads per lane: a window of 64 chunks
 
 // Two tables, entries [symbol][copy] with lane l using copy l (no bank conflicts): `len` =
-// (count << 16) | len for the length pass (with the fused histogram the lookup is a shared atomic
-// that adds 1 << 16), `code` = (code << 20) | len for the coding pass.
+// (count << 8) | len for the length pass (with the fused histogram the lookup is a shared atomic
+// that adds 1 << 8), `code` = (code << 20) | len for the coding pass.
 struct EncSmem {
   uint32_t len[256 * 32];
   uint32_t code[256 * 32];
@@ -286,7 +294,7 @@ __device__ __forceinline__ void reds_or_u32(uint32_t a, uint32_t x) {
 }
 
 // The bit count of the 16 bytes in v (count of them exist): the sum of their length-table entries
-// ((count << 16) | len; the low 16 bits of the sum are the bit count, at most 16 * 12). With HIST
+// ((count << 8) | len; the low 8 bits of the sum are the bit count, at most 16 * 12). With HIST
 // each lookup is a shared atomic that also adds 1 to the entry's count.
 template <bool HIST, bool COMPLETE, bool WHOLE>
 __device__ __forceinline__ uint32_t lengths16(uint32_t base, const uint4& v, uint32_t count,
@@ -302,13 +310,13 @@ __device__ __forceinline__ uint32_t lengths16(uint32_t base, const uint4& v, uin
                            : j == 1 ? row_addr<1>(w[q], base)
                            : j == 2 ? row_addr<2>(w[q], base)
                                     : row_addr<3>(w[q], base);
-        const uint32_t e = HIST ? atoms_add_u32(a, 1u << 16) : lds_u32(a);
+        const uint32_t e = HIST ? atoms_add_u32(a, 1u << kEncCountShift) : lds_u32(a);
         sum += e;
         if (!COMPLETE) uncodable |= (e & 0xffu) == 0;
       }
     }
   }
-  return sum & 0xffffu;
+  return HIST ? sum & ((1u << kEncCountShift) - 1u) : sum;  // without HIST every count is 0
 }
 
 // Word offset of chunk c (c > 0) from the chunks before it, read 32 * kLookLoads at a time by
@@ -538,42 +546,40 @@ __device__ void encode_chunks(const EncodeArgs& a, EncSmem& sm) {
     reinterpret_cast<uint4*>(buf)[q] = make_uint4(0, 0, 0, 0);
   __syncwarp();
   bool uncodable = false;
-  bool more = true;
-  for (uint32_t r = 0;; ++r) {
-    if (more) {
-      uint32_t c = 0;
-      if (lane == 0) c = atomicAdd(a.counter, 1u);
-      c = __shfl_sync(0xffffffffu, c, 0);
-      more = c < nchunks;
-      if (more) {
-        // the chunk a warp will most likely take one round from now, into L2
-        const uint64_t ahead = (uint64_t)c + gridDim.x * kEncWarps;
-        if (lane == 0 && ahead < full_chunks)
-          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.in + ahead * kChunk),
-                       "r"(kChunk)
-                       : "memory");
-        if (c < full_chunks) encode_chunk<HIST, COMPLETE, true>(a, sm, c, buf, sink, uncodable);
-        else encode_chunk<HIST, COMPLETE, false>(a, sm, c, buf, sink, uncodable);
+  for (uint32_t r = 1;; ++r) {
+    uint32_t c = 0;
+    if (lane == 0) c = atomicAdd(a.counter, 1u);
+    c = __shfl_sync(0xffffffffu, c, 0);
+    if (c >= nchunks) break;
+    // the chunk a warp will most likely take one round from now, into L2
+    const uint64_t ahead = (uint64_t)c + gridDim.x * kEncWarps;
+    if (lane == 0 && ahead < full_chunks)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.in + ahead * kChunk),
+                   "r"(kChunk)
+                   : "memory");
+    if (c < full_chunks) encode_chunk<HIST, COMPLETE, true>(a, sm, c, buf, sink, uncodable);
+    else encode_chunk<HIST, COMPLETE, false>(a, sm, c, buf, sink, uncodable);
+    if (HIST && r % a.flush == 0) {
+      // this warp clears every count into the histogram (the other warps keep counting)
+      const uint32_t t0 = (uint32_t)__cvta_generic_to_shared(sm.len);
+      for (int sym = 0; sym < 256; ++sym) {
+        uint32_t old;
+        asm volatile("atom.shared.and.b32 %0, [%1], %2;"
+                     : "=r"(old)
+                     : "r"(t0 + 4u * (32u * sym + lane)), "r"(0xffu)
+                     : "memory");
+        const uint32_t cnt = __reduce_add_sync(0xffffffffu, old >> kEncCountShift);
+        if (lane == 0 && cnt) atomicAdd(&a.hist[sym], cnt);
       }
     }
-    if (HIST) {
-      // the 16-bit counts go to the histogram every kEncFlushRounds rounds (a warp without a
-      // chunk left just counts rounds); the block leaves together once no warp has one
-      if ((r + 1) % kEncFlushRounds == 0) {
-        __syncthreads();
-        for (int sym = tid; sym < 256; sym += kEncThreads) {
-          uint32_t sum = 0;
-          for (int l = 0; l < 32; ++l) {
-            const uint32_t e = sm.len[sym * 32 + l];
-            sum += e >> 16;
-            sm.len[sym * 32 + l] = e & 0xffffu;
-          }
-          if (sum) atomicAdd(&a.hist[sym], sum);
-        }
-        if (!__syncthreads_or(more)) break;
-      }
-    } else if (!more) {
-      break;
+  }
+  if (HIST) {
+    // the counts since the warps' last flushes, once every warp is done
+    __syncthreads();
+    for (int sym = tid; sym < 256; sym += kEncThreads) {
+      uint32_t sum = 0;
+      for (int l = 0; l < 32; ++l) sum += sm.len[sym * 32 + l] >> kEncCountShift;
+      if (sum) atomicAdd(&a.hist[sym], sum);
     }
   }
   if (!COMPLETE && __any_sync(0xffffffffu, uncodable) && lane == 0)
@@ -1652,7 +1658,7 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
                   // the single pass: u64 look[nchunks], then the u32 chunk counter
                   static_cast<uint64_t*>(d_scratch),
                   reinterpret_cast<uint32_t*>(static_cast<uint64_t*>(d_scratch) + nchunks),
-                  kDefaultWaitNs, ~0ull};
+                  kDefaultWaitNs, ~0ull, kEncFlushRounds};
   return HX_OK;
 }
 
@@ -1682,7 +1688,7 @@ int launch_shannonic(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s
 int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                   void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
                   uint32_t* d_status, void* stream, uint64_t wait_ns = kDefaultWaitNs,
-                  uint64_t withhold = ~0ull) {
+                  uint64_t withhold = ~0ull, uint32_t flush = kEncFlushRounds) {
   EncodeArgs a;
   DeviceInfo info;
   const int rc = encode_args(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
@@ -1692,6 +1698,7 @@ int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint
   if (kind != HX_KIND_SHANNONIC) {
     a.wait_ns = wait_ns;
     a.withhold = withhold;
+    a.flush = flush;
     return launch_encode(a, info, s);
   }
   return launch_shannonic(a, info, s);
@@ -1822,10 +1829,11 @@ int hx_qlc_encode(const void* d_tables, const uint8_t* d_in, uint64_t n, void* d
 
 int hx_encode_bounded(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                       void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
-                      uint32_t* d_status, uint64_t wait_ns, uint64_t withhold, void* stream) {
-  if (kind == HX_KIND_SHANNONIC) return HX_ERR_ARG;
+                      uint32_t* d_status, uint64_t wait_ns, uint64_t withhold,
+                      uint32_t flush_rounds, void* stream) {
+  if (kind == HX_KIND_SHANNONIC || flush_rounds > kEncFlushRoundsMax) return HX_ERR_ARG;
   return encode_common(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
-                       stream, wait_ns, withhold);
+                       stream, wait_ns, withhold, flush_rounds ? flush_rounds : kEncFlushRounds);
 }
 
 int hx_decode(const void* d_tables, const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,

@@ -76,7 +76,7 @@ def lib():
             "hx_qlc_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
             "hx_qlc_decode": (i32, [P, P, u64, P, u64, P, P]),
             "hx_encode_noalloc": (i32, [P, P, u64, P, u64, P, P, P]),
-            "hx_encode_bounded": (i32, [u32, P, P, u64, P, u64, P, P, P, u64, u64, P]),
+            "hx_encode_bounded": (i32, [u32, P, P, u64, P, u64, P, P, P, u64, u64, u32, P]),
             "hx_shannonic_build": (i32, [P, i32, u32, CB]),
             "hx_expgolomb_build": (i32, [i32, i32, CB]),
             "hx_expgolomb_encode": (i32, [P, P, u64, P, u64, P, P, P, P]),
@@ -314,9 +314,11 @@ def encode(tables, x, out=None, scratch=None, hist=None, status=None, kind: int 
 
 
 def encode_bounded(tables, x, out, scratch, wait_ns: int, withhold: int = (1 << 64) - 1,
-                   hist=None, status=None, kind: int = KIND_HUFFMAN):
+                   hist=None, status=None, kind: int = KIND_HUFFMAN, flush_rounds: int = 0):
     """hx_encode_bounded: encode() with the chunks' wait limit in nanoseconds and, for failure
-    tests, one chunk (`withhold`) that never publishes its word count. Returns (out, status)."""
+    tests, one chunk (`withhold`) that never publishes its word count; `flush_rounds` is the
+    chunks a warp codes between its flushes of the fused histogram (0: the default). Returns
+    (out, status)."""
     x = _dev_u8(x, "x")
     out = _dev_u8(out, "out")
     if status is None:
@@ -324,7 +326,8 @@ def encode_bounded(tables, x, out, scratch, wait_ns: int, withhold: int = (1 << 
     _check(lib().hx_encode_bounded(kind, tables.data_ptr(), x.data_ptr(), x.numel(),
                                    out.data_ptr(), out.numel(), scratch.data_ptr(),
                                    hist.data_ptr() if hist is not None else None,
-                                   status.data_ptr(), int(wait_ns), int(withhold), _stream(x)),
+                                   status.data_ptr(), int(wait_ns), int(withhold),
+                                   int(flush_rounds), _stream(x)),
            "hx_encode_bounded")
     return out, status
 

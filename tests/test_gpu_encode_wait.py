@@ -1,4 +1,5 @@
-"""The single-pass encoder's bounded wait (failure detection without a GPU fault).
+"""The single-pass encoder's bounded wait (failure detection without a GPU fault), and the other
+knob hx_encode_bounded exposes, the fused histogram's flush interval.
 
 Each chunk learns its word offset from the chunks before it. A chunk that never publishes its
 word count (the `withhold` argument of hx_encode_bounded) makes every later chunk's wait run out:
@@ -64,3 +65,21 @@ def test_generous_limit_and_no_withheld_chunk_equals_oracle(setup):
     torch.cuda.synchronize()
     ref = orc.encode(ocb, x)[1]
     assert int(st.item()) == 0 and (out[:ref.size].cpu().numpy() == ref).all()
+
+
+@pytest.mark.parametrize("flush_rounds", [1, 2])
+def test_fused_histogram_flushed_every_chunk(setup, flush_rounds):
+    """Each warp clears the shared counts into the histogram after every (or every second) chunk
+    it codes, while the other warps keep counting: the histogram and the stream still equal the
+    oracle's."""
+    orc, tables, ocb = setup
+    n = (1 << 24) + 777
+    x = datagen.data(4, n=n)
+    out, scratch = _buffers(n)
+    hist = torch.zeros(256, dtype=torch.int32, device="cuda")
+    _, st = hx.encode_bounded(tables, torch.from_numpy(x).cuda(), out, scratch, wait_ns=10 ** 9,
+                              hist=hist, flush_rounds=flush_rounds)
+    torch.cuda.synchronize()
+    ref = orc.encode(ocb, x)[1]
+    assert int(st.item()) == 0 and (out[:ref.size].cpu().numpy() == ref).all()
+    assert (hist.cpu().numpy().astype(np.uint64) == orc.histogram(x)).all()
