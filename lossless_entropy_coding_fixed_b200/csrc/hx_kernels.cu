@@ -15,8 +15,8 @@
 //                and the chunk's word count, which it publishes at once; the coding pass joins two
 //                codes per 32-bit register, appends them to a 64-bit accumulator and ORs each
 //                finished word into the warp's chunk buffer; a decoupled look-back over the
-//                chunks before it (bounded wait) gives the chunk's word offset, and the chunk
-//                leaves with coalesced stores.
+//                chunks before it (64 per round trip to L2, bounded wait) gives the chunk's word
+//                offset, and the chunk leaves with coalesced stores.
 //
 //   k_decode     one thread per sub-stream (8 per chunk, 128 chunks per 1024-thread block). The
 //                two payload words in use and a bit offset into them give the next 32 bits with
