@@ -792,18 +792,46 @@ constexpr uint32_t kReaderReach16 = 4 * (1 + kReaderPulls16 / 4);
 constexpr uint32_t kCrowdedReaders = 16;
 
 // The decode table in shared memory: for every 12-bit window, (symbol << 8) | hx::kDecValid |
-// length of the code word it starts with; 0 when none does (an incomplete code).
-struct DecLut {
+// length of the code word it starts with; 0 when none does (an incomplete code). A warp's 32
+// lookups hit random banks, about 3.8 wavefronts per lookup. For QLC and Exp-Golomb codes, whose
+// few distinct lengths make the windows of a warp crowd more, the table is held 8 times, copy k
+// confined to banks 4k .. 4k + 3 and read by lanes 4k .. 4k + 3, so only 4 lanes can meet in a
+// bank (measured: QLC 0.922 -> 0.909 ms per GiB, Exp-Golomb 1.12 -> 0.95 ms; Huffman codes lose
+// 2 % to the longer address arithmetic and the L1 the copies take, and keep the one table).
+template <int COPIES>
+struct DecLut;
+template <>
+struct DecLut<1> {
   const uint16_t* full;
   __device__ __forceinline__ uint32_t operator()(uint32_t x) const { return full[x >> 20]; }
 };
+template <>
+struct DecLut<8> {
+  // entry i of copy k at byte ((i >> 3) << 7) + (k << 4) + ((i & 7) << 1): each 128-byte row holds
+  // 8 entries of every copy; `base` is the table's shared address + 16 * (lane / 4)
+  uint32_t base;
+  __device__ __forceinline__ uint32_t operator()(uint32_t x) const {
+    const uint32_t a = base + ((x >> 23) << 7) + ((x >> 19) & 14u);
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+  }
+};
+template <int KIND>
+__host__ __device__ constexpr int dec_copies() {
+  return KIND == HX_KIND_HUFFMAN ? 1 : 8;
+}
+// dynamic shared memory of the decoder of a kind (the one-table decoder's table is static)
+constexpr size_t dec_lut_bytes(uint32_t kind) {
+  return kind == HX_KIND_HUFFMAN ? 0 : 8 * 4096 * 2;
+}
 
 // Two symbols from the reader: table entries (symbol << 8) | kDecValid | length for either kind
 // (for a QLC table the length is 3 + the width of the area in the top 3 bits; the table holds it
 // already). An entry of 0 (no code word starts the window) only occurs for an incomplete code:
 // `valid` is the AND of the entries used, so its kDecValid bit ends up clear if any was 0.
-template <bool COMPLETE, class Reader>
-__device__ __forceinline__ void decode_pair(Reader& rd, uint32_t& valid, const DecLut& lut,
+template <bool COMPLETE, class Reader, class Lut>
+__device__ __forceinline__ void decode_pair(Reader& rd, uint32_t& valid, const Lut& lut,
                                             uint32_t& e1, uint32_t& e2) {
   const uint32_t x = rd.peek();
   e1 = lut(x);
@@ -816,9 +844,9 @@ __device__ __forceinline__ void decode_pair(Reader& rd, uint32_t& valid, const D
 
 // 32 symbols -> 32 output bytes, one 32-byte streaming store (a whole sector) when the output is
 // 32-byte aligned, else two 16-byte stores. The symbol bytes are gathered with byte permutes.
-template <bool COMPLETE, class Reader>
+template <bool COMPLETE, class Reader, class Lut>
 __device__ __forceinline__ void decode_group32(Reader& rd, uint32_t& valid, uint8_t* dst,
-                                               bool out32, const DecLut& lut) {
+                                               bool out32, const Lut& lut) {
   uint32_t o[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
@@ -840,10 +868,10 @@ __device__ __forceinline__ void decode_group32(Reader& rd, uint32_t& valid, uint
 
 // Decodes `mine` symbols of one sub-stream from a started reader to dst; returns the reader's
 // final bit position. Sets *invalid when a window started no code word.
-template <bool COMPLETE, class Reader>
+template <bool COMPLETE, class Reader, class Lut>
 __device__ __forceinline__ uint64_t decode_substream(Reader& rd, uint32_t mine, uint8_t* dst,
                                                      bool out32, bool& invalid,
-                                                     const DecLut& lut) {
+                                                     const Lut& lut) {
   uint32_t valid = hx::kDecValid;
   const uint32_t groups = mine / 32;
   for (uint32_t g = 0; g < groups; ++g)
@@ -861,8 +889,8 @@ __device__ __forceinline__ uint64_t decode_substream(Reader& rd, uint32_t mine, 
 // The block's chunks in a grid-stride loop, 8 lanes per chunk (one per sub-stream). COMPLETE:
 // every window starts a code word, so no entry is checked. VOTE: the block's first chunk looked
 // crowded (crowded_chunk), so the lanes about to decode vote on the 16-byte reader.
-template <int THREADS, bool COMPLETE, bool VOTE>
-__device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const DecLut& lut,
+template <int THREADS, bool COMPLETE, bool VOTE, class Lut>
+__device__ __forceinline__ void decode_chunks(const DecodeArgs& a, const Lut& lut,
                                               uint32_t total) {
   const int tid = threadIdx.x;
   const uint64_t n = a.n;
@@ -959,7 +987,9 @@ __device__ bool crowded_chunk(const DecodeArgs& a, uint64_t c) {
 // (decode_common picks).
 template <int KIND, int THREADS>
 __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a) {
-  __shared__ __align__(16) uint16_t s_lut[4096];
+  constexpr int kCopies = dec_copies<KIND>();
+  __shared__ __align__(16) uint16_t s_lut[kCopies == 1 ? 4096 : 8];
+  extern __shared__ __align__(16) uint16_t s_lut_copies[];  // dec_lut_bytes(KIND) bytes
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
   __shared__ bool s_crowded;
@@ -977,11 +1007,20 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a
     return;
   }
   const hx::Tables* tables = s_tables;
-  const uint4* src = reinterpret_cast<const uint4*>(tables->dec);
-  uint4* dst = reinterpret_cast<uint4*>(s_lut);
-  for (int i = tid; i < 4096 * 2 / 16; i += THREADS) dst[i] = src[i];
+  DecLut<kCopies> lut;
+  if constexpr (kCopies == 1) {
+    const uint4* src = reinterpret_cast<const uint4*>(tables->dec);
+    uint4* dst = reinterpret_cast<uint4*>(s_lut);
+    for (int i = tid; i < 4096 * 2 / 16; i += THREADS) dst[i] = src[i];
+    lut.full = s_lut;
+  } else {
+    for (int j = tid; j < 8 * 4096; j += THREADS) {
+      const int i = j >> 3, k = j & 7;
+      s_lut_copies[(((i >> 3) << 7) + (k << 4) + ((i & 7) << 1)) >> 1] = tables->dec[i];
+    }
+    lut.base = (uint32_t)__cvta_generic_to_shared(s_lut_copies) + 16u * ((tid & 31) >> 2);
+  }
   __syncthreads();
-  const DecLut lut{s_lut};
   const bool crowded = s_crowded;
   if (tables->complete) {
     if (crowded) decode_chunks<THREADS, true, true>(a, lut, (uint32_t)total);
@@ -1539,7 +1578,9 @@ struct DeviceInfo {
   int sms = 0;
   int hist_per_sm = 0;
   int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0;
-  int dec_per_sm[3] = {0, 0, 0};  // prefix-code decode blocks per SM at 1024, 256, 64 threads
+  // prefix-code decode blocks per SM at 1024, 256, 64 threads: [0] with one table (Huffman),
+  // [1] with the 8 bank-confined copies (QLC, Exp-Golomb)
+  int dec_per_sm[2][3] = {{0, 0, 0}, {0, 0, 0}};
   int enc_per_sm = 0;
 };
 
@@ -1579,12 +1620,22 @@ bool device_info(DeviceInfo* out) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return false;
-    for (int i = 0; i < 3; ++i)
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-              &d.dec_per_sm[i], reinterpret_cast<const void*>(prefix_decoder(HX_KIND_HUFFMAN, i)),
-              kDecodeBlock[i], 0) != cudaSuccess ||
-          d.dec_per_sm[i] < 1)
-        return false;
+    for (uint32_t kind : {HX_KIND_HUFFMAN, HX_KIND_QLC, HX_KIND_EXPGOLOMB})
+      for (int i = 0; i < 3; ++i)
+        if (dec_lut_bytes(kind) &&
+            cudaFuncSetAttribute(reinterpret_cast<const void*>(prefix_decoder(kind, i)),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dec_lut_bytes(kind)) != cudaSuccess)
+          return false;
+    for (int l = 0; l < 2; ++l) {
+      const uint32_t kind = l == 0 ? HX_KIND_HUFFMAN : HX_KIND_QLC;
+      for (int i = 0; i < 3; ++i)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                &d.dec_per_sm[l][i], reinterpret_cast<const void*>(prefix_decoder(kind, i)),
+                kDecodeBlock[i], dec_lut_bytes(kind)) != cudaSuccess ||
+            d.dec_per_sm[l][i] < 1)
+          return false;
+    }
     if (
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
                                                       0) != cudaSuccess ||
@@ -1614,7 +1665,8 @@ bool device_info(DeviceInfo* out) {
     for (uint32_t kind : {HX_KIND_HUFFMAN, HX_KIND_QLC, HX_KIND_EXPGOLOMB})
       for (int i = 0; i < 3; ++i)
         if (!prefer_l1(dev, reinterpret_cast<const void*>(prefix_decoder(kind, i)),
-                       d.dec_per_sm[i], kDecodeBlock[i], 0))
+                       d.dec_per_sm[dec_lut_bytes(kind) ? 1 : 0][i], kDecodeBlock[i],
+                       dec_lut_bytes(kind)))
           return false;
     d.sms = sms;
   }
@@ -1724,7 +1776,8 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   if (nchunks >= (uint64_t)info.sms * 64) bi = 0;
   else if (nchunks >= (uint64_t)info.sms * 16) bi = 1;
   const int threads = kind == HX_KIND_SHANNONIC ? kDecThreads : kDecodeBlock[bi];
-  const int per_sm = kind == HX_KIND_SHANNONIC ? info.sh_decode_per_sm : info.dec_per_sm[bi];
+  const int per_sm = kind == HX_KIND_SHANNONIC ? info.sh_decode_per_sm
+                                               : info.dec_per_sm[dec_lut_bytes(kind) ? 1 : 0][bi];
   const uint64_t per_block = threads / 8;
   const uint64_t want = (nchunks + per_block - 1) / per_block;
   const uint32_t grid =
@@ -1741,7 +1794,7 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   if (kind == HX_KIND_SHANNONIC)
     k_sh_decode<<<grid, kDecThreads, 0, s>>>(a);
   else
-    prefix_decoder(kind, bi)<<<grid, threads, 0, s>>>(a);
+    prefix_decoder(kind, bi)<<<grid, threads, dec_lut_bytes(kind), s>>>(a);
   return launched();
 }
 
