@@ -796,7 +796,7 @@ constexpr uint32_t kCrowdedReaders = 16;
 // lookups hit random banks, about 3.8 wavefronts per lookup. For QLC and Exp-Golomb codes, whose
 // few distinct lengths make the windows of a warp crowd more, the table is held 8 times, copy k
 // confined to banks 4k .. 4k + 3 and read by lanes 4k .. 4k + 3, so only 4 lanes can meet in a
-// bank (measured: QLC 0.922 -> 0.909 ms per GiB, Exp-Golomb 1.12 -> 0.95 ms; Huffman codes lose
+// bank (measured: QLC 0.918 -> 0.895 ms per GiB, Exp-Golomb 1.12 -> 0.94 ms; Huffman codes lose
 // 2 % to the longer address arithmetic and the L1 the copies take, and keep the one table).
 template <int COPIES>
 struct DecLut;
@@ -817,13 +817,16 @@ struct DecLut<8> {
     return v;
   }
 };
-template <int KIND>
+// The copies go to the blocks of 1024 threads (large inputs); the smaller blocks of small inputs
+// would spend more on filling 64 KB than the lookups gain (1 MiB of QLC: 28.8 -> 32.8 us).
+template <int KIND, int THREADS>
 __host__ __device__ constexpr int dec_copies() {
-  return KIND == HX_KIND_HUFFMAN ? 1 : 8;
+  return KIND == HX_KIND_HUFFMAN || THREADS != 1024 ? 1 : 8;
 }
-// dynamic shared memory of the decoder of a kind (the one-table decoder's table is static)
-constexpr size_t dec_lut_bytes(uint32_t kind) {
-  return kind == HX_KIND_HUFFMAN ? 0 : 8 * 4096 * 2;
+// dynamic shared memory of the decoder of a kind at block size index i (the one-table decoder's
+// table is static)
+constexpr size_t dec_lut_bytes(uint32_t kind, int i) {
+  return kind == HX_KIND_HUFFMAN || i != 0 ? 0 : 8 * 4096 * 2;
 }
 
 // Two symbols from the reader: table entries (symbol << 8) | kDecValid | length for either kind
@@ -987,9 +990,9 @@ __device__ bool crowded_chunk(const DecodeArgs& a, uint64_t c) {
 // (decode_common picks).
 template <int KIND, int THREADS>
 __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a) {
-  constexpr int kCopies = dec_copies<KIND>();
+  constexpr int kCopies = dec_copies<KIND, THREADS>();
   __shared__ __align__(16) uint16_t s_lut[kCopies == 1 ? 4096 : 8];
-  extern __shared__ __align__(16) uint16_t s_lut_copies[];  // dec_lut_bytes(KIND) bytes
+  extern __shared__ __align__(16) uint16_t s_lut_copies[];  // dec_lut_bytes(KIND, .) bytes
   __shared__ int64_t s_total;
   __shared__ const hx::Tables* s_tables;
   __shared__ bool s_crowded;
@@ -1014,9 +1017,14 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a
     for (int i = tid; i < 4096 * 2 / 16; i += THREADS) dst[i] = src[i];
     lut.full = s_lut;
   } else {
-    for (int j = tid; j < 8 * 4096; j += THREADS) {
-      const int i = j >> 3, k = j & 7;
-      s_lut_copies[(((i >> 3) << 7) + (k << 4) + ((i & 7) << 1)) >> 1] = tables->dec[i];
+    // entries 8r .. 8r + 7 fill bytes 16k .. 16k + 15 of row r in every copy k: one 16-byte load,
+    // eight 16-byte stores
+    const uint4* src = reinterpret_cast<const uint4*>(tables->dec);
+    uint4* dst = reinterpret_cast<uint4*>(s_lut_copies);
+    for (int r = tid; r < 4096 / 8; r += THREADS) {
+      const uint4 v = src[r];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) dst[8 * r + k] = v;
     }
     lut.base = (uint32_t)__cvta_generic_to_shared(s_lut_copies) + 16u * ((tid & 31) >> 2);
   }
@@ -1578,8 +1586,8 @@ struct DeviceInfo {
   int sms = 0;
   int hist_per_sm = 0;
   int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0;
-  // prefix-code decode blocks per SM at 1024, 256, 64 threads: [0] with one table (Huffman),
-  // [1] with the 8 bank-confined copies (QLC, Exp-Golomb)
+  // prefix-code decode blocks per SM at 1024, 256, 64 threads: [0] Huffman, [1] QLC and
+  // Exp-Golomb (whose 1024-thread blocks hold the 8 bank-confined table copies)
   int dec_per_sm[2][3] = {{0, 0, 0}, {0, 0, 0}};
   int enc_per_sm = 0;
 };
@@ -1622,17 +1630,17 @@ bool device_info(DeviceInfo* out) {
       return false;
     for (uint32_t kind : {HX_KIND_HUFFMAN, HX_KIND_QLC, HX_KIND_EXPGOLOMB})
       for (int i = 0; i < 3; ++i)
-        if (dec_lut_bytes(kind) &&
+        if (dec_lut_bytes(kind, i) &&
             cudaFuncSetAttribute(reinterpret_cast<const void*>(prefix_decoder(kind, i)),
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)dec_lut_bytes(kind)) != cudaSuccess)
+                                 (int)dec_lut_bytes(kind, i)) != cudaSuccess)
           return false;
     for (int l = 0; l < 2; ++l) {
       const uint32_t kind = l == 0 ? HX_KIND_HUFFMAN : HX_KIND_QLC;
       for (int i = 0; i < 3; ++i)
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
                 &d.dec_per_sm[l][i], reinterpret_cast<const void*>(prefix_decoder(kind, i)),
-                kDecodeBlock[i], dec_lut_bytes(kind)) != cudaSuccess ||
+                kDecodeBlock[i], dec_lut_bytes(kind, i)) != cudaSuccess ||
             d.dec_per_sm[l][i] < 1)
           return false;
     }
@@ -1665,8 +1673,8 @@ bool device_info(DeviceInfo* out) {
     for (uint32_t kind : {HX_KIND_HUFFMAN, HX_KIND_QLC, HX_KIND_EXPGOLOMB})
       for (int i = 0; i < 3; ++i)
         if (!prefer_l1(dev, reinterpret_cast<const void*>(prefix_decoder(kind, i)),
-                       d.dec_per_sm[dec_lut_bytes(kind) ? 1 : 0][i], kDecodeBlock[i],
-                       dec_lut_bytes(kind)))
+                       d.dec_per_sm[kind == HX_KIND_HUFFMAN ? 0 : 1][i], kDecodeBlock[i],
+                       dec_lut_bytes(kind, i)))
           return false;
     d.sms = sms;
   }
@@ -1777,7 +1785,7 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   else if (nchunks >= (uint64_t)info.sms * 16) bi = 1;
   const int threads = kind == HX_KIND_SHANNONIC ? kDecThreads : kDecodeBlock[bi];
   const int per_sm = kind == HX_KIND_SHANNONIC ? info.sh_decode_per_sm
-                                               : info.dec_per_sm[dec_lut_bytes(kind) ? 1 : 0][bi];
+                                               : info.dec_per_sm[kind == HX_KIND_HUFFMAN ? 0 : 1][bi];
   const uint64_t per_block = threads / 8;
   const uint64_t want = (nchunks + per_block - 1) / per_block;
   const uint32_t grid =
@@ -1794,7 +1802,7 @@ int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const 
   if (kind == HX_KIND_SHANNONIC)
     k_sh_decode<<<grid, kDecThreads, 0, s>>>(a);
   else
-    prefix_decoder(kind, bi)<<<grid, threads, dec_lut_bytes(kind), s>>>(a);
+    prefix_decoder(kind, bi)<<<grid, threads, dec_lut_bytes(kind, bi), s>>>(a);
   return launched();
 }
 
