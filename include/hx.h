@@ -203,17 +203,18 @@ int hx_decode_set(uint32_t kind, const void* const* d_tables, uint32_t n_tables,
                   const void* d_stream, uint64_t stream_bytes, uint8_t* d_out,
                   uint64_t n_expected, uint32_t* d_status, void* stream);
 
-/* hx_encode (and hx_qlc_encode, hx_expgolomb_encode) with its bounded wait exposed, for
- * failure-detection tests; the pages have no counterpart (they describe no GPU encoder). The
- * encoder reads its input once: each chunk publishes its word count as soon as it has measured
- * it, and learns its word offset from the chunks before it (they are always running, so the wait
- * ends). Every such wait is still bounded: after wait_ns nanoseconds (hx_encode uses 2 s) the
- * chunk raises HX_ERR_TIMEOUT in *d_status and writes no payload, and every chunk still waiting
- * gives up at once; the kernel completes and the context stays usable. withhold: a chunk that
- * never publishes its count (UINT64_MAX: none), so that the chunks after it time out.
- * flush_rounds: with d_hist, the chunks a warp codes between its flushes of the fused counts into
- * d_hist (0: the 128 of hx_encode; at most 4096, else HX_ERR_ARG), so that a test can make the
- * flush run often. kind 0, 1 or 3 (HX_ERR_ARG for kind 2); other arguments and errors as
+/* hx_encode (and hx_qlc_encode, hx_expgolomb_encode, hx_shannonic_encode) with its bounded wait
+ * exposed, for failure-detection tests; the pages have no counterpart (they describe no GPU
+ * encoder). The encoder reads its input once: each chunk (kind 2: each group of 4 chunks)
+ * publishes its word count as soon as it has measured it, and learns its word offset from the
+ * ones before it (they are always running, so the wait ends). Every such wait is still bounded:
+ * after wait_ns nanoseconds (hx_encode uses 2 s) the chunk raises HX_ERR_TIMEOUT in *d_status and
+ * writes no payload, and every chunk still waiting gives up at once; the kernel completes and the
+ * context stays usable. withhold: a chunk (kind 2: a group) that never publishes its count
+ * (UINT64_MAX: none), so that the ones after it time out. flush_rounds: with d_hist and kinds 0,
+ * 1, 3, the chunks a warp codes between its flushes of the fused counts into d_hist (0: the 128
+ * of hx_encode; at most 4096, else HX_ERR_ARG), so that a test can make the flush run often;
+ * kind 2 counts into 32-bit tables per warp and flushes once. Other arguments and errors as
  * hx_encode. */
 int hx_encode_bounded(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64_t n,
                       void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,

@@ -110,24 +110,19 @@ __global__ void __launch_bounds__(kHistThreads) k_histogram(const uint8_t* __res
 }
 
 // ---------------------------------------------------------------------------------- encode
-// The arguments of an encode: k_encode (kinds 0, 1, 3) reads the look-back fields, the Shannonic
-// passes (kind 2) the measure-block fields.
+// The arguments of an encode (k_encode for kinds 0, 1, 3; k_sh_encode for kind 2, whose
+// look-back unit is a group of 4 chunks).
 struct EncodeArgs {
   const hx::Tables* tables;
   const uint8_t* in;
   uint64_t n;
   uint8_t* out;
   uint64_t cap;
-  uint32_t* local;   // Shannonic scratch: block-local word offset of every chunk
-  uint32_t* btotal;  // Shannonic scratch: words of each measure block
-  uint32_t mblocks;  // Shannonic measure blocks
-  uint32_t cpb;      // chunks per Shannonic measure block
-  uint32_t* hist;    // optional fused histogram
+  uint32_t* hist;  // optional fused histogram
   uint32_t* status;
   uint32_t kind;
-  // single-pass encoder (k_encode)
-  uint64_t* look;     // scratch: each chunk's published word count or word offset (zeroed)
-  uint32_t* counter;  // scratch: next chunk to take (zeroed)
+  uint64_t* look;     // scratch: each chunk's (group's) published word count or offset (zeroed)
+  uint32_t* counter;  // scratch: next chunk (group) to take (zeroed)
   uint64_t wait_ns;   // limit of one chunk's wait for its predecessors
   uint64_t withhold;  // a chunk that publishes nothing (failure tests), else ~0
   uint32_t flush;     // fused histogram: a warp's chunks between its flushes of the counts
@@ -181,43 +176,6 @@ __device__ __forceinline__ uint32_t load16(const EncodeArgs& a, uint32_t c, uint
   return valid;
 }
 
-// Exclusive scan of cnt[0..m) in place with the whole block (m <= 16 * blockDim.x); returns the
-// sum. `red` holds one word per warp.
-template <int THREADS>
-__device__ uint32_t block_exclusive_scan(uint32_t* cnt, uint32_t m, uint32_t* red) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t seg = (m + THREADS - 1) / THREADS;
-  const uint32_t lo = min(m, tid * seg), hi = min(m, lo + seg);
-  uint32_t s = 0;
-  for (uint32_t i = lo; i < hi; ++i) s += cnt[i];
-  uint32_t incl = s;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d);
-    if (lane >= d) incl += t;
-  }
-  if (lane == 31) red[warp] = incl;
-  __syncthreads();
-  uint32_t before = 0, total = 0;
-#pragma unroll
-  for (int w = 0; w < THREADS / 32; ++w) {
-    const uint32_t r = red[w];
-    before += w < warp ? r : 0u;
-    total += r;
-  }
-  uint32_t run = before + incl - s;
-  for (uint32_t i = lo; i < hi; ++i) {
-    const uint32_t v = cnt[i];
-    cnt[i] = run;
-    run += v;
-  }
-  __syncthreads();
-  return total;
-}
-
-// Limits of the Shannonic coder's measure blocks (the two-pass encoder of kind 2).
-constexpr uint32_t kMaxChunksPerBlock = 1024;  // chunks of one measure block
-constexpr uint32_t kMaxMeasureBlocks = 2048;
 constexpr uint32_t kMaxChunkWords = HX_CHUNK * HX_LMAX_MAX / 32;  // 1536: a chunk's largest size
 
 // ---------------------------------------------------------------------------------- encode, one pass
@@ -1043,32 +1001,24 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a
 // The review page's range-partitioned coder: a byte's range index is coded by tANS with 128
 // states (the table variant of asymmetric numeral systems), its offset inside the range in
 // ceil(log2 size) bits. tANS runs from a sub-stream's last symbol to its first, so its bit count
-// is known only after the whole sub-stream has been run: the encoder's first pass runs it to
-// count (k_sh_measure, two sub-streams per thread), the second runs it again and writes
-// (k_sh_pack, one per thread, as in the decoder, k_sh_decode, which reads each sub-stream
-// backwards).
+// is known only after the whole sub-stream has been run: the encoder (k_sh_encode) parks each
+// sub-stream's bits in shared memory until the offsets before it are known. The decoder,
+// k_sh_decode, reads each sub-stream backwards.
 
-constexpr int kShThreads = 256;  // pack and decode: 8 threads per chunk, 32 chunks per block
-constexpr int kShCopies = 16;    // symbol table copies: lane l reads copy l % 16 (<= 2-way)
+constexpr int kShCopies = 16;  // symbol table copies: lane l reads copy l % 16 (<= 2-way)
 
 // Encoder tables in shared memory: per byte value [byte][copy] the step's fields (sh_sym) and,
-// at a fixed distance, its offset in its range (sh_off); the ranges' states (sh_enc). The
-// measure pass needs no offsets (ShCount).
+// at a fixed distance, its offset in its range (sh_off); the ranges' states (sh_enc).
 struct ShEnc {
   uint32_t sym[256 * kShCopies];
   uint32_t off[256 * kShCopies];
   uint8_t enc[128];
 };
-struct ShCount {
-  uint32_t sym[256 * kShCopies];
-  uint8_t enc[128];
-};
 
-template <class T>
-__device__ __forceinline__ void sh_load_tables(const hx::Tables* t, T& s) {
+__device__ __forceinline__ void sh_load_tables(const hx::Tables* t, ShEnc& s) {
   for (int i = threadIdx.x; i < 256 * kShCopies; i += blockDim.x) {
     s.sym[i] = t->sh_sym[i / kShCopies];
-    if constexpr (sizeof(T) == sizeof(ShEnc)) s.off[i] = t->sh_off[i / kShCopies];
+    s.off[i] = t->sh_off[i / kShCopies];
   }
   for (int i = threadIdx.x; i < 128; i += blockDim.x) s.enc[i] = t->sh_enc[i];
 }
@@ -1085,8 +1035,7 @@ struct ShLane {
   uint32_t sym, enc;
 };
 constexpr uint32_t kOffDist = 4 * 256 * kShCopies;
-template <class T>
-__device__ __forceinline__ ShLane sh_lane(const T& s, uint32_t lane) {
+__device__ __forceinline__ ShLane sh_lane(const ShEnc& s, uint32_t lane) {
   return {(uint32_t)__cvta_generic_to_shared(s.sym) + 4 * (lane % kShCopies),
           (uint32_t)__cvta_generic_to_shared(s.enc) - 128u};
 }
@@ -1110,144 +1059,17 @@ __device__ __forceinline__ uint32_t sh_value(uint32_t e, uint32_t off, uint32_t 
   return __funnelshift_r((((off - hi) << len) + xo), 0u, e);
 }
 
-// Bytes of sub-stream k of chunk c, last first: calls fn(byte) for each.
-template <class Fn>
-__device__ __forceinline__ void sh_reverse(const EncodeArgs& a, uint32_t c, uint32_t k,
-                                           uint32_t m, Fn&& fn) {
-  const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
-  if (m == kSubLen) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.in + first);
-    uint4 nxt = __ldg(src + kSubLen / 16 - 1);
-#pragma unroll 1
-    for (int g = kSubLen / 16 - 1; g >= 0; --g) {
-      const uint4 v = nxt;
-      if (g > 0) nxt = __ldg(src + g - 1);
-      const uint32_t w[4] = {v.w, v.z, v.y, v.x};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        fn(w[q] >> 24);
-        fn((w[q] >> 16) & 0xffu);
-        fn((w[q] >> 8) & 0xffu);
-        fn(w[q] & 0xffu);
-      }
-    }
-  } else {
-    for (uint32_t i = m; i-- > 0;) fn((uint32_t)a.in[first + i]);
-  }
-}
-
 // Symbols in sub-stream k of chunk c (0 past the end of the input).
 __device__ __forceinline__ uint32_t sh_count(uint64_t n, uint32_t c, uint32_t k) {
   const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
   return first < n ? (uint32_t)min((uint64_t)kSubLen, n - first) : 0u;
 }
 
-struct ShMeasureSmem {
-  ShCount t;
-  uint32_t cnt[kMaxChunksPerBlock];
-  uint32_t red[kShThreads / 32];
-  uint32_t hist[kShThreads / 32][256];
-};
-
-__global__ void __launch_bounds__(kShThreads) k_sh_measure(EncodeArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  ShMeasureSmem& sm = *reinterpret_cast<ShMeasureSmem*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
-    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
-    return;
-  }
-  sh_load_tables(a.tables, sm.t);
-  const bool hist = a.hist != nullptr;
-  if (hist)
-    for (int i = tid; i < (kShThreads / 32) * 256; i += kShThreads) (&sm.hist[0][0])[i] = 0;
-  __syncthreads();
-  const ShLane tl = sh_lane(sm.t, lane);
-  const uint64_t n = a.n;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  const uint32_t c0 = blockIdx.x * a.cpb;
-  const uint32_t m_chunks = c0 < nchunks ? min(a.cpb, nchunks - c0) : 0u;
-  uint16_t* sync = reinterpret_cast<uint16_t*>(a.out + sync_offset(n));
-  // two sub-streams per thread, q and q + 4, their tANS chains interleaved (each step waits on
-  // the table load of the one before it)
-  const uint32_t q = tid & 3, slot = tid >> 2;
-  const uint32_t rounds = (m_chunks + 63) / 64;
-  for (uint32_t r = 0; r < rounds; ++r) {
-    const uint32_t i = r * 64 + slot;
-    const bool live = i < m_chunks;
-    const uint32_t c = c0 + (live ? i : 0);
-    const uint32_t m0 = live ? sh_count(n, c, q) : 0u, m1 = live ? sh_count(n, c, q + 4) : 0u;
-    uint32_t b0 = 0, b1 = 0;
-    auto step = [&](uint32_t s, uint32_t& x) -> uint32_t {
-      uint32_t xo, hi;
-      if (hist) atomicAdd(&sm.hist[warp][s], 1u);
-      return sh_next(lds_u32(tl.sym + s * (4 * kShCopies)), x, tl.enc, xo, hi);
-    };
-    if (m1 == kSubLen) {  // both whole
-      const uint4* s0 =
-          reinterpret_cast<const uint4*>(a.in + (uint64_t)c * kChunk + (uint64_t)q * kSubLen);
-      const uint4* s1 = s0 + 4 * kSubLen / 16;
-      uint4 n0 = __ldg(s0 + kSubLen / 16 - 1), n1 = __ldg(s1 + kSubLen / 16 - 1);
-      uint32_t x0 = 128, x1 = 128;
-#pragma unroll 1
-      for (int g = kSubLen / 16 - 1; g >= 0; --g) {
-        const uint4 v0 = n0, v1 = n1;
-        if (g > 0) {
-          n0 = __ldg(s0 + g - 1);
-          n1 = __ldg(s1 + g - 1);
-        }
-        const uint32_t w0[4] = {v0.w, v0.z, v0.y, v0.x}, w1[4] = {v1.w, v1.z, v1.y, v1.x};
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-#pragma unroll
-          for (int h = 3; h >= 0; --h) {
-            b0 += step(__byte_perm(w0[qq], 0u, 0x4440 + h), x0);
-            b1 += step(__byte_perm(w1[qq], 0u, 0x4440 + h), x1);
-          }
-        }
-      }
-    } else {
-      uint32_t x0 = 128, x1 = 128;
-      if (m0) sh_reverse(a, c, q, m0, [&](uint32_t s) { b0 += step(s, x0); });
-      if (m1) sh_reverse(a, c, q + 4, m1, [&](uint32_t s) { b1 += step(s, x1); });
-    }
-    if (m0) b0 += HX_SHN_R;  // the final states
-    if (m1) b1 += HX_SHN_R;
-    // the chunk's 8 sub-streams: sync offsets by prefix sums over its 4 threads
-    uint32_t i0 = b0, i1 = b1;
-#pragma unroll
-    for (int d = 1; d < 4; d <<= 1) {
-      const uint32_t t0 = __shfl_up_sync(0xffffffffu, i0, d, 4);
-      const uint32_t t1 = __shfl_up_sync(0xffffffffu, i1, d, 4);
-      if (q >= (uint32_t)d) {
-        i0 += t0;
-        i1 += t1;
-      }
-    }
-    const uint32_t tot0 = __shfl_sync(0xffffffffu, i0, 3, 4);
-    const uint32_t total = tot0 + __shfl_sync(0xffffffffu, i1, 3, 4);
-    if (live) {
-      sync[(uint64_t)c * HX_SUBSTREAMS + q] = (uint16_t)(q == 0 ? total : i0 - b0);
-      sync[(uint64_t)c * HX_SUBSTREAMS + q + 4] = (uint16_t)(tot0 + i1 - b1);
-      if (q == 0) sm.cnt[i] = (total + 31) >> 5;
-    }
-  }
-  __syncthreads();
-  const uint32_t total = block_exclusive_scan<kShThreads>(sm.cnt, m_chunks, sm.red);
-  for (uint32_t i = tid; i < m_chunks; i += kShThreads) a.local[c0 + i] = sm.cnt[i];
-  if (tid == 0) a.btotal[blockIdx.x] = total;
-  if (hist) {
-    __syncthreads();
-    for (int sym = tid; sym < 256; sym += kShThreads) {
-      uint32_t sum = 0;
-#pragma unroll
-      for (int w = 0; w < kShThreads / 32; ++w) sum += sm.hist[w][sym];
-      if (sum) atomicAdd(&a.hist[sym], sum);
-    }
-  }
+__device__ __forceinline__ void reds_add_u32(uint32_t a, uint32_t x) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(a), "r"(x) : "memory");
 }
 
-// Predicated global stores (no branch around them).
+// Predicated stores (no branch around them).
 __device__ __forceinline__ void st_global_if(bool p, uint32_t* a, uint32_t v) {
   asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q st.global.u32 [%0], %1;\n}"
                ::"l"(a), "r"(v), "r"((uint32_t)p) : "memory");
@@ -1257,136 +1079,280 @@ __device__ __forceinline__ void st_global_v4_if(bool p, uint32_t* a, uint4 v) {
       "{\n .reg .pred q;\n setp.ne.u32 q, %5, 0;\n @q st.global.v4.u32 [%0], {%1, %2, %3, %4};\n}"
       ::"l"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"((uint32_t)p) : "memory");
 }
+__device__ __forceinline__ void sts_if(bool p, uint32_t a, uint32_t v) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q st.shared.u32 [%0], %1;\n}"
+               ::"r"(a), "r"(v), "r"((uint32_t)p) : "memory");
+}
 
-struct ShPackSmem {
-  ShEnc t;
-  uint32_t bpre[kMaxMeasureBlocks];
-  uint32_t red[kShThreads / 32];
-};
-
-__global__ void __launch_bounds__(kShThreads) k_sh_pack(EncodeArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  ShPackSmem& sm = *reinterpret_cast<ShPackSmem*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31;
-  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) return;  // measure said so
-  const uint64_t n = a.n;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  const uint64_t P = payload_offset(n);
-  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
-  const uint16_t* sync = reinterpret_cast<const uint16_t*>(a.out + sync_offset(n));
-  uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
-  sh_load_tables(a.tables, sm.t);
-  for (uint32_t i = tid; i < a.mblocks; i += kShThreads) sm.bpre[i] = a.btotal[i];
-  __syncthreads();
-  const uint32_t total = block_exclusive_scan<kShThreads>(sm.bpre, a.mblocks, sm.red);
-  const bool fits = P + 4ull * ((uint64_t)total + 2) <= a.cap;
-  if (blockIdx.x == 0 && tid == 0) {
-    write_header(a);
-    reinterpret_cast<uint64_t*>(a.out)[4] = total;
-    word_off[nchunks] = total;
-    if (fits) {
-      payload[total] = 0;
-      payload[total + 1] = 0;
-    } else {
-      atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
-    }
-  }
-  if (!fits) {  // the index still, but no payload word
-    for (uint32_t c = blockIdx.x * kShThreads + tid; c < nchunks; c += gridDim.x * kShThreads)
-      word_off[c] = sm.bpre[c / a.cpb] + a.local[c];
-    return;
-  }
-  const ShLane tl = sh_lane(sm.t, lane);
-  const uint32_t k = tid & 7;
-  const uint32_t groups = (nchunks + 31) / 32;
-  for (uint32_t gi = blockIdx.x; gi < groups; gi += gridDim.x) {
-    const uint32_t c = gi * 32 + (tid >> 3);
-    const bool live = c < nchunks;
-    const uint32_t m = live ? sh_count(n, c, k) : 0u;
-    uint32_t widx = 0, nacc = 0, tail = 0;
-    bool last = false;
-    if (live) {
-      const uint32_t woff = sm.bpre[c / a.cpb] + a.local[c];
-      if (k == 0) word_off[c] = woff;
-      const uint16_t* row = sync + (uint64_t)c * HX_SUBSTREAMS;
-      const uint32_t chunk_bits = row[0];
-      const uint32_t s = k == 0 ? 0u : row[k];
-      const uint32_t e = k + 1 < HX_SUBSTREAMS ? row[k + 1] : chunk_bits;
-      last = m != 0 && e == chunk_bits;
-      widx = woff + (s >> 5);
-      nacc = s & 31;  // the first bits belong to earlier sub-streams (zeros here)
-      uint32_t hi = 0, lo = 0;
-      // Finished words leave in aligned groups of 4 (one 16-byte store; q0..q2 hold the three
-      // words before the current one), those before the sub-stream's first whole group one by one.
-      const uint32_t gfirst = (widx + 3) & ~3u;
-      uint32_t q0 = 0, q1 = 0, q2 = 0;
-      // appends len (<= 30) bits
-      auto put = [&](uint32_t value, uint32_t len) {
-        hi = __funnelshift_l(lo, hi, len);
-        lo = (lo << len) | value;
-        nacc += len;
-        const bool full = nacc >= 32;
-        nacc -= full ? 32u : 0u;
-        const uint32_t w = __funnelshift_r(lo, hi, nacc);
-        st_global_if(full && widx < gfirst, payload + widx, w);
-        st_global_v4_if(full && widx >= gfirst && (widx & 3) == 3, payload + widx - 3,
-                        make_uint4(q0, q1, q2, w));
-        q0 = full ? q1 : q0;
-        q1 = full ? q2 : q1;
-        q2 = full ? w : q2;
-        widx += full ? 1u : 0u;
-      };
-      uint32_t state = 128;
-      // the bits of byte `sym` (as sh_value) and their count
-      auto code = [&](uint32_t sym, uint32_t& len) -> uint32_t {
-        const uint32_t ea = tl.sym + sym * (4 * kShCopies);
-        const uint32_t e = lds_u32(ea), off = lds_u32(ea + kOffDist);
-        uint32_t xo, xh;
-        len = sh_next(e, state, tl.enc, xo, xh);
-        return sh_value(e, off, xo, xh, len);
-      };
-      if (m == kSubLen) {
-        // whole sub-stream: 16 bytes at a time from the end, two codes joined per append
-        const uint4* src = reinterpret_cast<const uint4*>(a.in + (uint64_t)c * kChunk +
-                                                          (uint64_t)k * kSubLen);
-        uint4 nxt = __ldg(src + kSubLen / 16 - 1);
+// Runs tANS over sub-stream k of chunk c (m symbols, from the last to the first) and hands its
+// bits to put(value, len): two codes joined per call (at most 30 bits), the final state last.
+// With HIST every byte is also counted at hist + 4 * byte (shared memory).
+template <bool HIST, class Put>
+__device__ __forceinline__ void sh_run(const EncodeArgs& a, const ShLane& tl, uint32_t c,
+                                       uint32_t k, uint32_t m, uint32_t hist, Put&& put) {
+  uint32_t state = 128;
+  // the bits of byte `sym` (as sh_value) and their count
+  auto code = [&](uint32_t sym, uint32_t& len) -> uint32_t {
+    if (HIST) reds_add_u32(hist + 4u * sym, 1u);
+    const uint32_t ea = tl.sym + sym * (4 * kShCopies);
+    const uint32_t e = lds_u32(ea), off = lds_u32(ea + kOffDist);
+    uint32_t xo, xh;
+    len = sh_next(e, state, tl.enc, xo, xh);
+    return sh_value(e, off, xo, xh, len);
+  };
+  if (m == kSubLen) {
+    // a whole sub-stream: 16 bytes at a time from the end, the next 16 already requested
+    const uint4* src =
+        reinterpret_cast<const uint4*>(a.in + (uint64_t)c * kChunk + (uint64_t)k * kSubLen);
+    uint4 nxt = __ldg(src + kSubLen / 16 - 1);
 #pragma unroll 1
-        for (int g = kSubLen / 16 - 1; g >= 0; --g) {
-          const uint4 v = nxt;
-          if (g > 0) nxt = __ldg(src + g - 1);
-          const uint32_t w[4] = {v.w, v.z, v.y, v.x};
+    for (int g = kSubLen / 16 - 1; g >= 0; --g) {
+      const uint4 v = nxt;
+      if (g > 0) nxt = __ldg(src + g - 1);
+      const uint32_t w[4] = {v.w, v.z, v.y, v.x};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 4; ++q) {
 #pragma unroll
-            for (int h = 3; h > 0; h -= 2) {
-              uint32_t l0, l1;
-              const uint32_t v0 = code(__byte_perm(w[q], 0u, 0x4440 + h), l0);
-              const uint32_t v1 = code(__byte_perm(w[q], 0u, 0x4440 + h - 1), l1);
-              put((v0 << l1) | v1, l0 + l1);
-            }
-          }
-        }
-      } else if (m) {
-        const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
-        for (uint32_t i = m; i-- > 0;) {
-          uint32_t l;
-          const uint32_t v = code((uint32_t)a.in[first + i], l);
-          put(v, l);
+        for (int h = 3; h > 0; h -= 2) {
+          uint32_t l0, l1;
+          const uint32_t v0 = code(__byte_perm(w[q], 0u, 0x4440 + h), l0);
+          const uint32_t v1 = code(__byte_perm(w[q], 0u, 0x4440 + h - 1), l1);
+          put((v0 << l1) | v1, l0 + l1);
         }
       }
-      if (m) put(state - 128u, HX_SHN_R);
-      // the finished words of the last, incomplete group
-      const uint32_t g = max(gfirst, widx & ~3u);
-      if (widx >= g + 1) payload[widx - 1] = q2;
-      if (widx >= g + 2) payload[widx - 2] = q1;
-      if (widx >= g + 3) payload[widx - 3] = q0;
-      tail = nacc ? lo << (32 - nacc) : 0u;
-      // the chunk's last word is stored whole (zero padding)
-      if (last && nacc) payload[widx] = tail;
+    }
+  } else if (m) {
+    const uint64_t first = (uint64_t)c * kChunk + (uint64_t)k * kSubLen;
+    for (uint32_t i = m; i-- > 0;) {
+      uint32_t l;
+      const uint32_t v = code((uint32_t)a.in[first + i], l);
+      put(v, l);
+    }
+  }
+  if (m) put(state - 128u, HX_SHN_R);
+}
+
+// Sub-stream k of chunk c (m > 0 symbols) coded again, straight into the payload: its bits start
+// at bit s of the chunk, whose first word is woff; `last` when it ends the chunk. Finished words
+// leave in aligned groups of 4 (one 16-byte store; q0..q2 hold the three words before the
+// current one), those before the sub-stream's first whole group one by one, the stores predicated
+// rather than branched around. The first word's earlier bits are stored as zeros; the last,
+// unfinished word is stored whole when it ends the chunk, else returned in `tail` at `widx` for
+// the caller to OR in once the sub-stream after it has stored that word.
+__device__ __noinline__ void sh_write_direct(const EncodeArgs& a, const ShLane& tl, uint32_t c,
+                                             uint32_t k, uint32_t m, uint32_t* payload,
+                                             uint32_t woff, uint32_t s, bool last,
+                                             uint32_t& widx, uint32_t& tail) {
+  widx = woff + (s >> 5);
+  uint32_t nacc = s & 31, hi = 0, lo = 0;
+  const uint32_t gfirst = (widx + 3) & ~3u;
+  uint32_t q0 = 0, q1 = 0, q2 = 0;
+  sh_run<false>(a, tl, c, k, m, 0u, [&](uint32_t value, uint32_t len) {
+    hi = __funnelshift_l(lo, hi, len);
+    lo = (lo << len) | value;
+    nacc += len;
+    const bool full = nacc >= 32;
+    nacc -= full ? 32u : 0u;
+    const uint32_t w = __funnelshift_r(lo, hi, nacc);
+    st_global_if(full && widx < gfirst, payload + widx, w);
+    st_global_v4_if(full && widx >= gfirst && (widx & 3) == 3, payload + widx - 3,
+                    make_uint4(q0, q1, q2, w));
+    q0 = full ? q1 : q0;
+    q1 = full ? q2 : q1;
+    q2 = full ? w : q2;
+    widx += full ? 1u : 0u;
+  });
+  // the finished words of the last, incomplete group
+  const uint32_t g = max(gfirst, widx & ~3u);
+  if (widx >= g + 1) payload[widx - 1] = q2;
+  if (widx >= g + 2) payload[widx - 2] = q1;
+  if (widx >= g + 3) payload[widx - 3] = q0;
+  tail = nacc ? lo << (32 - nacc) : 0u;
+  if (last && nacc) payload[widx] = tail;
+}
+
+// The one-pass encoder of kind 2. A warp takes the next group of 4 chunks from a counter, one
+// sub-stream per lane, runs tANS over it and parks its bits in its own region of shared memory
+// (kShPark words, word-aligned from bit 0), counting the fused histogram. From the bit counts it
+// writes the sync rows and publishes the group's word count; it learns the group's word offset
+// from the groups before it (the decoupled look-back of k_encode, over groups) and copies each
+// chunk out, the warp writing 32 consecutive payload words per store instruction, each word
+// shifted together from the sub-stream's parked words. A word shared by two sub-streams is
+// carried from one to the next and stored once. When any sub-stream of the group codes to more
+// than kShPark words, its lane's writes have run into the regions after it (the last lane's into
+// a guard area sized for the longest sub-stream), so every lane of the group codes its sub-stream
+// again straight into the payload.
+constexpr int kShEncWarps = 12;
+constexpr int kShEncThreads = 32 * kShEncWarps;
+constexpr uint32_t kShPark = 113;  // words: 7.06 bits per symbol; odd, so the 32 regions start
+                                   // in 32 different banks
+constexpr uint32_t kShSubMaxWords = (kSubLen * 15 + HX_SHN_R + 31) / 32;  // 241
+constexpr uint32_t kShParkWords = 32 * kShPark + (kShSubMaxWords - kShPark);
+
+struct ShEncodeSmem {
+  ShEnc t;
+  uint32_t hist[kShEncWarps][256];
+  alignas(16) uint32_t park[kShEncWarps][kShParkWords];
+};
+static_assert(sizeof(ShEncodeSmem) <= 227 * 1024, "one block per SM");
+
+template <bool HIST>
+__device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint64_t n = a.n;
+  const uint32_t nchunks = (uint32_t)n_chunks_of(n), ngroups = (nchunks + 3) / 4;
+  const uint32_t full_chunks = (uint32_t)(n / kChunk);
+  const uint64_t P = payload_offset(n);
+  uint32_t* word_off = reinterpret_cast<uint32_t*>(a.out + 64);
+  uint16_t* sync = reinterpret_cast<uint16_t*>(a.out + sync_offset(n));
+  uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + P);
+  // payload words that fit before the 2 guard words at the end of the caller's buffer
+  const uint64_t room = a.cap >= P + 8 ? (a.cap - P - 8) / 4 : 0;
+  const ShLane tl = sh_lane(sm.t, lane);
+  const uint32_t park = (uint32_t)__cvta_generic_to_shared(sm.park[warp]);
+  const uint32_t hist = (uint32_t)__cvta_generic_to_shared(sm.hist[warp]);
+  const uint32_t j = lane >> 3, k = lane & 7;
+  const uint32_t region = park + 4u * kShPark * lane;
+  for (;;) {
+    uint32_t g = 0;
+    if (lane == 0) g = atomicAdd(a.counter, 1u);
+    g = __shfl_sync(0xffffffffu, g, 0);
+    if (g >= ngroups) break;
+    // the group this warp will most likely take next, into L2
+    const uint64_t ahead = (uint64_t)g + gridDim.x * kShEncWarps;
+    if (lane == 0 && 4 * ahead + 4 <= full_chunks)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.in + ahead * 4 * kChunk),
+                   "r"(4 * kChunk)
+                   : "memory");
+    const uint32_t c = 4 * g + j;
+    const uint32_t m = c < nchunks ? sh_count(n, c, k) : 0u;
+    // tANS into the lane's region; a word is stored once it is finished
+    uint32_t wa = region, hi = 0, lo = 0, nacc = 0;
+    sh_run<HIST>(a, tl, c, k, m, hist, [&](uint32_t value, uint32_t len) {
+      hi = __funnelshift_l(lo, hi, len);
+      lo = (lo << len) | value;
+      nacc += len;
+      const uint32_t f = nacc >> 5;  // 0 or 1: at most 30 bits join at most 31
+      nacc &= 31u;
+      sts_if(f != 0, wa, __funnelshift_r(lo, hi, nacc));
+      wa += 4u * f;
+    });
+    sts_if(nacc != 0, wa, nacc ? lo << (32 - nacc) : 0u);
+    const uint32_t bits = 8u * (wa - region) + nacc;
+    const bool spill = __any_sync(0xffffffffu, bits > 32u * kShPark);
+    // the chunk's sync row: its bit count, then where sub-streams 1..7 start
+    uint32_t incl = bits;
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d, 8);
+      if (k >= (uint32_t)d) incl += t;
+    }
+    const uint32_t s = incl - bits;
+    const uint32_t cbits = __shfl_sync(0xffffffffu, incl, 7, 8);
+    if (c < nchunks) sync[(uint64_t)c * HX_SUBSTREAMS + k] = (uint16_t)(k == 0 ? cbits : s);
+    // the group's word count, published before the wait; each chunk's offset inside the group
+    const uint32_t cw = (cbits + 31) >> 5;
+    const uint32_t w0 = __shfl_sync(0xffffffffu, cw, 0), w1 = __shfl_sync(0xffffffffu, cw, 8);
+    const uint32_t w2 = __shfl_sync(0xffffffffu, cw, 16), w3 = __shfl_sync(0xffffffffu, cw, 24);
+    const uint32_t gw = w0 + w1 + w2 + w3;
+    const uint32_t before = (j > 0 ? w0 : 0u) + (j > 1 ? w1 : 0u) + (j > 2 ? w2 : 0u);
+    if (lane == 0 && g != a.withhold)
+      st_relaxed_u64(a.look + g, (g == 0 ? kLookPre : kLookAgg) | gw);
+    __syncwarp();
+    uint64_t goff;
+    const bool ok = chunk_offset(a, g, gw, lane, goff);
+    // offsets are below 2^32 words (a stream holds fewer)
+    const uint32_t coff = (uint32_t)goff + before;
+    const bool fits = ok && (uint64_t)coff + cw <= room;
+    if (ok && c < nchunks && k == 0) {
+      word_off[c] = coff;
+      if (c + 1 == nchunks) {
+        reinterpret_cast<uint64_t*>(a.out)[4] = (uint64_t)coff + cw;
+        word_off[nchunks] = coff + cw;
+        if (fits) payload[coff + cw] = payload[coff + cw + 1] = 0;
+      }
+      if (!fits) atomicOr(a.status, (uint32_t)HX_ERR_CAPACITY);
+    }
+    if (!spill) {
+      // chunk by chunk, sub-stream by sub-stream: the lanes take 32 consecutive output words
+#pragma unroll 1
+      for (uint32_t jj = 0; jj < 4; ++jj) {
+        const uint32_t cc = 4 * g + jj;
+        if (cc >= nchunks || !__shfl_sync(0xffffffffu, fits, 8 * jj)) continue;
+        const uint32_t base = __shfl_sync(0xffffffffu, coff, 8 * jj);
+        const uint32_t ctot = __shfl_sync(0xffffffffu, cbits, 8 * jj);
+        uint32_t carry = 0;
+#pragma unroll 1
+        for (uint32_t q = 0; q < HX_SUBSTREAMS; ++q) {
+          const uint32_t src = 8 * jj + q;
+          const uint32_t sq = __shfl_sync(0xffffffffu, s, src);
+          const uint32_t bq = __shfl_sync(0xffffffffu, bits, src);
+          if (bq == 0) continue;  // an empty sub-stream at the end of the input
+          const uint32_t sh = sq & 31, e = sq + bq;
+          const uint32_t nin = (bq + 31) >> 5, nout = ((e + 31) >> 5) - (sq >> 5);
+          // its last word is finished by a later sub-stream
+          const bool open = (e & 31) != 0 && e < ctot;
+          const uint32_t rq = park + 4u * kShPark * src;
+          uint32_t* dst = payload + base + (sq >> 5);
+          uint32_t wlast = 0;
+          for (uint32_t i = lane; i < nout; i += 32) {
+            const uint32_t cur = i < nin ? lds_u32(rq + 4u * i) : 0u;
+            const uint32_t prev = i > 0 ? lds_u32(rq + 4u * (i - 1)) : 0u;
+            uint32_t w = __funnelshift_r(cur, prev, sh);
+            if (i == 0) w |= carry;
+            if (open && i + 1 == nout) wlast = w;
+            else dst[i] = w;
+          }
+          carry = open ? __shfl_sync(0xffffffffu, wlast, (nout - 1) & 31) : 0u;
+        }
+      }
+    } else {
+      // a sub-stream outgrew its region: code the group again, straight into the payload
+      const bool mine = fits && c < nchunks && m != 0;
+      const bool last = m != 0 && s + bits == cbits;
+      uint32_t widx = 0, tail = 0;
+      if (mine) sh_write_direct(a, tl, c, k, m, payload, coff, s, last, widx, tail);
+      __syncwarp();
+      if (mine && !last && tail) atomicOr(payload + widx, tail);
     }
     __syncwarp();
-    // any other unfinished word is OR-ed into the word the next sub-stream stored whole
-    if (live && m && !last && nacc) atomicOr(payload + widx, tail);
+  }
+}
+
+__global__ void __launch_bounds__(kShEncThreads, 1) k_sh_encode(EncodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ShEncodeSmem& sm = *reinterpret_cast<ShEncodeSmem*>(smem_raw);
+  const int tid = threadIdx.x;
+  if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
+    if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
+    return;
+  }
+  sh_load_tables(a.tables, sm.t);
+  if (a.hist)
+    for (int i = tid; i < kShEncWarps * 256; i += kShEncThreads) (&sm.hist[0][0])[i] = 0;
+  if (blockIdx.x == 0 && tid == 0) {
+    write_header(a);
+    if (a.n == 0) {  // no group writes the totals
+      reinterpret_cast<uint64_t*>(a.out)[4] = 0;
+      reinterpret_cast<uint32_t*>(a.out + 64)[0] = 0;
+      if (a.cap >= payload_offset(0) + 8) {
+        uint32_t* payload = reinterpret_cast<uint32_t*>(a.out + payload_offset(0));
+        payload[0] = payload[1] = 0;
+      }
+    }
+  }
+  __syncthreads();
+  if (a.hist) {
+    sh_encode_groups<true>(a, sm);
+    __syncthreads();
+    for (int sym = tid; sym < 256; sym += kShEncThreads) {
+      uint32_t sum = 0;
+#pragma unroll
+      for (int w = 0; w < kShEncWarps; ++w) sum += sm.hist[w][sym];
+      if (sum) atomicAdd(&a.hist[sym], sum);
+    }
+  } else {
+    sh_encode_groups<false>(a, sm);
   }
 }
 
@@ -1585,7 +1551,7 @@ DecodeKernel prefix_decoder(uint32_t kind, int i) {
 struct DeviceInfo {
   int sms = 0;
   int hist_per_sm = 0;
-  int sh_measure_per_sm = 0, sh_pack_per_sm = 0, sh_decode_per_sm = 0;
+  int sh_encode_per_sm = 0, sh_decode_per_sm = 0;
   // prefix-code decode blocks per SM at 1024, 256, 64 threads: [0] Huffman, [1] QLC and
   // Exp-Golomb (whose 1024-thread blocks hold the 8 bank-confined table copies)
   int dec_per_sm[2][3] = {{0, 0, 0}, {0, 0, 0}};
@@ -1647,15 +1613,11 @@ bool device_info(DeviceInfo* out) {
     if (
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
                                                       0) != cudaSuccess ||
-        cudaFuncSetAttribute(k_sh_measure, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(ShMeasureSmem)) != cudaSuccess ||
-        cudaFuncSetAttribute(k_sh_pack, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(ShPackSmem)) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_measure_per_sm, k_sh_measure,
-                                                      kShThreads,
-                                                      sizeof(ShMeasureSmem)) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_pack_per_sm, k_sh_pack, kShThreads,
-                                                      sizeof(ShPackSmem)) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sh_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(ShEncodeSmem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_encode_per_sm, k_sh_encode,
+                                                      kShEncThreads,
+                                                      sizeof(ShEncodeSmem)) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_decode_per_sm, k_sh_decode,
                                                       kDecThreads, 0) != cudaSuccess)
       return false;
@@ -1665,7 +1627,7 @@ bool device_info(DeviceInfo* out) {
                                                       sizeof(EncSmem)) != cudaSuccess ||
         d.enc_per_sm < 1)
       return false;
-    if (d.sh_measure_per_sm < 1 || d.sh_pack_per_sm < 1 || d.sh_decode_per_sm < 1) return false;
+    if (d.sh_encode_per_sm < 1 || d.sh_decode_per_sm < 1) return false;
     if (d.hist_per_sm < 1)
       return false;
     // The decoders' payload reads hit L1 most of the time: give L1 all the on-chip memory that
@@ -1700,23 +1662,10 @@ int encode_args(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint64
     return HX_ERR_ARG;
   if (!device_info(info)) return HX_ERR_CUDA;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n);
-  // the Shannonic coder's measure blocks: at least one wave of resident blocks, at most
-  // kMaxChunksPerBlock chunks each (n < 2^32 gives at most 2^20 chunks, so 1024 blocks always
-  // suffice)
-  const int per_sm = info->sh_measure_per_sm;
-  uint32_t mblocks = (uint32_t)std::min<uint64_t>(
-      {(uint64_t)nchunks, (uint64_t)kMaxMeasureBlocks,
-       std::max<uint64_t>((uint64_t)info->sms * per_sm,
-                          (nchunks + kMaxChunksPerBlock - 1) / kMaxChunksPerBlock)});
-  const uint32_t cpb = mblocks ? (nchunks + mblocks - 1) / mblocks : 1;
-  if (mblocks) mblocks = (nchunks + cpb - 1) / cpb;  // no block without chunks
-  // scratch (hx_scratch_bytes): Shannonic u32 local[nchunks], u32 btotal[mblocks] (mblocks <=
-  // nchunks); or the single pass's u64 look[nchunks] and u32 counter
-  auto* local = static_cast<uint32_t*>(d_scratch);
+  // scratch (hx_scratch_bytes): u64 look[nchunks] (kind 2 uses one per group of 4 chunks), then
+  // the u32 counter
   *a = EncodeArgs{static_cast<const hx::Tables*>(d_tables), d_in, n, static_cast<uint8_t*>(d_out),
-                  out_cap, local, local + nchunks, mblocks, cpb, d_hist, d_status, kind,
-                  // the single pass: u64 look[nchunks], then the u32 chunk counter
-                  static_cast<uint64_t*>(d_scratch),
+                  out_cap, d_hist, d_status, kind, static_cast<uint64_t*>(d_scratch),
                   reinterpret_cast<uint32_t*>(static_cast<uint64_t*>(d_scratch) + nchunks),
                   kDefaultWaitNs, ~0ull, kEncFlushRounds};
   return HX_OK;
@@ -1733,15 +1682,15 @@ int launch_encode(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
   return launched();
 }
 
-// The Shannonic coder's two passes (tANS runs backwards, so a sub-stream's length is known only
-// once it has been run): measure, then pack.
+// The Shannonic encode: zero the look-back words and the counter, then one block per SM (a
+// group of 4 chunks per warp and round).
 int launch_shannonic(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
-  if (a.mblocks) k_sh_measure<<<a.mblocks, kShThreads, sizeof(ShMeasureSmem), s>>>(a);
-  if (launched()) return HX_ERR_CUDA;
-  const uint32_t nchunks = (uint32_t)n_chunks_of(a.n);
-  const uint32_t grid = (uint32_t)std::max<uint64_t>(  // 32 chunks per block and round
-      1, std::min<uint64_t>((nchunks + 31) / 32, (uint64_t)info.sms * info.sh_pack_per_sm));
-  k_sh_pack<<<grid, kShThreads, sizeof(ShPackSmem), s>>>(a);
+  const uint64_t nchunks = n_chunks_of(a.n), ngroups = (nchunks + 3) / 4;
+  if (cudaMemsetAsync(a.look, 0, 8 * nchunks + 4, s) != cudaSuccess) return HX_ERR_CUDA;
+  const uint32_t grid = (uint32_t)std::max<uint64_t>(
+      1, std::min<uint64_t>((ngroups + kShEncWarps - 1) / kShEncWarps,
+                            (uint64_t)info.sms * info.sh_encode_per_sm));
+  k_sh_encode<<<grid, kShEncThreads, sizeof(ShEncodeSmem), s>>>(a);
   return launched();
 }
 
@@ -1755,13 +1704,10 @@ int encode_common(uint32_t kind, const void* d_tables, const uint8_t* d_in, uint
                              &a, &info);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (kind != HX_KIND_SHANNONIC) {
-    a.wait_ns = wait_ns;
-    a.withhold = withhold;
-    a.flush = flush;
-    return launch_encode(a, info, s);
-  }
-  return launch_shannonic(a, info, s);
+  a.wait_ns = wait_ns;
+  a.withhold = withhold;
+  a.flush = flush;  // k_encode's; k_sh_encode's warps count into tables of their own
+  return kind == HX_KIND_SHANNONIC ? launch_shannonic(a, info, s) : launch_encode(a, info, s);
 }
 
 int decode_common(uint32_t kind, const void* const* d_set, uint32_t nset, const void* d_stream,
@@ -1892,7 +1838,7 @@ int hx_encode_bounded(uint32_t kind, const void* d_tables, const uint8_t* d_in, 
                       void* d_out, uint64_t out_cap, void* d_scratch, uint32_t* d_hist,
                       uint32_t* d_status, uint64_t wait_ns, uint64_t withhold,
                       uint32_t flush_rounds, void* stream) {
-  if (kind == HX_KIND_SHANNONIC || flush_rounds > kEncFlushRoundsMax) return HX_ERR_ARG;
+  if (flush_rounds > kEncFlushRoundsMax) return HX_ERR_ARG;
   return encode_common(kind, d_tables, d_in, n, d_out, out_cap, d_scratch, d_hist, d_status,
                        stream, wait_ns, withhold, flush_rounds ? flush_rounds : kEncFlushRounds);
 }

@@ -83,3 +83,33 @@ def test_fused_histogram_flushed_every_chunk(setup, flush_rounds):
     ref = orc.encode(ocb, x)[1]
     assert int(st.item()) == 0 and (out[:ref.size].cpu().numpy() == ref).all()
     assert (hist.cpu().numpy().astype(np.uint64) == orc.histogram(x)).all()
+
+
+@pytest.mark.parametrize("withhold", [0, 4, 9])
+def test_shannonic_withheld_group_times_out_and_context_survives(setup, withhold):
+    """The Shannonic encoder's look-back runs over groups of 4 chunks: a group that never
+    publishes its word count makes the groups after it time out (group 9 is the last of 40
+    chunks: nothing waits for it)."""
+    orc = setup[0]
+    counts = sum(orc.histogram(b) for b in datagen.prior_batches(1))
+    tables = hx.shannonic_build(counts).upload(torch.device("cuda:0"))
+    ocb = orc.shannonic_codebook(counts)
+    n = 40 * 4096 - 100
+    x = datagen.data(1, n=n)
+    xd = torch.from_numpy(x).cuda()
+    k = hx.KIND_SHANNONIC
+    out = torch.zeros(hx.encode_bound(n, k), dtype=torch.uint8, device="cuda")
+    scratch = torch.empty(hx.scratch_bytes(n), dtype=torch.uint8, device="cuda")
+    _, st = hx.encode_bounded(tables, xd, out, scratch, wait_ns=2_000_000, withhold=withhold,
+                              kind=k)
+    torch.cuda.synchronize()
+    status = int(st.item())
+    ref = orc.encode(ocb, x)[1]
+    if withhold == 9:
+        assert status == 0 and (out[:ref.size].cpu().numpy() == ref).all()
+    else:
+        assert status & hx.HX_ERR_TIMEOUT
+    out2 = torch.zeros_like(out)
+    _, st2 = hx.encode(tables, xd, out=out2, scratch=scratch, kind=k)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0 and (out2[:ref.size].cpu().numpy() == ref).all()

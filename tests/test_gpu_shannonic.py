@@ -1,4 +1,4 @@
-"""The Shannonic coder on the GPU (k_sh_measure, k_sh_pack, k_sh_decode) against the oracle.
+"""The Shannonic coder on the GPU (k_sh_encode, k_sh_decode) against the oracle.
 
 Byte work, so the bar is bit-exact: the stream the GPU writes equals the oracle's byte for byte,
 decoding returns the input, the fused histogram equals the oracle's, and on damaged streams the
@@ -86,17 +86,43 @@ def test_adversarial_inputs(orc, cuda):
         assert st == 0 and (y == x).all()
 
 
+def test_parked_and_recoded_groups(orc, cuda):
+    """The encoder parks each sub-stream's bits in shared memory (113 words, 7.06 bits per
+    symbol) and codes a group of 4 chunks again, straight into the payload, when one of its
+    sub-streams is longer. Runs of the codebook's rarest byte make some groups long: a whole
+    chunk, a single sub-stream, and a run across a chunk boundary, among groups that fit."""
+    x = datagen.data(4, n=64 * 4096 + 123)
+    counts = sum(orc.histogram(b) for b in datagen.prior_batches(1))
+    tables, ocb = _book(orc, counts, cuda)
+    rare = np.uint8(np.argmin(counts))
+    x[20 * 4096:21 * 4096] = rare
+    x[41 * 4096 + 3 * 512:41 * 4096 + 4 * 512] = rare
+    x[51 * 4096 - 700:51 * 4096 + 300] = rare
+    x[-50:] = rare
+    hist = torch.zeros(256, dtype=torch.int32, device=cuda)
+    ref = orc.encode(ocb, x)[1]
+    got, st, _ = _enc(tables, x, hist=hist)
+    assert st == 0 and got.size == ref.size and (got == ref).all()
+    assert (hist.cpu().numpy().astype(np.uint64) == orc.histogram(x)).all()
+    st, y = _dec(tables, ref, x.size)
+    assert st == 0 and (y == x).all()
+
+
 def test_capacity_and_wrong_tables(orc, cuda):
     x = datagen.data(1, n=5 * 4096 + 3)
     tables, ocb = _book(orc, orc.histogram(x), cuda)
     full = orc.encode(ocb, x)[1]
     need = full.size
     P = hx.payload_offset(x.size)
-    for cap in (need - 4, P + 8):
+    for cap in (need - 4, need // 2, P + 8):
         got, st, total = _enc(tables, x, cap=cap)
         assert st == hx.HX_ERR_CAPACITY and hx.stream_bytes(x.size, total) == need
-        # the header and the index are those of the whole stream, and no payload word is written
-        assert got.size == cap and (got[:P] == full[:P]).all() and (got[P:] == 0).all()
+        # the header and the index are those of the whole stream; a payload word is either the
+        # stream's own (a chunk that fitted) or untouched (zero), and none lies past the buffer
+        assert got.size == cap and (got[:P] == full[:P]).all()
+        assert ((got[P:] == full[P:cap]) | (got[P:] == 0)).all()
+    got, st, _ = _enc(tables, x, cap=need)
+    assert st == 0 and (got == full).all()
     huff = hx.build_codebook(orc.histogram(x)).upload(cuda)
     _, st, _ = _enc(huff, x)
     assert st == hx.HX_ERR_ARG

@@ -141,8 +141,10 @@ def test_host_argument_checks_need_no_gpu():
     assert L.hx_encode(256, 257, 100, 256, 1 << 20, 256, None, 256, None) == hx.HX_ERR_ARG
     assert L.hx_encode(256, 256, 100, 256, 10, 256, None, 256, None) == hx.HX_ERR_ARG
     # the bounded-wait encode: same checks, plus the kind
-    assert L.hx_encode_bounded(2, 256, 256, 100, 256, 1 << 20, 256, None, 256, 10, 0, 0,
-                               None) == hx.HX_ERR_ARG  # the Shannonic coder has no bounded wait
+    assert L.hx_encode_bounded(4, 256, 256, 100, 256, 1 << 20, 256, None, 256, 10, 0, 0,
+                               None) == hx.HX_ERR_ARG  # no stream kind 4
+    assert L.hx_encode_bounded(2, 256, 256, 100, 256, 1 << 20, 256, None, 256, 10, 0, 4097,
+                               None) == hx.HX_ERR_ARG
     assert L.hx_encode_bounded(0, None, 256, 100, 256, 1 << 20, 256, None, 256, 10, 0, 0,
                                None) == hx.HX_ERR_ARG
     assert L.hx_encode_bounded(0, 256, 256, 100, 256, 1 << 20, 256, None, 256, 10, 0, 4097,
