@@ -1007,19 +1007,18 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) k_decode(DecodeArgs a
 
 constexpr int kShCopies = 16;  // symbol table copies: lane l reads copy l % 16 (<= 2-way)
 
-// Encoder tables in shared memory: per byte value [byte][copy] the step's fields (sh_sym) and,
-// at a fixed distance, its offset in its range (sh_off); the ranges' states (sh_enc).
+// Encoder tables in shared memory: per byte value [byte][copy] one 8-byte entry, the step's
+// fields (sh_sym) and the byte's offset in its range (sh_off), read with one load; the ranges'
+// states (sh_enc). A row of 16 copies is 128 bytes, so lanes l and l + 16 share banks and a warp's
+// lookup takes the 2 wavefronts its 256 bytes need.
 struct ShEnc {
-  uint32_t sym[256 * kShCopies];
-  uint32_t off[256 * kShCopies];
+  uint2 ent[256 * kShCopies];
   uint8_t enc[128];
 };
 
 __device__ __forceinline__ void sh_load_tables(const hx::Tables* t, ShEnc& s) {
-  for (int i = threadIdx.x; i < 256 * kShCopies; i += blockDim.x) {
-    s.sym[i] = t->sh_sym[i / kShCopies];
-    s.off[i] = t->sh_off[i / kShCopies];
-  }
+  for (int i = threadIdx.x; i < 256 * kShCopies; i += blockDim.x)
+    s.ent[i] = make_uint2(t->sh_sym[i / kShCopies], t->sh_off[i / kShCopies]);
   for (int i = threadIdx.x; i < 128; i += blockDim.x) s.enc[i] = t->sh_enc[i];
 }
 
@@ -1030,14 +1029,18 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
 }
 
 // Shared addresses of the encoder tables for this lane: its copy of byte b's entry is at
-// sym + 4 * kShCopies * b, b's offset kOffDist further; `enc` is sh_enc's address - 128.
+// sym + 8 * kShCopies * b; `enc` is sh_enc's address - 128.
 struct ShLane {
   uint32_t sym, enc;
 };
-constexpr uint32_t kOffDist = 4 * 256 * kShCopies;
 __device__ __forceinline__ ShLane sh_lane(const ShEnc& s, uint32_t lane) {
-  return {(uint32_t)__cvta_generic_to_shared(s.sym) + 4 * (lane % kShCopies),
+  return {(uint32_t)__cvta_generic_to_shared(s.ent) + 8 * (lane % kShCopies),
           (uint32_t)__cvta_generic_to_shared(s.enc) - 128u};
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
 }
 
 // One tANS step from state x (in [128, 256)) with the byte's entry e: returns the bit count
@@ -1079,6 +1082,9 @@ __device__ __forceinline__ void st_global_v4_if(bool p, uint32_t* a, uint4 v) {
       "{\n .reg .pred q;\n setp.ne.u32 q, %5, 0;\n @q st.global.v4.u32 [%0], {%1, %2, %3, %4};\n}"
       ::"l"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"((uint32_t)p) : "memory");
 }
+__device__ __forceinline__ void sts_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
 __device__ __forceinline__ void sts_if(bool p, uint32_t a, uint32_t v) {
   asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q st.shared.u32 [%0], %1;\n}"
                ::"r"(a), "r"(v), "r"((uint32_t)p) : "memory");
@@ -1094,11 +1100,10 @@ __device__ __forceinline__ void sh_run(const EncodeArgs& a, const ShLane& tl, ui
   // the bits of byte `sym` (as sh_value) and their count
   auto code = [&](uint32_t sym, uint32_t& len) -> uint32_t {
     if (HIST) reds_add_u32(hist + 4u * sym, 1u);
-    const uint32_t ea = tl.sym + sym * (4 * kShCopies);
-    const uint32_t e = lds_u32(ea), off = lds_u32(ea + kOffDist);
+    const uint2 eo = lds_v2(tl.sym + sym * (8 * kShCopies));
     uint32_t xo, xh;
-    len = sh_next(e, state, tl.enc, xo, xh);
-    return sh_value(e, off, xo, xh, len);
+    len = sh_next(eo.x, state, tl.enc, xo, xh);
+    return sh_value(eo.x, eo.y, xo, xh, len);
   };
   if (m == kSubLen) {
     // a whole sub-stream: 16 bytes at a time from the end, the next 16 already requested
@@ -1173,21 +1178,21 @@ __device__ __noinline__ void sh_write_direct(const EncodeArgs& a, const ShLane& 
 
 // The one-pass encoder of kind 2. A warp takes the next group of 4 chunks from a counter, one
 // sub-stream per lane, runs tANS over it and parks its bits in its own region of shared memory
-// (kShPark words, word-aligned from bit 0), counting the fused histogram. From the bit counts it
-// writes the sync rows and publishes the group's word count; it learns the group's word offset
-// from the groups before it (the decoupled look-back of k_encode, over groups) and copies each
-// chunk out, the warp writing 32 consecutive payload words per store instruction, each word
-// shifted together from the sub-stream's parked words. A word shared by two sub-streams is
-// carried from one to the next and stored once. When any sub-stream of the group codes to more
-// than kShPark words, its lane's writes have run into the regions after it (the last lane's into
-// a guard area sized for the longest sub-stream), so every lane of the group codes its sub-stream
-// again straight into the payload.
+// (a zero word, then up to kShPark words from bit 0), counting the fused histogram. From the bit
+// counts it writes the sync rows and publishes the group's word count; it learns the group's word
+// offset from the groups before it (the decoupled look-back of k_encode, over groups) and copies
+// each chunk out, sub-stream by sub-stream, each lane shifting two consecutive payload words
+// together from the parked words (the word before its pair from the lane before it). A word
+// shared by two sub-streams is carried from one to the next and stored once. When any
+// sub-stream of the group codes to more than kShPark words, its lane's writes have run into the
+// regions after it (the last lane's into a guard area sized for the longest sub-stream), so every
+// lane of the group codes its sub-stream again straight into the payload.
 constexpr int kShEncWarps = 12;
 constexpr int kShEncThreads = 32 * kShEncWarps;
-constexpr uint32_t kShPark = 113;  // words: 7.06 bits per symbol; odd, so the 32 regions start
-                                   // in 32 different banks
+constexpr uint32_t kShPark = 112;              // words: 7 bits per symbol
+constexpr uint32_t kShStride = kShPark + 1;    // odd: the 32 regions start in 32 different banks
 constexpr uint32_t kShSubMaxWords = (kSubLen * 15 + HX_SHN_R + 31) / 32;  // 241
-constexpr uint32_t kShParkWords = 32 * kShPark + (kShSubMaxWords - kShPark);
+constexpr uint32_t kShParkWords = 31 * kShStride + 1 + kShSubMaxWords;
 
 struct ShEncodeSmem {
   ShEnc t;
@@ -1212,7 +1217,7 @@ __device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
   const uint32_t park = (uint32_t)__cvta_generic_to_shared(sm.park[warp]);
   const uint32_t hist = (uint32_t)__cvta_generic_to_shared(sm.hist[warp]);
   const uint32_t j = lane >> 3, k = lane & 7;
-  const uint32_t region = park + 4u * kShPark * lane;
+  const uint32_t region = park + 4u * kShStride * lane;
   for (;;) {
     uint32_t g = 0;
     if (lane == 0) g = atomicAdd(a.counter, 1u);
@@ -1226,19 +1231,22 @@ __device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
                    : "memory");
     const uint32_t c = 4 * g + j;
     const uint32_t m = c < nchunks ? sh_count(n, c, k) : 0u;
-    // tANS into the lane's region; a word is stored once it is finished
-    uint32_t wa = region, hi = 0, lo = 0, nacc = 0;
+    // tANS into the lane's region. pos counts the bits from the start of the zero word (32 +
+    // the sub-stream's bits); hi:lo holds the last 64 of them, so the last finished word,
+    // (pos >> 5) - 1, is hi:lo >> (pos mod 32) (a wrapping shift reads only pos's low 5 bits):
+    // every append stores it, again and again until the next one is finished, with no
+    // condition.
+    uint32_t pos = 32, hi = 0, lo = 0;
     sh_run<HIST>(a, tl, c, k, m, hist, [&](uint32_t value, uint32_t len) {
       hi = __funnelshift_l(lo, hi, len);
       lo = (lo << len) | value;
-      nacc += len;
-      const uint32_t f = nacc >> 5;  // 0 or 1: at most 30 bits join at most 31
-      nacc &= 31u;
-      sts_if(f != 0, wa, __funnelshift_r(lo, hi, nacc));
-      wa += 4u * f;
+      pos += len;
+      sts_u32(region + ((pos >> 3) & ~3u) - 4u, __funnelshift_r(lo, hi, pos));
     });
-    sts_if(nacc != 0, wa, nacc ? lo << (32 - nacc) : 0u);
-    const uint32_t bits = 8u * (wa - region) + nacc;
+    const uint32_t part = pos & 31u;  // the unfinished word's bits
+    sts_if(part != 0, region + ((pos >> 3) & ~3u), part ? lo << (32 - part) : 0u);
+    sts_u32(region, 0u);
+    const uint32_t bits = pos - 32u;
     const bool spill = __any_sync(0xffffffffu, bits > 32u * kShPark);
     // the chunk's sync row: its bit count, then where sub-streams 1..7 start
     uint32_t incl = bits;
@@ -1281,7 +1289,7 @@ __device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
         if (cc >= nchunks || !__shfl_sync(0xffffffffu, fits, 8 * jj)) continue;
         const uint32_t base = __shfl_sync(0xffffffffu, coff, 8 * jj);
         const uint32_t ctot = __shfl_sync(0xffffffffu, cbits, 8 * jj);
-        uint32_t carry = 0;
+        uint32_t carry = 0;  // the unfinished word of the sub-stream before (its bits on top)
 #pragma unroll 1
         for (uint32_t q = 0; q < HX_SUBSTREAMS; ++q) {
           const uint32_t src = 8 * jj + q;
@@ -1290,20 +1298,28 @@ __device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
           if (bq == 0) continue;  // an empty sub-stream at the end of the input
           const uint32_t sh = sq & 31, e = sq + bq;
           const uint32_t nin = (bq + 31) >> 5, nout = ((e + 31) >> 5) - (sq >> 5);
-          // its last word is finished by a later sub-stream
+          // its last word is finished by a later sub-stream: carried, not stored
           const bool open = (e & 31) != 0 && e < ctot;
-          const uint32_t rq = park + 4u * kShPark * src;
-          uint32_t* dst = payload + base + (sq >> 5);
-          uint32_t wlast = 0;
-          for (uint32_t i = lane; i < nout; i += 32) {
-            const uint32_t cur = i < nin ? lds_u32(rq + 4u * i) : 0u;
-            const uint32_t prev = i > 0 ? lds_u32(rq + 4u * (i - 1)) : 0u;
-            uint32_t w = __funnelshift_r(cur, prev, sh);
-            if (i == 0) w |= carry;
-            if (open && i + 1 == nout) wlast = w;
-            else dst[i] = w;
+          const uint32_t lim = nout - (open ? 1u : 0u);
+          const uint32_t rq = park + 4u * kShStride * src + 4u;  // its word 0
+          const uint32_t w0 = base + (sq >> 5);                   // the payload word of output 0
+          // output word i = parked words i - 1 : i >> sh; before word 0 stand the carried bits
+          uint32_t before = sh ? carry >> (32 - sh) : 0u;
+          uint32_t wa = 0, wb = 0;
+          for (uint32_t i0 = 0; i0 < nout; i0 += 64) {
+            const uint32_t i = i0 + 2 * lane;
+            const uint32_t ca = i < nin ? lds_u32(rq + 4u * i) : 0u;
+            const uint32_t cb = i + 1 < nin ? lds_u32(rq + 4u * i + 4u) : 0u;
+            uint32_t pa = __shfl_up_sync(0xffffffffu, cb, 1);
+            if (lane == 0) pa = before;
+            before = __shfl_sync(0xffffffffu, cb, 31);
+            wa = __funnelshift_r(ca, pa, sh);
+            wb = __funnelshift_r(cb, ca, sh);
+            if (i < lim) payload[w0 + i] = wa;
+            if (i + 1 < lim) payload[w0 + i + 1] = wb;
           }
-          carry = open ? __shfl_sync(0xffffffffu, wlast, (nout - 1) & 31) : 0u;
+          const uint32_t t = (nout - 1) & 63;  // the last word's place in the last round
+          carry = open ? __shfl_sync(0xffffffffu, (t & 1) ? wb : wa, t >> 1) : 0u;
         }
       }
     } else {
