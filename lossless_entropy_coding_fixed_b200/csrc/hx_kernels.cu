@@ -1187,22 +1187,27 @@ __device__ __noinline__ void sh_write_direct(const EncodeArgs& a, const ShLane& 
 // sub-stream of the group codes to more than kShPark words, its lane's writes have run into the
 // regions after it (the last lane's into a guard area sized for the longest sub-stream), so every
 // lane of the group codes its sub-stream again straight into the payload.
-constexpr int kShEncWarps = 12;
-constexpr int kShEncThreads = 32 * kShEncWarps;
+// warps per block (one block per SM): as many as the shared memory holds, with and without the
+// fused histogram's tables
+template <bool HIST>
+__host__ __device__ constexpr int sh_enc_warps() { return HIST ? 12 : 13; }
 constexpr uint32_t kShPark = 112;              // words: 7 bits per symbol
 constexpr uint32_t kShStride = kShPark + 1;    // odd: the 32 regions start in 32 different banks
 constexpr uint32_t kShSubMaxWords = (kSubLen * 15 + HX_SHN_R + 31) / 32;  // 241
 constexpr uint32_t kShParkWords = 31 * kShStride + 1 + kShSubMaxWords;
 
+template <bool HIST>
 struct ShEncodeSmem {
+  static constexpr int kWarps = sh_enc_warps<HIST>();
   ShEnc t;
-  uint32_t hist[kShEncWarps][256];
-  alignas(16) uint32_t park[kShEncWarps][kShParkWords];
+  uint32_t hist[HIST ? kWarps : 1][256];
+  alignas(16) uint32_t park[kWarps][kShParkWords];
 };
-static_assert(sizeof(ShEncodeSmem) <= 227 * 1024, "one block per SM");
+static_assert(sizeof(ShEncodeSmem<true>) <= 227 * 1024, "one block per SM");
+static_assert(sizeof(ShEncodeSmem<false>) <= 227 * 1024, "one block per SM");
 
 template <bool HIST>
-__device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
+__device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem<HIST>& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint64_t n = a.n;
   const uint32_t nchunks = (uint32_t)n_chunks_of(n), ngroups = (nchunks + 3) / 4;
@@ -1224,7 +1229,7 @@ __device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
     g = __shfl_sync(0xffffffffu, g, 0);
     if (g >= ngroups) break;
     // the group this warp will most likely take next, into L2
-    const uint64_t ahead = (uint64_t)g + gridDim.x * kShEncWarps;
+    const uint64_t ahead = (uint64_t)g + gridDim.x * ShEncodeSmem<HIST>::kWarps;
     if (lane == 0 && 4 * ahead + 4 <= full_chunks)
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.in + ahead * 4 * kChunk),
                    "r"(4 * kChunk)
@@ -1335,17 +1340,19 @@ __device__ void sh_encode_groups(const EncodeArgs& a, ShEncodeSmem& sm) {
   }
 }
 
-__global__ void __launch_bounds__(kShEncThreads, 1) k_sh_encode(EncodeArgs a) {
+template <bool HIST>
+__global__ void __launch_bounds__(32 * sh_enc_warps<HIST>(), 1) k_sh_encode(EncodeArgs a) {
+  constexpr int kWarps = sh_enc_warps<HIST>(), kThreads = 32 * kWarps;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  ShEncodeSmem& sm = *reinterpret_cast<ShEncodeSmem*>(smem_raw);
+  ShEncodeSmem<HIST>& sm = *reinterpret_cast<ShEncodeSmem<HIST>*>(smem_raw);
   const int tid = threadIdx.x;
   if (a.tables->magic != hx::kTablesMagic || a.tables->kind != a.kind) {
     if (blockIdx.x == 0 && tid == 0) atomicOr(a.status, (uint32_t)HX_ERR_ARG);
     return;
   }
   sh_load_tables(a.tables, sm.t);
-  if (a.hist)
-    for (int i = tid; i < kShEncWarps * 256; i += kShEncThreads) (&sm.hist[0][0])[i] = 0;
+  if (HIST)
+    for (int i = tid; i < kWarps * 256; i += kThreads) (&sm.hist[0][0])[i] = 0;
   if (blockIdx.x == 0 && tid == 0) {
     write_header(a);
     if (a.n == 0) {  // no group writes the totals
@@ -1358,17 +1365,15 @@ __global__ void __launch_bounds__(kShEncThreads, 1) k_sh_encode(EncodeArgs a) {
     }
   }
   __syncthreads();
-  if (a.hist) {
-    sh_encode_groups<true>(a, sm);
+  sh_encode_groups<HIST>(a, sm);
+  if (HIST) {
     __syncthreads();
-    for (int sym = tid; sym < 256; sym += kShEncThreads) {
+    for (int sym = tid; sym < 256; sym += kThreads) {
       uint32_t sum = 0;
 #pragma unroll
-      for (int w = 0; w < kShEncWarps; ++w) sum += sm.hist[w][sym];
+      for (int w = 0; w < kWarps; ++w) sum += sm.hist[HIST ? w : 0][sym];
       if (sum) atomicAdd(&a.hist[sym], sum);
     }
-  } else {
-    sh_encode_groups<false>(a, sm);
   }
 }
 
@@ -1567,7 +1572,8 @@ DecodeKernel prefix_decoder(uint32_t kind, int i) {
 struct DeviceInfo {
   int sms = 0;
   int hist_per_sm = 0;
-  int sh_encode_per_sm = 0, sh_decode_per_sm = 0;
+  int sh_encode_per_sm[2] = {0, 0};  // without, with the fused histogram
+  int sh_decode_per_sm = 0;
   // prefix-code decode blocks per SM at 1024, 256, 64 threads: [0] Huffman, [1] QLC and
   // Exp-Golomb (whose 1024-thread blocks hold the 8 bank-confined table copies)
   int dec_per_sm[2][3] = {{0, 0, 0}, {0, 0, 0}};
@@ -1629,11 +1635,16 @@ bool device_info(DeviceInfo* out) {
     if (
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.hist_per_sm, k_histogram, kHistThreads,
                                                       0) != cudaSuccess ||
-        cudaFuncSetAttribute(k_sh_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(ShEncodeSmem)) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_encode_per_sm, k_sh_encode,
-                                                      kShEncThreads,
-                                                      sizeof(ShEncodeSmem)) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sh_encode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(ShEncodeSmem<false>)) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sh_encode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(ShEncodeSmem<true>)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &d.sh_encode_per_sm[0], k_sh_encode<false>, 32 * sh_enc_warps<false>(),
+            sizeof(ShEncodeSmem<false>)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &d.sh_encode_per_sm[1], k_sh_encode<true>, 32 * sh_enc_warps<true>(),
+            sizeof(ShEncodeSmem<true>)) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.sh_decode_per_sm, k_sh_decode,
                                                       kDecThreads, 0) != cudaSuccess)
       return false;
@@ -1643,7 +1654,8 @@ bool device_info(DeviceInfo* out) {
                                                       sizeof(EncSmem)) != cudaSuccess ||
         d.enc_per_sm < 1)
       return false;
-    if (d.sh_encode_per_sm < 1 || d.sh_decode_per_sm < 1) return false;
+    if (d.sh_encode_per_sm[0] < 1 || d.sh_encode_per_sm[1] < 1 || d.sh_decode_per_sm < 1)
+      return false;
     if (d.hist_per_sm < 1)
       return false;
     // The decoders' payload reads hit L1 most of the time: give L1 all the on-chip memory that
@@ -1702,11 +1714,14 @@ int launch_encode(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
 // group of 4 chunks per warp and round).
 int launch_shannonic(const EncodeArgs& a, const DeviceInfo& info, cudaStream_t s) {
   const uint64_t nchunks = n_chunks_of(a.n), ngroups = (nchunks + 3) / 4;
+  const int hist = a.hist != nullptr;
+  const uint64_t warps = hist ? sh_enc_warps<true>() : sh_enc_warps<false>();
   if (cudaMemsetAsync(a.look, 0, 8 * nchunks + 4, s) != cudaSuccess) return HX_ERR_CUDA;
   const uint32_t grid = (uint32_t)std::max<uint64_t>(
-      1, std::min<uint64_t>((ngroups + kShEncWarps - 1) / kShEncWarps,
-                            (uint64_t)info.sms * info.sh_encode_per_sm));
-  k_sh_encode<<<grid, kShEncThreads, sizeof(ShEncodeSmem), s>>>(a);
+      1, std::min<uint64_t>((ngroups + warps - 1) / warps,
+                            (uint64_t)info.sms * info.sh_encode_per_sm[hist]));
+  if (hist) k_sh_encode<true><<<grid, 32 * warps, sizeof(ShEncodeSmem<true>), s>>>(a);
+  else k_sh_encode<false><<<grid, 32 * warps, sizeof(ShEncodeSmem<false>), s>>>(a);
   return launched();
 }
 
