@@ -303,8 +303,8 @@ int shannonic_tables(const hx_codebook& cb, hx::Tables* t) {
     const int size = cb.sh_lo[r + 1] - cb.sh_lo[r];
     const int tot = nb + bits_for(size);
     t->sh_dec[u][0] = (1u << tot) - 1u;
-    t->sh_dec[u][1] = (uint32_t)tot | ((uint32_t)(xs << nb) << 16);
-    t->sh_dec[u][2] = (uint32_t)nb;
+    t->sh_dec[u][1] = (uint32_t)tot;
+    t->sh_dec[u][2] = (uint32_t)nb | ((uint32_t)(xs << nb) << 16);
     t->sh_dec[u][3] = (uint32_t)cb.sh_lo[r] | ((uint32_t)(0x8000 - size) << 16);
   }
   for (int r = 0; r < nr; ++r) {

@@ -1516,9 +1516,10 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
           const uint4 d = lds_v4(tab + 16u * kShDecCopies * state);
           const uint32_t v = x & d.x;       // offset and state bits
           x = __funnelshift_r(x, 0u, d.y);  // x >> (nb + ob)
-          used += d.y;                      // (the count is its low 16 bits)
+          used += d.y;
+          // the shifts by nb read d.z's low 5 bits
           const uint32_t off = __funnelshift_r(v, 0u, d.z);                  // v >> nb
-          state = (d.y >> 16) + v - __funnelshift_l(0u, off, d.z);          // base + v mod 2^nb
+          state = (d.z >> 16) + v - __funnelshift_l(0u, off, d.z);          // base + v mod 2^nb
           const uint32_t r = off * 0x10001u + d.w;
           over |= r;
           return r;
@@ -1534,7 +1535,7 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
               uint32_t x = rd.peek(), used = 0;
               const uint32_t b0 = one(x, used);
               const uint32_t b1 = one(x, used);
-              rd.skip(used & 0xffffu);
+              rd.skip(used);
               pair[h] = __byte_perm(b0, b1, 0x0040);
             }
             o[q] = __byte_perm(pair[0], pair[1], 0x5410);
@@ -1544,7 +1545,7 @@ __global__ void __launch_bounds__(kDecThreads, 5) k_sh_decode(DecodeArgs a) {
         for (uint32_t i = groups * 16; i < mine; ++i) {
           uint32_t x = rd.peek(), used = 0;
           dst[i] = (uint8_t)one(x, used);
-          rd.skip(used & 0xffffu);
+          rd.skip(used);
         }
         // the chain must end in state 128 exactly at the sub-stream's first bit
         bad |= (over >> 31) || state != 128u ||

@@ -22,9 +22,9 @@ struct Tables {
     // Shannonic (kind 2) instead:
     struct {
       // per decoding state 128 + u, four words: the mask of the bits its symbol took (the
-      // offset and the state bits, 2^(nb + ob) - 1); their count nb + ob (bits 0-4) | the base of
-      // the next state (xs << nb, bits 16-23: the next state is base + the nb state bits); nb;
-      // first byte value of the range (bits 0-15) | 0x8000 - range size (16-31), so that
+      // offset and the state bits, 2^(nb + ob) - 1); their count nb + ob; nb (bits 0-4) | the
+      // base of the next state (xs << nb, bits 16-23: the next state is base + the nb state
+      // bits); first byte value of the range (bits 0-15) | 0x8000 - range size (16-31), so that
       // offset * 0x10001 + this word holds the byte in bits 0-7 and sets bit 31 exactly when the
       // offset is not inside the range
       uint32_t sh_dec[128][4];
