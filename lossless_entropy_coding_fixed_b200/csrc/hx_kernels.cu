@@ -29,10 +29,15 @@
 //                bank of their lines (codes of one length) vote per warp and may read 16-byte
 //                blocks instead.
 //
-//   k_sh_*       the Shannonic range coder: tANS over range indices with one table entry per
-//                step; a measure pass (two sub-streams per thread) and a pack pass (one per
-//                thread, 16-byte stores), since a tANS sub-stream's length is known only once it
-//                has been run; the decoder reads each sub-stream backwards, one thread each.
+//   k_sh_encode  the Shannonic range coder's encoder: tANS over range indices with one table
+//                entry per step. A warp takes the next group of 4 chunks, runs one sub-stream per
+//                lane and parks its bits in shared memory (a tANS sub-stream's length is known
+//                only once it has been run), publishes the group's word count, learns its offset
+//                by the same look-back as k_encode, and copies the chunks out with coalesced
+//                stores; a group with a sub-stream too long for its region is coded again
+//                straight into the payload.
+//   k_sh_decode  reads each sub-stream backwards, one thread each, with 16-byte payload blocks
+//                one block ahead and a 16-byte state entry per symbol.
 #include <cuda_runtime.h>
 
 #include <algorithm>
