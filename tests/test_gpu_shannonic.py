@@ -106,6 +106,14 @@ def test_parked_and_recoded_groups(orc, cuda):
     assert (hist.cpu().numpy().astype(np.uint64) == orc.histogram(x)).all()
     st, y = _dec(tables, ref, x.size)
     assert st == 0 and (y == x).all()
+    # a buffer that ends inside the stream: the header and the index are whole, a payload word is
+    # the stream's own or untouched (zero), in recoded groups as in the others
+    P = hx.payload_offset(x.size)
+    for cap in (ref.size // 2, ref.size - 4):
+        got, st, total = _enc(tables, x, cap=cap)
+        assert st == hx.HX_ERR_CAPACITY and hx.stream_bytes(x.size, total) == ref.size
+        assert got.size == cap and (got[:P] == ref[:P]).all()
+        assert ((got[P:] == ref[P:cap]) | (got[P:] == 0)).all()
 
 
 def test_capacity_and_wrong_tables(orc, cuda):
