@@ -1192,6 +1192,7 @@ __device__ __noinline__ void sh_write_direct(const EncodeArgs& a, const ShLane& 
 // sub-stream of the group codes to more than kShPark words, its lane's writes have run into the
 // regions after it (the last lane's into a guard area sized for the longest sub-stream), so every
 // lane of the group codes its sub-stream again straight into the payload.
+
 // warps per block (one block per SM): as many as the shared memory holds, with and without the
 // fused histogram's tables
 template <bool HIST>
