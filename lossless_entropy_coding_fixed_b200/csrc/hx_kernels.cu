@@ -1383,8 +1383,8 @@ __global__ void __launch_bounds__(32 * sh_enc_warps<HIST>(), 1) k_sh_encode(Enco
   }
 }
 
-// Reads a sub-stream backwards: the unread bits end at bit 32 * j + t of the payload (t in
-// 1..32 unread bits in word j, MSB first); cur = word j, prv = word j - 1. The words below come
+// Reads a sub-stream backwards: the unread bits end at bit 32 * j + 32 - u of the payload (the
+// last u, 0..31, bits of word j are read, MSB first); cur = word j, prv = word j - 1. The words below come
 // in aligned 16-byte blocks: r is block rb, the one that holds the next word to come in, and the
 // block below it is already requested (nx), so a block is moved only once it has had a whole
 // block's worth of symbols to arrive. Words outside the caller's buffer read as 0.
@@ -1394,7 +1394,7 @@ struct BackBits {
   const uint32_t* words;  // 16-byte aligned
   uint32_t wlimit;
   int32_t j, rb;
-  uint32_t t, cur, prv;
+  uint32_t u, cur, prv;
   uint4 r, nx;
   __device__ __forceinline__ uint32_t word(int32_t i) const {
     return (uint32_t)i < wlimit ? __ldg(words + (uint32_t)i) : 0u;
@@ -1407,7 +1407,7 @@ struct BackBits {
   __device__ __forceinline__ void start(uint64_t end_bit) {
     const uint64_t last = end_bit - 1;  // the first bit to read (backwards)
     j = (int32_t)(last >> 5);
-    t = (uint32_t)(last & 31) + 1;
+    u = 31u - (uint32_t)(last & 31);
     cur = word(j);
     prv = word(j - 1);
     rb = (j - 2) >> 2;  // floor: the block of word j - 2
@@ -1416,7 +1416,7 @@ struct BackBits {
   }
   // the 32 bits before the read position, the last of them in bit 0 (bits before the payload's
   // first word read as 0)
-  __device__ __forceinline__ uint32_t peek() const { return __funnelshift_r(cur, prv, 32 - t); }
+  __device__ __forceinline__ uint32_t peek() const { return __funnelshift_r(cur, prv, u); }
   __device__ __forceinline__ void advance() {
     --j;
     cur = prv;
@@ -1431,10 +1431,9 @@ struct BackBits {
   }
   // moves the read position back by len (<= 31) bits
   __device__ __forceinline__ void skip(uint32_t len) {
-    if (t > len) {
-      t -= len;
-    } else {
-      t += 32 - len;
+    u += len;
+    if (u >= 32) {
+      u -= 32;
       advance();
     }
   }
@@ -1444,7 +1443,7 @@ struct BackBits {
     skip(len);
     return v;
   }
-  __device__ __forceinline__ int64_t position() const { return 32ll * j + t; }
+  __device__ __forceinline__ int64_t position() const { return 32ll * j + 32 - u; }
 };
 
 
