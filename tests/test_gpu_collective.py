@@ -1,6 +1,6 @@
-"""The compressed all-gather on a GPU with NCCL and the real coder, as one rank (the exchange
-between two ranks is covered on CPU ranks), in a child process so the process group does not
-outlive the test."""
+"""The compressed all-gather on a GPU with NCCL and the real coder (each of the four stream
+kinds), as one rank (the exchange between two ranks is covered on CPU ranks), in a child process
+so the process group does not outlive the test."""
 import os
 import socket
 
@@ -33,13 +33,14 @@ def _rank(port, q):
                             timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda:0"))
     try:
         res = {}
-        for kind in (hx.KIND_HUFFMAN, hx.KIND_QLC):
+        prior = sum(oracle.histogram(b) for b in datagen.prior_batches(1))
+        books = {hx.KIND_HUFFMAN: (hx.build_codebook(prior), oracle.huffman_codebook(prior)),
+                 hx.KIND_QLC: (hx.qlc_build(prior), oracle.qlc_codebook(prior)),
+                 hx.KIND_SHANNONIC: (hx.shannonic_build(prior), oracle.shannonic_codebook(prior)),
+                 hx.KIND_EXPGOLOMB: (hx.expgolomb_build(6, 0), oracle.ExpGolombBook(6, 0))}
+        for kind, (cb, ocb) in books.items():
             for parts in (1, 3):
                 x = datagen.data(1, n=(1 << 20) - 77)
-                prior = sum(oracle.histogram(b) for b in datagen.prior_batches(1))
-                cb = hx.build_codebook(prior) if kind == hx.KIND_HUFFMAN else hx.qlc_build(prior)
-                ocb = (oracle.huffman_codebook(prior) if kind == hx.KIND_HUFFMAN
-                       else oracle.qlc_codebook(prior))
                 out, sizes = collective.compressed_all_gather(
                     torch.from_numpy(x).cuda(), cb.upload("cuda"), codec=collective.Codec(kind),
                     parts=parts)
@@ -71,6 +72,6 @@ def test_one_rank_round_trip():
     res = q.get(timeout=300)
     p.join(120)
     assert p.exitcode == 0
-    assert len(res) == 4
+    assert len(res) == 8
     for case, (ok, sizes, ref_size, same_stream) in res.items():
         assert ok and sizes == [ref_size] and same_stream, case
