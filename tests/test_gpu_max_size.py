@@ -40,13 +40,15 @@ def chunk_bytes(tile, c):
     return np.concatenate([tile, tile])[lo % TILE:lo % TILE + (hi - lo)]
 
 
-@pytest.mark.parametrize("kind", ["huffman", "qlc"])
+@pytest.mark.parametrize("kind", ["huffman", "qlc", "shannonic"])
 def test_max_size_stream(orc, setup, kind):
     tile, counts, x, hist_expected = setup
     if kind == "huffman":
         cb, ocb = hx.build_codebook(counts), orc.huffman_codebook(counts)
-    else:
+    elif kind == "qlc":
         cb, ocb = hx.qlc_build(counts), orc.qlc_codebook(counts)
+    else:  # 2^18 groups of 4 chunks in the Shannonic encoder's look-back
+        cb, ocb = hx.shannonic_build(counts), orc.shannonic_codebook(counts)
     tables = cb.upload()
     hist = torch.zeros(256, dtype=torch.int32, device="cuda")
     out, st = hx.encode(tables, x, hist=hist, kind=cb.kind)
